@@ -1,0 +1,178 @@
+/*
+ * kda.h -- C ABI of libkda: the Kimi Delta Attention (KDA) operator on one NVIDIA B200 (sm_100a).
+ *
+ * The operator.  KDA is Gated DeltaNet with the scalar per-head gate replaced by a per-channel gate
+ * on the key dimension ("Kimi K3 구조 분석" page, key messages; llm-wiki "Kimi K3" chapter, section 1
+ * "GatedDeltaNet과 KDA의 차이").  Per (sequence, head) it keeps a fixed-size state S (dk x dv) that is
+ * updated once per token and read by multiplying the query into it (same chapter, section 1):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,        o_t = S_t^T q_t,
+ *
+ * with alpha_t = exp(max(log_alpha_t, ln 0.0067)): every step keeps at least 0.67 % of what it held
+ * (orkas.ai "Kimi K3 architecture" post, section "GPU 코드 경로 하나를 없앤 하한").  There is no scale
+ * on q.  A NaN log-decay is treated as the floor (fmaxf semantics).
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers unless the argument says "host".  The caller owns every buffer; the
+ *    library never allocates device memory and keeps no state between calls apart from one status
+ *    word per device (see kda_get_device_status).
+ *  - Layouts are dense row-major, token-major with heads interleaved:
+ *        q, k, log_alpha: [T_tot, H, dk]     v, o: [T_tot, H, dv]     beta: [T_tot, H]
+ *        states: [N, H, dk, dv] fp32 (dv contiguous)
+ *    Alignment: states, checkpoints, transitions, the chunk path's q/k/v/log_alpha/o and the
+ *    decode state must be 16-byte aligned (TMA tiles and 16-byte vectors); beta, the int32 tables and
+ *    the decode step's per-token inputs need only their natural alignment.  The workspace must be
+ *    256-byte aligned.
+ *  - dtype (kda_dtype_t) is the element type of q, k, v and o.  log_alpha, beta and all states are
+ *    fp32 always.
+ *  - Calls are asynchronous on `stream`.  Argument errors that the host can see are returned before
+ *    anything is launched.  Errors that only the device can see (a bad cu_seqlens table, a bounded
+ *    wait that ran out) are recorded in the per-device status word and read with
+ *    kda_get_device_status; the kernels never trap.
+ *  - Supported sizes: dk, dv in {64, 128} for KDA_F32; dk = 128 and dv in {64, 128} for KDA_BF16.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kda_stream_t;   /* same type as cudaStream_t; NULL = legacy default */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_ARG = -1,          /* null pointer, bad size, non-monotone host table, ... */
+    KDA_ERR_ALIGN = -2,        /* a pointer is not aligned as documented above */
+    KDA_ERR_UNSUPPORTED = -3,  /* dk/dv/dtype combination not built */
+    KDA_ERR_CUDA = -4,         /* a CUDA runtime call failed (launch, symbol, attribute) */
+    KDA_ERR_TIMEOUT = -5,      /* device: a bounded wait inside a kernel ran out */
+    KDA_ERR_WORKSPACE = -6,    /* workspace too small for even one chunk window */
+    KDA_ERR_DEVICE_INPUT = -7  /* device: cu_seqlens / seg_cu / ckpt_cu inconsistent */
+} kda_status_t;
+
+typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype_t;
+
+/* Token count of one chunk of the chunked form (fixed) and of the tiles inside it. */
+#define KDA_CHUNK 64
+#define KDA_TILE 16
+
+/*
+ * Workspace bytes that let kda_chunk_fwd process the whole batch in one pass.  A smaller workspace
+ * (at least kda_chunk_fwd_min_workspace_bytes) makes the call process the chunks in windows, one
+ * after another, carrying the state between windows; results are identical.
+ */
+KDA_API size_t kda_chunk_fwd_workspace_bytes(int64_t total_tokens, int n_seqs, int H, int dk, int dv,
+                                     kda_dtype_t dtype);
+KDA_API size_t kda_chunk_fwd_min_workspace_bytes(int n_seqs, int H, int dk, int dv, kda_dtype_t dtype);
+
+/*
+ * Chunked (prefill) form over a packed batch of N sequences.
+ *
+ * The sequences are packed along the token axis; cu_seqlens (device, int32 [N+1], cu[0] = 0,
+ * non-decreasing, cu[N] = total_tokens) gives their offsets.  Each sequence is cut into chunks of
+ * KDA_CHUNK tokens; inside a chunk the cumulative log-decay is anchored at 16-token tile boundaries
+ * so that the inverse decay inside a tile stays below e^80.09 and the diagonal tiles use the same
+ * dense bf16 tensor-core product as all other tiles (orkas.ai post, decay-floor section).  The
+ * intra-chunk system (I + strict_tril(beta K Gamma K^T))^-1 is solved by blocked forward
+ * substitution over 16x16 tiles, and the state is carried across chunks in fp32.
+ *
+ *   initial_state   [N,H,dk,dv] fp32, or NULL for zero.
+ *   o               [T_tot,H,dv] of `dtype` (written for every token).
+ *   final_state     [N,H,dk,dv] fp32, or NULL.
+ *   ckpt_stride     0 = no checkpoints, else a positive multiple of KDA_CHUNK (512 for the prefix
+ *                   cache of the orkas.ai post's serving section: hashes every 512 tokens, sparse
+ *                   state checkpoints at hash ends).  Checkpoint j (1-based) of sequence i is the state
+ *                   after j*ckpt_stride tokens, stored at checkpoints[ckpt_cu[i] + j - 1]
+ *                   ([*,H,dk,dv] fp32); ckpt_cu is the device copy of the table that
+ *                   kda_ckpt_offsets fills.  When the stride divides len_i the last checkpoint equals
+ *                   final_state.
+ *   final_transition [N,H,dk,dk] fp32 or NULL: prod_t (I - beta_t k_t k_t^T) Diag(alpha_t) over the
+ *                   sequence (the "cumulative transition" of the sequence-split paragraph of the
+ *                   orkas.ai serving section; input of kda_segment_compose).
+ *   workspace       device scratch of ws_bytes (see above), 256-byte aligned; contents on entry are
+ *                   ignored.
+ * Resuming from a checkpoint: run the suffix [b, len) with initial_state = the checkpoint at b; when b
+ * is a multiple of KDA_CHUNK the chunk grid coincides with that of the unsplit run.
+ */
+KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v,
+                           const float* log_alpha, const float* beta,
+                           const float* initial_state,
+                           const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
+                           int H, int dk, int dv, kda_dtype_t dtype,
+                           int ckpt_stride,
+                           void* o, float* final_state,
+                           float* checkpoints, const int32_t* ckpt_cu,
+                           float* final_transition,
+                           void* workspace, size_t ws_bytes, kda_stream_t stream);
+
+/*
+ * One recurrent (decode) step for n sequences x H heads, state updated in place: the fixed-size
+ * state of the llm-wiki chapter's section 1 (O(1) memory per token).  state [n,H,dk,dv] fp32;
+ * q, k [n,H,dk], v [n,H,dv] of `dtype`; log_alpha [n,H,dk] fp32; beta [n,H] fp32; o [n,H,dv] of
+ * `dtype`.  Memory-bound: each call reads and writes the whole state once.
+ */
+KDA_API kda_status_t kda_recurrent_step(float* state, const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta,
+                                int n, int H, int dk, int dv, kda_dtype_t dtype,
+                                void* o, kda_stream_t stream);
+
+/*
+ * Segment composition (orkas.ai serving section, sequence split): each segment s of a sequence is
+ * summarised by its cumulative transition M_s [dk,dk] and its zero-start final state Z_s [dk,dv]
+ * (both from kda_chunk_fwd run on the segment from a zero state with final_transition set).  An
+ * exclusive prefix scan X_0 = init, X_{s+1} = M_s X_s + Z_s recovers every segment's start state.
+ *   transitions  [S,H,dk,dk] fp32;  zero_states [S,H,dk,dv] fp32  (S = total segments)
+ *   seg_cu       device int32 [n_seqs+1]: segments of sequence i are seg_cu[i] .. seg_cu[i+1]-1
+ *   init         [n_seqs,H,dk,dv] fp32 or NULL (zero)
+ *   start_states [S,H,dk,dv] fp32 (X_s of each segment);  end_states [n_seqs,H,dk,dv] or NULL.
+ */
+KDA_API kda_status_t kda_segment_compose(const float* transitions, const float* zero_states,
+                                 const int32_t* seg_cu, const float* init,
+                                 int n_seqs, int n_segs, int H, int dk, int dv,
+                                 float* start_states, float* end_states, kda_stream_t stream);
+
+/*
+ * Host-only, pure: checkpoint offsets for kda_chunk_fwd.  host_ckpt_cu[0] = 0 and
+ * host_ckpt_cu[i+1] = host_ckpt_cu[i] + floor(len_i / stride) with len_i from host_cu_seqlens
+ * (host int32 [n+1]).  Returns KDA_ERR_ARG on a bad stride or a decreasing table.
+ */
+KDA_API kda_status_t kda_ckpt_offsets(const int32_t* host_cu_seqlens, int n, int stride,
+                              int32_t* host_ckpt_cu);
+
+/* Synchronises `stream`, returns the current device's status word (KDA_OK if no kernel recorded an
+ * error) and clears it. */
+KDA_API kda_status_t kda_get_device_status(kda_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+KDA_API const char* kda_status_string(kda_status_t status);
+
+/* Version string of the library build. */
+KDA_API const char* kda_version(void);
+
+/*
+ * Diagnostics (no KDA arithmetic).
+ *  kda_selftest_wait_timeout: launches one tiny kernel that waits on an mbarrier nothing will
+ *  complete, with a wait limit of limit_us microseconds; returns KDA_ERR_TIMEOUT when the bounded
+ *  wait ran out as designed (and leaves the status word clear).  Shows on a live GPU that the
+ *  kernels' waits end without a fault.
+ *  kda_selftest_umma: one 128 x n x 64 bf16 tcgen05 product D = A B^T through the same shared-memory
+ *  descriptors, TMEM allocation and load path the chunk kernels use. a [128,64], b [n,64] bf16
+ *  row-major (device), d [128,n] fp32 (device); n in {16, 32, ..., 256}.
+ */
+KDA_API kda_status_t kda_selftest_wait_timeout(int limit_us, kda_stream_t stream);
+KDA_API kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H_ */

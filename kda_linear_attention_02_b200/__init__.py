@@ -1,0 +1,244 @@
+"""kda_linear_attention_02_b200 -- Kimi Delta Attention (KDA) on one NVIDIA B200.
+
+A thin Python binding over the C ABI of ``libkda.so`` (see ``include/kda.h``).  Every function here
+has the name of the C entry point it calls and only marshals arguments: it checks shapes, dtypes
+and devices of torch tensors, turns them into raw pointers and passes the current CUDA stream.  All
+of the operator's arithmetic runs in the library's CUDA kernels; there is no fallback.  If the
+library has not been built the import of any entry point fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "KDA_BF16", "KDA_F32", "KDA_CHUNK", "KDAError", "lib_path",
+    "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd",
+    "kda_recurrent_step", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
+    "kda_status_string", "kda_version", "kda_selftest_wait_timeout", "kda_selftest_umma",
+]
+
+KDA_BF16 = 0
+KDA_F32 = 1
+KDA_CHUNK = 64
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libkda.so")
+_lib = None
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {kda_status_string(status)} ({status})")
+        self.status = status
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"libkda.so is not built ({_LIB_PATH}); run "
+                           "`python -m kda_linear_attention_02_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    L.kda_chunk_fwd_workspace_bytes.restype = sz
+    L.kda_chunk_fwd_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i32]
+    L.kda_chunk_fwd_min_workspace_bytes.restype = sz
+    L.kda_chunk_fwd_min_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    L.kda_chunk_fwd.restype = i32
+    L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32,
+                                vp, vp, vp, vp, vp, vp, sz, vp]
+    L.kda_recurrent_step.restype = i32
+    L.kda_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
+    L.kda_segment_compose.restype = i32
+    L.kda_segment_compose.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.kda_ckpt_offsets.restype = i32
+    L.kda_ckpt_offsets.argtypes = [vp, i32, i32, vp]
+    L.kda_get_device_status.restype = i32
+    L.kda_get_device_status.argtypes = [vp]
+    L.kda_status_string.restype = ctypes.c_char_p
+    L.kda_status_string.argtypes = [i32]
+    L.kda_version.restype = ctypes.c_char_p
+    L.kda_version.argtypes = []
+    L.kda_selftest_wait_timeout.restype = i32
+    L.kda_selftest_wait_timeout.argtypes = [i32, vp]
+    L.kda_selftest_umma.restype = i32
+    L.kda_selftest_umma.argtypes = [vp, vp, vp, i32, vp]
+    _lib = L
+    return L
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"q/k/v/o must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need(t, name, shape=None, dtype=None, device=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+
+
+def _opt(t, name, shape, dtype, device):
+    if t is not None:
+        _need(t, name, shape, dtype, device)
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise KDAError(st, where)
+
+
+def kda_status_string(status: int) -> str:
+    return _load().kda_status_string(int(status)).decode()
+
+
+def kda_version() -> str:
+    return _load().kda_version().decode()
+
+
+def kda_chunk_fwd_workspace_bytes(total_tokens, n_seqs, H, dk, dv, dtype=KDA_BF16) -> int:
+    return int(_load().kda_chunk_fwd_workspace_bytes(int(total_tokens), int(n_seqs), int(H), int(dk), int(dv),
+                                                     int(dtype)))
+
+
+def kda_chunk_fwd_min_workspace_bytes(n_seqs, H, dk, dv, dtype=KDA_BF16) -> int:
+    return int(_load().kda_chunk_fwd_min_workspace_bytes(int(n_seqs), int(H), int(dk), int(dv), int(dtype)))
+
+
+def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, o, final_state=None, *,
+                  ckpt_stride=0, checkpoints=None, ckpt_cu=None, final_transition=None, workspace=None,
+                  stream=None):
+    """Chunked KDA forward over a packed batch (C: kda_chunk_fwd).
+
+    q, k, log_alpha [T,H,dk]; v, o [T,H,dv]; beta [T,H]; cu_seqlens int32 [N+1] (device);
+    initial_state / final_state [N,H,dk,dv] fp32 or None; checkpoints [*,H,dk,dv] fp32 with
+    ckpt_cu int32 [N+1] (device); final_transition [N,H,dk,dk] fp32 or None; workspace: uint8
+    device tensor (allocated here from torch's allocator when None).  Outputs are written in place.
+    """
+    _need(q, "q")
+    dev = q.device
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    n = cu_seqlens.numel() - 1
+    _need(k, "k", (T, H, dk), q.dtype, dev)
+    _need(v, "v", (T, H, dv), q.dtype, dev)
+    _need(o, "o", (T, H, dv), q.dtype, dev)
+    _need(log_alpha, "log_alpha", (T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (T, H), torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", (n + 1,), torch.int32, dev)
+    _opt(initial_state, "initial_state", (n, H, dk, dv), torch.float32, dev)
+    _opt(final_state, "final_state", (n, H, dk, dv), torch.float32, dev)
+    _opt(final_transition, "final_transition", (n, H, dk, dk), torch.float32, dev)
+    if ckpt_stride:
+        _need(checkpoints, "checkpoints", None, torch.float32, dev)
+        if checkpoints.dim() != 4 or tuple(checkpoints.shape[1:]) != (H, dk, dv):
+            raise ValueError("checkpoints must be [n_ckpt, H, dk, dv]")
+        _need(ckpt_cu, "ckpt_cu", (n + 1,), torch.int32, dev)
+    if workspace is None:
+        nbytes = kda_chunk_fwd_workspace_bytes(T, n, H, dk, dv, dt)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", None, torch.uint8, dev)
+    st = _load().kda_chunk_fwd(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(initial_state), _p(cu_seqlens),
+                               n, T, H, dk, dv, dt, int(ckpt_stride), _p(o), _p(final_state),
+                               _p(checkpoints if ckpt_stride else None), _p(ckpt_cu if ckpt_stride else None),
+                               _p(final_transition), _p(workspace), workspace.numel(), _stream(stream))
+    _check(st, "kda_chunk_fwd")
+    return o
+
+
+def kda_recurrent_step(state, q, k, v, log_alpha, beta, o, *, stream=None):
+    """One decode step, state [n,H,dk,dv] fp32 updated in place (C: kda_recurrent_step).
+
+    q, k [n,H,dk]; v, o [n,H,dv] (bf16 or fp32); log_alpha [n,H,dk] fp32; beta [n,H] fp32.
+    """
+    _need(state, "state", None, torch.float32)
+    dev = state.device
+    n, H, dk, dv = state.shape
+    dt = _dtype_code(q)
+    _need(q, "q", (n, H, dk), q.dtype, dev)
+    _need(k, "k", (n, H, dk), q.dtype, dev)
+    _need(v, "v", (n, H, dv), q.dtype, dev)
+    _need(o, "o", (n, H, dv), q.dtype, dev)
+    _need(log_alpha, "log_alpha", (n, H, dk), torch.float32, dev)
+    _need(beta, "beta", (n, H), torch.float32, dev)
+    st = _load().kda_recurrent_step(_p(state), _p(q), _p(k), _p(v), _p(log_alpha), _p(beta), n, H, dk, dv, dt,
+                                    _p(o), _stream(stream))
+    _check(st, "kda_recurrent_step")
+    return o
+
+
+def kda_segment_compose(transitions, zero_states, seg_cu, init, start_states, end_states=None, *, stream=None):
+    """Prefix scan X_{s+1} = M_s X_s + Z_s over each sequence's segments (C: kda_segment_compose).
+
+    transitions [S,H,dk,dk]; zero_states, start_states [S,H,dk,dv]; seg_cu int32 [N+1] (device);
+    init / end_states [N,H,dk,dv] or None.  All fp32.
+    """
+    _need(zero_states, "zero_states", None, torch.float32)
+    dev = zero_states.device
+    S, H, dk, dv = zero_states.shape
+    n = seg_cu.numel() - 1
+    _need(transitions, "transitions", (S, H, dk, dk), torch.float32, dev)
+    _need(seg_cu, "seg_cu", (n + 1,), torch.int32, dev)
+    _need(start_states, "start_states", (S, H, dk, dv), torch.float32, dev)
+    _opt(init, "init", (n, H, dk, dv), torch.float32, dev)
+    _opt(end_states, "end_states", (n, H, dk, dv), torch.float32, dev)
+    st = _load().kda_segment_compose(_p(transitions), _p(zero_states), _p(seg_cu), _p(init), n, S, H, dk, dv,
+                                     _p(start_states), _p(end_states), _stream(stream))
+    _check(st, "kda_segment_compose")
+    return start_states
+
+
+def kda_ckpt_offsets(cu_seqlens_host, stride: int) -> torch.Tensor:
+    """Host-only checkpoint offsets (C: kda_ckpt_offsets); returns an int32 CPU tensor [N+1]."""
+    cu = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous().cpu()
+    n = cu.numel() - 1
+    out = torch.empty(n + 1, dtype=torch.int32)
+    _check(_load().kda_ckpt_offsets(_p(cu), n, int(stride), _p(out)), "kda_ckpt_offsets")
+    return out
+
+
+def kda_get_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status word."""
+    return int(_load().kda_get_device_status(_stream(stream)))
+
+
+def kda_selftest_wait_timeout(limit_us: int = 2000, stream=None) -> int:
+    return int(_load().kda_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def kda_selftest_umma(a, b, d, *, stream=None):
+    n = b.shape[0]
+    _need(a, "a", (128, 64), torch.bfloat16)
+    _need(b, "b", (n, 64), torch.bfloat16, a.device)
+    _need(d, "d", (128, n), torch.float32, a.device)
+    _check(_load().kda_selftest_umma(_p(a), _p(b), _p(d), n, _stream(stream)), "kda_selftest_umma")
+    return d

@@ -1,0 +1,62 @@
+// kda_internal.h -- host-side launch functions shared between the libkda translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+// Decode step (kda_decode.cu).
+cudaError_t launch_decode(float* state, const void* q, const void* k, const void* v, const float* la,
+                          const float* beta, void* o, int nh, int dk, int dv, bool bf16, cudaStream_t s);
+
+// Segment compose (kda_compose.cu).
+cudaError_t launch_compose(const float* M, const float* Z, const int32_t* seg_cu, const float* init, int n_seqs,
+                           int n_segs, int H, int dk, int dv, float* starts, float* ends, int* status,
+                           cudaStream_t s);
+
+// Everything one chunk-path launch needs (kda_chunk_f32.cu / kda_chunk_bf16.cu).
+struct ChunkArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_alpha;
+    const float* beta;
+    const float* initial_state;
+    const int32_t* cu_seqlens;
+    const int32_t* cu_chunks;   // device [N+1], filled by launch_chunk_index
+    int n_seqs;
+    int64_t total_tokens;
+    int H, dk, dv;
+    int ckpt_stride;
+    void* o;
+    float* final_state;
+    float* checkpoints;
+    const int32_t* ckpt_cu;
+    float* final_transition;
+    float* carry;               // [N,H,dk,dv+dk] fp32 state carried between windows (or null)
+    void* packets;              // window of per-(chunk, head) packets
+    long long win_lo, win_hi;   // global chunk index window [lo, hi)
+    bool multi_window;
+    int* status;                // device status word
+};
+
+// Builds cu_chunks[i] = sum_{j<i} ceil(len_j / 64) from cu_seqlens and validates the table.
+cudaError_t launch_chunk_index(const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens, int32_t* cu_chunks,
+                               int* status, cudaStream_t s);
+
+// fp32 path: SIMT fp32 intra-chunk prep + inter-chunk state pass.
+size_t chunk_packet_bytes_f32(int dk, int dv);
+cudaError_t launch_chunk_f32(const ChunkArgs& a, cudaStream_t s);
+
+// bf16 path: tcgen05 intra-chunk prep + tcgen05 inter-chunk state pass.
+size_t chunk_packet_bytes_bf16(int dk, int dv);
+cudaError_t launch_chunk_bf16(const ChunkArgs& a, cudaStream_t s);
+
+// Diagnostics.
+cudaError_t launch_selftest_wait(int limit_us, int* d_result, cudaStream_t s);
+cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int* status, cudaStream_t s);
+
+}  // namespace kda

@@ -1,0 +1,78 @@
+// kda_umma_selftest.cu -- diagnostic: one tcgen05 bf16 product through the same shared-memory
+// descriptors (K-major, 128-byte swizzle), TMEM allocation, commit and TMEM-load path that the chunk
+// kernels use.  D[128, n] = A[128, 64] * B[n, 64]^T.  No KDA arithmetic.
+#include "kda_device.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+__global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16* __restrict__ a,
+                                                            const __nv_bfloat16* __restrict__ b,
+                                                            float* __restrict__ d, int n, int* status) {
+    extern __shared__ __align__(1024) uint8_t raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = base;                 // 128 rows x 128 B
+    uint8_t* sB = base + 128 * 128;     // n rows x 128 B
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t tbase;
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+
+    // stage rows into the K-major 128B-swizzled layout: 16-byte chunk c of row r goes to chunk c ^ (r % 8)
+    for (int e = t; e < 128 * 8; e += 128) {
+        const int r = e >> 3, c = e & 7;
+        const uint4 x = reinterpret_cast<const uint4*>(a + r * 64)[c];
+        *reinterpret_cast<uint4*>(sA + sw128_offset(r, c * 8, 128)) = x;
+    }
+    for (int e = t; e < n * 8; e += 128) {
+        const int r = e >> 3, c = e & 7;
+        const uint4 x = reinterpret_cast<const uint4*>(b + r * 64)[c];
+        *reinterpret_cast<uint4*>(sB + sw128_offset(r, c * 8, n)) = x;
+    }
+    fence_proxy_async_smem();
+    if (t == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    if (w == 0) {
+        tmem_alloc(&tbase, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tbase;
+    if (t == 0) {
+        const uint32_t idesc = idesc_bf16(128, n);
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = sdesc_k_sw128(smem_u32(sA) + kk * 32);
+            const uint64_t db = sdesc_k_sw128(smem_u32(sB) + kk * 32);
+            umma_f16(tm, da, db, idesc, kk > 0);
+        }
+        umma_commit(&bar);
+    }
+    __syncwarp();
+    const bool ok = mbar_wait(&bar, 0, status);
+    tc_fence_after();
+    if (ok) {
+        for (int c0 = 0; c0 < n; c0 += 16) {
+            float r[16];
+            tmem_ld16(tm + (static_cast<uint32_t>(32 * w) << 16) + c0, r);
+            tmem_wait_ld();
+            for (int j = 0; j < 16; ++j) d[(32 * w + lane) * n + c0 + j] = r[j];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tm, 256);
+}
+
+cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int* status, cudaStream_t s) {
+    const int smem = 1024 + 128 * 128 + n * 128;
+    cudaError_t e = cudaFuncSetAttribute(selftest_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    selftest_umma_kernel<<<1, 128, smem, s>>>(static_cast<const __nv_bfloat16*>(a),
+                                              static_cast<const __nv_bfloat16*>(b), d, n, status);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

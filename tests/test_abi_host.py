@@ -1,0 +1,135 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every entry point that
+include/kda.h declares, computes the checkpoint table, sizes its workspace, and rejects bad
+arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import kda_linear_attention_02_b200 as kda
+from kda_linear_attention_02_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda._load()
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "kda.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = _declared_symbols()
+    assert len(syms) >= 10
+    for s in syms:
+        assert hasattr(lib, s), f"libkda.so does not export {s}"
+    # and nothing else leaks out besides the declared entry points
+    assert ctypes.CDLL(kda.lib_path()).kda_version() != 0
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in kda.kda_version()
+    assert kda.kda_status_string(0) == "KDA_OK"
+    assert kda.kda_status_string(-5) == "KDA_ERR_TIMEOUT"
+    assert kda.kda_status_string(-7) == "KDA_ERR_DEVICE_INPUT"
+
+
+def _brute_ckpt_cu(cu, stride):
+    out = [0]
+    for i in range(len(cu) - 1):
+        L = cu[i + 1] - cu[i]
+        out.append(out[-1] + sum(1 for j in range(1, L + 1) if j % stride == 0))
+    return out
+
+
+@pytest.mark.parametrize("stride", [64, 512, 1024])
+def test_ckpt_offsets_bit_exact(lib, stride):
+    from kda_linear_attention_02_b200 import synth
+    lengths = synth.varlen_lengths(64, 1024, 65536, 1) + [0, 511, 512, 513, 1]
+    cu = synth.cu_from_lengths(lengths).tolist()
+    got = kda.kda_ckpt_offsets(cu, stride).tolist()
+    assert got == _brute_ckpt_cu(cu, stride)
+
+
+def test_ckpt_offsets_rejects_bad_tables(lib):
+    with pytest.raises(kda.KDAError):
+        kda.kda_ckpt_offsets([0, 10, 5], 64)
+    with pytest.raises(kda.KDAError):
+        kda.kda_ckpt_offsets([1, 10], 64)
+    with pytest.raises(kda.KDAError):
+        kda.kda_ckpt_offsets([0, 10], 0)
+
+
+def test_varlen_lengths_recipe():
+    from kda_linear_attention_02_b200 import synth
+    L = synth.varlen_lengths(64, 1024, 65536, 1)
+    assert len(L) == 64 and min(L) >= 1024 and max(L) <= 65536
+    assert L == synth.varlen_lengths(64, 1024, 65536, 1)
+
+
+def test_workspace_sizes(lib):
+    full = kda.kda_chunk_fwd_workspace_bytes(4 * 4096, 4, 32, 128, 128, kda.KDA_BF16)
+    mini = kda.kda_chunk_fwd_min_workspace_bytes(4, 32, 128, 128, kda.KDA_BF16)
+    assert full > mini > 0
+    assert kda.kda_chunk_fwd_workspace_bytes(100, 1, 2, 64, 64, kda.KDA_F32) > 0
+    # unsupported combinations report 0
+    assert kda.kda_chunk_fwd_workspace_bytes(100, 1, 2, 96, 64, kda.KDA_F32) == 0
+    assert kda.kda_chunk_fwd_workspace_bytes(100, 1, 2, 64, 64, kda.KDA_BF16) == 0
+
+
+def _call_chunk(lib, **over):
+    """Raw C call with fake (never dereferenced) pointers: all of these must fail on the host."""
+    a = dict(q=0x1000, k=0x2000, v=0x3000, la=0x4000, b=0x5000, s0=None, cu=0x6000, n=2, T=100, H=4, dk=128,
+             dv=128, dt=0, stride=0, o=0x7000, fs=None, ck=None, ckcu=None, tr=None, ws=0x10000, wsb=1 << 30)
+    a.update(over)
+    vp = ctypes.c_void_p
+    return lib.kda_chunk_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["la"]), vp(a["b"]), vp(a["s0"]),
+                             vp(a["cu"]), a["n"], a["T"], a["H"], a["dk"], a["dv"], a["dt"], a["stride"], vp(a["o"]),
+                             vp(a["fs"]), vp(a["ck"]), vp(a["ckcu"]), vp(a["tr"]), vp(a["ws"]), a["wsb"], None)
+
+
+def test_chunk_fwd_host_argument_errors(lib):
+    assert _call_chunk(lib, H=0) == -1
+    assert _call_chunk(lib, n=-1) == -1
+    assert _call_chunk(lib, T=-5) == -1
+    assert _call_chunk(lib, dt=7) == -1
+    assert _call_chunk(lib, dk=96) == -3
+    assert _call_chunk(lib, dk=64, dt=0) == -3            # bf16 path needs dk = 128
+    assert _call_chunk(lib, stride=100, ck=0x8000, ckcu=0x9000) == -1   # not a multiple of 64
+    assert _call_chunk(lib, stride=512) == -1             # checkpoints missing
+    assert _call_chunk(lib, q=None) == -1
+    assert _call_chunk(lib, cu=None) == -1
+    assert _call_chunk(lib, ws=None) == -1
+    assert _call_chunk(lib, q=0x1004) == -2               # misaligned
+    assert _call_chunk(lib, ws=0x10010) == -2             # workspace must be 256-byte aligned
+    assert _call_chunk(lib, wsb=100) == -6                # workspace too small
+    assert _call_chunk(lib, n=0) == 0                     # empty batch: nothing to do
+
+
+def test_decode_and_compose_host_argument_errors(lib):
+    vp = ctypes.c_void_p
+    ok = [vp(0x1000)] * 6
+    assert lib.kda_recurrent_step(*ok, 1, 0, 128, 128, 0, vp(0x2000), None) == -1
+    assert lib.kda_recurrent_step(*ok, 1, 1, 96, 128, 0, vp(0x2000), None) == -3
+    assert lib.kda_recurrent_step(vp(0x1004), *ok[1:], 1, 1, 128, 128, 0, vp(0x2000), None) == -2
+    assert lib.kda_recurrent_step(*ok, 0, 1, 128, 128, 0, vp(0x2000), None) == 0
+    assert lib.kda_segment_compose(vp(0x1000), vp(0x2000), None, None, 1, 1, 1, 128, 128, vp(0x3000), None,
+                                   None) == -1
+    assert lib.kda_segment_compose(vp(0x1000), vp(0x2000), vp(0x4000), None, 1, 1, 1, 128, 80, vp(0x3000), None,
+                                   None) == -3
+    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 20, None) == -1
+
+
+def test_binding_checks_shapes_on_cpu_tensors(lib):
+    q = torch.zeros(64, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        kda.kda_chunk_fwd(q, q, q[:, :1], torch.zeros(64, 2, 128), torch.zeros(64, 2),
+                          None, torch.tensor([0, 64], dtype=torch.int32), q)

@@ -1,0 +1,160 @@
+"""GPU parity for the decode step, segment compose, the fp32 chunk path and the diagnostics,
+against the fp64 oracle on the same seeded inputs (all calls go through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import kda_linear_attention_02_b200 as kda
+from kda_linear_attention_02_b200 import synth
+from kda_testlib import assert_close, f32np, oracle_slices
+import oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(autouse=True)
+def _clear_status():
+    kda.kda_get_device_status()
+    yield
+    assert kda.kda_get_device_status() == 0, "a kernel recorded an error in the status word"
+
+
+@pytest.mark.parametrize("n", [16, 64, 128, 256])
+def test_selftest_umma_matches_matmul(n):
+    g = torch.Generator(DEV).manual_seed(n)
+    a = torch.randn(128, 64, device=DEV, generator=g).to(torch.bfloat16)
+    b = torch.randn(n, 64, device=DEV, generator=g).to(torch.bfloat16)
+    d = torch.full((128, n), float("nan"), device=DEV)
+    kda.kda_selftest_umma(a, b, d)
+    ref = a.double().cpu() @ b.double().cpu().T
+    np.testing.assert_allclose(d.cpu().numpy(), ref.numpy(), rtol=1e-4, atol=1e-4)
+
+
+def test_bounded_wait_times_out_cleanly():
+    st = kda.kda_selftest_wait_timeout(2000)
+    assert kda.kda_status_string(st) == "KDA_ERR_TIMEOUT"
+    # the context is still usable and the status word is clear
+    x = torch.ones(4, device=DEV) * 2
+    assert float(x.sum()) == 8.0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (128, 64), (64, 64)])
+def test_decode_steps_match_oracle(dtype, dk, dv):
+    n, H, steps = 5, 3, 6
+    s0, q, k, v, la, b = synth.make_decode_inputs(n, H, dk, dv, dtype=dtype, device=DEV, seed=3, steps=steps)
+    state = s0.clone()
+    outs = []
+    for t in range(steps):
+        o = torch.empty(n, H, dv, dtype=dtype, device=DEV)
+        kda.kda_recurrent_step(state, q[t], k[t], v[t], la[t], b[t], o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    O = torch.stack(outs)                       # [steps, n, H, dv]
+    for i in range(n):
+        for h in range(H):
+            r = oracle.kda_seq(f32np(q[:, i, h]), f32np(k[:, i, h]), f32np(v[:, i, h]), f32np(la[:, i, h]),
+                               f32np(b[:, i, h]), s0=s0[i, h].double().cpu().numpy())
+            assert_close(f32np(O[:, i, h]), r["o"], dtype, f"decode o ({i},{h})")
+            assert_close(f32np(state[i, h]), r["state"], dtype, f"decode state ({i},{h})")
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128)])
+def test_segment_compose_matches_oracle(dk, dv):
+    H = 3
+    nseg = [3, 1, 0, 5]
+    S = sum(nseg)
+    g = torch.Generator(DEV).manual_seed(11)
+    M = torch.randn(S, H, dk, dk, device=DEV, generator=g) / (dk ** 0.5)
+    Z = torch.randn(S, H, dk, dv, device=DEV, generator=g)
+    init = torch.randn(len(nseg), H, dk, dv, device=DEV, generator=g)
+    seg_cu = synth.cu_from_lengths(nseg, DEV)
+    starts = torch.full((S, H, dk, dv), float("nan"), device=DEV)
+    ends = torch.full((len(nseg), H, dk, dv), float("nan"), device=DEV)
+    kda.kda_segment_compose(M, Z, seg_cu, init, starts, ends)
+    torch.cuda.synchronize()
+    cu = seg_cu.cpu().tolist()
+    for i in range(len(nseg)):
+        for h in range(H):
+            a, z = cu[i], cu[i + 1]
+            st, en = oracle.segment_compose(M[a:z, h].double().cpu().numpy(), Z[a:z, h].double().cpu().numpy(),
+                                            init[i, h].double().cpu().numpy())
+            if z > a:
+                assert_close(f32np(starts[a:z, h]), st, torch.float32, "compose starts")
+            assert_close(f32np(ends[i, h]), en, torch.float32, "compose end")
+
+
+def _run_chunk(inp, dtype, *, ckpt_stride=0, transition=False, ws_bytes=None, init=True):
+    T, H, dk = inp.q.shape
+    dv = inp.v.shape[-1]
+    n = inp.n_seqs
+    o = torch.full((T, H, dv), float("nan"), dtype=dtype, device=DEV)
+    fs = torch.full((n, H, dk, dv), float("nan"), device=DEV)
+    tr = torch.full((n, H, dk, dk), float("nan"), device=DEV) if transition else None
+    ck = ckcu = None
+    if ckpt_stride:
+        ckcu_h = kda.kda_ckpt_offsets(inp.cu_seqlens.cpu(), ckpt_stride)
+        ck = torch.full((max(1, int(ckcu_h[-1])), H, dk, dv), float("nan"), device=DEV)
+        ckcu = ckcu_h.to(DEV)
+    ws = None
+    if ws_bytes is not None:
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=DEV)
+    kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.state0 if init else None,
+                      inp.cu_seqlens, o, fs, ckpt_stride=ckpt_stride, checkpoints=ck, ckpt_cu=ckcu,
+                      final_transition=tr, workspace=ws)
+    torch.cuda.synchronize()
+    return o, fs, ck, ckcu, tr
+
+
+def _check_chunk(inp, dtype, outs, seqs, heads, ckpt_stride=0, transition=False):
+    o, fs, ck, ckcu, tr = outs
+    res = oracle_slices(inp, seqs, heads, ckpt_stride=ckpt_stride, want_transition=transition)
+    cu = inp.cu_seqlens.cpu().tolist()
+    ckcu = None if ckcu is None else ckcu.cpu().tolist()
+    for (i, h), r in res.items():
+        a, b = cu[i], cu[i + 1]
+        if b > a:
+            assert_close(f32np(o[a:b, h]), r["o"], dtype, f"o seq {i} head {h}")
+        assert_close(f32np(fs[i, h]), r["state"], dtype, f"final state seq {i} head {h}")
+        if ckpt_stride and "marks" in r:
+            nck = len(r["marks"])
+            assert ckcu[i + 1] - ckcu[i] == nck
+            for j in range(nck):
+                assert_close(f32np(ck[ckcu[i] + j, h]), r["marks"][j], dtype, f"ckpt {j} seq {i} head {h}")
+        if transition:
+            assert_close(f32np(tr[i, h]), r["transition"], dtype, f"transition seq {i} head {h}")
+
+
+def test_chunk_f32_pr1_workload():
+    # B=1, T=256, H=2, dk=dv=64, fp32, zero initial state, seed 0
+    inp = synth.make_inputs([256], 2, 64, 64, dtype=torch.float32, device=DEV, seed=0)
+    outs = _run_chunk(inp, torch.float32, init=False)
+    _check_chunk(inp, torch.float32, outs, [0], [0, 1])
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+def test_chunk_f32_varlen_ragged(dk, dv):
+    lengths = [1, 63, 64, 65, 200, 0, 130, 16]
+    inp = synth.make_inputs(lengths, 2, dk, dv, dtype=torch.float32, device=DEV, seed=5, with_state0=True)
+    outs = _run_chunk(inp, torch.float32, ckpt_stride=64, transition=True)
+    _check_chunk(inp, torch.float32, outs, range(len(lengths)), [0, 1], ckpt_stride=64, transition=True)
+
+
+def test_chunk_f32_windows_are_bit_identical():
+    lengths = [300, 5, 129, 64]
+    inp = synth.make_inputs(lengths, 2, 64, 64, dtype=torch.float32, device=DEV, seed=6, with_state0=True)
+    full = _run_chunk(inp, torch.float32, ckpt_stride=128, transition=True)
+    small = kda.kda_chunk_fwd_min_workspace_bytes(4, 2, 64, 64, kda.KDA_F32) + 3 * 2 * 40000
+    win = _run_chunk(inp, torch.float32, ckpt_stride=128, transition=True, ws_bytes=small)
+    for a, b in zip(full, win):
+        if a is not None and a.dtype != torch.int32:
+            assert torch.equal(a, b)
+
+
+def test_chunk_bad_cu_seqlens_is_reported():
+    inp = synth.make_inputs([64, 64], 2, 64, 64, dtype=torch.float32, device=DEV, seed=1)
+    inp.cu_seqlens = torch.tensor([0, 100, 64], dtype=torch.int32, device=DEV)   # not monotone, wrong total
+    o = torch.zeros(128, 2, 64, device=DEV)
+    kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, inp.cu_seqlens, o, None)
+    assert kda.kda_get_device_status() == -7
