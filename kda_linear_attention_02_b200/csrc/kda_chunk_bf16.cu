@@ -1,11 +1,798 @@
-// kda_chunk_bf16.cu -- chunked KDA forward for bf16 inputs on tcgen05 (placeholder during bring-up).
+// kda_chunk_bf16.cu -- chunked KDA forward for bf16 inputs on the sm_100a tensor cores (tcgen05).
+//
+// The chunk algebra (per chunk of C = 64 tokens, positions r; lambda = max(log_alpha, ln 0.0067),
+// g = chunk-local inclusive cumsum of lambda, gamma = exp(g)):
+//   A[r,s]   = beta_r sum_c k_rc k_sc exp(g_rc - g_sc)   (s < r),     Aqk[r,s] = sum_c q_rc k_sc exp(..)  (s <= r)
+//   X = (I + A)^-1 (blocked forward substitution over 16 x 16 tiles),  Y = Aqk X
+//   W = X diag(beta) (K * gamma),  U = X diag(beta) V
+//   P = Q * gamma - Y diag(beta) (K * gamma)  (= Q gamma - Aqk W),   O_intra = Y diag(beta) V  (= Aqk U)
+// and across chunks, with the fp32 state S:
+//   U' = U - W S,   O = P S + O_intra,   S <- Diag(gamma_C) S + (K * exp(g_C - g))^T U'.
+// Folding Aqk into P and O_intra takes the output off the chunk-to-chunk critical path: the
+// inter-chunk step is two dependent products ([-W; P] S, then Kdec^T U').
+//
+// Decay floor (orkas.ai "Kimi K3 architecture" post, section "GPU 코드 경로 하나를 없앤 하한"): with
+// lambda >= ln 0.0067 the cumulative log-decay of a 16-token tile lies in [-80.09, 0], so with the
+// tile anchor b_t (g just before tile t) every factor exp(g_r - b_t) <= 1 and exp(b_t - g_s) <= e^80.09
+// < 3.39e38 fits bf16.  Diagonal 16 x 16 tiles therefore go through the same dense bf16 tensor-core
+// product as every other tile; nothing is computed per position pair in log space.  With row r in
+// tile t the key-side operand of tile t is
+//   s in tile t:          k_s exp(b_t - g_s)                          (<= e^80.09)
+//   s in tile j < t:      k_s exp(b_{j+1} - g_s) exp(b_t - b_{j+1})   (both <= 1)
+// and the row side is k_r exp(g_r - b_t) or q_r exp(g_r - b_t) (<= 1).  Entries with s > r are
+// finite (|.| <= 128 e^80.09 < fp32 max) and are dropped after the product.
+//
+// Kernels:
+//  prep_bf16_kernel   persistent, one (chunk, head) item at a time per CTA: TMA tensor loads of the
+//                     raw tiles (prefetched one item ahead), SIMT exponentials and operand
+//                     construction, tcgen05 products for A/Aqk (4 anchored variants) and for
+//                     [X; Y] (beta K gamma | beta V), fp32 blocked forward substitution in between,
+//                     and a bulk TMA store of the MMA-ready packet.
+//  state_bf16_kernel  one CTA per (sequence, head, dv-slice), warp-specialised: a producer warp
+//                     streams packets through a shared-memory ring with bulk TMA, one thread issues
+//                     the two tcgen05 products per chunk, eight epilogue warps hold the fp32 state in
+//                     registers and feed bf16 copies of S and U' back as the next operands.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "kda_chunk_common.cuh"
 #include "kda_internal.h"
 
 namespace kda {
+namespace {
 
-size_t chunk_packet_bytes_bf16(int dk, int dv) { return 82944; }
+constexpr int kDK = 128;
 
-cudaError_t launch_chunk_bf16(const ChunkArgs& a, cudaStream_t s) { return cudaErrorNotSupported; }
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+__device__ __forceinline__ void st_b32(uint8_t* p, uint32_t v) { *reinterpret_cast<uint32_t*>(p) = v; }
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
+    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+    return __bfloat1622float2(h);
+}
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+    const float2 a = bf2_to_f2(u.x), b = bf2_to_f2(u.y), c = bf2_to_f2(u.z), d = bf2_to_f2(u.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+}
+
+// ------------------------------------------------------------------------------------------------
+// Packet: everything the inter-chunk pass needs for one (chunk, head), laid out exactly as its
+// shared-memory stage so that it moves with plain bulk copies.
+template <int DV>
+struct Pk {
+    static constexpr uint32_t AW = 0;                 // [-W; P]: 128 x 128 bf16, K-major, 128B swizzle, 2 K atoms
+    static constexpr uint32_t KD = 32768;             // Kdec^T:  128 x 64 bf16, K-major, 128B swizzle
+    static constexpr uint32_t U = 49152;              // U:       [DV/8][64][8] bf16 (8-column chunks)
+    static constexpr uint32_t OI = U + DV * 128;      // O_intra: [DV/8][64][8] bf16
+    static constexpr uint32_t G = OI + DV * 128;      // gamma_C: [128] fp32
+    static constexpr uint32_t BYTES = ((G + 512 + 1023) / 1024) * 1024;
+};
+
+// ------------------------------------------------------------------------------------------------
+// prep kernel shared memory (bytes from a 1024-aligned base)
+namespace ps {
+constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_V = 32768, STG_L = 49152;   // raw TMA tiles
+constexpr uint32_t RALL = 81920;     // row side [K e^(g-b); Q e^(g-b)]: 128 x 128 bf16 (A operand)
+constexpr uint32_t BVAR = 114688;    // key side, variant i (rows 16(i+1)) at BVAR + 2048 i (i+1)
+constexpr uint32_t QT = 155648;      // Q * gamma, [64][128] bf16, 16-byte chunks swizzled by row
+constexpr uint32_t BKV = 172032;     // [beta K gamma | beta V]^T: (128+DV) x 64 bf16 (B operand)
+constexpr uint32_t MISC = 204800;    // beta[64] fp32, tile totals [4][128] fp32
+constexpr uint32_t AF = 81920, AQF = 98560, XF = 115200, XY = 132096, TMP = 148480;   // solve (aliases)
+constexpr uint32_t AWS = 81920, US = 114688, OIS = 131072;                           // packet staging
+constexpr uint32_t BYTES = MISC + 256 + 2048;
+constexpr int LDA = 65;              // fp32 row pitch of A, Aqk, X
+}  // namespace ps
+
+template <int DV>
+__device__ __forceinline__ void issue_tile_loads(uint8_t* sm, const CUtensorMap* mq, const CUtensorMap* mk,
+                                                 const CUtensorMap* mv, const CUtensorMap* ml, uint64_t* bar,
+                                                 int h, long long tok0) {
+    const int tok = static_cast<int>(tok0);
+    mbar_arrive_expect_tx(bar, 2 * 16384 + DV * 128 + 32768);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        tma_load_3d(sm + ps::STG_Q + hf * 8192, mq, hf * 64, h, tok, bar);
+        tma_load_3d(sm + ps::STG_K + hf * 8192, mk, hf * 64, h, tok, bar);
+    }
+#pragma unroll
+    for (int hf = 0; hf < DV / 64; ++hf) tma_load_3d(sm + ps::STG_V + hf * 8192, mv, hf * 64, h, tok, bar);
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) tma_load_3d(sm + ps::STG_L + qq * 8192, ml, qq * 32, h, tok, bar);
+}
+
+template <int DV>
+__global__ void __launch_bounds__(256, 1)
+prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_l,
+                 const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
+                 const int32_t* __restrict__ cu_chunks, int n_seqs, int H, long long win_lo, long long n_items,
+                 uint8_t* __restrict__ packets, int* status) {
+    using P = Pk<DV>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    __shared__ __align__(8) uint64_t bar_load, bar_mma;
+    __shared__ uint32_t tmem_slot;
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    float* bet = reinterpret_cast<float*>(sm + ps::MISC);
+    float* tot = bet + 64;
+    float* AF = reinterpret_cast<float*>(sm + ps::AF);
+    float* AQF = reinterpret_cast<float*>(sm + ps::AQF);
+    float* XF = reinterpret_cast<float*>(sm + ps::XF);
+    float* TMP = reinterpret_cast<float*>(sm + ps::TMP);
+    constexpr int LDA = ps::LDA;
+
+    if (t == 0) {
+        mbar_init(&bar_load, 1);
+        mbar_init(&bar_mma, 1);
+        fence_barrier_init();
+        prefetch_tmap(&map_q); prefetch_tmap(&map_k); prefetch_tmap(&map_v); prefetch_tmap(&map_l);
+    }
+    if (w == 0) {
+        tmem_alloc(&tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_slot;
+    uint32_t ph_load = 0, ph_mma = 0;
+    bool load_pending = false;   // meaningful in thread 0 only
+
+    long long item = blockIdx.x;
+    ChunkLoc loc{};
+    int h = static_cast<int>(item % H);
+    bool valid = item < n_items && locate_chunk(cu_chunks, cu_seqlens, n_seqs, win_lo + item / H, loc);
+    if (t == 0 && valid) {
+        issue_tile_loads<DV>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, h, loc.tok0);
+        load_pending = true;
+    }
+
+    while (valid) {
+        const int n = loc.n;
+        uint8_t* pkt = packets + static_cast<size_t>(item) * P::BYTES;
+        if (t < 64) bet[t] = t < n ? beta[(static_cast<size_t>(loc.tok0) + t) * H + h] : 0.f;
+        {
+            const bool ok = mbar_wait(&bar_load, ph_load, status);
+            if (__syncthreads_or(!ok)) break;
+        }
+        ph_load ^= 1;
+        if (t == 0) load_pending = false;
+
+        // ---------------- column pass: thread = (channel pair, 16-token tile)
+        {
+            const int cp = t & 63, tq = t >> 6, c0 = 2 * cp;
+            float2 p[16];
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int r = 16 * tq + j;
+                const float2 la =
+                    *reinterpret_cast<const float2*>(sm + ps::STG_L + (c0 >> 5) * 8192 + r * 128 + (c0 & 31) * 4);
+                if (r < n) {
+                    acc.x += floor_log_decay(la.x);
+                    acc.y += floor_log_decay(la.y);
+                }
+                p[j] = acc;   // g_r - b_tq: the log-decay inside the tile up to r
+            }
+            tot[tq * 128 + c0] = acc.x;
+            tot[tq * 128 + c0 + 1] = acc.y;
+            __syncthreads();
+            float bx[5], by[5];
+            bx[0] = 0.f; by[0] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                bx[i + 1] = bx[i] + tot[i * 128 + c0];
+                by[i + 1] = by[i] + tot[i * 128 + c0 + 1];
+            }
+            // per-(tile, channel) factors, all in [e^-320, 1] or underflowing only when negligible
+            const float ebx = __expf(bx[tq]), eby = __expf(by[tq]);                         // e^{b_t}
+            const float ftx = __expf(bx[tq + 1] - bx[tq]), fty = __expf(by[tq + 1] - by[tq]);   // e^{b_{t+1}-b_t}
+            const float ecx = __expf(bx[4] - bx[tq + 1]), ecy = __expf(by[4] - by[tq + 1]);     // e^{g_C-b_{t+1}}
+            float dvx[4], dvy[4];   // e^{b_i - b_{t+1}}, i > t
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                dvx[i] = i > tq ? __expf(bx[i] - bx[tq + 1]) : 0.f;
+                dvy[i] = i > tq ? __expf(by[i] - by[tq + 1]) : 0.f;
+            }
+            if (tq == 3)
+                *reinterpret_cast<float2*>(pkt + P::G + c0 * 4) = make_float2(__expf(bx[4]), __expf(by[4]));
+
+#pragma unroll
+            for (int grp = 0; grp < 2; ++grp) {
+                float tk[2][8], tv[2][8], td[2][8];   // beta K gamma, beta V, Kdec along 8 tokens
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int j = 8 * grp + jj, r = 16 * tq + j;
+                    const bool in = r < n;
+                    const uint32_t kb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 +
+                                                                           r * 128 + (c0 & 63) * 2);
+                    const uint32_t qb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 +
+                                                                           r * 128 + (c0 & 63) * 2);
+                    const float2 kf = in ? bf2_to_f2(kb) : make_float2(0.f, 0.f);
+                    const float2 qf = in ? bf2_to_f2(qb) : make_float2(0.f, 0.f);
+                    float2 vf = make_float2(0.f, 0.f);
+                    if (c0 < DV && in) {
+                        const uint32_t vb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 +
+                                                                               r * 128 + (c0 & 63) * 2);
+                        vf = bf2_to_f2(vb);
+                    }
+                    const float Ex = __expf(p[j].x), Ey = __expf(p[j].y);     // e^{g_r - b_t} <= 1
+                    const float Ix = __expf(-p[j].x), Iy = __expf(-p[j].y);   // e^{b_t - g_r} <= e^80.09
+                    const float Fx = ftx * Ix, Fy = fty * Iy;                 // e^{b_{t+1} - g_r} <= 1
+                    const float Gx = ebx * Ex, Gy = eby * Ey;                 // e^{g_r}
+                    const float bt = bet[r];
+                    // row side of A / Aqk
+                    st_b32(sm + ps::RALL + sw128_offset(r, c0, 128), pack_bf16x2(kf.x * Ex, kf.y * Ey));
+                    st_b32(sm + ps::RALL + sw128_offset(64 + r, c0, 128), pack_bf16x2(qf.x * Ex, qf.y * Ey));
+                    // key side: own tile (diagonal) and the variants of later row tiles
+                    st_b32(sm + ps::BVAR + 2048 * tq * (tq + 1) + sw128_offset(r, c0, 16 * (tq + 1)),
+                           pack_bf16x2(kf.x * Ix, kf.y * Iy));
+#pragma unroll
+                    for (int i = 1; i < 4; ++i)
+                        if (i > tq)
+                            st_b32(sm + ps::BVAR + 2048 * i * (i + 1) + sw128_offset(r, c0, 16 * (i + 1)),
+                                   pack_bf16x2(kf.x * Fx * dvx[i], kf.y * Fy * dvy[i]));
+                    // Q * gamma for the epilogue (P = Q gamma - ...)
+                    st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2,
+                           pack_bf16x2(qf.x * Gx, qf.y * Gy));
+                    tk[0][jj] = bt * kf.x * Gx; tk[1][jj] = bt * kf.y * Gy;
+                    tv[0][jj] = bt * vf.x;      tv[1][jj] = bt * vf.y;
+                    td[0][jj] = kf.x * ecx * Fx; td[1][jj] = kf.y * ecy * Fy;
+                }
+                const int kc = 2 * tq + grp;   // 8-token chunk index along the 64-token K extent
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    const int c = c0 + ch;
+                    const uint32_t sw = static_cast<uint32_t>((kc ^ (c & 7)) << 4);
+                    *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + sw) = pack8(tk[ch]);
+                    if (c < DV) *reinterpret_cast<uint4*>(sm + ps::BKV + (128 + c) * 128 + sw) = pack8(tv[ch]);
+                    *reinterpret_cast<uint4*>(pkt + P::KD + c * 128 + sw) = pack8(td[ch]);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // prefetch the next item's tiles into the (now free) staging area
+        const long long nitem = item + gridDim.x;
+        ChunkLoc nloc{};
+        const int nh = static_cast<int>(nitem % H);
+        const bool nvalid = nitem < n_items && locate_chunk(cu_chunks, cu_seqlens, n_seqs, win_lo + nitem / H, nloc);
+        if (t == 0 && nvalid) {
+            issue_tile_loads<DV>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.tok0);
+            load_pending = true;
+        }
+
+        // ---------------- phase A: D[m, off_i + s] = RALL[m, :] . BVAR_i[s, :]  (M=128, N=16(i+1), K=128)
+        if (t == 0) {
+            tc_fence_after();
+            const uint32_t ra = smem_u32(sm + ps::RALL);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int nrow = 16 * (i + 1);
+                const uint32_t bv = smem_u32(sm + ps::BVAR + 2048 * i * (i + 1));
+                const uint32_t idesc = idesc_bf16(128, nrow);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
+                    umma_f16(tm + 8 * i * (i + 1), sdesc_k_sw128(ra + ka * 16384 + kb),
+                             sdesc_k_sw128(bv + ka * nrow * 128 + kb), idesc, ks > 0);
+                }
+            }
+            umma_commit(&bar_mma);
+        }
+        {
+            const bool ok = mbar_wait(&bar_mma, ph_mma, status);
+            if (__syncthreads_or(!ok)) break;
+        }
+        ph_mma ^= 1;
+        tc_fence_after();
+
+        // ---------------- TMEM -> fp32 A (strict lower, beta rows) and Aqk (inclusive lower)
+        {
+            const int qw = w & 3, role = w >> 2;
+            const int vi = 2 * (qw & 1) + role;
+            const int nv = 16 * (vi + 1);
+            const int off = 8 * vi * (vi + 1);
+            const int r = (32 * qw + lane) & 63;
+            const bool is_q = qw >= 2;
+            const bool mine = (lane >> 4) == role;
+            float* dst = is_q ? AQF : AF;
+            const float br = bet[r];
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) {
+                float v[16];
+                if (cb < nv) {
+                    tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + off + cb, v);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                }
+                if (mine) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int s = cb + j;
+                        dst[r * LDA + s] = is_q ? (s <= r ? v[j] : 0.f) : (s < r ? br * v[j] : 0.f);
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------- X = (I + A)^-1: diagonal blocks by forward substitution (lane = column) ...
+        if (t < 128 && lane < 16) {
+            const int o0 = 16 * w, col = lane;
+            for (int r = 0; r < 16; ++r) {
+                float x = (r == col) ? 1.f : 0.f;
+                for (int m = col; m < r; ++m) x = fmaf(-AF[(o0 + r) * LDA + o0 + m], XF[(o0 + m) * LDA + o0 + col], x);
+                XF[(o0 + r) * LDA + o0 + col] = x;
+            }
+        }
+        for (int e = t; e < 64 * 64; e += 256) {
+            const int r = e >> 6, s = e & 63;
+            if ((s >> 4) > (r >> 4)) XF[r * LDA + s] = 0.f;
+        }
+        __syncthreads();
+        // ... then the off-diagonal blocks by block diagonal: X_ij = -X_ii sum_{j<=m<i} A_im X_mj
+        for (int d = 1; d < 4; ++d) {
+            const int nb = 4 - d;
+            for (int e = t; e < nb * 256; e += 256) {
+                const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, i = bi + d, j = bi;
+                float a = 0.f;
+                for (int m = 16 * j; m < 16 * i; ++m) a = fmaf(AF[(16 * i + rr) * LDA + m], XF[m * LDA + 16 * j + cc], a);
+                TMP[e] = a;
+            }
+            __syncthreads();
+            for (int e = t; e < nb * 256; e += 256) {
+                const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, i = bi + d, j = bi;
+                float a = 0.f;
+                for (int m = 0; m <= rr; ++m) a = fmaf(XF[(16 * i + rr) * LDA + 16 * i + m], TMP[bi * 256 + m * 16 + cc], a);
+                XF[(16 * i + rr) * LDA + 16 * j + cc] = -a;
+            }
+            __syncthreads();
+        }
+        // [X; Y] (Y = Aqk X) as the bf16 A operand of phase B: 128 x 64, K-major, 128B swizzle
+        for (int e = t; e < 128 * 8; e += 256) {
+            const int m = e >> 3, mc = e & 7;
+            float v[8];
+            if (m < 64) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = XF[m * LDA + 8 * mc + j];
+            } else {
+                const int r = m - 64;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = 0.f;
+                for (int u = 8 * mc; u <= r; ++u) {
+                    const float a = AQF[r * LDA + u];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[j] = fmaf(a, XF[u * LDA + 8 * mc + j], v[j]);
+                }
+            }
+            *reinterpret_cast<uint4*>(sm + ps::XY + m * 128 + ((mc ^ (m & 7)) << 4)) = pack8(v);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---------------- phase B: D[m, n] = [X; Y][m, :] . [beta K gamma | beta V]^T[n, :]  (N = 128 + DV, K = 64)
+        if (t == 0) {
+            tc_fence_after();
+            const uint32_t xa = smem_u32(sm + ps::XY), kb = smem_u32(sm + ps::BKV);
+            const uint32_t idesc = idesc_bf16(128, 128 + DV);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma_f16(tm, sdesc_k_sw128(xa + ks * 32), sdesc_k_sw128(kb + ks * 32), idesc, ks > 0);
+            umma_commit(&bar_mma);
+        }
+        {
+            const bool ok = mbar_wait(&bar_mma, ph_mma, status);
+            if (__syncthreads_or(!ok)) break;
+        }
+        ph_mma ^= 1;
+        tc_fence_after();
+
+        // ---------------- epilogue: rows 0..63 -> -W | U, rows 64..127 -> P = Q gamma - Y bK gamma | O_intra
+        {
+            const int qw = w & 3, half = w >> 2;
+            const int m = 32 * qw + lane;
+            const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
+            if (half == 0) {
+#pragma unroll 1
+                for (int c16 = 0; c16 < 8; ++c16) {
+                    float v[16];
+                    tmem_ld16(lane_base + 16 * c16, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const int cc = 2 * c16 + sub;
+                        float o8[8];
+                        if (m < 64) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) o8[j] = -v[8 * sub + j];
+                        } else {
+                            const int r = m - 64;
+                            float q8[8];
+                            unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + ((cc ^ (r & 7)) << 4)), q8);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) o8[j] = q8[j] - v[8 * sub + j];
+                        }
+                        *reinterpret_cast<uint4*>(sm + ps::AWS + (cc >> 3) * 16384 + m * 128 +
+                                                  (((cc & 7) ^ (m & 7)) << 4)) = pack8(o8);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c16 = 0; c16 < DV / 16; ++c16) {
+                    float v[16];
+                    tmem_ld16(lane_base + 128 + 16 * c16, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const int cc = 2 * c16 + sub;
+                        float o8[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) o8[j] = v[8 * sub + j];
+                        const uint32_t dst = (m < 64 ? ps::US + m * 16 : ps::OIS + (m - 64) * 16) + cc * 1024;
+                        *reinterpret_cast<uint4*>(sm + dst) = pack8(o8);
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (t == 0) {
+            bulk_s2g(pkt + P::AW, sm + ps::AWS, 32768);
+            bulk_s2g(pkt + P::U, sm + ps::US, DV * 128);
+            bulk_s2g(pkt + P::OI, sm + ps::OIS, DV * 128);
+            bulk_commit();
+            bulk_wait_read0();   // staging is overwritten by the next column pass
+        }
+        __syncthreads();
+        item = nitem;
+        loc = nloc;
+        h = nh;
+        valid = nvalid;
+    }
+    if (t == 0) {
+        if (load_pending) mbar_wait(&bar_load, ph_load, nullptr);   // never leave a TMA write in flight
+        bulk_wait0();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tm, 256);
+}
+
+// ------------------------------------------------------------------------------------------------
+// inter-chunk state pass
+template <int DV, int DVS>
+struct SCfg {
+    static constexpr int NCW = DVS / 2;   // state columns per epilogue warp (two warps share a lane quarter)
+    static constexpr int NST = DVS == 128 ? 2 : 3;
+    static constexpr uint32_t AW = 0, KD = 32768, U = 49152, OI = U + DVS * 128, G = OI + DVS * 128;
+    static constexpr uint32_t STAGE = ((G + 512 + 1023) / 1024) * 1024;
+    static constexpr uint32_t SOP = NST * STAGE;      // S^T as B operand: 2 K atoms x DVS rows x 128 B
+    static constexpr uint32_t UOP = SOP + DVS * 256;  // U'^T as B operand: 1 K atom x DVS rows x 128 B
+    static constexpr uint32_t BYTES = UOP + DVS * 128;
+    static constexpr uint32_t TMEM_COLS = 2 * DVS <= 32 ? 32 : (2 * DVS <= 64 ? 64 : (2 * DVS <= 128 ? 128 : 256));
+};
+
+template <int DV, int DVS>
+__global__ void __launch_bounds__(320, 1)
+state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict__ cu_seqlens,
+                  const int32_t* __restrict__ cu_chunks, int n_seqs, int H, long long win_lo, long long win_hi,
+                  const float* __restrict__ initial_state, __nv_bfloat16* __restrict__ o,
+                  float* __restrict__ final_state, float* __restrict__ final_transition, int ckpt_stride,
+                  float* __restrict__ checkpoints, const int32_t* __restrict__ ckpt_cu, float* __restrict__ carry,
+                  int* status) {
+    using C = SCfg<DV, DVS>;
+    using P = Pk<DV>;
+    constexpr int NST = C::NST, NCW = C::NCW, NSV = DV / DVS, CW = DV + kDK;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    __shared__ __align__(8) uint64_t full[NST], empty[NST], d1_full, d2_full, s_ready, up_ready;
+    __shared__ uint32_t tmem_slot;
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    const int seq = blockIdx.x / H, h = blockIdx.x % H, slice = blockIdx.y;
+    const bool trans = slice >= NSV;
+    const int j0 = (trans ? slice - NSV : slice) * DVS;
+    if (trans && !final_transition) return;
+    const long long ch_lo = cu_chunks[seq], ch_hi = cu_chunks[seq + 1];
+    const long long lo = ch_lo > win_lo ? ch_lo : win_lo;
+    const long long hi = ch_hi < win_hi ? ch_hi : win_hi;
+    const bool empty_seq = ch_lo == ch_hi;
+    if (!(lo < hi) && !(empty_seq && win_lo == 0)) return;
+    const bool first = empty_seq || ch_lo >= win_lo;
+    const bool last = empty_seq || ch_hi <= win_hi;
+    const int nch = static_cast<int>(hi > lo ? hi - lo : 0);
+    const size_t sh = static_cast<size_t>(seq) * H + h;
+    const long long seq_tok0 = cu_seqlens[seq];
+    const long long seq_len = static_cast<long long>(cu_seqlens[seq + 1]) - seq_tok0;
+
+    if (t == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + 8);
+        }
+        mbar_init(&d1_full, 1);
+        mbar_init(&d2_full, 1);
+        mbar_init(&s_ready, 8);
+        mbar_init(&up_ready, 8);
+        fence_barrier_init();
+    }
+    if (w == 0) {
+        tmem_alloc(&tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_slot;
+
+    if (w == 8) {
+        // ---------------- producer: packets -> shared-memory ring (bulk TMA)
+        if (lane == 0) {
+            int issued = 0;
+            for (int ci = 0; ci < nch; ++ci) {
+                const int st = ci % NST;
+                if (!mbar_wait(&empty[st], ((ci / NST) & 1) ^ 1, status)) break;
+                const uint8_t* pk = packets + static_cast<size_t>((lo + ci - win_lo) * H + h) * P::BYTES;
+                uint8_t* sb = sm + st * C::STAGE;
+                const uint32_t bytes = 32768 + 16384 + 512 + (trans ? 0u : 2u * DVS * 128);
+                mbar_arrive_expect_tx(&full[st], bytes);
+                bulk_g2s(sb + C::AW, pk + P::AW, 32768, &full[st]);
+                bulk_g2s(sb + C::KD, pk + P::KD, 16384, &full[st]);
+                if (!trans) {
+                    bulk_g2s(sb + C::U, pk + P::U + (j0 / 8) * 1024, DVS * 128, &full[st]);
+                    bulk_g2s(sb + C::OI, pk + P::OI + (j0 / 8) * 1024, DVS * 128, &full[st]);
+                }
+                bulk_g2s(sb + C::G, pk + P::G, 512, &full[st]);
+                issued = ci + 1;
+            }
+            // never leave a copy in flight: wait (bounded, quietly) for the last fill of every stage
+            for (int ci = issued - NST < 0 ? 0 : issued - NST; ci < issued; ++ci)
+                mbar_wait(&full[ci % NST], (ci / NST) & 1, nullptr);
+        }
+    } else if (w == 9) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, DVS);
+            const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP);
+            for (int ci = 0; ci < nch; ++ci) {
+                const int st = ci % NST;
+                if (!mbar_wait(&s_ready, ci & 1, status)) break;
+                if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
+                tc_fence_after();
+                const uint32_t sb = smem_u32(sm + st * C::STAGE);
+                // D1 = [-W; P] S   (M = 128, N = DVS, K = 128)
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
+                    umma_f16(tm, sdesc_k_sw128(sb + C::AW + ka * 16384 + kb),
+                             sdesc_k_sw128(sop + ka * (DVS * 128) + kb), idesc, ks > 0);
+                }
+                umma_commit(&d1_full);
+                if (!mbar_wait(&up_ready, ci & 1, status)) break;
+                tc_fence_after();
+                // D2 = Kdec^T U'   (M = 128, N = DVS, K = 64)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), sdesc_k_sw128(uop + ks * 32), idesc,
+                             ks > 0);
+                umma_commit(&d2_full);
+                umma_commit(&empty[st]);
+            }
+        }
+    } else {
+        // ---------------- epilogue warps: lane quarter qw, columns [jw, jw + NCW) of the slice
+        const int qw = w & 3, jw = (w >> 2) * NCW;
+        const int i = 32 * qw + lane;   // TMEM lane: row of D1 (token row / P row), channel of D2 and S
+        const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
+        float S[NCW];
+#pragma unroll
+        for (int j = 0; j < NCW; ++j) {
+            const int col = j0 + jw + j;
+            float x;
+            if (!first) x = carry[(sh * kDK + i) * CW + (trans ? DV : 0) + col];
+            else if (trans) x = (i == col) ? 1.f : 0.f;
+            else x = initial_state ? initial_state[(sh * kDK + i) * DV + col] : 0.f;
+            S[j] = x;
+        }
+        auto write_sop = [&]() {
+#pragma unroll
+            for (int j = 0; j < NCW; ++j)
+                *reinterpret_cast<__nv_bfloat16*>(sm + C::SOP + sw128_offset(jw + j, i, DVS)) = __float2bfloat16_rn(S[j]);
+        };
+        write_sop();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_ready);
+        for (int ci = 0; ci < nch; ++ci) {
+            const int st = ci % NST;
+            const uint8_t* sb = sm + st * C::STAGE;
+            const int c = static_cast<int>(lo + ci - ch_lo);
+            const long long rem = seq_len - static_cast<long long>(c) * 64;
+            const int n = rem < 64 ? static_cast<int>(rem) : 64;
+            if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
+            if (!mbar_wait(&d1_full, ci & 1, status)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int cb = 0; cb < NCW; cb += 16) {
+                float v[16];
+                tmem_ld16(lane_base + jw + cb, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    const int cc = (jw + cb) / 8 + sub;   // 8-column chunk within the slice
+                    if (i < 64) {
+                        float u8[8];
+                        if (trans) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) u8[e] = 0.f;
+                        } else {
+                            unpack8(*reinterpret_cast<const uint4*>(sb + C::U + cc * 1024 + i * 16), u8);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            *reinterpret_cast<__nv_bfloat16*>(sm + C::UOP + sw128_offset(jw + cb + 8 * sub + e, i, DVS)) =
+                                __float2bfloat16_rn(u8[e] + v[8 * sub + e]);
+                    } else if (!trans && i - 64 < n) {
+                        const int r = i - 64;
+                        float o8[8];
+                        unpack8(*reinterpret_cast<const uint4*>(sb + C::OI + cc * 1024 + r * 16), o8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o8[e] += v[8 * sub + e];
+                        *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + j0 + jw +
+                                                  cb + 8 * sub) = pack8(o8);
+                    }
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&up_ready);
+            if (!mbar_wait(&d2_full, ci & 1, status)) break;
+            tc_fence_after();
+            const float gam = *reinterpret_cast<const float*>(sb + C::G + i * 4);
+#pragma unroll
+            for (int cb = 0; cb < NCW; cb += 16) {
+                float v[16];
+                tmem_ld16(lane_base + DVS + jw + cb, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) S[cb + e] = fmaf(gam, S[cb + e], v[e]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);   // done with this stage's U, O_intra and gamma
+            write_sop();
+            if (!trans && ckpt_stride > 0 && checkpoints && n == 64) {
+                const long long end = static_cast<long long>(c + 1) * 64;
+                if (end % ckpt_stride == 0) {
+                    const long long slot = ckpt_cu[seq] + end / ckpt_stride - 1;
+                    if (slot >= ckpt_cu[seq] && slot < ckpt_cu[seq + 1]) {
+                        float4* dst = reinterpret_cast<float4*>(checkpoints +
+                                                                ((static_cast<size_t>(slot) * H + h) * kDK + i) * DV + j0 + jw);
+#pragma unroll
+                        for (int e = 0; e < NCW / 4; ++e)
+                            dst[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
+                    } else if (lane == 0) {
+                        set_status(status, KDA_ERR_DEVICE_INPUT);
+                    }
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_ready);
+        }
+#pragma unroll
+        for (int j = 0; j < NCW; ++j) {
+            const int col = j0 + jw + j;
+            if (last) {
+                if (trans) final_transition[(sh * kDK + i) * kDK + col] = S[j];
+                else if (final_state) final_state[(sh * kDK + i) * DV + col] = S[j];
+            } else {
+                carry[(sh * kDK + i) * CW + (trans ? DV : 0) + col] = S[j];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tm, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------------------------------
+// host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3D map over a [T, H, d] tensor (d innermost), box {box_d, 1, 64 tokens}, no swizzle.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int d, int H, long long T,
+              int box_d) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize, static_cast<cuuint64_t>(H) * d * esize};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_d), 1u, 64u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+template <int DV, int DVS>
+cudaError_t launch_state(const ChunkArgs& a, cudaStream_t s) {
+    using C = SCfg<DV, DVS>;
+    const int smem = static_cast<int>(C::BYTES) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(state_bf16_kernel<DV, DVS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int slices = DV / DVS + (a.final_transition ? kDK / DVS : 0);
+    dim3 grid(a.n_seqs * a.H, slices);
+    state_bf16_kernel<DV, DVS><<<grid, 320, smem, s>>>(
+        static_cast<const uint8_t*>(a.packets), a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, a.win_hi,
+        a.initial_state, static_cast<__nv_bfloat16*>(a.o), a.final_state, a.final_transition, a.ckpt_stride,
+        a.checkpoints, a.ckpt_cu, a.carry, a.status);
+    return cudaGetLastError();
+}
+
+template <int DV>
+cudaError_t launch_bf16_t(const ChunkArgs& a, cudaStream_t s) {
+    const long long items = (a.win_hi - a.win_lo) * a.H;
+    if (a.total_tokens > 0 && items > 0) {
+        CUtensorMap mq, mk, mv, ml;
+        if (!make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, a.H, a.total_tokens, 64) ||
+            !make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, a.H, a.total_tokens, 64) ||
+            !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, a.total_tokens, 64) ||
+            !make_map(&ml, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, a.H, a.total_tokens, 32))
+            return cudaErrorInvalidValue;
+        const int smem = static_cast<int>(ps::BYTES) + 1024;
+        cudaError_t e = cudaFuncSetAttribute(prep_bf16_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        const long long grid = items < num_sms() ? items : num_sms();
+        prep_bf16_kernel<DV><<<static_cast<unsigned>(grid), 256, smem, s>>>(
+            mq, mk, mv, ml, a.beta, a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, items,
+            static_cast<uint8_t*>(a.packets), a.status);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // dv slice per state CTA: as wide as possible while the (sequence, head) chains fill the GPU
+    const long long chains = static_cast<long long>(a.n_seqs) * a.H;
+    const int sms = num_sms();
+    if (DV == 128 && chains >= (sms * 3) / 4) return launch_state<DV, DV>(a, s);
+    if (chains * (DV / 64) >= (sms * 3) / 4) return launch_state<DV, 64>(a, s);
+    return launch_state<DV, 32>(a, s);
+}
+
+}  // namespace
+
+size_t chunk_packet_bytes_bf16(int dk, int dv) { return dv == 64 ? Pk<64>::BYTES : Pk<128>::BYTES; }
+
+cudaError_t launch_chunk_bf16(const ChunkArgs& a, cudaStream_t s) {
+    if (a.dk != kDK) return cudaErrorInvalidValue;
+    return a.dv == 64 ? launch_bf16_t<64>(a, s) : launch_bf16_t<128>(a, s);
+}
 
 }  // namespace kda

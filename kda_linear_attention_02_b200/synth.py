@@ -57,7 +57,7 @@ def cu_from_lengths(lengths, device="cpu") -> torch.Tensor:
 def _draw(shape, gen, device, mean=0.0, std=1.0, slab_rows=None):
     out = torch.empty(shape, dtype=torch.float32, device=device)
     rows = shape[0]
-    step = rows if slab_rows is None else max(1, slab_rows)
+    step = max(1, rows if slab_rows is None else slab_rows)
     for r0 in range(0, rows, step):
         r1 = min(rows, r0 + step)
         out[r0:r1].normal_(mean, std, generator=gen)
