@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""bench.py -- KDA operator throughput on B200: chunked prefill tokens/s (headline) and recurrent
+decode steps/s, each against its HBM roofline, plus end-to-end and CPU-oracle baselines.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One timed step = one kda_chunk_fwd call over the prefill workload (B=4 sequences x T=4096 tokens,
+H=32 heads, dk=dv=128, bf16 q/k/v, fp32 log_alpha/beta, zero initial state, fp32 final state and
+fp32 state checkpoints every 512 tokens): the per-chunk decay prep, the intra-chunk tcgen05 pass,
+the inter-chunk tcgen05 state pass and the checkpoint writes.  The decode workload (256 sequences x
+32 heads of 128 x 128 fp32 state, 1024 consecutive kda_recurrent_step calls) and a segment compose
+are timed alongside and reported under "decode" and "compose".  Inputs are seeded synthetic data
+drawn on the device; every input and output set is larger than the 126 MB L2, so no flush is needed.
+
+Under torchrun (N > 1) every rank runs its own batch on its own GPU (weak scaling, no data-path
+collective); the step time is the max over ranks (one NCCL all-reduce of a scalar outside the timed
+region).  --impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (H=32,d=128,bf16) & decode steps/s; % of TC/HBM roofline"
+B, T, H, D = 4, 4096, 32, 128
+CKPT = 512
+DEC_N, DEC_STEPS = 256, 1024
+# Algorithmic bytes per (token, head) of the prefill path.  Reads: q, k, v bf16 (3 x 256 B),
+# log_alpha fp32 (512 B), beta fp32 (4 B).  Writes: o bf16 (256 B), the 512-token checkpoint
+# (128 x 128 x 4 B / 512 = 128 B) and the final state (64 KiB per 4096 tokens = 16 B).
+PREFILL_READ_B = 3 * 256 + 512 + 4
+PREFILL_WRITE_B = 256 + 128 + 16
+# Decode bytes per (sequence, head) step: state read + write (2 x 64 KiB), q/k/v bf16, log_alpha,
+# beta, o bf16.
+DECODE_B = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampler (read-only queries) running while the measured work runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.path = tempfile.mktemp(prefix="kda_clocks_", suffix=".csv")
+        self.f = open(self.path, "w")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "100", "-i", str(index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except Exception:
+                self.p.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            c = [x.strip() for x in line.split(",")]
+            if len(c) < 9:
+                continue
+            try:
+                sm.append(float(c[1]))
+                mx.append(float(c[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, c[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(x, world):
+    import torch
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_sample(inp, budget_s=12.0, max_slices=None):
+    """Times the fp64 oracle (as it stands) on whole (sequence, head) slices of the workload,
+    as many as fit the time budget (estimated from one calibration slice)."""
+    import oracle
+    cu = inp.cu_seqlens.cpu().tolist()
+    nseq = len(cu) - 1
+    Hh = inp.q.shape[1]
+
+    def job(i, h):
+        a, b = cu[i], cu[i + 1]
+        f = lambda t: t.float().cpu().numpy()
+        return dict(q=f(inp.q[a:b, h]), k=f(inp.k[a:b, h]), v=f(inp.v[a:b, h]),
+                    log_alpha=f(inp.log_alpha[a:b, h]), beta=f(inp.beta[a:b, h]), want_o=True)
+
+    threads = oracle.threads_used()
+    t0 = time.perf_counter()
+    oracle.kda_seq(**job(0, 0))
+    one = time.perf_counter() - t0
+    n = max(1, min(nseq * Hh, int(budget_s * threads / max(one, 1e-3))))
+    if max_slices:
+        n = min(n, max_slices)
+    keys = [(i, h) for i in range(nseq) for h in range(Hh)][:n]
+    jobs = [(key, job(*key)) for key in keys]
+    t0 = time.perf_counter()
+    oracle.run_slices(jobs, threads)
+    dt = time.perf_counter() - t0
+    toks = sum(cu[i + 1] - cu[i] for i, _ in keys)
+    return {"value": toks / Hh / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {nseq * Hh} (sequence, head) slices x {cu[1] - cu[0]} tokens, fp64, "
+                      f"{dt:.1f} s on {threads} threads; tokens/s = token-heads/s / {Hh}"}
+
+
+def run_ours(args):
+    import torch
+    import kda_linear_attention_02_b200 as kda
+    from kda_linear_attention_02_b200 import synth
+
+    rank, world, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    hbm, tc, tc_sus, peak_kind = peaks()
+    stream = torch.cuda.current_stream()
+
+    # ------------------------------------------------------------------ prefill workload
+    inp = synth.make_inputs([T] * B, H, D, D, dtype=torch.bfloat16, device=dev, seed=rank)
+    ckcu_h = kda.kda_ckpt_offsets(inp.cu_seqlens.cpu(), CKPT)
+    ckcu = ckcu_h.to(dev)
+    ck = torch.empty(int(ckcu_h[-1]), H, D, D, device=dev)
+    o = torch.empty(B * T, H, D, dtype=torch.bfloat16, device=dev)
+    fs = torch.empty(B, H, D, D, device=dev)
+    ws = torch.empty(kda.kda_chunk_fwd_workspace_bytes(B * T, B, H, D, D, kda.KDA_BF16), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, inp.cu_seqlens, o, fs,
+                          ckpt_stride=CKPT, checkpoints=ck, ckpt_cu=ckcu, workspace=ws)
+
+    clocks = Clocks(dev.index if world == 1 else local)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    kda.kda_profile_begin(min(args.steps, 256))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_idx, ms_prep, ms_state, ncalls = kda.kda_profile_end()
+    barrier(world)
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = max_over_ranks(ms, world)
+    st = kda.kda_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {kda.kda_status_string(st)}")
+    tokens_job = B * T * world
+    value = tokens_job / (ms_max / 1e3)
+
+    # per-kernel roofline (live CUDA events on the launching stream, averaged over the timed calls)
+    th = B * T * H
+    prep_ms, state_ms, idx_ms = ms_prep / ncalls, ms_state / ncalls, ms_idx / ncalls
+    prep_bytes, state_bytes = PREFILL_READ_B * th, PREFILL_WRITE_B * th
+    kernels = {
+        "kda_chunk_index": {"ms": idx_ms},
+        "prep_bf16_kernel": {"ms": prep_ms, "alg_bytes": prep_bytes,
+                             "achieved_gbs": prep_bytes / (prep_ms / 1e3) / 1e9},
+        "state_bf16_kernel": {"ms": state_ms, "alg_bytes": state_bytes,
+                              "achieved_gbs": state_bytes / (state_ms / 1e3) / 1e9},
+    }
+    dom = "prep_bf16_kernel" if prep_ms >= state_ms else "state_bf16_kernel"
+    ach = kernels[dom]["achieved_gbs"]
+    whole_bytes = (PREFILL_READ_B + PREFILL_WRITE_B) * th
+    whole_gbs = whole_bytes / (ms / 1e3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get(dom)
+        except Exception:
+            traffic = None
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach / hbm, 4), "traffic": traffic, "peak_kind": peak_kind,
+                "alg_bytes_per_launch": kernels[dom]["alg_bytes"],
+                "whole_step": {"alg_bytes": whole_bytes, "achieved_gbs": round(whole_gbs, 1),
+                               "frac": round(whole_gbs / hbm, 4)},
+                "kernels": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                            for k, v in kernels.items()}}
+
+    # ------------------------------------------------------------------ end to end from host buffers
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
+    hq, hk, hv, hla, hb = pin(inp.q), pin(inp.k), pin(inp.v), pin(inp.log_alpha), pin(inp.beta)
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hfs = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hla, hb))
+    d2h = ho.numel() * ho.element_size() + hfs.numel() * hfs.element_size()
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        inp.q.copy_(hq, non_blocking=True); inp.k.copy_(hk, non_blocking=True); inp.v.copy_(hv, non_blocking=True)
+        inp.log_alpha.copy_(hla, non_blocking=True); inp.beta.copy_(hb, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True); hfs.copy_(fs, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e = {"value": tokens_job / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+    del hq, hk, hv, hla, hb, ho, hfs
+
+    # ------------------------------------------------------------------ decode workload
+    s0, dq, dk_, dv_, dla, db = synth.make_decode_inputs(DEC_N, H, D, D, dtype=torch.bfloat16, device=dev,
+                                                         seed=100 + rank, steps=DEC_STEPS)
+    state = s0.clone()
+    do = torch.empty(DEC_N, H, D, dtype=torch.bfloat16, device=dev)
+    for t_ in range(3):
+        kda.kda_recurrent_step(state, dq[t_], dk_[t_], dv_[t_], dla[t_], db[t_], do)
+    state.copy_(s0)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for t_ in range(DEC_STEPS):
+        kda.kda_recurrent_step(state, dq[t_], dk_[t_], dv_[t_], dla[t_], db[t_], do)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dec_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    step_ms = dec_ms / DEC_STEPS
+    dec_bytes = DECODE_B * DEC_N * H
+    dec_gbs = dec_bytes / (step_ms / 1e3) / 1e9
+    decode = {"metric": "KDA decode steps/s (256 seqs x H=32, 128x128 fp32 state, 1024 steps)",
+              "value": world * DEC_STEPS / (dec_ms / 1e3), "unit": "steps/s",
+              "tokens_per_s": DEC_N * world * DEC_STEPS / (dec_ms / 1e3), "ms_per_step": round(step_ms, 5),
+              "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": round(dec_gbs, 1),
+                           "peak": hbm, "unit": "GB/s", "frac": round(dec_gbs / hbm, 4),
+                           "alg_bytes_per_launch": dec_bytes}}
+    del s0, dq, dk_, dv_, dla, db, state, do
+
+    # ------------------------------------------------------------------ segment compose (64 seqs x 8 segments)
+    nseg = 8
+    M = torch.randn(64 * nseg, H, D, D, device=dev) * (1.0 / D ** 0.5)
+    Z = torch.randn(64 * nseg, H, D, D, device=dev)
+    seg_cu = synth.cu_from_lengths([nseg] * 64, dev)
+    starts = torch.empty_like(Z)
+    ends = torch.empty(64, H, D, D, device=dev)
+    kda.kda_segment_compose(M, Z, seg_cu, None, starts, ends)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    kda.kda_segment_compose(M, Z, seg_cu, None, starts, ends)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    comp_ms = e0.elapsed_time(e1)
+    comp_bytes = 64 * nseg * H * 3 * D * D * 4
+    compose = {"workload": "64 sequences x 8 segments x H=32, dk=dv=128 fp32", "ms": round(comp_ms, 4),
+               "achieved_gbs": round(comp_bytes / (comp_ms / 1e3) / 1e9, 1)}
+    del M, Z, starts, ends
+    clk = clocks.stop()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(inp)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "KDA prefill B=4 T=4096 H=32 dk=dv=128 bf16, zero initial state, fp32 final "
+                                   "state, fp32 checkpoints every 512 tokens",
+                       "global_batch": B * world, "seq_len": T, "heads": H, "dk": D, "dv": D, "ckpt_stride": CKPT,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs and outputs larger than L2 (1.1 GB per step), no flush"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+            "gpu_launches": 3 * args.steps, "decode": decode, "compose": compose,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """fp64 CPU oracle, as it stands, on the host cores: each step is a bounded sample of the same
+    prefill workload (whole (sequence, head) slices)."""
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from kda_linear_attention_02_b200 import synth
+    import oracle
+    oracle.build()
+    inp = synth.make_inputs([T] * B, H, D, D, dtype=torch.bfloat16, device="cpu", seed=0)
+    per_step_slices = oracle.threads_used()          # one slice per host thread per step
+    samples = []
+    for it in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(inp, budget_s=1e9, max_slices=per_step_slices)
+        if it >= args.warmup:
+            samples.append(r)
+    val = statistics.median(s["value"] for s in samples)
+    ms = per_step_slices * T / H / val * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "KDA prefill B=4 T=4096 H=32 dk=dv=128 bf16 inputs, zero initial state",
+                       "global_batch": B, "seq_len": T, "heads": H},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": samples[0]["cores"], "kind": "oracle",
+                             "sample": f"each step: {per_step_slices} (sequence, head) slices x {T} tokens"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

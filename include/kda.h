@@ -160,6 +160,17 @@ KDA_API const char* kda_status_string(kda_status_t status);
 KDA_API const char* kda_version(void);
 
 /*
+ * Per-kernel timing of kda_chunk_fwd (measurement plumbing, no KDA arithmetic).  After
+ * kda_profile_begin(max_calls), the next max_calls calls of kda_chunk_fwd on this thread record CUDA
+ * events on their stream around each of their kernels (chunk index, intra-chunk prep, inter-chunk
+ * state).  kda_profile_end synchronises those events, writes the summed milliseconds of each kernel
+ * over the recorded calls and the number of recorded calls, and stops recording.  The events are
+ * created once per process (no device memory is allocated).
+ */
+KDA_API kda_status_t kda_profile_begin(int max_calls);
+KDA_API kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_state, int* n_calls);
+
+/*
  * Diagnostics (no KDA arithmetic).
  *  kda_selftest_wait_timeout: launches one tiny kernel that waits on an mbarrier nothing will
  *  complete, with a wait limit of limit_us microseconds; returns KDA_ERR_TIMEOUT when the bounded

@@ -17,7 +17,8 @@ __all__ = [
     "KDA_BF16", "KDA_F32", "KDA_CHUNK", "KDAError", "lib_path",
     "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd",
     "kda_recurrent_step", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
-    "kda_status_string", "kda_version", "kda_selftest_wait_timeout", "kda_selftest_umma",
+    "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
+    "kda_selftest_umma",
 ]
 
 KDA_BF16 = 0
@@ -67,6 +68,10 @@ def _load():
     L.kda_status_string.argtypes = [i32]
     L.kda_version.restype = ctypes.c_char_p
     L.kda_version.argtypes = []
+    L.kda_profile_begin.restype = i32
+    L.kda_profile_begin.argtypes = [i32]
+    L.kda_profile_end.restype = i32
+    L.kda_profile_end.argtypes = [vp, vp, vp, vp]
     L.kda_selftest_wait_timeout.restype = i32
     L.kda_selftest_wait_timeout.argtypes = [i32, vp]
     L.kda_selftest_umma.restype = i32
@@ -229,6 +234,19 @@ def kda_ckpt_offsets(cu_seqlens_host, stride: int) -> torch.Tensor:
 def kda_get_device_status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device status word."""
     return int(_load().kda_get_device_status(_stream(stream)))
+
+
+def kda_profile_begin(max_calls: int):
+    """Record per-kernel CUDA events in the next max_calls kda_chunk_fwd calls (C: kda_profile_begin)."""
+    _check(_load().kda_profile_begin(int(max_calls)), "kda_profile_begin")
+
+
+def kda_profile_end():
+    """Returns (ms_index, ms_prep, ms_state, n_calls) summed over the recorded calls (C: kda_profile_end)."""
+    a, b, c, n = ctypes.c_float(), ctypes.c_float(), ctypes.c_float(), ctypes.c_int()
+    _check(_load().kda_profile_end(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), ctypes.byref(n)),
+           "kda_profile_end")
+    return a.value, b.value, c.value, n.value
 
 
 def kda_selftest_wait_timeout(limit_us: int = 2000, stream=None) -> int:

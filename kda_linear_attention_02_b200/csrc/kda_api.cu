@@ -91,6 +91,17 @@ cudaError_t launch_selftest_wait(int limit_us, int* d_result, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// ---- optional per-kernel timing of kda_chunk_fwd (see kda_profile_begin)
+constexpr int kProfileMax = 256;
+static ChunkEvents g_prof[kProfileMax];
+static bool g_prof_created = false;
+static thread_local int t_prof_limit = 0, t_prof_used = 0;
+
+ChunkEvents* profile_slot() {
+    if (t_prof_used >= t_prof_limit) return nullptr;
+    return &g_prof[t_prof_used++];
+}
+
 }  // namespace kda
 
 using namespace kda;
@@ -213,6 +224,8 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
     }
     a.status = status_ptr();
     if (!a.status) return KDA_ERR_CUDA;
+    a.events = profile_slot();
+    if (a.events) cudaEventRecord(a.events->ev[0], s);
     cudaError_t e = launch_chunk_index(cu_seqlens, n_seqs, total_tokens, reinterpret_cast<int32_t*>(ws), a.status, s);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     long long lo = 0;
@@ -284,6 +297,38 @@ kda_status_t kda_get_device_status(kda_stream_t stream) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
     return static_cast<kda_status_t>(h);
+}
+
+kda_status_t kda_profile_begin(int max_calls) {
+    if (max_calls < 0 || max_calls > kProfileMax) return KDA_ERR_ARG;
+    if (!g_prof_created) {
+        for (auto& c : g_prof)
+            for (auto& ev : c.ev)
+                if (cudaEventCreate(&ev) != cudaSuccess) return KDA_ERR_CUDA;
+        g_prof_created = true;
+    }
+    t_prof_limit = max_calls;
+    t_prof_used = 0;
+    return KDA_OK;
+}
+
+kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_state, int* n_calls) {
+    if (!ms_index || !ms_prep || !ms_state || !n_calls) return KDA_ERR_ARG;
+    float a = 0.f, b = 0.f, c = 0.f;
+    for (int i = 0; i < t_prof_used; ++i) {
+        float x = 0.f;
+        if (cudaEventSynchronize(g_prof[i].ev[3]) != cudaSuccess) return KDA_ERR_CUDA;
+        if (cudaEventElapsedTime(&x, g_prof[i].ev[0], g_prof[i].ev[1]) != cudaSuccess) return KDA_ERR_CUDA;
+        a += x;
+        if (cudaEventElapsedTime(&x, g_prof[i].ev[1], g_prof[i].ev[2]) != cudaSuccess) return KDA_ERR_CUDA;
+        b += x;
+        if (cudaEventElapsedTime(&x, g_prof[i].ev[2], g_prof[i].ev[3]) != cudaSuccess) return KDA_ERR_CUDA;
+        c += x;
+    }
+    *ms_index = a; *ms_prep = b; *ms_state = c; *n_calls = t_prof_used;
+    t_prof_limit = 0;
+    t_prof_used = 0;
+    return KDA_OK;
 }
 
 kda_status_t kda_selftest_wait_timeout(int limit_us, kda_stream_t stream) {

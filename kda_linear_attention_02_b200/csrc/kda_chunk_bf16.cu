@@ -761,6 +761,7 @@ cudaError_t launch_state(const ChunkArgs& a, cudaStream_t s) {
 template <int DV>
 cudaError_t launch_bf16_t(const ChunkArgs& a, cudaStream_t s) {
     const long long items = (a.win_hi - a.win_lo) * a.H;
+    if (a.events) cudaEventRecord(a.events->ev[1], s);
     if (a.total_tokens > 0 && items > 0) {
         CUtensorMap mq, mk, mv, ml;
         if (!make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, a.H, a.total_tokens, 64) ||
@@ -778,12 +779,16 @@ cudaError_t launch_bf16_t(const ChunkArgs& a, cudaStream_t s) {
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    if (a.events) cudaEventRecord(a.events->ev[2], s);
     // dv slice per state CTA: as wide as possible while the (sequence, head) chains fill the GPU
     const long long chains = static_cast<long long>(a.n_seqs) * a.H;
     const int sms = num_sms();
-    if (DV == 128 && chains >= (sms * 3) / 4) return launch_state<DV, DV>(a, s);
-    if (chains * (DV / 64) >= (sms * 3) / 4) return launch_state<DV, 64>(a, s);
-    return launch_state<DV, 32>(a, s);
+    cudaError_t e;
+    if (DV == 128 && chains >= (sms * 3) / 4) e = launch_state<DV, DV>(a, s);
+    else if (chains * (DV / 64) >= (sms * 3) / 4) e = launch_state<DV, 64>(a, s);
+    else e = launch_state<DV, 32>(a, s);
+    if (a.events) cudaEventRecord(a.events->ev[3], s);
+    return e;
 }
 
 }  // namespace

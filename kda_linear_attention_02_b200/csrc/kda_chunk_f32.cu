@@ -361,6 +361,7 @@ cudaError_t launch_f32_t(const ChunkArgs& a, cudaStream_t s) {
                              static_cast<int>(SS::BYTES));
     if (e != cudaSuccess) return e;
     const long long items = (a.win_hi - a.win_lo) * a.H;
+    if (a.events) cudaEventRecord(a.events->ev[1], s);
     if (items > 0)
         chunk_prep_f32_kernel<DK, DV><<<static_cast<unsigned>(items), 256, SM::BYTES, s>>>(
             static_cast<const float*>(a.q), static_cast<const float*>(a.k), static_cast<const float*>(a.v),
@@ -369,10 +370,12 @@ cudaError_t launch_f32_t(const ChunkArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int slices = DV / kF32Cols + (a.final_transition ? DK / kF32Cols : 0);
     dim3 grid(a.n_seqs * a.H, slices);
+    if (a.events) cudaEventRecord(a.events->ev[2], s);
     chunk_state_f32_kernel<DK, DV><<<grid, 256, SS::BYTES, s>>>(
         static_cast<const float*>(a.packets), a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, a.win_hi,
         a.multi_window, a.initial_state, static_cast<float*>(a.o), a.final_state, a.final_transition, a.ckpt_stride,
         a.checkpoints, a.ckpt_cu, a.carry, a.status);
+    if (a.events) cudaEventRecord(a.events->ev[3], s);
     return cudaGetLastError();
 }
 

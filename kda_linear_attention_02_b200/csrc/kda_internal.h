@@ -17,6 +17,10 @@ cudaError_t launch_compose(const float* M, const float* Z, const int32_t* seg_cu
                            int n_segs, int H, int dk, int dv, float* starts, float* ends, int* status,
                            cudaStream_t s);
 
+// Optional per-kernel events of one kda_chunk_fwd call (null = not recording).
+struct ChunkEvents {
+    cudaEvent_t ev[4];   // before index, before prep, before state, after state
+};
 // Everything one chunk-path launch needs (kda_chunk_f32.cu / kda_chunk_bf16.cu).
 struct ChunkArgs {
     const void* q;
@@ -41,6 +45,7 @@ struct ChunkArgs {
     long long win_lo, win_hi;   // global chunk index window [lo, hi)
     bool multi_window;
     int* status;                // device status word
+    struct ChunkEvents* events; // per-kernel timing events of this call, or null
 };
 
 // Builds cu_chunks[i] = sum_{j<i} ceil(len_j / 64) from cu_seqlens and validates the table.
@@ -54,6 +59,8 @@ cudaError_t launch_chunk_f32(const ChunkArgs& a, cudaStream_t s);
 // bf16 path: tcgen05 intra-chunk prep + tcgen05 inter-chunk state pass.
 size_t chunk_packet_bytes_bf16(int dk, int dv);
 cudaError_t launch_chunk_bf16(const ChunkArgs& a, cudaStream_t s);
+
+ChunkEvents* profile_slot();   // events for the current call, or null
 
 // Diagnostics.
 cudaError_t launch_selftest_wait(int limit_us, int* d_result, cudaStream_t s);
