@@ -178,10 +178,12 @@ KDA_API kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_
  *  kernels' waits end without a fault.
  *  kda_selftest_umma: one 128 x n x 64 bf16 tcgen05 product D = A B^T through the same shared-memory
  *  descriptors, TMEM allocation and load path the chunk kernels use. a [128,64], b [n,64] bf16
- *  row-major (device), d [128,n] fp32 (device); n in {16, 32, ..., 256}.
+ *  row-major (device), d [128,n] fp32 (device); n in {16, 32, ..., 256}.  b_mn_major != 0 stages B
+ *  MN-major instead of K-major (then n must be a multiple of 64).
  */
 KDA_API kda_status_t kda_selftest_wait_timeout(int limit_us, kda_stream_t stream);
-KDA_API kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, kda_stream_t stream);
+KDA_API kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, int b_mn_major,
+                                       kda_stream_t stream);
 
 #ifdef __cplusplus
 }

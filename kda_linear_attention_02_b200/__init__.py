@@ -75,7 +75,7 @@ def _load():
     L.kda_selftest_wait_timeout.restype = i32
     L.kda_selftest_wait_timeout.argtypes = [i32, vp]
     L.kda_selftest_umma.restype = i32
-    L.kda_selftest_umma.argtypes = [vp, vp, vp, i32, vp]
+    L.kda_selftest_umma.argtypes = [vp, vp, vp, i32, i32, vp]
     _lib = L
     return L
 
@@ -253,10 +253,11 @@ def kda_selftest_wait_timeout(limit_us: int = 2000, stream=None) -> int:
     return int(_load().kda_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
-def kda_selftest_umma(a, b, d, *, stream=None):
+def kda_selftest_umma(a, b, d, *, b_mn_major=False, stream=None):
     n = b.shape[0]
     _need(a, "a", (128, 64), torch.bfloat16)
     _need(b, "b", (n, 64), torch.bfloat16, a.device)
     _need(d, "d", (128, n), torch.float32, a.device)
-    _check(_load().kda_selftest_umma(_p(a), _p(b), _p(d), n, _stream(stream)), "kda_selftest_umma")
+    _check(_load().kda_selftest_umma(_p(a), _p(b), _p(d), n, int(bool(b_mn_major)), _stream(stream)),
+           "kda_selftest_umma")
     return d

@@ -25,13 +25,13 @@
 // Kernels:
 //  prep_bf16_kernel   persistent, one (chunk, head) item at a time per CTA: TMA tensor loads of the
 //                     raw tiles (prefetched one item ahead), SIMT exponentials and operand
-//                     construction, tcgen05 products for A/Aqk (4 anchored variants) and for
-//                     [X; Y] (beta K gamma | beta V), fp32 blocked forward substitution in between,
-//                     and a bulk TMA store of the MMA-ready packet.
+//                     construction, tcgen05 products for A/Aqk (4 anchored variants), for
+//                     [X; Y] = [I; Aqk] X and for [X; Y] (beta K gamma | beta V), fp32 blocked
+//                     forward substitution for X, and a bulk TMA store of the MMA-ready packet.
 //  state_bf16_kernel  one CTA per (sequence, head, dv-slice), warp-specialised: a producer warp
 //                     streams packets through a shared-memory ring with bulk TMA, one thread issues
-//                     the two tcgen05 products per chunk, eight epilogue warps hold the fp32 state in
-//                     registers and feed bf16 copies of S and U' back as the next operands.
+//                     the two tcgen05 products per chunk, 8 or 16 epilogue warps hold the fp32 state
+//                     in registers and feed bf16 copies of S and U' back as the next operands.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -82,11 +82,14 @@ constexpr uint32_t RALL = 81920;     // row side [K e^(g-b); Q e^(g-b)]: 128 x 1
 constexpr uint32_t BVAR = 114688;    // key side, variant i (rows 16(i+1)) at BVAR + 2048 i (i+1)
 constexpr uint32_t QT = 155648;      // Q * gamma, [64][128] bf16, 16-byte chunks swizzled by row
 constexpr uint32_t BKV = 172032;     // [beta K gamma | beta V]^T: (128+DV) x 64 bf16 (B operand)
-constexpr uint32_t MISC = 204800;    // beta[64] fp32, tile totals [4][128] fp32
-constexpr uint32_t AF = 81920, AQF = 98560, XF = 115200, XY = 132096, TMP = 148480;   // solve (aliases)
-constexpr uint32_t AWS = 81920, US = 114688, OIS = 131072;                           // packet staging
-constexpr uint32_t BYTES = MISC + 256 + 2048;
-constexpr int LDA = 65;              // fp32 row pitch of A, Aqk, X
+constexpr uint32_t MISC = 204800;    // beta[64] fp32, half-tile totals [8][128] fp32
+constexpr uint32_t IAQ = 209920;     // [I; Aqk]: 128 x 64 bf16 (A operand of the Y product)
+// aliases of RALL/BVAR once phase A has completed
+constexpr uint32_t AF = 81920, XF = 98560, TMP = 115200, XT = 118784, XY = 126976;   // solve
+constexpr uint32_t AWS = 81920, US = 114688, OIS = 131072;                          // packet staging
+constexpr uint32_t BYTES = IAQ + 16384;
+constexpr int LDA = 65;              // fp32 row pitch of A and X
+constexpr int NT = 512;              // threads per CTA
 }  // namespace ps
 
 template <int DV>
@@ -106,26 +109,63 @@ __device__ __forceinline__ void issue_tile_loads(uint8_t* sm, const CUtensorMap*
     for (int qq = 0; qq < 4; ++qq) tma_load_3d(sm + ps::STG_L + qq * 8192, ml, qq * 32, h, tok, bar);
 }
 
+// One block diagonal of the off-diagonal inverse blocks, d = i - j:
+//   T_ij = sum_{j <= m < i} A_im X_mj   (16 x 16, K = 16 d),   X_ij = -X_ii T_ij.
+template <int D>
+__device__ __forceinline__ void solve_level(const float* __restrict__ AF, float* __restrict__ XF,
+                                            float* __restrict__ TMP, int t) {
+    constexpr int LDA = ps::LDA;
+    constexpr int NB = 4 - D;
+    for (int e = t; e < NB * 256; e += ps::NT) {
+        const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, i = bi + D, j = bi;
+        const float* a = AF + (16 * i + rr) * LDA + 16 * j;
+        const float* x = XF + (16 * j) * LDA + 16 * j + cc;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16 * D; m += 4) {
+            s0 = fmaf(a[m], x[m * LDA], s0);
+            s1 = fmaf(a[m + 1], x[(m + 1) * LDA], s1);
+            s2 = fmaf(a[m + 2], x[(m + 2) * LDA], s2);
+            s3 = fmaf(a[m + 3], x[(m + 3) * LDA], s3);
+        }
+        TMP[e] = (s0 + s1) + (s2 + s3);
+    }
+    __syncthreads();
+    for (int e = t; e < NB * 256; e += ps::NT) {
+        const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, i = bi + D, j = bi;
+        const float* xi = XF + (16 * i + rr) * LDA + 16 * i;   // row rr of X_ii (zero above the diagonal)
+        const float* tm = TMP + bi * 256 + cc;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; m += 2) {
+            s0 = fmaf(xi[m], tm[m * 16], s0);
+            s1 = fmaf(xi[m + 1], tm[(m + 1) * 16], s1);
+        }
+        XF[(16 * i + rr) * LDA + 16 * j + cc] = -(s0 + s1);
+    }
+    __syncthreads();
+}
+
 template <int DV>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(512, 1)
 prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_l,
                  const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                  const int32_t* __restrict__ cu_chunks, int n_seqs, int H, long long win_lo, long long n_items,
                  uint8_t* __restrict__ packets, int* status) {
     using P = Pk<DV>;
+    constexpr int NT = ps::NT;
+    constexpr int LDA = ps::LDA;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     __shared__ __align__(8) uint64_t bar_load, bar_mma;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     float* bet = reinterpret_cast<float*>(sm + ps::MISC);
-    float* tot = bet + 64;
+    float* tot = bet + 64;   // [8 half-tiles][128 channels]
     float* AF = reinterpret_cast<float*>(sm + ps::AF);
-    float* AQF = reinterpret_cast<float*>(sm + ps::AQF);
     float* XF = reinterpret_cast<float*>(sm + ps::XF);
     float* TMP = reinterpret_cast<float*>(sm + ps::TMP);
-    constexpr int LDA = ps::LDA;
 
     if (t == 0) {
         mbar_init(&bar_load, 1);
@@ -137,6 +177,18 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tmem_alloc(&tmem_slot, 256);
         tmem_relinquish();
     }
+    // identity rows 0..63 of [I; Aqk] (rows 64..127 are rewritten for every item)
+    for (int e = t; e < 64 * 8; e += NT) {
+        const int r = e >> 3, sc = e & 7;
+        uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        if ((r >> 3) == sc) {
+            const uint32_t one = 0x3F80u << (16 * (r & 1));   // bf16 1.0 in the low or high half
+            const int word = (r & 7) >> 1;
+            if (word == 0) z.x = one; else if (word == 1) z.y = one; else if (word == 2) z.z = one; else z.w = one;
+        }
+        *reinterpret_cast<uint4*>(sm + ps::IAQ + r * 128 + ((sc ^ (r & 7)) << 4)) = z;
+    }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -164,34 +216,39 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         ph_load ^= 1;
         if (t == 0) load_pending = false;
 
-        // ---------------- column pass: thread = (channel pair, 16-token tile)
+        // ---------------- column pass: thread = (channel pair, 8-token half tile)
         {
-            const int cp = t & 63, tq = t >> 6, c0 = 2 * cp;
-            float2 p[16];
+            const int cp = t & 63, q8 = t >> 6, tq = q8 >> 1, hh = q8 & 1, c0 = 2 * cp;
+            float2 p[8];
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int r = 16 * tq + j;
+            for (int j = 0; j < 8; ++j) {
+                const int r = 8 * q8 + j;
                 const float2 la =
                     *reinterpret_cast<const float2*>(sm + ps::STG_L + (c0 >> 5) * 8192 + r * 128 + (c0 & 31) * 4);
                 if (r < n) {
                     acc.x += floor_log_decay(la.x);
                     acc.y += floor_log_decay(la.y);
                 }
-                p[j] = acc;   // g_r - b_tq: the log-decay inside the tile up to r
+                p[j] = acc;
             }
-            tot[tq * 128 + c0] = acc.x;
-            tot[tq * 128 + c0 + 1] = acc.y;
+            tot[q8 * 128 + c0] = acc.x;
+            tot[q8 * 128 + c0 + 1] = acc.y;
             __syncthreads();
+            if (hh) {   // second half of the tile: add the first half's total
+                const float ox = tot[(q8 - 1) * 128 + c0], oy = tot[(q8 - 1) * 128 + c0 + 1];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) { p[j].x += ox; p[j].y += oy; }
+            }
+            // p[j] = g_r - b_tq: the log-decay inside the tile up to r
             float bx[5], by[5];
             bx[0] = 0.f; by[0] = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                bx[i + 1] = bx[i] + tot[i * 128 + c0];
-                by[i + 1] = by[i] + tot[i * 128 + c0 + 1];
+                bx[i + 1] = bx[i] + tot[(2 * i) * 128 + c0] + tot[(2 * i + 1) * 128 + c0];
+                by[i + 1] = by[i] + tot[(2 * i) * 128 + c0 + 1] + tot[(2 * i + 1) * 128 + c0 + 1];
             }
-            // per-(tile, channel) factors, all in [e^-320, 1] or underflowing only when negligible
-            const float ebx = __expf(bx[tq]), eby = __expf(by[tq]);                         // e^{b_t}
+            const float ebx = __expf(bx[tq]), eby = __expf(by[tq]);                             // e^{b_t}
             const float ftx = __expf(bx[tq + 1] - bx[tq]), fty = __expf(by[tq + 1] - by[tq]);   // e^{b_{t+1}-b_t}
             const float ecx = __expf(bx[4] - bx[tq + 1]), ecy = __expf(by[4] - by[tq + 1]);     // e^{g_C-b_{t+1}}
             float dvx[4], dvy[4];   // e^{b_i - b_{t+1}}, i > t
@@ -200,60 +257,56 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 dvx[i] = i > tq ? __expf(bx[i] - bx[tq + 1]) : 0.f;
                 dvy[i] = i > tq ? __expf(by[i] - by[tq + 1]) : 0.f;
             }
-            if (tq == 3)
+            if (q8 == 7)
                 *reinterpret_cast<float2*>(pkt + P::G + c0 * 4) = make_float2(__expf(bx[4]), __expf(by[4]));
 
+            float tk[2][8], tv[2][8], td[2][8];   // beta K gamma, beta V, Kdec along the 8 tokens
 #pragma unroll
-            for (int grp = 0; grp < 2; ++grp) {
-                float tk[2][8], tv[2][8], td[2][8];   // beta K gamma, beta V, Kdec along 8 tokens
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const int j = 8 * grp + jj, r = 16 * tq + j;
-                    const bool in = r < n;
-                    const uint32_t kb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 +
+            for (int j = 0; j < 8; ++j) {
+                const int r = 8 * q8 + j;
+                const bool in = r < n;
+                const uint32_t kb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 +
+                                                                       r * 128 + (c0 & 63) * 2);
+                const uint32_t qb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 +
+                                                                       r * 128 + (c0 & 63) * 2);
+                const float2 kf = in ? bf2_to_f2(kb) : make_float2(0.f, 0.f);
+                const float2 qf = in ? bf2_to_f2(qb) : make_float2(0.f, 0.f);
+                float2 vf = make_float2(0.f, 0.f);
+                if (c0 < DV && in) {
+                    const uint32_t vb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 +
                                                                            r * 128 + (c0 & 63) * 2);
-                    const uint32_t qb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 +
-                                                                           r * 128 + (c0 & 63) * 2);
-                    const float2 kf = in ? bf2_to_f2(kb) : make_float2(0.f, 0.f);
-                    const float2 qf = in ? bf2_to_f2(qb) : make_float2(0.f, 0.f);
-                    float2 vf = make_float2(0.f, 0.f);
-                    if (c0 < DV && in) {
-                        const uint32_t vb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 +
-                                                                               r * 128 + (c0 & 63) * 2);
-                        vf = bf2_to_f2(vb);
-                    }
-                    const float Ex = __expf(p[j].x), Ey = __expf(p[j].y);     // e^{g_r - b_t} <= 1
-                    const float Ix = __expf(-p[j].x), Iy = __expf(-p[j].y);   // e^{b_t - g_r} <= e^80.09
-                    const float Fx = ftx * Ix, Fy = fty * Iy;                 // e^{b_{t+1} - g_r} <= 1
-                    const float Gx = ebx * Ex, Gy = eby * Ey;                 // e^{g_r}
-                    const float bt = bet[r];
-                    // row side of A / Aqk
-                    st_b32(sm + ps::RALL + sw128_offset(r, c0, 128), pack_bf16x2(kf.x * Ex, kf.y * Ey));
-                    st_b32(sm + ps::RALL + sw128_offset(64 + r, c0, 128), pack_bf16x2(qf.x * Ex, qf.y * Ey));
-                    // key side: own tile (diagonal) and the variants of later row tiles
-                    st_b32(sm + ps::BVAR + 2048 * tq * (tq + 1) + sw128_offset(r, c0, 16 * (tq + 1)),
-                           pack_bf16x2(kf.x * Ix, kf.y * Iy));
-#pragma unroll
-                    for (int i = 1; i < 4; ++i)
-                        if (i > tq)
-                            st_b32(sm + ps::BVAR + 2048 * i * (i + 1) + sw128_offset(r, c0, 16 * (i + 1)),
-                                   pack_bf16x2(kf.x * Fx * dvx[i], kf.y * Fy * dvy[i]));
-                    // Q * gamma for the epilogue (P = Q gamma - ...)
-                    st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2,
-                           pack_bf16x2(qf.x * Gx, qf.y * Gy));
-                    tk[0][jj] = bt * kf.x * Gx; tk[1][jj] = bt * kf.y * Gy;
-                    tv[0][jj] = bt * vf.x;      tv[1][jj] = bt * vf.y;
-                    td[0][jj] = kf.x * ecx * Fx; td[1][jj] = kf.y * ecy * Fy;
+                    vf = bf2_to_f2(vb);
                 }
-                const int kc = 2 * tq + grp;   // 8-token chunk index along the 64-token K extent
+                const float Ex = __expf(p[j].x), Ey = __expf(p[j].y);     // e^{g_r - b_t} <= 1
+                const float Ix = __expf(-p[j].x), Iy = __expf(-p[j].y);   // e^{b_t - g_r} <= e^80.09
+                const float Fx = ftx * Ix, Fy = fty * Iy;                 // e^{b_{t+1} - g_r} <= 1
+                const float Gx = ebx * Ex, Gy = eby * Ey;                 // e^{g_r}
+                const float bt = bet[r];
+                // row side of A / Aqk
+                st_b32(sm + ps::RALL + sw128_offset(r, c0, 128), pack_bf16x2(kf.x * Ex, kf.y * Ey));
+                st_b32(sm + ps::RALL + sw128_offset(64 + r, c0, 128), pack_bf16x2(qf.x * Ex, qf.y * Ey));
+                // key side: own tile (diagonal) and the variants of later row tiles
+                st_b32(sm + ps::BVAR + 2048 * tq * (tq + 1) + sw128_offset(r, c0, 16 * (tq + 1)),
+                       pack_bf16x2(kf.x * Ix, kf.y * Iy));
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    const int c = c0 + ch;
-                    const uint32_t sw = static_cast<uint32_t>((kc ^ (c & 7)) << 4);
-                    *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + sw) = pack8(tk[ch]);
-                    if (c < DV) *reinterpret_cast<uint4*>(sm + ps::BKV + (128 + c) * 128 + sw) = pack8(tv[ch]);
-                    *reinterpret_cast<uint4*>(pkt + P::KD + c * 128 + sw) = pack8(td[ch]);
-                }
+                for (int i = 1; i < 4; ++i)
+                    if (i > tq)
+                        st_b32(sm + ps::BVAR + 2048 * i * (i + 1) + sw128_offset(r, c0, 16 * (i + 1)),
+                               pack_bf16x2(kf.x * Fx * dvx[i], kf.y * Fy * dvy[i]));
+                // Q * gamma for the epilogue (P = Q gamma - ...)
+                st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2,
+                       pack_bf16x2(qf.x * Gx, qf.y * Gy));
+                tk[0][j] = bt * kf.x * Gx; tk[1][j] = bt * kf.y * Gy;
+                tv[0][j] = bt * vf.x;      tv[1][j] = bt * vf.y;
+                td[0][j] = kf.x * ecx * Fx; td[1][j] = kf.y * ecy * Fy;
+            }
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                const int c = c0 + ch;
+                const uint32_t sw = static_cast<uint32_t>((q8 ^ (c & 7)) << 4);   // 8-token chunk q8 of row c
+                *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + sw) = pack8(tk[ch]);
+                if (c < DV) *reinterpret_cast<uint4*>(sm + ps::BKV + (128 + c) * 128 + sw) = pack8(tv[ch]);
+                *reinterpret_cast<uint4*>(pkt + P::KD + c * 128 + sw) = pack8(td[ch]);
             }
         }
         fence_proxy_async_smem();
@@ -294,8 +347,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         ph_mma ^= 1;
         tc_fence_after();
 
-        // ---------------- TMEM -> fp32 A (strict lower, beta rows) and Aqk (inclusive lower)
-        {
+        // ---------------- TMEM -> fp32 A (strict lower, beta rows) and bf16 Aqk (inclusive lower) into [I; Aqk]
+        if (w < 8) {
             const int qw = w & 3, role = w >> 2;
             const int vi = 2 * (qw & 1) + role;
             const int nv = 16 * (vi + 1);
@@ -303,7 +356,6 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const int r = (32 * qw + lane) & 63;
             const bool is_q = qw >= 2;
             const bool mine = (lane >> 4) == role;
-            float* dst = is_q ? AQF : AF;
             const float br = bet[r];
 #pragma unroll
             for (int cb = 0; cb < 64; cb += 16) {
@@ -316,10 +368,21 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 }
                 if (mine) {
+                    if (is_q) {
+                        float o8[8];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int s = cb + j;
-                        dst[r * LDA + s] = is_q ? (s <= r ? v[j] : 0.f) : (s < r ? br * v[j] : 0.f);
+                        for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) o8[j] = (cb + 8 * hf + j <= r) ? v[8 * hf + j] : 0.f;
+                            const int sc = (cb >> 3) + hf;
+                            *reinterpret_cast<uint4*>(sm + ps::IAQ + (64 + r) * 128 + ((sc ^ (r & 7)) << 4)) = pack8(o8);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int s = cb + j;
+                            AF[r * LDA + s] = s < r ? br * v[j] : 0.f;
+                        }
                     }
                 }
             }
@@ -327,57 +390,72 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tc_fence_before();
         __syncthreads();
 
-        // ---------------- X = (I + A)^-1: diagonal blocks by forward substitution (lane = column) ...
-        if (t < 128 && lane < 16) {
+        // ---------------- X = (I + A)^-1: diagonal 16x16 blocks, column held in registers (lane = column)
+        if (w < 4 && lane < 16) {
             const int o0 = 16 * w, col = lane;
-            for (int r = 0; r < 16; ++r) {
-                float x = (r == col) ? 1.f : 0.f;
-                for (int m = col; m < r; ++m) x = fmaf(-AF[(o0 + r) * LDA + o0 + m], XF[(o0 + m) * LDA + o0 + col], x);
-                XF[(o0 + r) * LDA + o0 + col] = x;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) x[r] = (r == col) ? 1.f : 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float xm = x[m];
+#pragma unroll
+                for (int r = m + 1; r < 16; ++r) x[r] = fmaf(-AF[(o0 + r) * LDA + o0 + m], xm, x[r]);
             }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) XF[(o0 + r) * LDA + o0 + col] = x[r];
         }
-        for (int e = t; e < 64 * 64; e += 256) {
+        for (int e = t; e < 64 * 64; e += NT) {   // strictly upper blocks are zero
             const int r = e >> 6, s = e & 63;
             if ((s >> 4) > (r >> 4)) XF[r * LDA + s] = 0.f;
         }
         __syncthreads();
-        // ... then the off-diagonal blocks by block diagonal: X_ij = -X_ii sum_{j<=m<i} A_im X_mj
-        for (int d = 1; d < 4; ++d) {
-            const int nb = 4 - d;
-            for (int e = t; e < nb * 256; e += 256) {
-                const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, i = bi + d, j = bi;
-                float a = 0.f;
-                for (int m = 16 * j; m < 16 * i; ++m) a = fmaf(AF[(16 * i + rr) * LDA + m], XF[m * LDA + 16 * j + cc], a);
-                TMP[e] = a;
-            }
-            __syncthreads();
-            for (int e = t; e < nb * 256; e += 256) {
-                const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, i = bi + d, j = bi;
-                float a = 0.f;
-                for (int m = 0; m <= rr; ++m) a = fmaf(XF[(16 * i + rr) * LDA + 16 * i + m], TMP[bi * 256 + m * 16 + cc], a);
-                XF[(16 * i + rr) * LDA + 16 * j + cc] = -a;
-            }
-            __syncthreads();
-        }
-        // [X; Y] (Y = Aqk X) as the bf16 A operand of phase B: 128 x 64, K-major, 128B swizzle
-        for (int e = t; e < 128 * 8; e += 256) {
-            const int m = e >> 3, mc = e & 7;
+        solve_level<1>(AF, XF, TMP, t);
+        solve_level<2>(AF, XF, TMP, t);
+        solve_level<3>(AF, XF, TMP, t);
+        // X^T as the bf16 B operand of the Y product: row m = column m of X, K = 64 rows of X
+        {
+            const int m = t >> 3, uc = t & 7;
             float v[8];
-            if (m < 64) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = XF[m * LDA + 8 * mc + j];
-            } else {
-                const int r = m - 64;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = 0.f;
-                for (int u = 8 * mc; u <= r; ++u) {
-                    const float a = AQF[r * LDA + u];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) v[j] = fmaf(a, XF[u * LDA + 8 * mc + j], v[j]);
-                }
-            }
-            *reinterpret_cast<uint4*>(sm + ps::XY + m * 128 + ((mc ^ (m & 7)) << 4)) = pack8(v);
+            for (int j = 0; j < 8; ++j) v[j] = XF[(8 * uc + j) * LDA + m];
+            *reinterpret_cast<uint4*>(sm + ps::XT + m * 128 + ((uc ^ (m & 7)) << 4)) = pack8(v);
         }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---------------- phase Y: [X; Y] = [I; Aqk] X   (M = 128, N = 64, K = 64)
+        if (t == 0) {
+            tc_fence_after();
+            const uint32_t ia = smem_u32(sm + ps::IAQ), xt = smem_u32(sm + ps::XT);
+            const uint32_t idesc = idesc_bf16(128, 64);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma_f16(tm, sdesc_k_sw128(ia + ks * 32), sdesc_k_sw128(xt + ks * 32), idesc, ks > 0);
+            umma_commit(&bar_mma);
+        }
+        {
+            const bool ok = mbar_wait(&bar_mma, ph_mma, status);
+            if (__syncthreads_or(!ok)) break;
+        }
+        ph_mma ^= 1;
+        tc_fence_after();
+        {   // 16 warps: lane quarter qw, 16-column group cg
+            const int qw = w & 3, cg = w >> 2;
+            const int m = 32 * qw + lane;
+            float v[16];
+            tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 16 * cg, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float o8[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o8[j] = v[8 * hf + j];
+                const int sc = 2 * cg + hf;
+                *reinterpret_cast<uint4*>(sm + ps::XY + m * 128 + ((sc ^ (m & 7)) << 4)) = pack8(o8);
+            }
+        }
+        tc_fence_before();
         fence_proxy_async_smem();
         __syncthreads();
 
@@ -400,12 +478,12 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
         // ---------------- epilogue: rows 0..63 -> -W | U, rows 64..127 -> P = Q gamma - Y bK gamma | O_intra
         {
-            const int qw = w & 3, half = w >> 2;
+            const int qw = w & 3, cg = w >> 2;   // 64-column group: 0,1 -> K part, 2,3 -> V part
             const int m = 32 * qw + lane;
             const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
-            if (half == 0) {
+            if (cg < 2) {
 #pragma unroll 1
-                for (int c16 = 0; c16 < 8; ++c16) {
+                for (int c16 = 4 * cg; c16 < 4 * cg + 4; ++c16) {
                     float v[16];
                     tmem_ld16(lane_base + 16 * c16, v);
                     tmem_wait_ld();
@@ -427,9 +505,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                                                   (((cc & 7) ^ (m & 7)) << 4)) = pack8(o8);
                     }
                 }
-            } else {
+            } else if (64 * (cg - 2) < DV) {
 #pragma unroll 1
-                for (int c16 = 0; c16 < DV / 16; ++c16) {
+                for (int c16 = 4 * (cg - 2); c16 < 4 * (cg - 2) + 4; ++c16) {
                     float v[16];
                     tmem_ld16(lane_base + 128 + 16 * c16, v);
                     tmem_wait_ld();
@@ -474,18 +552,23 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 // inter-chunk state pass
 template <int DV, int DVS>
 struct SCfg {
-    static constexpr int NCW = DVS / 2;   // state columns per epilogue warp (two warps share a lane quarter)
+    static constexpr int NEW = DVS >= 64 ? 16 : 8;        // epilogue warps (NEW/4 share each TMEM lane quarter)
+    static constexpr int NCW = DVS * 4 / NEW;              // state columns per epilogue warp (>= 16)
+    static constexpr int NT = 32 * (NEW + 2);              // + producer warp + MMA warp
+    static constexpr bool MN = DVS >= 64;                  // S and U' staged MN-major (row = channel / token)
     static constexpr int NST = DVS == 128 ? 2 : 3;
     static constexpr uint32_t AW = 0, KD = 32768, U = 49152, OI = U + DVS * 128, G = OI + DVS * 128;
     static constexpr uint32_t STAGE = ((G + 512 + 1023) / 1024) * 1024;
-    static constexpr uint32_t SOP = NST * STAGE;      // S^T as B operand: 2 K atoms x DVS rows x 128 B
-    static constexpr uint32_t UOP = SOP + DVS * 256;  // U'^T as B operand: 1 K atom x DVS rows x 128 B
+    static constexpr uint32_t SOP = NST * STAGE;      // S as B operand (N = DVS, K = 128)
+    static constexpr uint32_t UOP = SOP + DVS * 256;  // U' as B operand (N = DVS, K = 64)
     static constexpr uint32_t BYTES = UOP + DVS * 128;
+    static constexpr uint32_t S_LBO = 128 * 128;      // MN-major: 64 columns x 128 K rows per block
+    static constexpr uint32_t U_LBO = 64 * 128;       // MN-major: 64 columns x 64 K rows per block
     static constexpr uint32_t TMEM_COLS = 2 * DVS <= 32 ? 32 : (2 * DVS <= 64 ? 64 : (2 * DVS <= 128 ? 128 : 256));
 };
 
 template <int DV, int DVS>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(SCfg<DV, DVS>::NT, 1)
 state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict__ cu_seqlens,
                   const int32_t* __restrict__ cu_chunks, int n_seqs, int H, long long win_lo, long long win_hi,
                   const float* __restrict__ initial_state, __nv_bfloat16* __restrict__ o,
@@ -494,7 +577,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                   int* status) {
     using C = SCfg<DV, DVS>;
     using P = Pk<DV>;
-    constexpr int NST = C::NST, NCW = C::NCW, NSV = DV / DVS, CW = DV + kDK;
+    constexpr int NST = C::NST, NCW = C::NCW, NEW = C::NEW, NSV = DV / DVS, CW = DV + kDK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     __shared__ __align__(8) uint64_t full[NST], empty[NST], d1_full, d2_full, s_ready, up_ready;
@@ -519,12 +602,12 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
     if (t == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + 8);
+            mbar_init(&empty[s], 1 + NEW);
         }
         mbar_init(&d1_full, 1);
         mbar_init(&d2_full, 1);
-        mbar_init(&s_ready, 8);
-        mbar_init(&up_ready, 8);
+        mbar_init(&s_ready, NEW);
+        mbar_init(&up_ready, NEW / 2);   // only the warps that produce U' (TMEM lanes 0..63)
         fence_barrier_init();
     }
     if (w == 0) {
@@ -536,7 +619,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
     tc_fence_after();
     const uint32_t tm = tmem_slot;
 
-    if (w == 8) {
+    if (w == NEW) {
         // ---------------- producer: packets -> shared-memory ring (bulk TMA)
         if (lane == 0) {
             int issued = 0;
@@ -560,10 +643,10 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             for (int ci = issued - NST < 0 ? 0 : issued - NST; ci < issued; ++ci)
                 mbar_wait(&full[ci % NST], (ci / NST) & 1, nullptr);
         }
-    } else if (w == 9) {
+    } else if (w == NEW + 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, DVS);
+            const uint32_t idesc = idesc_bf16(128, DVS, false, C::MN);
             const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP);
             for (int ci = 0; ci < nch; ++ci) {
                 const int st = ci % NST;
@@ -575,17 +658,20 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
-                    umma_f16(tm, sdesc_k_sw128(sb + C::AW + ka * 16384 + kb),
-                             sdesc_k_sw128(sop + ka * (DVS * 128) + kb), idesc, ks > 0);
+                    const uint64_t bdesc = C::MN ? sdesc_mn_sw128(sop + ks * 2048, C::S_LBO)
+                                                 : sdesc_k_sw128(sop + ka * (DVS * 128) + kb);
+                    umma_f16(tm, sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc, ks > 0);
                 }
                 umma_commit(&d1_full);
                 if (!mbar_wait(&up_ready, ci & 1, status)) break;
                 tc_fence_after();
                 // D2 = Kdec^T U'   (M = 128, N = DVS, K = 64)
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), sdesc_k_sw128(uop + ks * 32), idesc,
-                             ks > 0);
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t bdesc = C::MN ? sdesc_mn_sw128(uop + ks * 2048, C::U_LBO)
+                                                 : sdesc_k_sw128(uop + ks * 32);
+                    umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), bdesc, idesc, ks > 0);
+                }
                 umma_commit(&d2_full);
                 umma_commit(&empty[st]);
             }
@@ -605,10 +691,22 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             else x = initial_state ? initial_state[(sh * kDK + i) * DV + col] : 0.f;
             S[j] = x;
         }
+        // S (and later U') as a B operand: MN-major rows are written 8 columns at a time
         auto write_sop = [&]() {
+            if constexpr (C::MN) {
 #pragma unroll
-            for (int j = 0; j < NCW; ++j)
-                *reinterpret_cast<__nv_bfloat16*>(sm + C::SOP + sw128_offset(jw + j, i, DVS)) = __float2bfloat16_rn(S[j]);
+                for (int j = 0; j < NCW; j += 8) {
+                    float f8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f8[e] = S[j + e];
+                    *reinterpret_cast<uint4*>(sm + C::SOP + sw128_mn_offset(jw + j, i, C::S_LBO)) = pack8(f8);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < NCW; ++j)
+                    *reinterpret_cast<__nv_bfloat16*>(sm + C::SOP + sw128_offset(jw + j, i, DVS)) =
+                        __float2bfloat16_rn(S[j]);
+            }
         };
         write_sop();
         fence_proxy_async_smem();
@@ -640,24 +738,32 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                             unpack8(*reinterpret_cast<const uint4*>(sb + C::U + cc * 1024 + i * 16), u8);
                         }
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            *reinterpret_cast<__nv_bfloat16*>(sm + C::UOP + sw128_offset(jw + cb + 8 * sub + e, i, DVS)) =
-                                __float2bfloat16_rn(u8[e] + v[8 * sub + e]);
+                        for (int e = 0; e < 8; ++e) u8[e] += v[8 * sub + e];
+                        if constexpr (C::MN) {
+                            *reinterpret_cast<uint4*>(sm + C::UOP + sw128_mn_offset(8 * cc, i, C::U_LBO)) = pack8(u8);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                *reinterpret_cast<__nv_bfloat16*>(sm + C::UOP + sw128_offset(8 * cc + e, i, DVS)) =
+                                    __float2bfloat16_rn(u8[e]);
+                        }
                     } else if (!trans && i - 64 < n) {
                         const int r = i - 64;
                         float o8[8];
                         unpack8(*reinterpret_cast<const uint4*>(sb + C::OI + cc * 1024 + r * 16), o8);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) o8[e] += v[8 * sub + e];
-                        *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + j0 + jw +
-                                                  cb + 8 * sub) = pack8(o8);
+                        *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + j0 +
+                                                  8 * cc) = pack8(o8);
                     }
                 }
             }
             tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&up_ready);
+            if (qw < 2) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&up_ready);
+            }
             if (!mbar_wait(&d2_full, ci & 1, status)) break;
             tc_fence_after();
             const float gam = *reinterpret_cast<const float*>(sb + C::G + i * 4);
@@ -751,7 +857,7 @@ cudaError_t launch_state(const ChunkArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int slices = DV / DVS + (a.final_transition ? kDK / DVS : 0);
     dim3 grid(a.n_seqs * a.H, slices);
-    state_bf16_kernel<DV, DVS><<<grid, 320, smem, s>>>(
+    state_bf16_kernel<DV, DVS><<<grid, C::NT, smem, s>>>(
         static_cast<const uint8_t*>(a.packets), a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, a.win_hi,
         a.initial_state, static_cast<__nv_bfloat16*>(a.o), a.final_state, a.final_transition, a.ckpt_stride,
         a.checkpoints, a.ckpt_cu, a.carry, a.status);
@@ -773,7 +879,7 @@ cudaError_t launch_bf16_t(const ChunkArgs& a, cudaStream_t s) {
         cudaError_t e = cudaFuncSetAttribute(prep_bf16_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         const long long grid = items < num_sms() ? items : num_sms();
-        prep_bf16_kernel<DV><<<static_cast<unsigned>(grid), 256, smem, s>>>(
+        prep_bf16_kernel<DV><<<static_cast<unsigned>(grid), ps::NT, smem, s>>>(
             mq, mk, mv, ml, a.beta, a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, items,
             static_cast<uint8_t*>(a.packets), a.status);
         e = cudaGetLastError();

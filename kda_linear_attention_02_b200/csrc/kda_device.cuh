@@ -173,13 +173,34 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(2u) << 61;              // SWIZZLE_128B
     return d;
 }
-// Instruction descriptor: kind::f16 with A = B = bf16, D = fp32, both K-major, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool negate_a = false) {
+// Shared-memory matrix descriptor, MN-major operand with the 128-byte swizzle: each K row holds
+// 64 consecutive MN elements (128 B, 16-byte chunks XOR-permuted by (k % 8)); 8 K rows form a
+// 1024-byte atom; atoms follow each other along K (SBO = 1024); the next 64 MN elements start
+// lbo_bytes further.  Stepping K by 16 adds 2048 B to the start address.
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((1024u >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+// Instruction descriptor: kind::f16 with A = B = bf16, D = fp32, shape M x N; A K-major, B K-major
+// unless b_mn (then MN-major).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool negate_a = false, bool b_mn = false) {
     return (1u << 4)                       // D format: f32
            | (1u << 7)                     // A format: bf16
            | (1u << 10)                    // B format: bf16
            | ((negate_a ? 1u : 0u) << 13)  // negate A
+           | ((b_mn ? 1u : 0u) << 16)      // B major-ness
            | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+// Byte offset of element (mn, k) in an MN-major 128B-swizzled tile ([mn/64 blocks of lbo bytes]
+// [k/8 atoms of 1024 B][k%8 rows of 128 B]).
+__host__ __device__ __forceinline__ uint32_t sw128_mn_offset(int mn, int k, uint32_t lbo_bytes) {
+    return static_cast<uint32_t>((mn >> 6) * lbo_bytes + (k >> 3) * 1024 + (k & 7) * 128 +
+                                 ((((mn & 63) >> 3) ^ (k & 7)) << 4) + (mn & 7) * 2);
 }
 
 // Byte offset of element (row, k) in a K-major 128B-swizzled tile of `rows` rows whose K extent is

@@ -64,6 +64,7 @@ ChunkEvents* profile_slot();   // events for the current call, or null
 
 // Diagnostics.
 cudaError_t launch_selftest_wait(int limit_us, int* d_result, cudaStream_t s);
-cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int* status, cudaStream_t s);
+cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int b_mn, int* status,
+                                 cudaStream_t s);
 
 }  // namespace kda

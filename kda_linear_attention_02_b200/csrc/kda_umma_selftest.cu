@@ -1,6 +1,6 @@
 // kda_umma_selftest.cu -- diagnostic: one tcgen05 bf16 product through the same shared-memory
-// descriptors (K-major, 128-byte swizzle), TMEM allocation, commit and TMEM-load path that the chunk
-// kernels use.  D[128, n] = A[128, 64] * B[n, 64]^T.  No KDA arithmetic.
+// descriptors (128-byte swizzle; B K-major or MN-major), TMEM allocation, commit and TMEM-load path
+// that the chunk kernels use.  D[128, n] = A[128, 64] * B[n, 64]^T.  No KDA arithmetic.
 #include "kda_device.cuh"
 #include "kda_internal.h"
 
@@ -8,7 +8,7 @@ namespace kda {
 
 __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16* __restrict__ a,
                                                             const __nv_bfloat16* __restrict__ b,
-                                                            float* __restrict__ d, int n, int* status) {
+                                                            float* __restrict__ d, int n, int b_mn, int* status) {
     extern __shared__ __align__(1024) uint8_t raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = base;                 // 128 rows x 128 B
@@ -23,10 +23,18 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
         const uint4 x = reinterpret_cast<const uint4*>(a + r * 64)[c];
         *reinterpret_cast<uint4*>(sA + sw128_offset(r, c * 8, 128)) = x;
     }
-    for (int e = t; e < n * 8; e += 128) {
-        const int r = e >> 3, c = e & 7;
-        const uint4 x = reinterpret_cast<const uint4*>(b + r * 64)[c];
-        *reinterpret_cast<uint4*>(sB + sw128_offset(r, c * 8, n)) = x;
+    const uint32_t lbo = 8 * 1024;   // MN-major: 64 K rows = 8 atoms per 64-element MN block
+    if (b_mn) {
+        for (int e = t; e < n * 64; e += 128) {
+            const int r = e >> 6, k = e & 63;
+            *reinterpret_cast<__nv_bfloat16*>(sB + sw128_mn_offset(r, k, lbo)) = b[r * 64 + k];
+        }
+    } else {
+        for (int e = t; e < n * 8; e += 128) {
+            const int r = e >> 3, c = e & 7;
+            const uint4 x = reinterpret_cast<const uint4*>(b + r * 64)[c];
+            *reinterpret_cast<uint4*>(sB + sw128_offset(r, c * 8, n)) = x;
+        }
     }
     fence_proxy_async_smem();
     if (t == 0) {
@@ -42,10 +50,11 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
     tc_fence_after();
     const uint32_t tm = tbase;
     if (t == 0) {
-        const uint32_t idesc = idesc_bf16(128, n);
+        const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0);
         for (int kk = 0; kk < 4; ++kk) {
             const uint64_t da = sdesc_k_sw128(smem_u32(sA) + kk * 32);
-            const uint64_t db = sdesc_k_sw128(smem_u32(sB) + kk * 32);
+            const uint64_t db = b_mn ? sdesc_mn_sw128(smem_u32(sB) + kk * 2048, lbo)
+                                     : sdesc_k_sw128(smem_u32(sB) + kk * 32);
             umma_f16(tm, da, db, idesc, kk > 0);
         }
         umma_commit(&bar);
@@ -66,12 +75,13 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
     if (w == 0) tmem_dealloc(tm, 256);
 }
 
-cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int* status, cudaStream_t s) {
-    const int smem = 1024 + 128 * 128 + n * 128;
+cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int b_mn, int* status,
+                                 cudaStream_t s) {
+    const int smem = 1024 + 128 * 128 + ((n + 63) / 64) * 64 * 128;
     cudaError_t e = cudaFuncSetAttribute(selftest_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     selftest_umma_kernel<<<1, 128, smem, s>>>(static_cast<const __nv_bfloat16*>(a),
-                                              static_cast<const __nv_bfloat16*>(b), d, n, status);
+                                              static_cast<const __nv_bfloat16*>(b), d, n, b_mn, status);
     return cudaGetLastError();
 }
 

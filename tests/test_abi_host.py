@@ -125,7 +125,8 @@ def test_decode_and_compose_host_argument_errors(lib):
                                    None) == -1
     assert lib.kda_segment_compose(vp(0x1000), vp(0x2000), vp(0x4000), None, 1, 1, 1, 128, 80, vp(0x3000), None,
                                    None) == -3
-    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 20, None) == -1
+    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 20, 0, None) == -1
+    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 32, 1, None) == -1
 
 
 def test_binding_checks_shapes_on_cpu_tensors(lib):
