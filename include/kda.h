@@ -116,6 +116,34 @@ KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v,
                            void* workspace, size_t ws_bytes, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd without a workspace argument, for callers that may not allocate device memory (a
+ * serving engine that gives all device memory to its own pool at start-up, or a program with a
+ * fixed device-memory budget that forbids allocations while running).  The pages have no
+ * counterpart to this entry point; it is library plumbing.
+ *
+ * Arguments, layouts and results are those of kda_chunk_fwd.  The scratch is one array of
+ * KDA_NOALLOC_SCRATCH_BYTES (64 MiB) compiled into the library: every GPU that loads the library
+ * holds it until the process exits.  The chunks are processed in windows sized to that array.
+ * A batch whose minimum scratch (kda_chunk_fwd_min_workspace_bytes: chunk index, the carried state
+ * of every (sequence, head), one chunk of packets) exceeds it is refused with KDA_ERR_WORKSPACE;
+ * at dk = dv = 128 that allows up to 491 (sequence, head) pairs, e.g. 15 sequences of 32 heads.
+ * The first call on each device looks the array's device address up (with that device current)
+ * and keeps it; make that first call before any stream capture.  All calls share the one array and
+ * it keeps the last call's contents (nothing in it needs to start at zero): calls that may overlap
+ * on the GPU -- on different streams, or from different host threads -- race and must not be issued.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u << 20)
+KDA_API kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                   const float* log_alpha, const float* beta,
+                                   const float* initial_state,
+                                   const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
+                                   int H, int dk, int dv, kda_dtype_t dtype,
+                                   int ckpt_stride,
+                                   void* o, float* final_state,
+                                   float* checkpoints, const int32_t* ckpt_cu,
+                                   float* final_transition, kda_stream_t stream);
+
+/*
  * One recurrent (decode) step for n sequences x H heads, state updated in place: the fixed-size
  * state of the llm-wiki chapter's section 1 (O(1) memory per token).  state [n,H,dk,dv] fp32;
  * q, k [n,H,dk], v [n,H,dv] of `dtype`; log_alpha [n,H,dk] fp32; beta [n,H] fp32; o [n,H,dv] of

@@ -15,7 +15,7 @@ import torch
 
 __all__ = [
     "KDA_BF16", "KDA_F32", "KDA_CHUNK", "KDAError", "lib_path",
-    "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd",
+    "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
     "kda_recurrent_step", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
     "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
     "kda_selftest_umma",
@@ -56,6 +56,9 @@ def _load():
     L.kda_chunk_fwd.restype = i32
     L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32,
                                 vp, vp, vp, vp, vp, vp, sz, vp]
+    L.kda_chunk_fwd_noalloc.restype = i32
+    L.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32,
+                                        vp, vp, vp, vp, vp, vp]
     L.kda_recurrent_step.restype = i32
     L.kda_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
     L.kda_segment_compose.restype = i32
@@ -177,6 +180,41 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, o, final_
                                _p(checkpoints if ckpt_stride else None), _p(ckpt_cu if ckpt_stride else None),
                                _p(final_transition), _p(workspace), workspace.numel(), _stream(stream))
     _check(st, "kda_chunk_fwd")
+    return o
+
+
+def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, initial_state, cu_seqlens, o, final_state=None, *,
+                          ckpt_stride=0, checkpoints=None, ckpt_cu=None, final_transition=None, stream=None):
+    """kda_chunk_fwd for callers that may not allocate device memory (C: kda_chunk_fwd_noalloc).
+
+    Same arguments and results as kda_chunk_fwd, without a workspace: the library uses its own
+    fixed 64 MiB device array instead, so nothing is allocated here or in the library.  Calls that
+    could overlap on the GPU share that array and must not be issued concurrently.
+    """
+    _need(q, "q")
+    dev = q.device
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    n = cu_seqlens.numel() - 1
+    _need(k, "k", (T, H, dk), q.dtype, dev)
+    _need(v, "v", (T, H, dv), q.dtype, dev)
+    _need(o, "o", (T, H, dv), q.dtype, dev)
+    _need(log_alpha, "log_alpha", (T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (T, H), torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", (n + 1,), torch.int32, dev)
+    _opt(initial_state, "initial_state", (n, H, dk, dv), torch.float32, dev)
+    _opt(final_state, "final_state", (n, H, dk, dv), torch.float32, dev)
+    _opt(final_transition, "final_transition", (n, H, dk, dk), torch.float32, dev)
+    if ckpt_stride:
+        _need(checkpoints, "checkpoints", None, torch.float32, dev)
+        _need(ckpt_cu, "ckpt_cu", (n + 1,), torch.int32, dev)
+    st = _load().kda_chunk_fwd_noalloc(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(initial_state),
+                                       _p(cu_seqlens), n, T, H, dk, dv, dt, int(ckpt_stride), _p(o),
+                                       _p(final_state), _p(checkpoints if ckpt_stride else None),
+                                       _p(ckpt_cu if ckpt_stride else None), _p(final_transition),
+                                       _stream(stream))
+    _check(st, "kda_chunk_fwd_noalloc")
     return o
 
 
