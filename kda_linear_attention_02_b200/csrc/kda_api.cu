@@ -164,15 +164,20 @@ const char* kda_status_string(kda_status_t st) {
     return "KDA_ERR_UNKNOWN";
 }
 
+// Per window chunk: H packets and one chunk-table entry.
+size_t chunk_bytes(kda_dtype_t dt, int H, int dk, int dv) {
+    return static_cast<size_t>(H) * packet_bytes(dt, dk, dv) + sizeof(int2);
+}
+
 size_t kda_chunk_fwd_workspace_bytes(int64_t total_tokens, int n_seqs, int H, int dk, int dv, kda_dtype_t dt) {
     if (total_tokens < 0 || n_seqs < 0 || H <= 0 || !supported(dt, dk, dv)) return 0;
     return index_bytes(n_seqs) +
-           static_cast<size_t>(chunk_upper_bound(total_tokens, n_seqs)) * H * packet_bytes(dt, dk, dv);
+           static_cast<size_t>(chunk_upper_bound(total_tokens, n_seqs)) * chunk_bytes(dt, H, dk, dv);
 }
 
 size_t kda_chunk_fwd_min_workspace_bytes(int n_seqs, int H, int dk, int dv, kda_dtype_t dt) {
     if (n_seqs < 0 || H <= 0 || !supported(dt, dk, dv)) return 0;
-    return index_bytes(n_seqs) + carry_bytes(n_seqs, H, dk, dv) + static_cast<size_t>(H) * packet_bytes(dt, dk, dv);
+    return index_bytes(n_seqs) + carry_bytes(n_seqs, H, dk, dv) + chunk_bytes(dt, H, dk, dv);
 }
 
 kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
@@ -208,20 +213,23 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
     a.final_state = final_state; a.checkpoints = checkpoints; a.ckpt_cu = ckpt_cu;
     a.final_transition = final_transition;
 
+    const size_t cbytes = chunk_bytes(dtype, H, dk, dv);
     long long win;   // chunks per window
-    if (ws_bytes >= ib + static_cast<size_t>(ub) * H * pb) {
+    if (ws_bytes >= ib + static_cast<size_t>(ub) * cbytes) {
         win = ub > 0 ? ub : 1;
         a.carry = nullptr;
         a.packets = ws + ib;
         a.multi_window = false;
     } else {
         const size_t cb = carry_bytes(n_seqs, H, dk, dv);
-        if (ws_bytes < ib + cb + static_cast<size_t>(H) * pb) return KDA_ERR_WORKSPACE;
-        win = static_cast<long long>((ws_bytes - ib - cb) / (static_cast<size_t>(H) * pb));
+        if (ws_bytes < ib + cb + cbytes) return KDA_ERR_WORKSPACE;
+        win = static_cast<long long>((ws_bytes - ib - cb) / cbytes);
         a.carry = reinterpret_cast<float*>(ws + ib);
         a.packets = ws + ib + cb;
         a.multi_window = true;
     }
+    // the chunk table of a window follows its packets
+    a.chunk_tab = reinterpret_cast<int2*>(static_cast<char*>(a.packets) + static_cast<size_t>(win) * H * pb);
     a.status = status_ptr();
     if (!a.status) return KDA_ERR_CUDA;
     a.events = profile_slot();

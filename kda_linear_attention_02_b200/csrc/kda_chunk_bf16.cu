@@ -34,6 +34,7 @@
 //                     in registers and feed bf16 copies of S and U' back as the next operands.
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "kda_chunk_common.cuh"
@@ -44,8 +45,11 @@ namespace {
 
 constexpr int kDK = 128;
 
+// 1024-byte aligned base inside a dynamic shared-memory array.  Offsetting the array pointer itself
+// (instead of rounding an integer) keeps the shared address space visible to the compiler, so the
+// accesses through it stay shared-memory loads and stores.
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+    return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
 }
 __device__ __forceinline__ void st_b32(uint8_t* p, uint32_t v) { *reinterpret_cast<uint32_t*>(p) = v; }
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
@@ -69,7 +73,7 @@ struct Pk {
     static constexpr uint32_t AW = 0;                 // [-W; P]: 128 x 128 bf16, K-major, 128B swizzle, 2 K atoms
     static constexpr uint32_t KD = 32768;             // Kdec^T:  128 x 64 bf16, K-major, 128B swizzle
     static constexpr uint32_t U = 49152;              // U:       [DV/8][64][8] bf16 (8-column chunks)
-    static constexpr uint32_t OI = U + DV * 128;      // O_intra: [DV/8][64][8] bf16
+    static constexpr uint32_t OI = U + DV * 128;      // O_intra: [DV/64][64 rows][128 B], 16-byte chunks ^ (row % 8)
     static constexpr uint32_t G = OI + DV * 128;      // gamma_C: [128] fp32
     static constexpr uint32_t BYTES = ((G + 512 + 1023) / 1024) * 1024;
 };
@@ -79,16 +83,18 @@ struct Pk {
 namespace ps {
 constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_V = 32768, STG_L = 49152;   // raw TMA tiles
 constexpr uint32_t RALL = 81920;     // row side [K e^(g-b); Q e^(g-b)]: 128 x 128 bf16 (A operand)
-constexpr uint32_t BVAR = 114688;    // key side, variant i (rows 16(i+1)) at BVAR + 2048 i (i+1)
+constexpr uint32_t BVAR = 114688;    // key side: variants 0..3 stacked as rows [0,16) [16,48) [48,96) [96,160)
+                                     // of one 160-row B operand, [2 K atoms][160 rows][128 B]
 constexpr uint32_t QT = 155648;      // Q * gamma, [64][128] bf16, 16-byte chunks swizzled by row
 constexpr uint32_t BKV = 172032;     // [beta K gamma | beta V]^T: (128+DV) x 64 bf16 (B operand)
 constexpr uint32_t MISC = 204800;    // beta[64] fp32, half-tile totals [8][128] fp32
 constexpr uint32_t IAQ = 209920;     // [I; Aqk]: 128 x 64 bf16 (A operand of the Y product)
 // aliases of RALL/BVAR once phase A has completed
-constexpr uint32_t AF = 81920, XF = 98560, TMP = 115200, XT = 118784, XY = 126976;   // solve
+constexpr uint32_t AT = 81920, XF = 99328, TMP = 116224, XT = 124928, XY = 133120;   // solve
 constexpr uint32_t AWS = 81920, US = 114688, OIS = 131072;                          // packet staging
 constexpr uint32_t BYTES = IAQ + 16384;
-constexpr int LDA = 65;              // fp32 row pitch of A and X
+constexpr int LDT = 68;              // fp32 row pitch of A^T (float4-aligned rows)
+constexpr int LDA = 65;              // fp32 row pitch of X
 constexpr int NT = 512;              // threads per CTA
 }  // namespace ps
 
@@ -109,53 +115,16 @@ __device__ __forceinline__ void issue_tile_loads(uint8_t* sm, const CUtensorMap*
     for (int qq = 0; qq < 4; ++qq) tma_load_3d(sm + ps::STG_L + qq * 8192, ml, qq * 32, h, tok, bar);
 }
 
-// One block diagonal of the off-diagonal inverse blocks, d = i - j:
-//   T_ij = sum_{j <= m < i} A_im X_mj   (16 x 16, K = 16 d),   X_ij = -X_ii T_ij.
-template <int D>
-__device__ __forceinline__ void solve_level(const float* __restrict__ AF, float* __restrict__ XF,
-                                            float* __restrict__ TMP, int t) {
-    constexpr int LDA = ps::LDA;
-    constexpr int NB = 4 - D;
-    for (int e = t; e < NB * 256; e += ps::NT) {
-        const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, i = bi + D, j = bi;
-        const float* a = AF + (16 * i + rr) * LDA + 16 * j;
-        const float* x = XF + (16 * j) * LDA + 16 * j + cc;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16 * D; m += 4) {
-            s0 = fmaf(a[m], x[m * LDA], s0);
-            s1 = fmaf(a[m + 1], x[(m + 1) * LDA], s1);
-            s2 = fmaf(a[m + 2], x[(m + 2) * LDA], s2);
-            s3 = fmaf(a[m + 3], x[(m + 3) * LDA], s3);
-        }
-        TMP[e] = (s0 + s1) + (s2 + s3);
-    }
-    __syncthreads();
-    for (int e = t; e < NB * 256; e += ps::NT) {
-        const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, i = bi + D, j = bi;
-        const float* xi = XF + (16 * i + rr) * LDA + 16 * i;   // row rr of X_ii (zero above the diagonal)
-        const float* tm = TMP + bi * 256 + cc;
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; m += 2) {
-            s0 = fmaf(xi[m], tm[m * 16], s0);
-            s1 = fmaf(xi[m + 1], tm[(m + 1) * 16], s1);
-        }
-        XF[(16 * i + rr) * LDA + 16 * j + cc] = -(s0 + s1);
-    }
-    __syncthreads();
-}
-
 template <int DV>
 __global__ void __launch_bounds__(512, 1)
 prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_l,
-                 const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
-                 const int32_t* __restrict__ cu_chunks, int n_seqs, int H, long long win_lo, long long n_items,
+                 const float* __restrict__ beta, const int2* __restrict__ chunk_tab, int H, long long n_items,
                  uint8_t* __restrict__ packets, int* status) {
     using P = Pk<DV>;
     constexpr int NT = ps::NT;
     constexpr int LDA = ps::LDA;
+    constexpr int LDT = ps::LDT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     __shared__ __align__(8) uint64_t bar_load, bar_mma;
@@ -163,7 +132,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     float* bet = reinterpret_cast<float*>(sm + ps::MISC);
     float* tot = bet + 64;   // [8 half-tiles][128 channels]
-    float* AF = reinterpret_cast<float*>(sm + ps::AF);
+    float* AT = reinterpret_cast<float*>(sm + ps::AT);    // AT[s][r] = beta_r A[r][s]
     float* XF = reinterpret_cast<float*>(sm + ps::XF);
     float* TMP = reinterpret_cast<float*>(sm + ps::TMP);
 
@@ -196,19 +165,23 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint32_t ph_load = 0, ph_mma = 0;
     bool load_pending = false;   // meaningful in thread 0 only
 
+    // chunk table entry {first token, valid tokens} of a window item (n = 0: past the last chunk)
+    auto entry = [&](long long it) -> int2 { return it < n_items ? chunk_tab[it / H] : make_int2(0, 0); };
     long long item = blockIdx.x;
-    ChunkLoc loc{};
+    int2 loc = entry(item);
     int h = static_cast<int>(item % H);
-    bool valid = item < n_items && locate_chunk(cu_chunks, cu_seqlens, n_seqs, win_lo + item / H, loc);
+    bool valid = loc.y > 0;
+    int2 nloc = entry(item + gridDim.x);   // one item ahead
     if (t == 0 && valid) {
-        issue_tile_loads<DV>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, h, loc.tok0);
+        issue_tile_loads<DV>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, h, loc.x);
         load_pending = true;
     }
 
     while (valid) {
-        const int n = loc.n;
+        const int n = loc.y;
+        const long long tok0 = loc.x;
         uint8_t* pkt = packets + static_cast<size_t>(item) * P::BYTES;
-        if (t < 64) bet[t] = t < n ? beta[(static_cast<size_t>(loc.tok0) + t) * H + h] : 0.f;
+        if (t < 64) bet[t] = t < n ? beta[(static_cast<size_t>(tok0) + t) * H + h] : 0.f;
         {
             const bool ok = mbar_wait(&bar_load, ph_load, status);
             if (__syncthreads_or(!ok)) break;
@@ -217,6 +190,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         if (t == 0) load_pending = false;
 
         // ---------------- column pass: thread = (channel pair, 8-token half tile)
+        uint4 kd_pk[2];
         {
             const int cp = t & 63, q8 = t >> 6, tq = q8 >> 1, hh = q8 & 1, c0 = 2 * cp;
             float2 p[8];
@@ -234,6 +208,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
             tot[q8 * 128 + c0] = acc.x;
             tot[q8 * 128 + c0 + 1] = acc.y;
+            if (t == 0) bulk_wait_read0();   // the previous item's packet staging has been read out
             __syncthreads();
             if (hh) {   // second half of the tile: add the first half's total
                 const float ox = tot[(q8 - 1) * 128 + c0], oy = tot[(q8 - 1) * 128 + c0 + 1];
@@ -285,13 +260,12 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 // row side of A / Aqk
                 st_b32(sm + ps::RALL + sw128_offset(r, c0, 128), pack_bf16x2(kf.x * Ex, kf.y * Ey));
                 st_b32(sm + ps::RALL + sw128_offset(64 + r, c0, 128), pack_bf16x2(qf.x * Ex, qf.y * Ey));
-                // key side: own tile (diagonal) and the variants of later row tiles
-                st_b32(sm + ps::BVAR + 2048 * tq * (tq + 1) + sw128_offset(r, c0, 16 * (tq + 1)),
-                       pack_bf16x2(kf.x * Ix, kf.y * Iy));
+                // key side: own tile (diagonal) and the variants of later row tiles (variant i: rows 8 i (i+1) + r)
+                st_b32(sm + ps::BVAR + sw128_offset(8 * tq * (tq + 1) + r, c0, 160), pack_bf16x2(kf.x * Ix, kf.y * Iy));
 #pragma unroll
                 for (int i = 1; i < 4; ++i)
                     if (i > tq)
-                        st_b32(sm + ps::BVAR + 2048 * i * (i + 1) + sw128_offset(r, c0, 16 * (i + 1)),
+                        st_b32(sm + ps::BVAR + sw128_offset(8 * i * (i + 1) + r, c0, 160),
                                pack_bf16x2(kf.x * Fx * dvx[i], kf.y * Fy * dvy[i]));
                 // Q * gamma for the epilogue (P = Q gamma - ...)
                 st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2,
@@ -306,40 +280,34 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 const uint32_t sw = static_cast<uint32_t>((q8 ^ (c & 7)) << 4);   // 8-token chunk q8 of row c
                 *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + sw) = pack8(tk[ch]);
                 if (c < DV) *reinterpret_cast<uint4*>(sm + ps::BKV + (128 + c) * 128 + sw) = pack8(tv[ch]);
-                *reinterpret_cast<uint4*>(pkt + P::KD + c * 128 + sw) = pack8(td[ch]);
+                kd_pk[ch] = pack8(td[ch]);   // Kdec^T chunk: staged for the packet store after phase B
             }
         }
         fence_proxy_async_smem();
         __syncthreads();
 
-        // prefetch the next item's tiles into the (now free) staging area
-        const long long nitem = item + gridDim.x;
-        ChunkLoc nloc{};
-        const int nh = static_cast<int>(nitem % H);
-        const bool nvalid = nitem < n_items && locate_chunk(cu_chunks, cu_seqlens, n_seqs, win_lo + nitem / H, nloc);
-        if (t == 0 && nvalid) {
-            issue_tile_loads<DV>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.tok0);
-            load_pending = true;
-        }
-
-        // ---------------- phase A: D[m, off_i + s] = RALL[m, :] . BVAR_i[s, :]  (M=128, N=16(i+1), K=128)
+        // ---------------- phase A: D[m, n] = RALL[m, :] . BVAR[n, :]  (M = 128, N = 160, K = 128); the
+        // columns of variant i (row tile i's key side) are [8 i (i+1), 8 (i+1)(i+2))
         if (t == 0) {
             tc_fence_after();
-            const uint32_t ra = smem_u32(sm + ps::RALL);
+            const uint32_t ra = smem_u32(sm + ps::RALL), bv = smem_u32(sm + ps::BVAR);
+            const uint32_t idesc = idesc_bf16(128, 160);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int nrow = 16 * (i + 1);
-                const uint32_t bv = smem_u32(sm + ps::BVAR + 2048 * i * (i + 1));
-                const uint32_t idesc = idesc_bf16(128, nrow);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
-                    umma_f16(tm + 8 * i * (i + 1), sdesc_k_sw128(ra + ka * 16384 + kb),
-                             sdesc_k_sw128(bv + ka * nrow * 128 + kb), idesc, ks > 0);
-                }
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
+                umma_f16(tm, sdesc_k_sw128(ra + ka * 16384 + kb), sdesc_k_sw128(bv + ka * 160 * 128 + kb), idesc, ks > 0);
             }
             umma_commit(&bar_mma);
         }
+        // prefetch the next item's tiles into the (now free) staging area; look one more item ahead
+        const long long nitem = item + gridDim.x;
+        const int nh = static_cast<int>(nitem % H);
+        const bool nvalid = nloc.y > 0;
+        if (t == 0 && nvalid) {
+            issue_tile_loads<DV>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.x);
+            load_pending = true;
+        }
+        const int2 nnloc = entry(nitem + gridDim.x);
         {
             const bool ok = mbar_wait(&bar_mma, ph_mma, status);
             if (__syncthreads_or(!ok)) break;
@@ -362,7 +330,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 float v[16];
                 if (cb < nv) {
                     tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + off + cb, v);
-                    tmem_wait_ld();
+                    tmem_wait_ld_regs<16>(v);
                 } else {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = 0.f;
@@ -381,7 +349,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int s = cb + j;
-                            AF[r * LDA + s] = s < r ? br * v[j] : 0.f;
+                            AT[s * LDT + r] = s < r ? br * v[j] : 0.f;
                         }
                     }
                 }
@@ -390,29 +358,64 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tc_fence_before();
         __syncthreads();
 
-        // ---------------- X = (I + A)^-1: diagonal 16x16 blocks, column held in registers (lane = column)
-        if (w < 4 && lane < 16) {
-            const int o0 = 16 * w, col = lane;
-            float x[16];
+        // ---------------- X = (I + A)^-1.  Diagonal 32x32 blocks by forward substitution, one warp per
+        // block, lane = column, the column held in registers; A^T rows come as float4 broadcasts.
+        if (w < 2) {
+            const int o0 = 32 * w, col = lane;
+            float x[32];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) x[r] = (r == col) ? 1.f : 0.f;
+            for (int r = 0; r < 32; ++r) x[r] = (r == col) ? 1.f : 0.f;
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
+            for (int m = 0; m < 31; ++m) {
                 const float xm = x[m];
+                const float4* arow = reinterpret_cast<const float4*>(AT + (o0 + m) * LDT + o0);
 #pragma unroll
-                for (int r = m + 1; r < 16; ++r) x[r] = fmaf(-AF[(o0 + r) * LDA + o0 + m], xm, x[r]);
+                for (int r4 = (m + 1) >> 2; r4 < 8; ++r4) {
+                    const float4 a = arow[r4];
+                    if (4 * r4 + 0 > m) x[4 * r4 + 0] = fmaf(-a.x, xm, x[4 * r4 + 0]);
+                    if (4 * r4 + 1 > m) x[4 * r4 + 1] = fmaf(-a.y, xm, x[4 * r4 + 1]);
+                    if (4 * r4 + 2 > m) x[4 * r4 + 2] = fmaf(-a.z, xm, x[4 * r4 + 2]);
+                    if (4 * r4 + 3 > m) x[4 * r4 + 3] = fmaf(-a.w, xm, x[4 * r4 + 3]);
+                }
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) XF[(o0 + r) * LDA + o0 + col] = x[r];
-        }
-        for (int e = t; e < 64 * 64; e += NT) {   // strictly upper blocks are zero
-            const int r = e >> 6, s = e & 63;
-            if ((s >> 4) > (r >> 4)) XF[r * LDA + s] = 0.f;
+            for (int r = 0; r < 32; ++r) XF[(o0 + r) * LDA + o0 + col] = x[r];
+        } else {
+            for (int e = t - 64; e < 32 * 32; e += NT - 64) XF[(e >> 5) * LDA + 32 + (e & 31)] = 0.f;   // X_01 = 0
         }
         __syncthreads();
-        solve_level<1>(AF, XF, TMP, t);
-        solve_level<2>(AF, XF, TMP, t);
-        solve_level<3>(AF, XF, TMP, t);
+        // off-diagonal block: X_10 = -X_11 (A_10 X_00).  Warp w owns rows 2w, 2w+1, lane = column;
+        // the A (and X_11) values are warp-wide broadcasts, the loop is unrolled with independent sums.
+        {
+            const int r0 = 2 * w, c = lane;
+            float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 32; m += 2) {
+                const float2 a0 = *reinterpret_cast<const float2*>(AT + m * LDT + 32 + r0);         // A[32+r0(+1)][m]
+                const float2 a1 = *reinterpret_cast<const float2*>(AT + (m + 1) * LDT + 32 + r0);
+                const float x0 = XF[m * LDA + c], x1 = XF[(m + 1) * LDA + c];                        // X_00[m][c]
+                s0 = fmaf(a0.x, x0, s0); s1 = fmaf(a0.y, x0, s1);
+                u0 = fmaf(a1.x, x1, u0); u1 = fmaf(a1.y, x1, u1);
+            }
+            TMP[r0 * 33 + c] = s0 + u0;
+            TMP[(r0 + 1) * 33 + c] = s1 + u1;
+        }
+        __syncthreads();
+        {
+            const int r0 = 2 * w, c = lane;
+            const float* x11a = XF + (32 + r0) * LDA + 32;   // X_11 rows r0, r0 + 1 (zero above the diagonal)
+            const float* x11b = x11a + LDA;
+            float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 32; m += 2) {
+                const float t0 = TMP[m * 33 + c], t1 = TMP[(m + 1) * 33 + c];
+                s0 = fmaf(x11a[m], t0, s0); s1 = fmaf(x11b[m], t0, s1);
+                u0 = fmaf(x11a[m + 1], t1, u0); u1 = fmaf(x11b[m + 1], t1, u1);
+            }
+            XF[(32 + r0) * LDA + c] = -(s0 + u0);
+            XF[(33 + r0) * LDA + c] = -(s1 + u1);
+        }
+        __syncthreads();
         // X^T as the bf16 B operand of the Y product: row m = column m of X, K = 64 rows of X
         {
             const int m = t >> 3, uc = t & 7;
@@ -445,7 +448,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const int m = 32 * qw + lane;
             float v[16];
             tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 16 * cg, v);
-            tmem_wait_ld();
+            tmem_wait_ld_regs<16>(v);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 float o8[8];
@@ -486,7 +489,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 for (int c16 = 4 * cg; c16 < 4 * cg + 4; ++c16) {
                     float v[16];
                     tmem_ld16(lane_base + 16 * c16, v);
-                    tmem_wait_ld();
+                    tmem_wait_ld_regs<16>(v);
 #pragma unroll
                     for (int sub = 0; sub < 2; ++sub) {
                         const int cc = 2 * c16 + sub;
@@ -510,17 +513,27 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 for (int c16 = 4 * (cg - 2); c16 < 4 * (cg - 2) + 4; ++c16) {
                     float v[16];
                     tmem_ld16(lane_base + 128 + 16 * c16, v);
-                    tmem_wait_ld();
+                    tmem_wait_ld_regs<16>(v);
 #pragma unroll
                     for (int sub = 0; sub < 2; ++sub) {
                         const int cc = 2 * c16 + sub;
                         float o8[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) o8[j] = v[8 * sub + j];
-                        const uint32_t dst = (m < 64 ? ps::US + m * 16 : ps::OIS + (m - 64) * 16) + cc * 1024;
+                        const int r = m & 63;
+                        const uint32_t dst = m < 64 ? ps::US + cc * 1024 + r * 16
+                                                    : ps::OIS + (cc >> 3) * 8192 + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
                         *reinterpret_cast<uint4*>(sm + dst) = pack8(o8);
                     }
                 }
+            }
+        }
+        {   // Kdec^T (held in registers since the column pass) into the B operand area phase B has released
+            const int c0 = 2 * (t & 63), q8 = t >> 6;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                const int c = c0 + ch;
+                *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + ((q8 ^ (c & 7)) << 4)) = kd_pk[ch];
             }
         }
         tc_fence_before();
@@ -528,14 +541,14 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         __syncthreads();
         if (t == 0) {
             bulk_s2g(pkt + P::AW, sm + ps::AWS, 32768);
+            bulk_s2g(pkt + P::KD, sm + ps::BKV, 16384);
             bulk_s2g(pkt + P::U, sm + ps::US, DV * 128);
             bulk_s2g(pkt + P::OI, sm + ps::OIS, DV * 128);
-            bulk_commit();
-            bulk_wait_read0();   // staging is overwritten by the next column pass
+            bulk_commit();   // the next column pass waits for the read-out before reusing the staging
         }
-        __syncthreads();
         item = nitem;
         loc = nloc;
+        nloc = nnloc;
         h = nh;
         valid = nvalid;
     }
@@ -557,7 +570,8 @@ struct SCfg {
     static constexpr int NT = 32 * (NEW + 2);              // + producer warp + MMA warp
     static constexpr bool MN = DVS >= 64;                  // S and U' staged MN-major (row = channel / token)
     static constexpr int NST = DVS == 128 ? 2 : 3;
-    static constexpr uint32_t AW = 0, KD = 32768, U = 49152, OI = U + DVS * 128, G = OI + DVS * 128;
+    static constexpr uint32_t OI_BYTES = DVS >= 64 ? DVS * 128 : 8192;   // whole 64-column blocks of O_intra
+    static constexpr uint32_t AW = 0, KD = 32768, U = 49152, OI = U + DVS * 128, G = OI + OI_BYTES;
     static constexpr uint32_t STAGE = ((G + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SOP = NST * STAGE;      // S as B operand (N = DVS, K = 128)
     static constexpr uint32_t UOP = SOP + DVS * 256;  // U' as B operand (N = DVS, K = 64)
@@ -572,6 +586,7 @@ __global__ void __launch_bounds__(SCfg<DV, DVS>::NT, 1)
 state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict__ cu_seqlens,
                   const int32_t* __restrict__ cu_chunks, int n_seqs, int H, long long win_lo, long long win_hi,
                   const float* __restrict__ initial_state, __nv_bfloat16* __restrict__ o,
+                  const __grid_constant__ CUtensorMap map_o,
                   float* __restrict__ final_state, float* __restrict__ final_transition, int ckpt_stride,
                   float* __restrict__ checkpoints, const int32_t* __restrict__ ckpt_cu, float* __restrict__ carry,
                   int* status) {
@@ -628,13 +643,13 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 if (!mbar_wait(&empty[st], ((ci / NST) & 1) ^ 1, status)) break;
                 const uint8_t* pk = packets + static_cast<size_t>((lo + ci - win_lo) * H + h) * P::BYTES;
                 uint8_t* sb = sm + st * C::STAGE;
-                const uint32_t bytes = 32768 + 16384 + 512 + (trans ? 0u : 2u * DVS * 128);
+                const uint32_t bytes = 32768 + 16384 + 512 + (trans ? 0u : DVS * 128 + C::OI_BYTES);
                 mbar_arrive_expect_tx(&full[st], bytes);
                 bulk_g2s(sb + C::AW, pk + P::AW, 32768, &full[st]);
                 bulk_g2s(sb + C::KD, pk + P::KD, 16384, &full[st]);
                 if (!trans) {
                     bulk_g2s(sb + C::U, pk + P::U + (j0 / 8) * 1024, DVS * 128, &full[st]);
-                    bulk_g2s(sb + C::OI, pk + P::OI + (j0 / 8) * 1024, DVS * 128, &full[st]);
+                    bulk_g2s(sb + C::OI, pk + P::OI + (j0 / 64) * 8192, C::OI_BYTES, &full[st]);
                 }
                 bulk_g2s(sb + C::G, pk + P::G, 512, &full[st]);
                 issued = ci + 1;
@@ -712,20 +727,26 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_ready);
+        // full chunks leave through a TMA tensor store of the O tile, written in place over O_intra
+        const bool o_warp = qw >= 2;
+        const bool o_issuer = (w == 2) && lane == 0;
         for (int ci = 0; ci < nch; ++ci) {
             const int st = ci % NST;
-            const uint8_t* sb = sm + st * C::STAGE;
+            uint8_t* sb = sm + st * C::STAGE;
             const int c = static_cast<int>(lo + ci - ch_lo);
             const long long rem = seq_len - static_cast<long long>(c) * 64;
             const int n = rem < 64 ? static_cast<int>(rem) : 64;
+            const bool full_tma = C::MN && !trans && n == 64;
             if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
             if (!mbar_wait(&d1_full, ci & 1, status)) break;
             tc_fence_after();
+            float vv[NCW];   // D1 row i, columns jw .. jw + NCW: all loads in flight, one wait
+#pragma unroll
+            for (int cb = 0; cb < NCW; cb += 16) tmem_ld16(lane_base + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+            tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
             for (int cb = 0; cb < NCW; cb += 16) {
-                float v[16];
-                tmem_ld16(lane_base + jw + cb, v);
-                tmem_wait_ld();
+                const float* v = vv + cb;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {
                     const int cc = (jw + cb) / 8 + sub;   // 8-column chunk within the slice
@@ -749,12 +770,16 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                         }
                     } else if (!trans && i - 64 < n) {
                         const int r = i - 64;
+                        const int col = j0 + 8 * cc;   // first column of this 8-column chunk
+                        uint8_t* ot = sb + C::OI + ((col >> 6) - (j0 >> 6)) * 8192 + r * 128 +
+                                      ((((col & 63) >> 3) ^ (r & 7)) << 4);
                         float o8[8];
-                        unpack8(*reinterpret_cast<const uint4*>(sb + C::OI + cc * 1024 + r * 16), o8);
+                        unpack8(*reinterpret_cast<const uint4*>(ot), o8);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) o8[e] += v[8 * sub + e];
-                        *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + j0 +
-                                                  8 * cc) = pack8(o8);
+                        if (full_tma) *reinterpret_cast<uint4*>(ot) = pack8(o8);
+                        else *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + col) =
+                                 pack8(o8);
                     }
                 }
             }
@@ -763,18 +788,29 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&up_ready);
+            } else if (full_tma) {
+                fence_proxy_async_smem();
+                named_bar_sync(1, 32 * NEW / 2);   // every O warp has written its rows of the tile
+                if (o_issuer) {
+#pragma unroll
+                    for (int b = 0; b < DVS / 64; ++b)
+                        tma_store_3d(&map_o, j0 + 64 * b, h, static_cast<int>(seq_tok0 + c * 64), sb + C::OI + b * 8192);
+                    bulk_commit();
+                }
             }
             if (!mbar_wait(&d2_full, ci & 1, status)) break;
             tc_fence_after();
             const float gam = *reinterpret_cast<const float*>(sb + C::G + i * 4);
+            {
+                float vv[NCW];
 #pragma unroll
-            for (int cb = 0; cb < NCW; cb += 16) {
-                float v[16];
-                tmem_ld16(lane_base + DVS + jw + cb, v);
-                tmem_wait_ld();
+                for (int cb = 0; cb < NCW; cb += 16)
+                    tmem_ld16(lane_base + DVS + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+                tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) S[cb + e] = fmaf(gam, S[cb + e], v[e]);
+                for (int e = 0; e < NCW; ++e) S[e] = fmaf(gam, S[e], vv[e]);
             }
+            if (o_issuer) bulk_wait_read0();   // the O tile has been read out of this stage
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);   // done with this stage's U, O_intra and gamma
             write_sop();
@@ -798,6 +834,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_ready);
         }
+        if (o_issuer) bulk_wait0();
 #pragma unroll
         for (int j = 0; j < NCW; ++j) {
             const int col = j0 + jw + j;
@@ -812,6 +849,17 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
     tc_fence_before();
     __syncthreads();
     if (w == 0) tmem_dealloc(tm, C::TMEM_COLS);
+}
+
+// Per window chunk: {first token, valid tokens} (n = 0 past the last chunk), so that the prep
+// kernel finds any item with one load instead of a search.
+__global__ void chunk_table_kernel(const int32_t* __restrict__ cu_chunks, const int32_t* __restrict__ cu_seqlens,
+                                   int n_seqs, long long win_lo, long long win_hi, int2* __restrict__ tab) {
+    const long long gc = win_lo + static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gc >= win_hi) return;
+    ChunkLoc loc;
+    tab[gc - win_lo] = locate_chunk(cu_chunks, cu_seqlens, n_seqs, gc, loc)
+                           ? make_int2(static_cast<int>(loc.tok0), loc.n) : make_int2(0, 0);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -831,7 +879,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 
 // 3D map over a [T, H, d] tensor (d innermost), box {box_d, 1, 64 tokens}, no swizzle.
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int d, int H, long long T,
-              int box_d) {
+              int box_d, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
     auto enc = get_encode();
     if (!enc) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
@@ -839,7 +887,7 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_d), 1u, 64u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -857,9 +905,14 @@ cudaError_t launch_state(const ChunkArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int slices = DV / DVS + (a.final_transition ? kDK / DVS : 0);
     dim3 grid(a.n_seqs * a.H, slices);
+    CUtensorMap mo;   // o [T, H, DV]: 64-column x 64-token boxes with the 128-byte swizzle
+    memset(&mo, 0, sizeof(mo));
+    if (a.total_tokens > 0 &&
+        !make_map(&mo, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, a.total_tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
     state_bf16_kernel<DV, DVS><<<grid, C::NT, smem, s>>>(
         static_cast<const uint8_t*>(a.packets), a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, a.win_hi,
-        a.initial_state, static_cast<__nv_bfloat16*>(a.o), a.final_state, a.final_transition, a.ckpt_stride,
+        a.initial_state, static_cast<__nv_bfloat16*>(a.o), mo, a.final_state, a.final_transition, a.ckpt_stride,
         a.checkpoints, a.ckpt_cu, a.carry, a.status);
     return cudaGetLastError();
 }
@@ -878,10 +931,14 @@ cudaError_t launch_bf16_t(const ChunkArgs& a, cudaStream_t s) {
         const int smem = static_cast<int>(ps::BYTES) + 1024;
         cudaError_t e = cudaFuncSetAttribute(prep_bf16_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
+        const long long wchunks = a.win_hi - a.win_lo;
+        chunk_table_kernel<<<static_cast<unsigned>((wchunks + 255) / 256), 256, 0, s>>>(
+            a.cu_chunks, a.cu_seqlens, a.n_seqs, a.win_lo, a.win_hi, a.chunk_tab);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
         const long long grid = items < num_sms() ? items : num_sms();
         prep_bf16_kernel<DV><<<static_cast<unsigned>(grid), ps::NT, smem, s>>>(
-            mq, mk, mv, ml, a.beta, a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, items,
-            static_cast<uint8_t*>(a.packets), a.status);
+            mq, mk, mv, ml, a.beta, a.chunk_tab, a.H, items, static_cast<uint8_t*>(a.packets), a.status);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

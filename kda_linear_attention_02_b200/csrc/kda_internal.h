@@ -42,6 +42,7 @@ struct ChunkArgs {
     float* final_transition;
     float* carry;               // [N,H,dk,dv+dk] fp32 state carried between windows (or null)
     void* packets;              // window of per-(chunk, head) packets
+    int2* chunk_tab;            // window of per-chunk {first token, valid tokens} (bf16 path)
     long long win_lo, win_hi;   // global chunk index window [lo, hi)
     bool multi_window;
     int* status;                // device status word

@@ -10,7 +10,7 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
                                                             const __nv_bfloat16* __restrict__ b,
                                                             float* __restrict__ d, int n, int b_mn, int* status) {
     extern __shared__ __align__(1024) uint8_t raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);   // stays a shared-memory pointer
     uint8_t* sA = base;                 // 128 rows x 128 B
     uint8_t* sB = base + 128 * 128;     // n rows x 128 B
     __shared__ __align__(8) uint64_t bar;
@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
         for (int c0 = 0; c0 < n; c0 += 16) {
             float r[16];
             tmem_ld16(tm + (static_cast<uint32_t>(32 * w) << 16) + c0, r);
-            tmem_wait_ld();
+            tmem_wait_ld_regs<16>(r);
             for (int j = 0; j < 16; ++j) d[(32 * w + lane) * n + c0 + j] = r[j];
         }
     }
