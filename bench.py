@@ -97,6 +97,26 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def captured_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary (profiles/traffic.txt), or None
+    when the kernel's sources changed since that capture (their SHA-256 no longer matches)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    srcs = [os.path.join(ROOT, "kda_linear_attention_02_b200", "csrc", f) for f in ("kda_chunk_bf16.cu", "kda_device.cuh")]
+    digest = hashlib.sha256()
+    for f in srcs:
+        with open(f, "rb") as fh:
+            digest.update(fh.read())
+    now = digest.hexdigest()[:16]
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 3 and not line.startswith("#") and parts[0] == kernel:
+            return int(parts[1]) if parts[2] == now else None
+    return None
+
+
 def dist_setup(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -222,13 +242,7 @@ def run_ours(args):
     ach = kernels[dom]["achieved_gbs"]
     whole_bytes = (PREFILL_READ_B + PREFILL_WRITE_B) * th
     whole_gbs = whole_bytes / (ms / 1e3) / 1e9
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get(dom)
-        except Exception:
-            traffic = None
+    traffic = captured_traffic(dom)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(ach / hbm, 4), "traffic": traffic, "peak_kind": peak_kind,
                 "alg_bytes_per_launch": kernels[dom]["alg_bytes"],
