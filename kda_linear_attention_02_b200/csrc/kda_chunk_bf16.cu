@@ -90,7 +90,7 @@ constexpr uint32_t BKV = 172032;     // [beta K gamma | beta V]^T: (128+DV) x 64
 constexpr uint32_t MISC = 204800;    // beta[64] fp32, half-tile totals [8][128] fp32
 constexpr uint32_t IAQ = 209920;     // [I; Aqk]: 128 x 64 bf16 (A operand of the Y product)
 // aliases of RALL/BVAR once phase A has completed
-constexpr uint32_t AT = 81920, XF = 99328, TMP = 116224, XT = 124928, XY = 133120;   // solve
+constexpr uint32_t AT = 81920, XF = 99328, TMP = 116224, AL = 120448, XT = 124928, XY = 133120;   // solve
 constexpr uint32_t AWS = 81920, US = 114688, OIS = 131072;                          // packet staging
 constexpr uint32_t BYTES = IAQ + 16384;
 constexpr int LDT = 68;              // fp32 row pitch of A^T (float4-aligned rows)
@@ -135,6 +135,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     float* AT = reinterpret_cast<float*>(sm + ps::AT);    // AT[s][r] = beta_r A[r][s]
     float* XF = reinterpret_cast<float*>(sm + ps::XF);
     float* TMP = reinterpret_cast<float*>(sm + ps::TMP);
+    float* AL = reinterpret_cast<float*>(sm + ps::AL);    // A rows 32..63, cols 0..31: [32][32], float4 chunks ^ (row % 8)
 
     if (t == 0) {
         mbar_init(&bar_load, 1);
@@ -223,56 +224,68 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 bx[i + 1] = bx[i] + tot[(2 * i) * 128 + c0] + tot[(2 * i + 1) * 128 + c0];
                 by[i + 1] = by[i] + tot[(2 * i) * 128 + c0 + 1] + tot[(2 * i + 1) * 128 + c0 + 1];
             }
-            const float ebx = __expf(bx[tq]), eby = __expf(by[tq]);                             // e^{b_t}
-            const float ftx = __expf(bx[tq + 1] - bx[tq]), fty = __expf(by[tq + 1] - by[tq]);   // e^{b_{t+1}-b_t}
-            const float ecx = __expf(bx[4] - bx[tq + 1]), ecy = __expf(by[4] - by[tq + 1]);     // e^{g_C-b_{t+1}}
+            // anchors of this thread's tile, selected with compile-time indices (no local-memory arrays)
+            float btx = 0.f, bty = 0.f, bnx = 0.f, bny = 0.f;   // b_t and b_{t+1}
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (i == tq) { btx = bx[i]; bty = by[i]; bnx = bx[i + 1]; bny = by[i + 1]; }
+            const float ebx = __expf(btx), eby = __expf(bty);                 // e^{b_t}
+            const float ftx = __expf(bnx - btx), fty = __expf(bny - bty);     // e^{b_{t+1}-b_t}
+            const float ecx = __expf(bx[4] - bnx), ecy = __expf(by[4] - bny); // e^{g_C-b_{t+1}}
             float dvx[4], dvy[4];   // e^{b_i - b_{t+1}}, i > t
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                dvx[i] = i > tq ? __expf(bx[i] - bx[tq + 1]) : 0.f;
-                dvy[i] = i > tq ? __expf(by[i] - by[tq + 1]) : 0.f;
+                dvx[i] = i > tq ? __expf(bx[i] - bnx) : 0.f;
+                dvy[i] = i > tq ? __expf(by[i] - bny) : 0.f;
             }
             if (q8 == 7)
                 *reinterpret_cast<float2*>(pkt + P::G + c0 * 4) = make_float2(__expf(bx[4]), __expf(by[4]));
 
+            // all shared-memory loads of the 8 tokens first (the stores below cannot then delay them)
+            uint32_t kb8[8], qb8[8], vb8[8];
+            float bt8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = 8 * q8 + j;
+                kb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
+                qb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
+                vb8[j] = c0 < DV ? *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 + r * 128 +
+                                                                       (c0 & 63) * 2)
+                                 : 0u;
+                bt8[j] = bet[r];
+            }
             float tk[2][8], tv[2][8], td[2][8];   // beta K gamma, beta V, Kdec along the 8 tokens
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int r = 8 * q8 + j;
-                const bool in = r < n;
-                const uint32_t kb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 +
-                                                                       r * 128 + (c0 & 63) * 2);
-                const uint32_t qb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 +
-                                                                       r * 128 + (c0 & 63) * 2);
-                const float2 kf = in ? bf2_to_f2(kb) : make_float2(0.f, 0.f);
-                const float2 qf = in ? bf2_to_f2(qb) : make_float2(0.f, 0.f);
-                float2 vf = make_float2(0.f, 0.f);
-                if (c0 < DV && in) {
-                    const uint32_t vb = *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 +
-                                                                           r * 128 + (c0 & 63) * 2);
-                    vf = bf2_to_f2(vb);
-                }
+                // rows past the sequence end (n <= r) keep whatever the tile holds: their log-decay and beta are
+                // zero, so they add nothing to A, W, U, Kdec^T U' or the state, and their own P / O_intra rows
+                // are never stored as outputs
+                const float2 kf = bf2_to_f2(kb8[j]);
+                const float2 qf = bf2_to_f2(qb8[j]);
+                const float2 vf = bf2_to_f2(vb8[j]);
                 const float Ex = __expf(p[j].x), Ey = __expf(p[j].y);     // e^{g_r - b_t} <= 1
                 const float Ix = __expf(-p[j].x), Iy = __expf(-p[j].y);   // e^{b_t - g_r} <= e^80.09
                 const float Fx = ftx * Ix, Fy = fty * Iy;                 // e^{b_{t+1} - g_r} <= 1
                 const float Gx = ebx * Ex, Gy = eby * Ey;                 // e^{g_r}
-                const float bt = bet[r];
+                const float bt = bt8[j];
                 // row side of A / Aqk
                 st_b32(sm + ps::RALL + sw128_offset(r, c0, 128), pack_bf16x2(kf.x * Ex, kf.y * Ey));
                 st_b32(sm + ps::RALL + sw128_offset(64 + r, c0, 128), pack_bf16x2(qf.x * Ex, qf.y * Ey));
                 // key side: own tile (diagonal) and the variants of later row tiles (variant i: rows 8 i (i+1) + r)
                 st_b32(sm + ps::BVAR + sw128_offset(8 * tq * (tq + 1) + r, c0, 160), pack_bf16x2(kf.x * Ix, kf.y * Iy));
+                const float kFx = kf.x * Fx, kFy = kf.y * Fy;
 #pragma unroll
                 for (int i = 1; i < 4; ++i)
                     if (i > tq)
                         st_b32(sm + ps::BVAR + sw128_offset(8 * i * (i + 1) + r, c0, 160),
-                               pack_bf16x2(kf.x * Fx * dvx[i], kf.y * Fy * dvy[i]));
+                               pack_bf16x2(kFx * dvx[i], kFy * dvy[i]));
                 // Q * gamma for the epilogue (P = Q gamma - ...)
                 st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2,
                        pack_bf16x2(qf.x * Gx, qf.y * Gy));
                 tk[0][j] = bt * kf.x * Gx; tk[1][j] = bt * kf.y * Gy;
                 tv[0][j] = bt * vf.x;      tv[1][j] = bt * vf.y;
-                td[0][j] = kf.x * ecx * Fx; td[1][j] = kf.y * ecy * Fy;
+                td[0][j] = kFx * ecx;      td[1][j] = kFy * ecy;
             }
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
@@ -326,15 +339,23 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const bool mine = (lane >> 4) == role;
             const float br = bet[r];
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) {
-                float v[16];
-                if (cb < nv) {
-                    tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + off + cb, v);
-                    tmem_wait_ld_regs<16>(v);
-                } else {
+            for (int cb2 = 0; cb2 < 64; cb2 += 32) {
+                float v2[32];   // two 16-column loads in flight per wait
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                for (int hb = 0; hb < 2; ++hb) {
+                    if (cb2 + 16 * hb < nv) {
+                        tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + off + cb2 + 16 * hb,
+                                  *reinterpret_cast<float(*)[16]>(v2 + 16 * hb));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v2[16 * hb + j] = 0.f;
+                    }
                 }
+                tmem_wait_ld_regs<32>(v2);
+#pragma unroll
+              for (int hb = 0; hb < 2; ++hb) {
+                const int cb = cb2 + 16 * hb;
+                const float* v = v2 + 16 * hb;
                 if (mine) {
                     if (is_q) {
                         float o8[8];
@@ -351,8 +372,16 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                             const int s = cb + j;
                             AT[s * LDT + r] = s < r ? br * v[j] : 0.f;
                         }
+                        if (r >= 32 && cb < 32) {   // the off-diagonal block A_10, row-contiguous for the solve
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int s = cb + j;
+                                AL[(r - 32) * 32 + 4 * ((s >> 2) ^ (r & 7)) + (s & 3)] = br * v[j];
+                            }
+                        }
                     }
                 }
+              }
             }
         }
         tc_fence_before();
@@ -365,18 +394,27 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             float x[32];
 #pragma unroll
             for (int r = 0; r < 32; ++r) x[r] = (r == col) ? 1.f : 0.f;
+            float4 cur[8], nxt[8];   // row m of A^T in registers while row m + 1 is loading
+#pragma unroll
+            for (int r4 = 0; r4 < 8; ++r4) cur[r4] = reinterpret_cast<const float4*>(AT + o0 * LDT + o0)[r4];
 #pragma unroll
             for (int m = 0; m < 31; ++m) {
+                if (m + 1 < 31) {
+#pragma unroll
+                    for (int r4 = (m + 2) >> 2; r4 < 8; ++r4)
+                        nxt[r4] = reinterpret_cast<const float4*>(AT + (o0 + m + 1) * LDT + o0)[r4];
+                }
                 const float xm = x[m];
-                const float4* arow = reinterpret_cast<const float4*>(AT + (o0 + m) * LDT + o0);
 #pragma unroll
                 for (int r4 = (m + 1) >> 2; r4 < 8; ++r4) {
-                    const float4 a = arow[r4];
+                    const float4 a = cur[r4];
                     if (4 * r4 + 0 > m) x[4 * r4 + 0] = fmaf(-a.x, xm, x[4 * r4 + 0]);
                     if (4 * r4 + 1 > m) x[4 * r4 + 1] = fmaf(-a.y, xm, x[4 * r4 + 1]);
                     if (4 * r4 + 2 > m) x[4 * r4 + 2] = fmaf(-a.z, xm, x[4 * r4 + 2]);
                     if (4 * r4 + 3 > m) x[4 * r4 + 3] = fmaf(-a.w, xm, x[4 * r4 + 3]);
                 }
+#pragma unroll
+                for (int r4 = 0; r4 < 8; ++r4) cur[r4] = nxt[r4];
             }
 #pragma unroll
             for (int r = 0; r < 32; ++r) XF[(o0 + r) * LDA + o0 + col] = x[r];
@@ -384,36 +422,54 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             for (int e = t - 64; e < 32 * 32; e += NT - 64) XF[(e >> 5) * LDA + 32 + (e & 31)] = 0.f;   // X_01 = 0
         }
         __syncthreads();
-        // off-diagonal block: X_10 = -X_11 (A_10 X_00).  Warp w owns rows 2w, 2w+1, lane = column;
-        // the A (and X_11) values are warp-wide broadcasts, the loop is unrolled with independent sums.
+        // off-diagonal block: X_10 = -X_11 (A_10 X_00).  Warp w owns rows 2w, 2w+1, lane = column; every
+        // operand of a row is loaded into registers before its 32 FMAs.
         {
-            const int r0 = 2 * w, c = lane;
-            float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
+            const int c = lane;
+            float xc[32];
 #pragma unroll
-            for (int m = 0; m < 32; m += 2) {
-                const float2 a0 = *reinterpret_cast<const float2*>(AT + m * LDT + 32 + r0);         // A[32+r0(+1)][m]
-                const float2 a1 = *reinterpret_cast<const float2*>(AT + (m + 1) * LDT + 32 + r0);
-                const float x0 = XF[m * LDA + c], x1 = XF[(m + 1) * LDA + c];                        // X_00[m][c]
-                s0 = fmaf(a0.x, x0, s0); s1 = fmaf(a0.y, x0, s1);
-                u0 = fmaf(a1.x, x1, u0); u1 = fmaf(a1.y, x1, u1);
+            for (int m = 0; m < 32; ++m) xc[m] = XF[m * LDA + c];   // X_00[:, c]
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r0 = 2 * w + rr;
+                float4 a4[8];
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4)
+                    a4[c4] = reinterpret_cast<const float4*>(AL + r0 * 32)[c4 ^ (r0 & 7)];   // A[32 + r0][4 c4 ..]
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    s0 = fmaf(a4[c4].x, xc[4 * c4 + 0], s0);
+                    s1 = fmaf(a4[c4].y, xc[4 * c4 + 1], s1);
+                    s2 = fmaf(a4[c4].z, xc[4 * c4 + 2], s2);
+                    s3 = fmaf(a4[c4].w, xc[4 * c4 + 3], s3);
+                }
+                TMP[r0 * 33 + c] = (s0 + s1) + (s2 + s3);
             }
-            TMP[r0 * 33 + c] = s0 + u0;
-            TMP[(r0 + 1) * 33 + c] = s1 + u1;
         }
         __syncthreads();
         {
-            const int r0 = 2 * w, c = lane;
-            const float* x11a = XF + (32 + r0) * LDA + 32;   // X_11 rows r0, r0 + 1 (zero above the diagonal)
-            const float* x11b = x11a + LDA;
-            float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
+            const int c = lane;
+            float tc[32];
 #pragma unroll
-            for (int m = 0; m < 32; m += 2) {
-                const float t0 = TMP[m * 33 + c], t1 = TMP[(m + 1) * 33 + c];
-                s0 = fmaf(x11a[m], t0, s0); s1 = fmaf(x11b[m], t0, s1);
-                u0 = fmaf(x11a[m + 1], t1, u0); u1 = fmaf(x11b[m + 1], t1, u1);
+            for (int m = 0; m < 32; ++m) tc[m] = TMP[m * 33 + c];   // T[:, c]
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r0 = 2 * w + rr;
+                const float* x11 = XF + (32 + r0) * LDA + 32;   // X_11 row r0 (zero above the diagonal)
+                float xr[32];
+#pragma unroll
+                for (int m = 0; m < 32; ++m) xr[m] = x11[m];
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 32; m += 4) {
+                    s0 = fmaf(xr[m], tc[m], s0);
+                    s1 = fmaf(xr[m + 1], tc[m + 1], s1);
+                    s2 = fmaf(xr[m + 2], tc[m + 2], s2);
+                    s3 = fmaf(xr[m + 3], tc[m + 3], s3);
+                }
+                XF[(32 + r0) * LDA + c] = -((s0 + s1) + (s2 + s3));
             }
-            XF[(32 + r0) * LDA + c] = -(s0 + u0);
-            XF[(33 + r0) * LDA + c] = -(s1 + u1);
         }
         __syncthreads();
         // X^T as the bf16 B operand of the Y product: row m = column m of X, K = 64 rows of X
@@ -486,13 +542,15 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
             if (cg < 2) {
 #pragma unroll 1
-                for (int c16 = 4 * cg; c16 < 4 * cg + 4; ++c16) {
-                    float v[16];
-                    tmem_ld16(lane_base + 16 * c16, v);
-                    tmem_wait_ld_regs<16>(v);
+                for (int c32 = 2 * cg; c32 < 2 * cg + 2; ++c32) {
+                    float vv[32];
+                    tmem_ld16(lane_base + 32 * c32, *reinterpret_cast<float(*)[16]>(vv));
+                    tmem_ld16(lane_base + 32 * c32 + 16, *reinterpret_cast<float(*)[16]>(vv + 16));
+                    tmem_wait_ld_regs<32>(vv);
 #pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
-                        const int cc = 2 * c16 + sub;
+                    for (int sub = 0; sub < 4; ++sub) {
+                        const int cc = 4 * c32 + sub;
+                        const float* v = vv;
                         float o8[8];
                         if (m < 64) {
 #pragma unroll
@@ -510,13 +568,15 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 }
             } else if (64 * (cg - 2) < DV) {
 #pragma unroll 1
-                for (int c16 = 4 * (cg - 2); c16 < 4 * (cg - 2) + 4; ++c16) {
-                    float v[16];
-                    tmem_ld16(lane_base + 128 + 16 * c16, v);
-                    tmem_wait_ld_regs<16>(v);
+                for (int c32 = 2 * (cg - 2); c32 < 2 * (cg - 2) + 2; ++c32) {
+                    float vv[32];
+                    tmem_ld16(lane_base + 128 + 32 * c32, *reinterpret_cast<float(*)[16]>(vv));
+                    tmem_ld16(lane_base + 128 + 32 * c32 + 16, *reinterpret_cast<float(*)[16]>(vv + 16));
+                    tmem_wait_ld_regs<32>(vv);
 #pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
-                        const int cc = 2 * c16 + sub;
+                    for (int sub = 0; sub < 4; ++sub) {
+                        const int cc = 4 * c32 + sub;
+                        const float* v = vv;
                         float o8[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) o8[j] = v[8 * sub + j];
