@@ -90,11 +90,13 @@ constexpr uint32_t BKV = 172032;     // [beta K gamma | beta V]^T: (128+DV) x 64
 constexpr uint32_t MISC = 204800;    // beta[64] fp32, half-tile totals [8][128] fp32
 constexpr uint32_t IAQ = 209920;     // [I; Aqk]: 128 x 64 bf16 (A operand of the Y product)
 // aliases of RALL/BVAR once phase A has completed
-constexpr uint32_t AT = 81920, XF = 99328, TMP = 116224, AL = 120448, XT = 124928, XY = 133120;   // solve
-constexpr uint32_t AWS = 81920, US = 114688, OIS = 131072;                          // packet staging
+constexpr uint32_t AM = 81920, XF = 99328, TT = 118016, XT = 124928, XY = 133120;   // solve
+constexpr uint32_t AWS = 81920, US = 114688, OIS = 131072;                       // packet staging
 constexpr uint32_t BYTES = IAQ + 16384;
-constexpr int LDT = 68;              // fp32 row pitch of A^T (float4-aligned rows)
-constexpr int LDA = 65;              // fp32 row pitch of X
+constexpr int LDM = 68;              // fp32 row pitch of AM (float4-aligned rows; 4 rows apart = 16 banks)
+constexpr int LDX = 73;              // fp32 row pitch of X (odd: column reads of X^T spread over the banks)
+constexpr int LDTT = 40;             // fp32 row pitch of the product scratch (8 banks per row: B fragments clash-free)
+static_assert(XF + 64 * LDX * 4 <= TT && TT + 32 * LDTT * 4 <= XT && AM + 64 * LDM * 4 <= XF, "solve map");
 constexpr int NT = 512;              // threads per CTA
 }  // namespace ps
 
@@ -123,8 +125,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  uint8_t* __restrict__ packets, int* status) {
     using P = Pk<DV>;
     constexpr int NT = ps::NT;
-    constexpr int LDA = ps::LDA;
-    constexpr int LDT = ps::LDT;
+    constexpr int LDM = ps::LDM;
+    constexpr int LDX = ps::LDX;
+    constexpr int LDTT = ps::LDTT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     __shared__ __align__(8) uint64_t bar_load, bar_mma;
@@ -132,10 +135,12 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     float* bet = reinterpret_cast<float*>(sm + ps::MISC);
     float* tot = bet + 64;   // [8 half-tiles][128 channels]
-    float* AT = reinterpret_cast<float*>(sm + ps::AT);    // AT[s][r] = beta_r A[r][s]
-    float* XF = reinterpret_cast<float*>(sm + ps::XF);
-    float* TMP = reinterpret_cast<float*>(sm + ps::TMP);
-    float* AL = reinterpret_cast<float*>(sm + ps::AL);    // A rows 32..63, cols 0..31: [32][32], float4 chunks ^ (row % 8)
+    // AM holds the strictly lower A = beta_r (K e^g)_r . (K e^-g)_s in two forms that never overlap: the
+    // off-diagonal 16 x 16 blocks row-major (AM[r][s], tile(s) < tile(r)), and each diagonal block
+    // transposed into its upper triangle (AM[s][r] for s < r in the same tile)
+    float* AM = reinterpret_cast<float*>(sm + ps::AM);
+    float* XF = reinterpret_cast<float*>(sm + ps::XF);    // X = (I + A)^-1, fp32, pitch LDX
+    float* TT = reinterpret_cast<float*>(sm + ps::TT);    // T = A_10 X_00 of a merge, pitch LDTT
 
     if (t == 0) {
         mbar_init(&bar_load, 1);
@@ -366,19 +371,17 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                             const int sc = (cb >> 3) + hf;
                             *reinterpret_cast<uint4*>(sm + ps::IAQ + (64 + r) * 128 + ((sc ^ (r & 7)) << 4)) = pack8(o8);
                         }
-                    } else {
+                    } else if ((cb >> 4) == (r >> 4)) {   // diagonal block: transposed, strict lower part only
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int s = cb + j;
-                            AT[s * LDT + r] = s < r ? br * v[j] : 0.f;
+                            if (s < r) AM[s * LDM + r] = br * v[j];
                         }
-                        if (r >= 32 && cb < 32) {   // the off-diagonal block A_10, row-contiguous for the solve
+                    } else if ((cb >> 4) < (r >> 4)) {    // off-diagonal block: row-major
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int s = cb + j;
-                                AL[(r - 32) * 32 + 4 * ((s >> 2) ^ (r & 7)) + (s & 3)] = br * v[j];
-                            }
-                        }
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            reinterpret_cast<float4*>(AM + r * LDM + cb)[q4] =
+                                make_float4(br * v[4 * q4], br * v[4 * q4 + 1], br * v[4 * q4 + 2], br * v[4 * q4 + 3]);
                     }
                 }
               }
@@ -387,26 +390,27 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tc_fence_before();
         __syncthreads();
 
-        // ---------------- X = (I + A)^-1.  Diagonal 32x32 blocks by forward substitution, one warp per
-        // block, lane = column, the column held in registers; A^T rows come as float4 broadcasts.
-        if (w < 2) {
-            const int o0 = 32 * w, col = lane;
-            float x[32];
+        // ---------------- X = (I + A)^-1 by blocked forward substitution over 16 x 16 tiles.
+        // Level 0: each diagonal block by forward substitution, one warp per block, lane = column, the
+        // column held in registers; a column of A comes as float4 broadcasts of a row of the transposed block.
+        if (w < 4) {
+            const int o0 = 16 * w, col = lane & 15;
+            float x[16];
 #pragma unroll
-            for (int r = 0; r < 32; ++r) x[r] = (r == col) ? 1.f : 0.f;
-            float4 cur[8], nxt[8];   // row m of A^T in registers while row m + 1 is loading
+            for (int r = 0; r < 16; ++r) x[r] = (r == col) ? 1.f : 0.f;
+            float4 cur[4], nxt[4];
 #pragma unroll
-            for (int r4 = 0; r4 < 8; ++r4) cur[r4] = reinterpret_cast<const float4*>(AT + o0 * LDT + o0)[r4];
+            for (int r4 = 0; r4 < 4; ++r4) cur[r4] = reinterpret_cast<const float4*>(AM + o0 * LDM + o0)[r4];
 #pragma unroll
-            for (int m = 0; m < 31; ++m) {
-                if (m + 1 < 31) {
+            for (int m = 0; m < 15; ++m) {
+                if (m + 1 < 15) {
 #pragma unroll
-                    for (int r4 = (m + 2) >> 2; r4 < 8; ++r4)
-                        nxt[r4] = reinterpret_cast<const float4*>(AT + (o0 + m + 1) * LDT + o0)[r4];
+                    for (int r4 = (m + 2) >> 2; r4 < 4; ++r4)
+                        nxt[r4] = reinterpret_cast<const float4*>(AM + (o0 + m + 1) * LDM + o0)[r4];
                 }
                 const float xm = x[m];
 #pragma unroll
-                for (int r4 = (m + 1) >> 2; r4 < 8; ++r4) {
+                for (int r4 = (m + 1) >> 2; r4 < 4; ++r4) {
                     const float4 a = cur[r4];
                     if (4 * r4 + 0 > m) x[4 * r4 + 0] = fmaf(-a.x, xm, x[4 * r4 + 0]);
                     if (4 * r4 + 1 > m) x[4 * r4 + 1] = fmaf(-a.y, xm, x[4 * r4 + 1]);
@@ -414,62 +418,94 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     if (4 * r4 + 3 > m) x[4 * r4 + 3] = fmaf(-a.w, xm, x[4 * r4 + 3]);
                 }
 #pragma unroll
-                for (int r4 = 0; r4 < 8; ++r4) cur[r4] = nxt[r4];
+                for (int r4 = 0; r4 < 4; ++r4) cur[r4] = nxt[r4];
             }
+            if (lane < 16) {
 #pragma unroll
-            for (int r = 0; r < 32; ++r) XF[(o0 + r) * LDA + o0 + col] = x[r];
+                for (int r = 0; r < 16; ++r) XF[(o0 + r) * LDX + o0 + col] = x[r];
+            }
         } else {
-            for (int e = t - 64; e < 32 * 32; e += NT - 64) XF[(e >> 5) * LDA + 32 + (e & 31)] = 0.f;   // X_01 = 0
-        }
-        __syncthreads();
-        // off-diagonal block: X_10 = -X_11 (A_10 X_00).  Warp w owns rows 2w, 2w+1, lane = column; every
-        // operand of a row is loaded into registers before its 32 FMAs.
-        {
-            const int c = lane;
-            float xc[32];
-#pragma unroll
-            for (int m = 0; m < 32; ++m) xc[m] = XF[m * LDA + c];   // X_00[:, c]
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int r0 = 2 * w + rr;
-                float4 a4[8];
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4)
-                    a4[c4] = reinterpret_cast<const float4*>(AL + r0 * 32)[c4 ^ (r0 & 7)];   // A[32 + r0][4 c4 ..]
-                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    s0 = fmaf(a4[c4].x, xc[4 * c4 + 0], s0);
-                    s1 = fmaf(a4[c4].y, xc[4 * c4 + 1], s1);
-                    s2 = fmaf(a4[c4].z, xc[4 * c4 + 2], s2);
-                    s3 = fmaf(a4[c4].w, xc[4 * c4 + 3], s3);
-                }
-                TMP[r0 * 33 + c] = (s0 + s1) + (s2 + s3);
+            for (int e = t - 128; e < 64 * 64; e += NT - 128) {   // the blocks above the diagonal are zero
+                const int r = e >> 6, c = e & 63;
+                if ((c >> 4) > (r >> 4)) XF[r * LDX + c] = 0.f;
             }
         }
         __syncthreads();
-        {
-            const int c = lane;
-            float tc[32];
+        // Levels 1 and 2 merge two inverted diagonal blocks: X_10 = -X_11 (A_10 X_00).  The products are
+        // 16- and 32-row tiles, below the tensor-core MMA's smallest M, so they run as warp-level tf32
+        // m16n8k8 MMAs with fp32 accumulation on fragments loaded straight from shared memory.
+        const int fg = lane >> 2, ft = lane & 3;   // fragment row group and column pair of this lane
+        if (w < 4) {   // level 1: 16 -> 32, pair p (rows 32 p + 16 .., cols 32 p ..), column tile nt of 8
+            const int p = w >> 1, nt = w & 1, rb = 32 * p + 16, c0 = 32 * p;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int m = 0; m < 32; ++m) tc[m] = TMP[m * 33 + c];   // T[:, c]
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int r0 = 2 * w + rr;
-                const float* x11 = XF + (32 + r0) * LDA + 32;   // X_11 row r0 (zero above the diagonal)
-                float xr[32];
-#pragma unroll
-                for (int m = 0; m < 32; ++m) xr[m] = x11[m];
-                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-                for (int m = 0; m < 32; m += 4) {
-                    s0 = fmaf(xr[m], tc[m], s0);
-                    s1 = fmaf(xr[m + 1], tc[m + 1], s1);
-                    s2 = fmaf(xr[m + 2], tc[m + 2], s2);
-                    s3 = fmaf(xr[m + 3], tc[m + 3], s3);
-                }
-                XF[(32 + r0) * LDA + c] = -((s0 + s1) + (s2 + s3));
+            for (int ks = 0; ks < 2; ++ks) {
+                if (ks < nt) continue;   // X_00 is zero above its diagonal
+                const uint32_t a[4] = {to_tf32(AM[(rb + fg) * LDM + c0 + 8 * ks + ft]),
+                                       to_tf32(AM[(rb + fg + 8) * LDM + c0 + 8 * ks + ft]),
+                                       to_tf32(AM[(rb + fg) * LDM + c0 + 8 * ks + ft + 4]),
+                                       to_tf32(AM[(rb + fg + 8) * LDM + c0 + 8 * ks + ft + 4])};
+                const uint32_t b[2] = {to_tf32(XF[(c0 + 8 * ks + ft) * LDX + c0 + 8 * nt + fg]),
+                                       to_tf32(XF[(c0 + 8 * ks + ft + 4) * LDX + c0 + 8 * nt + fg])};
+                mma_tf32(d, a, b);
             }
+            float* tt = TT + 16 * p * LDTT + 8 * nt;
+            *reinterpret_cast<float2*>(tt + fg * LDTT + 2 * ft) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(tt + (fg + 8) * LDTT + 2 * ft) = make_float2(d[2], d[3]);
+            __syncwarp();
+            float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                const uint32_t a[4] = {to_tf32(XF[(rb + fg) * LDX + rb + 8 * ks + ft]),
+                                       to_tf32(XF[(rb + fg + 8) * LDX + rb + 8 * ks + ft]),
+                                       to_tf32(XF[(rb + fg) * LDX + rb + 8 * ks + ft + 4]),
+                                       to_tf32(XF[(rb + fg + 8) * LDX + rb + 8 * ks + ft + 4])};
+                const uint32_t b[2] = {to_tf32(tt[(8 * ks + ft) * LDTT + fg]), to_tf32(tt[(8 * ks + ft + 4) * LDTT + fg])};
+                mma_tf32(e, a, b);
+            }
+            float* xo = XF + rb * LDX + c0 + 8 * nt + 2 * ft;
+            xo[fg * LDX] = -e[0];
+            xo[fg * LDX + 1] = -e[1];
+            xo[(fg + 8) * LDX] = -e[2];
+            xo[(fg + 8) * LDX + 1] = -e[3];
+        }
+        __syncthreads();
+        if (w < 8) {   // level 2: 32 -> 64, row tile mt of 16 and column tile nt of 8
+            const int nt = w & 3, mt = w >> 2;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                if (ks < nt) continue;   // X_00 is zero above its diagonal
+                const int ra = 32 + 16 * mt + fg;
+                const uint32_t a[4] = {to_tf32(AM[ra * LDM + 8 * ks + ft]), to_tf32(AM[(ra + 8) * LDM + 8 * ks + ft]),
+                                       to_tf32(AM[ra * LDM + 8 * ks + ft + 4]),
+                                       to_tf32(AM[(ra + 8) * LDM + 8 * ks + ft + 4])};
+                const uint32_t b[2] = {to_tf32(XF[(8 * ks + ft) * LDX + 8 * nt + fg]),
+                                       to_tf32(XF[(8 * ks + ft + 4) * LDX + 8 * nt + fg])};
+                mma_tf32(d, a, b);
+            }
+            float* tt = TT + 16 * mt * LDTT + 8 * nt;
+            *reinterpret_cast<float2*>(tt + fg * LDTT + 2 * ft) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(tt + (fg + 8) * LDTT + 2 * ft) = make_float2(d[2], d[3]);
+            named_bar_sync(1 + nt, 64);   // the two row tiles of this column tile of T are written
+            float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                if (ks >= 2 * (mt + 1)) continue;   // X_11 is zero above its diagonal
+                const int ra = 32 + 16 * mt + fg;
+                const uint32_t a[4] = {to_tf32(XF[ra * LDX + 32 + 8 * ks + ft]),
+                                       to_tf32(XF[(ra + 8) * LDX + 32 + 8 * ks + ft]),
+                                       to_tf32(XF[ra * LDX + 32 + 8 * ks + ft + 4]),
+                                       to_tf32(XF[(ra + 8) * LDX + 32 + 8 * ks + ft + 4])};
+                const uint32_t b[2] = {to_tf32(TT[(8 * ks + ft) * LDTT + 8 * nt + fg]),
+                                       to_tf32(TT[(8 * ks + ft + 4) * LDTT + 8 * nt + fg])};
+                mma_tf32(e, a, b);
+            }
+            float* xo = XF + (32 + 16 * mt) * LDX + 8 * nt + 2 * ft;
+            xo[fg * LDX] = -e[0];
+            xo[fg * LDX + 1] = -e[1];
+            xo[(fg + 8) * LDX] = -e[2];
+            xo[(fg + 8) * LDX + 1] = -e[3];
         }
         __syncthreads();
         // X^T as the bf16 B operand of the Y product: row m = column m of X, K = 64 rows of X
@@ -477,7 +513,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const int m = t >> 3, uc = t & 7;
             float v[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = XF[(8 * uc + j) * LDA + m];
+            for (int j = 0; j < 8; ++j) v[j] = XF[(8 * uc + j) * LDX + m];
             *reinterpret_cast<uint4*>(sm + ps::XT + m * 128 + ((uc ^ (m & 7)) << 4)) = pack8(v);
         }
         fence_proxy_async_smem();
