@@ -60,6 +60,15 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
     const float2 a = bf2_to_f2(u.x), b = bf2_to_f2(u.y), c = bf2_to_f2(u.z), d = bf2_to_f2(u.w);
     f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
 }
+__device__ __forceinline__ uint32_t pack2(float2 f) { return pack_bf16x2(f.x, f.y); }
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+// 2^x by the ex2.approx instruction; e^x is taken as 2^(x log2 e) with the scaling done two lanes at a time
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                       pack_bf16x2(f[6], f[7]));
@@ -206,28 +215,37 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 const int r = 8 * q8 + j;
                 const float2 la =
                     *reinterpret_cast<const float2*>(sm + ps::STG_L + (c0 >> 5) * 8192 + r * 128 + (c0 & 31) * 4);
-                if (r < n) {
-                    acc.x += floor_log_decay(la.x);
-                    acc.y += floor_log_decay(la.y);
-                }
+                if (r < n) acc = __fadd2_rn(acc, make_float2(floor_log_decay(la.x), floor_log_decay(la.y)));
                 p[j] = acc;
             }
-            tot[q8 * 128 + c0] = acc.x;
-            tot[q8 * 128 + c0 + 1] = acc.y;
+            *reinterpret_cast<float2*>(tot + q8 * 128 + c0) = acc;
+            // the 8 tokens' inputs, loaded before the barrier (the staging tiles are not part of the packet)
+            uint32_t kb8[8], qb8[8], vb8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = 8 * q8 + j;
+                kb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
+                qb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
+                vb8[j] = c0 < DV ? *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 + r * 128 +
+                                                                       (c0 & 63) * 2)
+                                 : 0u;
+            }
             if (t == 0) bulk_wait_read0();   // the previous item's packet staging has been read out
             __syncthreads();
             if (hh) {   // second half of the tile: add the first half's total
-                const float ox = tot[(q8 - 1) * 128 + c0], oy = tot[(q8 - 1) * 128 + c0 + 1];
+                const float2 ob = *reinterpret_cast<const float2*>(tot + (q8 - 1) * 128 + c0);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) { p[j].x += ox; p[j].y += oy; }
+                for (int j = 0; j < 8; ++j) { p[j].x += ob.x; p[j].y += ob.y; }
             }
             // p[j] = g_r - b_tq: the log-decay inside the tile up to r
             float bx[5], by[5];
             bx[0] = 0.f; by[0] = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                bx[i + 1] = bx[i] + tot[(2 * i) * 128 + c0] + tot[(2 * i + 1) * 128 + c0];
-                by[i + 1] = by[i] + tot[(2 * i) * 128 + c0 + 1] + tot[(2 * i + 1) * 128 + c0 + 1];
+                const float2 t0 = *reinterpret_cast<const float2*>(tot + (2 * i) * 128 + c0);
+                const float2 t1 = *reinterpret_cast<const float2*>(tot + (2 * i + 1) * 128 + c0);
+                bx[i + 1] = bx[i] + t0.x + t1.x;
+                by[i + 1] = by[i] + t0.y + t1.y;
             }
             // anchors of this thread's tile, selected with compile-time indices (no local-memory arrays)
             float btx = 0.f, bty = 0.f, bnx = 0.f, bny = 0.f;   // b_t and b_{t+1}
@@ -245,21 +263,12 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
             if (q8 == 7)
                 *reinterpret_cast<float2*>(pkt + P::G + c0 * 4) = make_float2(__expf(bx[4]), __expf(by[4]));
-
-            // all shared-memory loads of the 8 tokens first (the stores below cannot then delay them)
-            uint32_t kb8[8], qb8[8], vb8[8];
             float bt8[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = 8 * q8 + j;
-                kb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
-                qb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
-                vb8[j] = c0 < DV ? *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 + r * 128 +
-                                                                       (c0 & 63) * 2)
-                                 : 0u;
-                bt8[j] = bet[r];
-            }
+            for (int j = 0; j < 8; ++j) bt8[j] = bet[8 * q8 + j];
+
             float tk[2][8], tv[2][8], td[2][8];   // beta K gamma, beta V, Kdec along the 8 tokens
+            const float2 ft2 = make_float2(ftx, fty), eb2 = make_float2(ebx, eby), ec2 = make_float2(ecx, ecy);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int r = 8 * q8 + j;
@@ -269,37 +278,48 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 const float2 kf = bf2_to_f2(kb8[j]);
                 const float2 qf = bf2_to_f2(qb8[j]);
                 const float2 vf = bf2_to_f2(vb8[j]);
-                const float Ex = __expf(p[j].x), Ey = __expf(p[j].y);     // e^{g_r - b_t} <= 1
-                const float Ix = __expf(-p[j].x), Iy = __expf(-p[j].y);   // e^{b_t - g_r} <= e^80.09
-                const float Fx = ftx * Ix, Fy = fty * Iy;                 // e^{b_{t+1} - g_r} <= 1
-                const float Gx = ebx * Ex, Gy = eby * Ey;                 // e^{g_r}
-                const float bt = bt8[j];
+                const float2 pl = __fmul2_rn(p[j], f2(kLog2e));
+                const float2 E = make_float2(ex2_approx(pl.x), ex2_approx(pl.y));     // e^{g_r - b_t} <= 1
+                const float2 I = make_float2(ex2_approx(-pl.x), ex2_approx(-pl.y));   // e^{b_t - g_r} <= e^80.09
+                const float2 F = __fmul2_rn(ft2, I);                                  // e^{b_{t+1} - g_r} <= 1
+                const float2 G = __fmul2_rn(eb2, E);                                  // e^{g_r}
+                const float2 bt = f2(bt8[j]);
                 // row side of A / Aqk
-                st_b32(sm + ps::RALL + sw128_offset(r, c0, 128), pack_bf16x2(kf.x * Ex, kf.y * Ey));
-                st_b32(sm + ps::RALL + sw128_offset(64 + r, c0, 128), pack_bf16x2(qf.x * Ex, qf.y * Ey));
+                st_b32(sm + ps::RALL + sw128_offset(r, c0, 128), pack2(__fmul2_rn(kf, E)));
+                st_b32(sm + ps::RALL + sw128_offset(64 + r, c0, 128), pack2(__fmul2_rn(qf, E)));
                 // key side: own tile (diagonal) and the variants of later row tiles (variant i: rows 8 i (i+1) + r)
-                st_b32(sm + ps::BVAR + sw128_offset(8 * tq * (tq + 1) + r, c0, 160), pack_bf16x2(kf.x * Ix, kf.y * Iy));
-                const float kFx = kf.x * Fx, kFy = kf.y * Fy;
+                st_b32(sm + ps::BVAR + sw128_offset(8 * tq * (tq + 1) + r, c0, 160), pack2(__fmul2_rn(kf, I)));
+                const float2 kF = __fmul2_rn(kf, F);
 #pragma unroll
                 for (int i = 1; i < 4; ++i)
                     if (i > tq)
                         st_b32(sm + ps::BVAR + sw128_offset(8 * i * (i + 1) + r, c0, 160),
-                               pack_bf16x2(kFx * dvx[i], kFy * dvy[i]));
+                               pack2(__fmul2_rn(kF, make_float2(dvx[i], dvy[i]))));
                 // Q * gamma for the epilogue (P = Q gamma - ...)
-                st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2,
-                       pack_bf16x2(qf.x * Gx, qf.y * Gy));
-                tk[0][j] = bt * kf.x * Gx; tk[1][j] = bt * kf.y * Gy;
-                tv[0][j] = bt * vf.x;      tv[1][j] = bt * vf.y;
-                td[0][j] = kFx * ecx;      td[1][j] = kFy * ecy;
+                st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2, pack2(__fmul2_rn(qf, G)));
+                const float2 tk2 = __fmul2_rn(__fmul2_rn(bt, kf), G);
+                const float2 tv2 = __fmul2_rn(bt, vf);
+                const float2 td2 = __fmul2_rn(kF, ec2);
+                tk[0][j] = tk2.x; tk[1][j] = tk2.y;
+                tv[0][j] = tv2.x; tv[1][j] = tv2.y;
+                td[0][j] = td2.x; td[1][j] = td2.y;
             }
+            // rows c of the transposed operands: lanes 4..7 of each quarter warp take their odd channel first,
+            // so that the 8 lanes of a quarter warp hit 8 different 16-byte bank groups
+            const bool odd_first = (cp >> 2) & 1;
+            {
+                const uint4 k0 = pack8(tk[0]), k1 = pack8(tk[1]), v0 = pack8(tv[0]), v1 = pack8(tv[1]);
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                const int c = c0 + ch;
-                const uint32_t sw = static_cast<uint32_t>((q8 ^ (c & 7)) << 4);   // 8-token chunk q8 of row c
-                *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + sw) = pack8(tk[ch]);
-                if (c < DV) *reinterpret_cast<uint4*>(sm + ps::BKV + (128 + c) * 128 + sw) = pack8(tv[ch]);
-                kd_pk[ch] = pack8(td[ch]);   // Kdec^T chunk: staged for the packet store after phase B
+                for (int it = 0; it < 2; ++it) {
+                    const int ch = it ^ static_cast<int>(odd_first);
+                    const int c = c0 + ch;
+                    const uint32_t sw = static_cast<uint32_t>((q8 ^ (c & 7)) << 4);   // 8-token chunk q8 of row c
+                    *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + sw) = (ch ? k1 : k0);
+                    if (c < DV) *reinterpret_cast<uint4*>(sm + ps::BKV + (128 + c) * 128 + sw) = (ch ? v1 : v0);
+                }
             }
+            kd_pk[0] = pack8(td[0]);   // Kdec^T chunks: staged for the packet store after phase B
+            kd_pk[1] = pack8(td[1]);
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -577,14 +597,15 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const int m = 32 * qw + lane;
             const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
             if (cg < 2) {
-#pragma unroll 1
-                for (int c32 = 2 * cg; c32 < 2 * cg + 2; ++c32) {
-                    float vv[32];
-                    tmem_ld16(lane_base + 32 * c32, *reinterpret_cast<float(*)[16]>(vv));
-                    tmem_ld16(lane_base + 32 * c32 + 16, *reinterpret_cast<float(*)[16]>(vv + 16));
-                    tmem_wait_ld_regs<32>(vv);
+                {   // the group's 64 columns: four loads in flight, one wait
+                    const int c32 = 2 * cg;
+                    float vv[64];
 #pragma unroll
-                    for (int sub = 0; sub < 4; ++sub) {
+                    for (int i = 0; i < 4; ++i)
+                        tmem_ld16(lane_base + 32 * c32 + 16 * i, *reinterpret_cast<float(*)[16]>(vv + 16 * i));
+                    tmem_wait_ld_regs<64>(vv);
+#pragma unroll
+                    for (int sub = 0; sub < 8; ++sub) {
                         const int cc = 4 * c32 + sub;
                         const float* v = vv;
                         float o8[8];
@@ -603,14 +624,15 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
             } else if (64 * (cg - 2) < DV) {
-#pragma unroll 1
-                for (int c32 = 2 * (cg - 2); c32 < 2 * (cg - 2) + 2; ++c32) {
-                    float vv[32];
-                    tmem_ld16(lane_base + 128 + 32 * c32, *reinterpret_cast<float(*)[16]>(vv));
-                    tmem_ld16(lane_base + 128 + 32 * c32 + 16, *reinterpret_cast<float(*)[16]>(vv + 16));
-                    tmem_wait_ld_regs<32>(vv);
+                {
+                    const int c32 = 2 * (cg - 2);
+                    float vv[64];
 #pragma unroll
-                    for (int sub = 0; sub < 4; ++sub) {
+                    for (int i = 0; i < 4; ++i)
+                        tmem_ld16(lane_base + 128 + 32 * c32 + 16 * i, *reinterpret_cast<float(*)[16]>(vv + 16 * i));
+                    tmem_wait_ld_regs<64>(vv);
+#pragma unroll
+                    for (int sub = 0; sub < 8; ++sub) {
                         const int cc = 4 * c32 + sub;
                         const float* v = vv;
                         float o8[8];
@@ -625,11 +647,13 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
         }
         {   // Kdec^T (held in registers since the column pass) into the B operand area phase B has released
-            const int c0 = 2 * (t & 63), q8 = t >> 6;
+            const int cp = t & 63, c0 = 2 * cp, q8 = t >> 6;
+            const int odd_first = (cp >> 2) & 1;
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int it = 0; it < 2; ++it) {
+                const int ch = it ^ odd_first;
                 const int c = c0 + ch;
-                *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + ((q8 ^ (c & 7)) << 4)) = kd_pk[ch];
+                *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + ((q8 ^ (c & 7)) << 4)) = ch ? kd_pk[1] : kd_pk[0];
             }
         }
         tc_fence_before();
@@ -824,7 +848,6 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_ready);
         // full chunks leave through a TMA tensor store of the O tile, written in place over O_intra
-        const bool o_warp = qw >= 2;
         const bool o_issuer = (w == 2) && lane == 0;
         for (int ci = 0; ci < nch; ++ci) {
             const int st = ci % NST;
@@ -855,7 +878,11 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                             unpack8(*reinterpret_cast<const uint4*>(sb + C::U + cc * 1024 + i * 16), u8);
                         }
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) u8[e] += v[8 * sub + e];
+                        for (int e = 0; e < 8; e += 2) {
+                            const float2 a = __fadd2_rn(make_float2(u8[e], u8[e + 1]),
+                                                        make_float2(v[8 * sub + e], v[8 * sub + e + 1]));
+                            u8[e] = a.x; u8[e + 1] = a.y;
+                        }
                         if constexpr (C::MN) {
                             *reinterpret_cast<uint4*>(sm + C::UOP + sw128_mn_offset(8 * cc, i, C::U_LBO)) = pack8(u8);
                         } else {
@@ -872,7 +899,11 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                         float o8[8];
                         unpack8(*reinterpret_cast<const uint4*>(ot), o8);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) o8[e] += v[8 * sub + e];
+                        for (int e = 0; e < 8; e += 2) {
+                            const float2 a = __fadd2_rn(make_float2(o8[e], o8[e + 1]),
+                                                        make_float2(v[8 * sub + e], v[8 * sub + e + 1]));
+                            o8[e] = a.x; o8[e + 1] = a.y;
+                        }
                         if (full_tma) *reinterpret_cast<uint4*>(ot) = pack8(o8);
                         else *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + col) =
                                  pack8(o8);
@@ -904,7 +935,10 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                     tmem_ld16(lane_base + DVS + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
                 tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
-                for (int e = 0; e < NCW; ++e) S[e] = fmaf(gam, S[e], vv[e]);
+                for (int e = 0; e < NCW; e += 2) {
+                    const float2 a = __ffma2_rn(f2(gam), make_float2(S[e], S[e + 1]), make_float2(vv[e], vv[e + 1]));
+                    S[e] = a.x; S[e + 1] = a.y;
+                }
             }
             if (o_issuer) bulk_wait_read0();   // the O tile has been read out of this stage
             __syncwarp();
