@@ -35,6 +35,7 @@ METRIC = "KDA prefill tokens/s (H=32,d=128,bf16) & decode steps/s; % of TC/HBM r
 B, T, H, D = 4, 4096, 32, 128
 CKPT = 512
 DEC_N, DEC_STEPS = 256, 1024
+SPEC_ND, SPEC_POOL, SPEC_ROUNDS = 4, 16, 256   # drafts per round, distinct draft sets, timed rounds
 # Algorithmic bytes per (token, head) of the prefill path.  Reads: q, k, v bf16 (3 x 256 B),
 # log_alpha fp32 (512 B), beta fp32 (4 B).  Writes: o bf16 (256 B), the 512-token checkpoint
 # (128 x 128 x 4 B / 512 = 128 B) and the final state (64 KiB per 4096 tokens = 16 B).
@@ -306,6 +307,56 @@ def run_ours(args):
                            "alg_bytes_per_launch": dec_bytes}}
     del s0, dq, dk_, dv_, dla, db, state, do
 
+    # ------------------------------------------------------------------ speculative decoding
+    # The decode workload's 256 sequences x 32 heads; each round verifies 4 drafts per sequence
+    # (kda_decode_verify) and commits an accepted prefix drawn uniformly from 0..4 (kda_decode_commit).
+    # A pool of 16 seeded draft sets (673 MB, larger than L2) is cycled through.
+    gen = torch.Generator("cpu").manual_seed(300 + rank)
+    s0, sq, sk, sv, sla, sb = synth.make_decode_inputs(DEC_N, H, D, D, dtype=torch.bfloat16, device=dev,
+                                                       seed=200 + rank, steps=SPEC_ND * SPEC_POOL)
+    pool = []
+    for r in range(SPEC_POOL):
+        sl = slice(r * SPEC_ND, (r + 1) * SPEC_ND)
+        acc_h = torch.randint(0, SPEC_ND + 1, (DEC_N,), generator=gen, dtype=torch.int32)
+        pool.append(tuple(synth.draft_layout(x[sl]) for x in (sq, sk, sv, sla, sb)) + (acc_h.to(dev), acc_h))
+    del sq, sk, sv, sla, sb
+    state = s0.clone()
+    so = torch.empty(DEC_N * SPEC_ND, H, D, dtype=torch.bfloat16, device=dev)
+
+    def spec_round(r):
+        q_, k_, v_, la_, b_, acc_d, _ = pool[r % SPEC_POOL]
+        kda.kda_decode_verify(state, q_, k_, v_, la_, b_, so)
+        kda.kda_decode_commit(state, k_, v_, la_, b_, acc_d)
+
+    for r in range(3):
+        spec_round(r)
+    state.copy_(s0)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for r in range(SPEC_ROUNDS):
+        spec_round(r)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    spec_ms = max_over_ranks(e0.elapsed_time(e1), world) / SPEC_ROUNDS
+    # algorithmic bytes per round: verify reads the state once and every draft's q, k, v (bf16), log_alpha
+    # and beta, and writes its output; commit reads and writes the state of the sequences that accepted
+    # at least one draft, reading the accepted drafts' k, v, log_alpha, beta.
+    st_b = D * D * 4
+    ver_b = DEC_N * H * (st_b + SPEC_ND * (3 * D * 2 + D * 4 + 4 + D * 2))
+    com_b = sum(H * sum((2 * st_b + int(a) * (2 * D * 2 + D * 4 + 4)) for a in p[6].tolist() if a > 0)
+                for p in pool) / SPEC_POOL
+    acc_mean = sum(float(p[6].float().mean()) for p in pool) / SPEC_POOL
+    spec_gbs = (ver_b + com_b) / (spec_ms / 1e3) / 1e9
+    speculative = {"workload": f"{DEC_N} seqs x H={H}, {D}x{D} fp32 state, {SPEC_ND} drafts per round, accepted "
+                               f"counts uniform in 0..{SPEC_ND}", "rounds_per_s": world / (spec_ms / 1e3),
+                   "accepted_tokens_per_s": world * DEC_N * acc_mean / (spec_ms / 1e3),
+                   "ms_per_round": round(spec_ms, 5), "mean_accepted": round(acc_mean, 3),
+                   "roofline": {"bound": "hbm", "kernel": "decode_multi_kernel (verify + commit)",
+                                "achieved": round(spec_gbs, 1), "peak": hbm, "unit": "GB/s",
+                                "frac": round(spec_gbs / hbm, 4), "alg_bytes_per_round": int(ver_b + com_b)}}
+    del s0, pool, state, so
+
     # ------------------------------------------------------------------ segment compose (64 seqs x 8 segments)
     nseg = 8
     M = torch.randn(64 * nseg, H, D, D, device=dev) * (1.0 / D ** 0.5)
@@ -341,7 +392,7 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs and outputs larger than L2 (1.1 GB per step), no flush"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-            "gpu_launches": 3 * args.steps, "decode": decode, "compose": compose,
+            "gpu_launches": 4 * args.steps, "decode": decode, "speculative": speculative, "compose": compose,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

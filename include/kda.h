@@ -155,6 +155,37 @@ KDA_API kda_status_t kda_recurrent_step(float* state, const void* q, const void*
                                 void* o, kda_stream_t stream);
 
 /*
+ * Speculative decoding (orkas.ai "Kimi K3 architecture" post, section "비용은 서빙 스택에서
+ * 돌아옵니다", speculative-decoding item).  The recurrent state is updated in place, so a rejected
+ * draft token cannot be rolled back.  Instead the caller keeps the drafts' projected inputs, which
+ * are far smaller than the state, and the state is rebuilt on chip from them.  Two calls:
+ *
+ *   kda_decode_verify  outputs of all n_draft draft tokens of every sequence, each o_d = S_d^T q_d
+ *                      with S_d the state after drafts 1..d applied to `state`; `state` is read once
+ *                      and never written (the recurrence of kda_recurrent_step, token after token);
+ *   kda_decode_commit  the state after the first n_accept[i] drafts of sequence i, written in place
+ *                      (one read and one write of the state; none at all when n_accept[i] = 0).
+ *
+ * Layouts: the drafts of sequence i are rows i*n_draft + d (d = 0..n_draft-1) of token-major arrays:
+ *   q, k [n*n_draft, H, dk] and v [n*n_draft, H, dv] of `dtype`; log_alpha [n*n_draft, H, dk] fp32;
+ *   beta [n*n_draft, H] fp32; o [n*n_draft, H, dv] of `dtype`;
+ *   state [n, H, dk, dv] fp32 (16-byte aligned); n_accept: device int32 [n], each in 0..n_draft.
+ * Supported: dk, dv in {64, 128}; n_draft >= 1.  Host-detectable errors return before any launch.
+ * A sequence whose n_accept is out of range keeps its state unchanged and sets the status word to
+ * KDA_ERR_DEVICE_INPUT (read it with kda_get_device_status); the other sequences are committed.
+ * Applying commit with n_accept[i] = a gives, bit for bit, the state of a consecutive
+ * kda_recurrent_step calls on the same inputs, and verify gives their outputs.
+ */
+KDA_API kda_status_t kda_decode_verify(const float* state, const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta,
+                               int n, int n_draft, int H, int dk, int dv, kda_dtype_t dtype,
+                               void* o, kda_stream_t stream);
+KDA_API kda_status_t kda_decode_commit(float* state, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, const int32_t* n_accept,
+                               int n, int n_draft, int H, int dk, int dv, kda_dtype_t dtype,
+                               kda_stream_t stream);
+
+/*
  * Segment composition (orkas.ai serving section, sequence split): each segment s of a sequence is
  * summarised by its cumulative transition M_s [dk,dk] and its zero-start final state Z_s [dk,dv]
  * (both from kda_chunk_fwd run on the segment from a zero state with final_transition set).  An

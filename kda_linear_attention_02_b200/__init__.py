@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "KDA_BF16", "KDA_F32", "KDA_CHUNK", "KDAError", "lib_path",
     "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
-    "kda_recurrent_step", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
+    "kda_recurrent_step", "kda_decode_verify", "kda_decode_commit", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
     "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
     "kda_selftest_umma",
 ]
@@ -61,6 +61,10 @@ def _load():
                                         vp, vp, vp, vp, vp, vp]
     L.kda_recurrent_step.restype = i32
     L.kda_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
+    L.kda_decode_verify.restype = i32
+    L.kda_decode_verify.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
+    L.kda_decode_commit.restype = i32
+    L.kda_decode_commit.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
     L.kda_segment_compose.restype = i32
     L.kda_segment_compose.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]
     L.kda_ckpt_offsets.restype = i32
@@ -237,6 +241,59 @@ def kda_recurrent_step(state, q, k, v, log_alpha, beta, o, *, stream=None):
                                     _p(o), _stream(stream))
     _check(st, "kda_recurrent_step")
     return o
+
+
+def _draft_shapes(state, k, name="k"):
+    _need(state, "state", None, torch.float32)
+    n, H, dk, dv = state.shape
+    if k.dim() != 3 or k.shape[1] != H or k.shape[2] != dk or (n > 0 and k.shape[0] % n):
+        raise ValueError(f"{name}: expected [n*n_draft, {H}, {dk}] for n = {n}, got {tuple(k.shape)}")
+    n_draft = k.shape[0] // n if n > 0 else 1
+    return n, n_draft, H, dk, dv
+
+
+def kda_decode_verify(state, q, k, v, log_alpha, beta, o, *, stream=None):
+    """Outputs of n_draft draft tokens per sequence from the committed state (C: kda_decode_verify).
+
+    state [n,H,dk,dv] fp32 (read only); drafts token-major, sequence i at rows i*n_draft ..:
+    q, k [n*n_draft,H,dk]; v, o [n*n_draft,H,dv] (bf16 or fp32); log_alpha [n*n_draft,H,dk] fp32;
+    beta [n*n_draft,H] fp32.
+    """
+    n, n_draft, H, dk, dv = _draft_shapes(state, k)
+    dev = state.device
+    dt = _dtype_code(q)
+    T = n * n_draft
+    _need(q, "q", (T, H, dk), q.dtype, dev)
+    _need(k, "k", (T, H, dk), q.dtype, dev)
+    _need(v, "v", (T, H, dv), q.dtype, dev)
+    _need(o, "o", (T, H, dv), q.dtype, dev)
+    _need(log_alpha, "log_alpha", (T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (T, H), torch.float32, dev)
+    st = _load().kda_decode_verify(_p(state), _p(q), _p(k), _p(v), _p(log_alpha), _p(beta), n, n_draft, H, dk, dv,
+                                   dt, _p(o), _stream(stream))
+    _check(st, "kda_decode_verify")
+    return o
+
+
+def kda_decode_commit(state, k, v, log_alpha, beta, n_accept, *, stream=None):
+    """State after the first n_accept[i] drafts of each sequence, in place (C: kda_decode_commit).
+
+    Same draft layout as kda_decode_verify (q is not needed); n_accept int32 [n] on the device,
+    each in 0..n_draft.
+    """
+    n, n_draft, H, dk, dv = _draft_shapes(state, k)
+    dev = state.device
+    dt = _dtype_code(k)
+    T = n * n_draft
+    _need(k, "k", (T, H, dk), k.dtype, dev)
+    _need(v, "v", (T, H, dv), k.dtype, dev)
+    _need(log_alpha, "log_alpha", (T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (T, H), torch.float32, dev)
+    _need(n_accept, "n_accept", (n,), torch.int32, dev)
+    st = _load().kda_decode_commit(_p(state), _p(k), _p(v), _p(log_alpha), _p(beta), _p(n_accept), n, n_draft, H,
+                                   dk, dv, dt, _stream(stream))
+    _check(st, "kda_decode_commit")
+    return state
 
 
 def kda_segment_compose(transitions, zero_states, seg_cu, init, start_states, end_states=None, *, stream=None):

@@ -265,6 +265,50 @@ kda_status_t kda_recurrent_step(float* state, const void* q, const void* k, cons
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// Shared argument checks of the two speculative-decoding calls.
+static kda_status_t check_multi(int n, int n_draft, int H, int dk, int dv, kda_dtype_t dtype) {
+    if (n < 0 || H <= 0 || n_draft <= 0) return KDA_ERR_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_ARG;
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(n) * H > 0x7fffffffLL) return KDA_ERR_ARG;
+    if (static_cast<long long>(n) * n_draft * H > (1LL << 40)) return KDA_ERR_ARG;
+    return KDA_OK;
+}
+
+kda_status_t kda_decode_verify(const float* state, const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, int n, int n_draft, int H, int dk, int dv,
+                               kda_dtype_t dtype, void* o, kda_stream_t stream) {
+    const kda_status_t c = check_multi(n, n_draft, H, dk, dv, dtype);
+    if (c != KDA_OK) return c;
+    if (n == 0) return KDA_OK;
+    if (!state || !q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_ARG;
+    const size_t es = dtype == KDA_BF16 ? 2 : 4;
+    if (!aligned16(state) || !aligned_to(q, es) || !aligned_to(k, es) || !aligned_to(v, es) || !aligned_to(o, es) ||
+        !aligned4(log_alpha) || !aligned4(beta))
+        return KDA_ERR_ALIGN;
+    int* st = status_ptr();
+    if (!st) return KDA_ERR_CUDA;
+    return from_cuda(launch_decode_multi(const_cast<float*>(state), q, k, v, log_alpha, beta, n, H, n_draft, nullptr, o,
+                                         dk, dv, dtype == KDA_BF16, st, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kda_status_t kda_decode_commit(float* state, const void* k, const void* v, const float* log_alpha,
+                               const float* beta, const int32_t* n_accept, int n, int n_draft, int H, int dk, int dv,
+                               kda_dtype_t dtype, kda_stream_t stream) {
+    const kda_status_t c = check_multi(n, n_draft, H, dk, dv, dtype);
+    if (c != KDA_OK) return c;
+    if (n == 0) return KDA_OK;
+    if (!state || !k || !v || !log_alpha || !beta || !n_accept) return KDA_ERR_ARG;
+    const size_t es = dtype == KDA_BF16 ? 2 : 4;
+    if (!aligned16(state) || !aligned_to(k, es) || !aligned_to(v, es) || !aligned4(log_alpha) || !aligned4(beta) ||
+        !aligned4(n_accept))
+        return KDA_ERR_ALIGN;
+    int* st = status_ptr();
+    if (!st) return KDA_ERR_CUDA;
+    return from_cuda(launch_decode_multi(state, nullptr, k, v, log_alpha, beta, n, H, n_draft, n_accept, nullptr, dk,
+                                         dv, dtype == KDA_BF16, st, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kda_status_t kda_segment_compose(const float* transitions, const float* zero_states, const int32_t* seg_cu,
                                  const float* init, int n_seqs, int n_segs, int H, int dk, int dv,
                                  float* start_states, float* end_states, kda_stream_t stream) {

@@ -1,4 +1,5 @@
-// kda_decode.cu -- one recurrent KDA step (decode), state updated in place.
+// kda_decode.cu -- recurrent KDA steps (decode): one step in place, and the two halves of speculative
+// decoding (verify drafts without touching the state; commit the accepted prefix).
 //
 // The fixed-size state of the llm-wiki "Kimi K3" chapter (section 1: S updated per token, the query
 // multiplied into S, O(1) memory) with the per-channel decay of section "GatedDeltaNet과 KDA의 차이"
@@ -7,118 +8,282 @@
 //   a = exp(max(log_alpha, ln 0.0067));  p = (Diag(a) S)^T k;  u = beta (v - p);
 //   S <- Diag(a) S + k u^T;              o = S^T q = (Diag(a) S)^T q + u (k . q)
 //
-// HBM-bound (about 1.75 flop/byte): the kernel streams each (sequence, head) state once in and once
-// out with 128-bit loads/stores, keeps it in registers between the column reduction and the rank-1
-// write, and reduces the two column sums (against a*k and a*q) over warps through shared memory.
+// HBM-bound (about 1.75 flop/byte): a kernel streams each (sequence, head) state once in with 128-bit
+// loads, keeps it in registers across the column reductions and rank-1 updates of every token it
+// applies, and (when the state changes) streams it once out.
+//
+// Speculative decoding (orkas.ai post, section "비용은 서빙 스택에서 돌아옵니다", speculative-decoding
+// item): the state is updated in place, so a rejected draft cannot be undone; the projected inputs of
+// the drafts, far smaller than the state, are kept instead and the state is rebuilt on chip.
+//   verify: outputs of all n_draft drafts from the committed state, which is read and never written;
+//   commit: the state after the first n_accept[i] drafts of sequence i, written once (nothing moves
+//           when n_accept[i] = 0).
 #include "kda_device.cuh"
 #include "kda_internal.h"
 
 namespace kda {
+
+namespace {
+
+// NT threads over a DK x DV state block: thread t holds float4 column group t % CG of rows
+// t / CG + r RG.  The column sums run over the same row groups in the same order whenever RG is the
+// same, so a 128-thread CTA over 64 columns reduces exactly like a 256-thread CTA over 128 columns.
+template <int DK, int DV, int NT>
+struct DecodeTiling {
+    static constexpr int CG = DV / 4;     // float4 column groups
+    static constexpr int RG = NT / CG;    // row groups
+    static constexpr int RPT = DK / RG;   // state rows per thread
+    static_assert(RG * CG == NT && RPT * RG == DK && DV <= NT, "tiling");
+};
+
+// Per-token staging, double-buffered by token parity so that token t + 1 can be staged while slower
+// threads still read token t's values.
+template <int DK, int DV, int NT>
+struct DecodeSmem {
+    float a[2][DK], k[2][DK], q[2][DK], v[2][DV], u[2][DV], beta[2];
+    float4 red[2][DecodeTiling<DK, DV, NT>::RG][DecodeTiling<DK, DV, NT>::CG];
+    float kq;
+};
+
+// One token's inputs as this thread loads them (element t of each vector; DK, DV <= NT).
+struct TokenIn {
+    float la, k, q, v, beta;
+};
+
+template <typename T, int DK, int DV, bool OUT>
+__device__ __forceinline__ void load_token(TokenIn& x, const T* __restrict__ q, const T* __restrict__ k,
+                                           const T* __restrict__ v, const float* __restrict__ la,
+                                           const float* __restrict__ beta) {
+    const int t = threadIdx.x;
+    if (t < DK) {
+        x.la = la[t];
+        x.k = to_f32(k[t]);
+        if (OUT) x.q = to_f32(q[t]);
+    }
+    if (t < DV) x.v = to_f32(v[t]);
+    if (t == 0) x.beta = *beta;
+}
+
+template <int DK, int DV, int NT, bool OUT>
+__device__ __forceinline__ void stage_token(DecodeSmem<DK, DV, NT>& sh, int par, const TokenIn& x) {
+    const int t = threadIdx.x;
+    if (t < DK) {
+        sh.a[par][t] = __expf(floor_log_decay(x.la));
+        sh.k[par][t] = x.k;
+        if (OUT) sh.q[par][t] = x.q;
+    }
+    if (t < DV) sh.v[par][t] = x.v;
+    if (t == 0) sh.beta[par] = x.beta;
+}
+
+// One token applied to the register-held state s (thread t holds rows rg + r RG, columns 4 cg ..),
+// its inputs staged in sh[par] and made visible by a barrier.  OUT: also o = S_t^T q for this token.
+template <typename T, int DK, int DV, int NT, bool OUT>
+__device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>::RPT], DecodeSmem<DK, DV, NT>& sh,
+                                           int par, T* __restrict__ o) {
+    using DT = DecodeTiling<DK, DV, NT>;
+    constexpr int CG = DT::CG, RG = DT::RG, RPT = DT::RPT;
+    const int t = threadIdx.x, cg = t % CG, rg = t / CG;
+    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = rg + r * RG;
+        const float ak = sh.a[par][i] * sh.k[par][i];
+        pk.x = fmaf(ak, s[r].x, pk.x); pk.y = fmaf(ak, s[r].y, pk.y);
+        pk.z = fmaf(ak, s[r].z, pk.z); pk.w = fmaf(ak, s[r].w, pk.w);
+        if (OUT) {
+            const float aq = sh.a[par][i] * sh.q[par][i];
+            pq.x = fmaf(aq, s[r].x, pq.x); pq.y = fmaf(aq, s[r].y, pq.y);
+            pq.z = fmaf(aq, s[r].z, pq.z); pq.w = fmaf(aq, s[r].w, pq.w);
+        }
+    }
+    sh.red[0][rg][cg] = pk;
+    if (OUT) {
+        sh.red[1][rg][cg] = pq;
+        if (t < 32) {
+            float kq = 0.f;
+            for (int i = t; i < DK; i += 32) kq = fmaf(sh.k[par][i], sh.q[par][i], kq);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+            if (t == 0) sh.kq = kq;
+        }
+    }
+    __syncthreads();
+
+    if (t < DV) {
+        const int j = t;
+        const float* red0 = reinterpret_cast<const float*>(sh.red[0]);
+        float p = 0.f;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) p += red0[g * DV + j];
+        const float u = sh.beta[par] * (sh.v[par][j] - p);
+        sh.u[par][j] = u;
+        if (OUT) {
+            const float* red1 = reinterpret_cast<const float*>(sh.red[1]);
+            float pqj = 0.f;
+#pragma unroll
+            for (int g = 0; g < RG; ++g) pqj += red1[g * DV + j];
+            o[j] = from_f32<T>(fmaf(u, sh.kq, pqj));
+        }
+    }
+    __syncthreads();
+
+    const float4 u4 = reinterpret_cast<const float4*>(sh.u[par])[cg];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = rg + r * RG;
+        const float a = sh.a[par][i], kk = sh.k[par][i];
+        s[r].x = fmaf(a, s[r].x, kk * u4.x);
+        s[r].y = fmaf(a, s[r].y, kk * u4.y);
+        s[r].z = fmaf(a, s[r].z, kk * u4.z);
+        s[r].w = fmaf(a, s[r].w, kk * u4.w);
+    }
+}
 
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(float* __restrict__ state, const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, const float* __restrict__ log_alpha,
                    const float* __restrict__ beta, T* __restrict__ o) {
-    constexpr int CG = DV / 4;     // float4 column groups
-    constexpr int RG = 256 / CG;   // row groups
-    constexpr int RPT = DK / RG;   // rows per thread
-    static_assert(RG * CG == 256 && RPT * RG == DK, "tiling");
+    using DT = DecodeTiling<DK, DV, 256>;
+    __shared__ DecodeSmem<DK, DV, 256> sh;
     const int head = blockIdx.x;   // sequence * H + h
-    const int t = threadIdx.x;
-    const int cg = t % CG;
-    const int rg = t / CG;
-
-    __shared__ float s_a[DK], s_k[DK], s_q[DK], s_u[DV];
-    __shared__ float4 s_red[2][RG][CG];
-    __shared__ float s_kq;
-
+    const int t = threadIdx.x, cg = t % DT::CG, rg = t / DT::CG;
     float4* S = reinterpret_cast<float4*>(state + static_cast<size_t>(head) * DK * DV);
-    float4 s[RPT];
+    float4 s[DT::RPT];
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) s[r] = __ldcs(S + (rg + r * RG) * CG + cg);
-
-    for (int i = t; i < DK; i += 256) {
-        s_a[i] = __expf(floor_log_decay(log_alpha[static_cast<size_t>(head) * DK + i]));
-        s_k[i] = to_f32(k[static_cast<size_t>(head) * DK + i]);
-        s_q[i] = to_f32(q[static_cast<size_t>(head) * DK + i]);
-    }
+    for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg + r * DT::RG) * DT::CG + cg);
+    const size_t hk = static_cast<size_t>(head) * DK, hv = static_cast<size_t>(head) * DV;
+    TokenIn x;
+    load_token<T, DK, DV, true>(x, q + hk, k + hk, v + hv, log_alpha + hk, beta + head);
+    stage_token<DK, DV, 256, true>(sh, 0, x);
     __syncthreads();
+    token_step<T, DK, DV, 256, true>(s, sh, 0, o + hv);
+#pragma unroll
+    for (int r = 0; r < DT::RPT; ++r) __stcs(S + (rg + r * DT::RG) * DT::CG + cg, s[r]);
+}
 
-    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        const int i = rg + r * RG;
-        const float ak = s_a[i] * s_k[i], aq = s_a[i] * s_q[i];
-        pk.x = fmaf(ak, s[r].x, pk.x); pk.y = fmaf(ak, s[r].y, pk.y);
-        pk.z = fmaf(ak, s[r].z, pk.z); pk.w = fmaf(ak, s[r].w, pk.w);
-        pq.x = fmaf(aq, s[r].x, pq.x); pq.y = fmaf(aq, s[r].y, pq.y);
-        pq.z = fmaf(aq, s[r].z, pq.z); pq.w = fmaf(aq, s[r].w, pq.w);
-    }
-    s_red[0][rg][cg] = pk;
-    s_red[1][rg][cg] = pq;
-    if (t < 32) {
-        float kq = 0.f;
-        for (int i = t; i < DK; i += 32) kq = fmaf(s_k[i], s_q[i], kq);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-        if (t == 0) s_kq = kq;
-    }
-    __syncthreads();
-
-    if (t < DV) {
-        const int j = t;
-        const float* red0 = reinterpret_cast<const float*>(s_red[0]);
-        const float* red1 = reinterpret_cast<const float*>(s_red[1]);
-        float p = 0.f, pqj = 0.f;
-#pragma unroll
-        for (int g = 0; g < RG; ++g) {
-            p += red0[g * DV + j];
-            pqj += red1[g * DV + j];
+// Draft inputs are token-major per sequence: token (i, d) of sequence i at row i * n_draft + d of
+// [n * n_draft, H, .] arrays.  VERIFY: all n_draft tokens, outputs written, state read only.
+// Otherwise (commit): the first n_accept[i] tokens, state written back; no outputs.
+// Columns of the state are independent in every step (p, u and o are per column; k . q is recomputed),
+// so a CTA takes one 64-column slice (blockIdx.y) with 256 * 64 / DV threads: the row groups, and so the
+// reduction order, are those of decode_step_kernel, and the results equal consecutive single steps bit
+// for bit.  At DV = 128 the smaller CTAs (128 threads) keep more state loads in flight per SM while
+// others apply their tokens.
+constexpr int kSpecSlice = 64;
+template <int DV>
+__host__ __device__ constexpr int spec_threads() { return 256 * kSpecSlice / DV; }
+template <typename T, int DK, int DV, bool VERIFY>
+__global__ void __launch_bounds__(spec_threads<DV>(), 1024 / spec_threads<DV>() / 2)
+decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T* __restrict__ k,
+                    const T* __restrict__ v, const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                    int H, int n_draft, const int32_t* __restrict__ n_accept, T* __restrict__ o, int* status) {
+    constexpr int DVS = kSpecSlice;
+    static_assert(DV % DVS == 0, "slice");
+    constexpr int NT = spec_threads<DV>();
+    using DT = DecodeTiling<DK, DVS, NT>;
+    static_assert(DT::RG == DecodeTiling<DK, DV, 256>::RG, "same row groups as the single step");
+    __shared__ DecodeSmem<DK, DVS, NT> sh;
+    const int head = blockIdx.x;   // sequence * H + h
+    const int seq = head / H, h = head % H, j0 = blockIdx.y * DVS;
+    const int t = threadIdx.x, cg = t % DT::CG, rg = t / DT::CG;
+    int steps = n_draft;
+    if (!VERIFY) {
+        steps = n_accept[seq];
+        if (steps < 0 || steps > n_draft) {   // the state of this sequence is left as it was
+            if (t == 0 && h == 0 && blockIdx.y == 0) set_status(status, KDA_ERR_DEVICE_INPUT);
+            return;
         }
-        const float vj = to_f32(v[static_cast<size_t>(head) * DV + j]);
-        const float u = beta[head] * (vj - p);
-        s_u[j] = u;
-        o[static_cast<size_t>(head) * DV + j] = from_f32<T>(fmaf(u, s_kq, pqj));
+        if (steps == 0) return;
     }
-    __syncthreads();
-
-    const float4 u4 = reinterpret_cast<const float4*>(s_u)[cg];
+    // state rows are DV wide; this CTA's float4 column groups start at j0
+    float4* S = reinterpret_cast<float4*>(state + static_cast<size_t>(head) * DK * DV + j0);
+    float4 s[DT::RPT];
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        const int i = rg + r * RG;
-        const float a = s_a[i], kk = s_k[i];
-        float4 x;
-        x.x = fmaf(a, s[r].x, kk * u4.x);
-        x.y = fmaf(a, s[r].y, kk * u4.y);
-        x.z = fmaf(a, s[r].z, kk * u4.z);
-        x.w = fmaf(a, s[r].w, kk * u4.w);
-        __stcs(S + i * CG + cg, x);
+    for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg + r * DT::RG) * (DV / 4) + cg);
+    // token d + 1's inputs are loaded into registers while token d is applied, then staged
+    auto row_of = [&](int d) { return (static_cast<size_t>(seq) * n_draft + d) * H + h; };
+    auto load = [&](TokenIn& x, int d) {
+        const size_t row = row_of(d);
+        load_token<T, DK, DVS, VERIFY>(x, VERIFY ? q + row * DK : nullptr, k + row * DK, v + row * DV + j0,
+                                       log_alpha + row * DK, beta + row);
+    };
+    TokenIn x;
+    load(x, 0);
+    stage_token<DK, DVS, NT, VERIFY>(sh, 0, x);
+    for (int d = 0; d < steps; ++d) {
+        const int par = d & 1;
+        if (d + 1 < steps) load(x, d + 1);
+        __syncthreads();   // token d staged (and every reader of the other half is past token d - 1)
+        token_step<T, DK, DVS, NT, VERIFY>(s, sh, par, VERIFY ? o + row_of(d) * DV + j0 : nullptr);
+        if (d + 1 < steps) stage_token<DK, DVS, NT, VERIFY>(sh, par ^ 1, x);
+    }
+    if (!VERIFY) {
+#pragma unroll
+        for (int r = 0; r < DT::RPT; ++r) __stcs(S + (rg + r * DT::RG) * (DV / 4) + cg, s[r]);
     }
 }
 
 template <typename T, int DK, int DV>
-static cudaError_t launch_decode_t(float* state, const void* q, const void* k, const void* v, const float* la,
-                                   const float* beta, void* o, int nh, cudaStream_t s) {
+cudaError_t launch_decode_t(float* state, const void* q, const void* k, const void* v, const float* la,
+                            const float* beta, void* o, int nh, cudaStream_t s) {
     decode_step_kernel<T, DK, DV><<<nh, 256, 0, s>>>(state, static_cast<const T*>(q), static_cast<const T*>(k),
                                                     static_cast<const T*>(v), la, beta, static_cast<T*>(o));
     return cudaGetLastError();
 }
 
-template <typename T>
-static cudaError_t launch_decode_dt(float* state, const void* q, const void* k, const void* v, const float* la,
-                                    const float* beta, void* o, int nh, int dk, int dv, cudaStream_t s) {
-    if (dk == 128 && dv == 128) return launch_decode_t<T, 128, 128>(state, q, k, v, la, beta, o, nh, s);
-    if (dk == 128 && dv == 64) return launch_decode_t<T, 128, 64>(state, q, k, v, la, beta, o, nh, s);
-    if (dk == 64 && dv == 128) return launch_decode_t<T, 64, 128>(state, q, k, v, la, beta, o, nh, s);
-    return launch_decode_t<T, 64, 64>(state, q, k, v, la, beta, o, nh, s);
+template <typename T, int DK, int DV>
+cudaError_t launch_multi_t(float* state, const void* q, const void* k, const void* v, const float* la,
+                           const float* beta, int n, int H, int n_draft, const int32_t* n_accept, void* o,
+                           int* status, cudaStream_t s) {
+    const T* qq = static_cast<const T*>(q);
+    const T* kk = static_cast<const T*>(k);
+    const T* vv = static_cast<const T*>(v);
+    const dim3 grid(n * H, DV / kSpecSlice);
+    if (n_accept)
+        decode_multi_kernel<T, DK, DV, false><<<grid, spec_threads<DV>(), 0, s>>>(state, qq, kk, vv, la, beta, H, n_draft, n_accept,
+                                                                  nullptr, status);
+    else
+        decode_multi_kernel<T, DK, DV, true><<<grid, spec_threads<DV>(), 0, s>>>(state, qq, kk, vv, la, beta, H, n_draft, nullptr,
+                                                                 static_cast<T*>(o), status);
+    return cudaGetLastError();
 }
+
+}  // namespace
 
 cudaError_t launch_decode(float* state, const void* q, const void* k, const void* v, const float* la,
                           const float* beta, void* o, int nh, int dk, int dv, bool bf16, cudaStream_t s) {
     if (nh == 0) return cudaSuccess;
-    return bf16 ? launch_decode_dt<__nv_bfloat16>(state, q, k, v, la, beta, o, nh, dk, dv, s)
-                : launch_decode_dt<float>(state, q, k, v, la, beta, o, nh, dk, dv, s);
+#define KDA_DECODE_CASE(T, DK, DV) \
+    if (dk == DK && dv == DV) return launch_decode_t<T, DK, DV>(state, q, k, v, la, beta, o, nh, s);
+    if (bf16) {
+        KDA_DECODE_CASE(__nv_bfloat16, 128, 128) KDA_DECODE_CASE(__nv_bfloat16, 128, 64)
+        KDA_DECODE_CASE(__nv_bfloat16, 64, 128) KDA_DECODE_CASE(__nv_bfloat16, 64, 64)
+    } else {
+        KDA_DECODE_CASE(float, 128, 128) KDA_DECODE_CASE(float, 128, 64)
+        KDA_DECODE_CASE(float, 64, 128) KDA_DECODE_CASE(float, 64, 64)
+    }
+#undef KDA_DECODE_CASE
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_multi(float* state, const void* q, const void* k, const void* v, const float* la,
+                                const float* beta, int n, int H, int n_draft, const int32_t* n_accept, void* o,
+                                int dk, int dv, bool bf16, int* status, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+#define KDA_MULTI_CASE(T, DK, DV)  \
+    if (dk == DK && dv == DV)      \
+        return launch_multi_t<T, DK, DV>(state, q, k, v, la, beta, n, H, n_draft, n_accept, o, status, s);
+    if (bf16) {
+        KDA_MULTI_CASE(__nv_bfloat16, 128, 128) KDA_MULTI_CASE(__nv_bfloat16, 128, 64)
+        KDA_MULTI_CASE(__nv_bfloat16, 64, 128) KDA_MULTI_CASE(__nv_bfloat16, 64, 64)
+    } else {
+        KDA_MULTI_CASE(float, 128, 128) KDA_MULTI_CASE(float, 128, 64)
+        KDA_MULTI_CASE(float, 64, 128) KDA_MULTI_CASE(float, 64, 64)
+    }
+#undef KDA_MULTI_CASE
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace kda

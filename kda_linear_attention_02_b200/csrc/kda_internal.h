@@ -11,6 +11,11 @@ namespace kda {
 // Decode step (kda_decode.cu).
 cudaError_t launch_decode(float* state, const void* q, const void* k, const void* v, const float* la,
                           const float* beta, void* o, int nh, int dk, int dv, bool bf16, cudaStream_t s);
+// Speculative decoding (kda_decode.cu): n_accept == nullptr verifies (outputs of all n_draft drafts, state
+// read only); otherwise commits the first n_accept[i] drafts of every sequence into the state.
+cudaError_t launch_decode_multi(float* state, const void* q, const void* k, const void* v, const float* la,
+                                const float* beta, int n, int H, int n_draft, const int32_t* n_accept, void* o,
+                                int dk, int dv, bool bf16, int* status, cudaStream_t s);
 
 // Segment compose (kda_compose.cu).
 cudaError_t launch_compose(const float* M, const float* Z, const int32_t* seg_cu, const float* init, int n_seqs,

@@ -121,3 +121,9 @@ def make_decode_inputs(n, H, dk, dv, *, dtype=torch.bfloat16, device="cpu", seed
     la = -5.0 * torch.sigmoid(_draw((steps, n, H, dk), gen, device, std=1.5))
     state0 = _draw((n, H, dk, dv), gen, device, std=state_sd)
     return state0, q, k, v, la, beta
+
+
+def draft_layout(x):
+    """[n_draft, n, H, ...] per-step decode inputs -> the token-major draft layout [n * n_draft, H, ...]
+    (sequence i's drafts at rows i * n_draft ..) of kda_decode_verify / kda_decode_commit."""
+    return x.transpose(0, 1).contiguous().reshape(x.shape[0] * x.shape[1], *x.shape[2:])

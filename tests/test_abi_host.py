@@ -129,6 +129,35 @@ def test_decode_and_compose_host_argument_errors(lib):
     assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 32, 1, None) == -1
 
 
+def test_speculative_decode_host_argument_errors(lib):
+    vp = ctypes.c_void_p
+    st, q, k, v, la, b, o, acc = (vp(0x1000 * (i + 1)) for i in range(8))
+    # verify: (state, q, k, v, la, beta, n, n_draft, H, dk, dv, dtype, o, stream)
+    assert lib.kda_decode_verify(st, q, k, v, la, b, 2, 0, 4, 128, 128, 0, o, None) == -1      # no drafts
+    assert lib.kda_decode_verify(st, q, k, v, la, b, 2, 3, 0, 128, 128, 0, o, None) == -1      # no heads
+    assert lib.kda_decode_verify(st, q, k, v, la, b, 2, 3, 4, 96, 128, 0, o, None) == -3       # dk
+    assert lib.kda_decode_verify(st, q, k, v, la, b, 2, 3, 4, 128, 128, 5, o, None) == -1      # dtype
+    assert lib.kda_decode_verify(vp(0x1004), q, k, v, la, b, 2, 3, 4, 128, 128, 0, o, None) == -2
+    assert lib.kda_decode_verify(st, None, k, v, la, b, 2, 3, 4, 128, 128, 0, o, None) == -1
+    assert lib.kda_decode_verify(st, q, k, v, la, b, 0, 3, 4, 128, 128, 0, o, None) == 0       # empty batch
+    # commit: (state, k, v, la, beta, n_accept, n, n_draft, H, dk, dv, dtype, stream)
+    assert lib.kda_decode_commit(st, k, v, la, b, None, 2, 3, 4, 128, 128, 0, None) == -1      # no counts
+    assert lib.kda_decode_commit(st, k, v, la, b, acc, 2, -1, 4, 128, 128, 0, None) == -1
+    assert lib.kda_decode_commit(st, k, v, la, b, vp(0x1002), 2, 3, 4, 128, 128, 0, None) == -2
+    assert lib.kda_decode_commit(st, k, v, la, b, acc, 2, 3, 4, 64, 80, 1, None) == -3
+    assert lib.kda_decode_commit(st, k, v, la, b, acc, 0, 3, 4, 128, 128, 0, None) == 0
+
+
+def test_draft_layout_is_token_major_per_sequence():
+    from kda_linear_attention_02_b200 import synth
+    x = torch.arange(3 * 2 * 5).reshape(3, 2, 5)        # [n_draft=3, n=2, H=5]
+    y = synth.draft_layout(x)
+    assert y.shape == (6, 5)
+    for i in range(2):
+        for d in range(3):
+            assert torch.equal(y[i * 3 + d], x[d, i])
+
+
 def test_binding_checks_shapes_on_cpu_tensors(lib):
     q = torch.zeros(64, 2, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
