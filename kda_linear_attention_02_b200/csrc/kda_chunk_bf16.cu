@@ -81,9 +81,11 @@ template <int DV>
 struct Pk {
     static constexpr uint32_t AW = 0;                 // [-W; P]: 128 x 128 bf16, K-major, 128B swizzle, 2 K atoms
     static constexpr uint32_t KD = 32768;             // Kdec^T:  128 x 64 bf16, K-major, 128B swizzle
-    static constexpr uint32_t U = 49152;              // U:       [DV/8][64][8] bf16 (8-column chunks)
-    static constexpr uint32_t OI = U + DV * 128;      // O_intra: [DV/64][64 rows][128 B], 16-byte chunks ^ (row % 8)
-    static constexpr uint32_t G = OI + DV * 128;      // gamma_C: [128] fp32
+    // [U; O_intra] per 64-column atom: [DV/64][128 rows: U rows 0..63, O_intra rows 64..127][128 B],
+    // 16-byte chunks ^ (row % 8) -- the K-major 128B-swizzle A operand that loads them into the state
+    // pass's accumulator, and the layout of the O tensor store
+    static constexpr uint32_t UO = 49152;
+    static constexpr uint32_t G = UO + DV * 256;      // gamma_C: [128] fp32
     static constexpr uint32_t BYTES = ((G + 512 + 1023) / 1024) * 1024;
 };
 
@@ -100,7 +102,7 @@ constexpr uint32_t MISC = 204800;    // beta[64] fp32, half-tile totals [8][128]
 constexpr uint32_t IAQ = 209920;     // [I; Aqk]: 128 x 64 bf16 (A operand of the Y product)
 // aliases of RALL/BVAR once phase A has completed
 constexpr uint32_t AM = 81920, XF = 99328, TT = 118016, XT = 124928, XY = 133120;   // solve
-constexpr uint32_t AWS = 81920, US = 114688, OIS = 131072;                       // packet staging
+constexpr uint32_t AWS = 81920, UOS = 114688;                                    // packet staging
 constexpr uint32_t BYTES = IAQ + 16384;
 constexpr int LDM = 68;              // fp32 row pitch of AM (float4-aligned rows; 4 rows apart = 16 banks)
 constexpr int LDX = 73;              // fp32 row pitch of X (odd: column reads of X^T spread over the banks)
@@ -638,10 +640,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         float o8[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) o8[j] = v[8 * sub + j];
-                        const int r = m & 63;
-                        const uint32_t dst = m < 64 ? ps::US + cc * 1024 + r * 16
-                                                    : ps::OIS + (cc >> 3) * 8192 + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
-                        *reinterpret_cast<uint4*>(sm + dst) = pack8(o8);
+                        *reinterpret_cast<uint4*>(sm + ps::UOS + (cc >> 3) * 16384 + m * 128 +
+                                                  (((cc & 7) ^ (m & 7)) << 4)) = pack8(o8);
                     }
                 }
             }
@@ -662,8 +662,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         if (t == 0) {
             bulk_s2g(pkt + P::AW, sm + ps::AWS, 32768);
             bulk_s2g(pkt + P::KD, sm + ps::BKV, 16384);
-            bulk_s2g(pkt + P::U, sm + ps::US, DV * 128);
-            bulk_s2g(pkt + P::OI, sm + ps::OIS, DV * 128);
+            bulk_s2g(pkt + P::UO, sm + ps::UOS, DV * 256);
             bulk_commit();   // the next column pass waits for the read-out before reusing the staging
         }
         item = nitem;
@@ -690,15 +689,18 @@ struct SCfg {
     static constexpr int NT = 32 * (NEW + 2);              // + producer warp + MMA warp
     static constexpr bool MN = DVS >= 64;                  // S and U' staged MN-major (row = channel / token)
     static constexpr int NST = DVS == 128 ? 2 : 3;
-    static constexpr uint32_t OI_BYTES = DVS >= 64 ? DVS * 128 : 8192;   // whole 64-column blocks of O_intra
-    static constexpr uint32_t AW = 0, KD = 32768, U = 49152, OI = U + DVS * 128, G = OI + OI_BYTES;
+    static constexpr uint32_t UO_BYTES = DVS >= 64 ? DVS * 256 : 16384;   // whole 64-column atoms of [U; O_intra]
+    static constexpr uint32_t AW = 0, KD = 32768, UO = 49152, G = UO + UO_BYTES;
     static constexpr uint32_t STAGE = ((G + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SOP = NST * STAGE;      // S as B operand (N = DVS, K = 128)
     static constexpr uint32_t UOP = SOP + DVS * 256;  // U' as B operand (N = DVS, K = 64)
-    static constexpr uint32_t BYTES = UOP + DVS * 128;
+    static constexpr uint32_t IDN = UOP + DVS * 128;  // 16 x 64 bf16 B operand, row n = 1 where k % 16 == n
+    static constexpr uint32_t BYTES = IDN + 2048;
+    // TMEM: D1 double-buffered at columns [0, DVS) and [2 DVS, 3 DVS), D2 at [DVS, 2 DVS)
     static constexpr uint32_t S_LBO = 128 * 128;      // MN-major: 64 columns x 128 K rows per block
     static constexpr uint32_t U_LBO = 64 * 128;       // MN-major: 64 columns x 64 K rows per block
-    static constexpr uint32_t TMEM_COLS = 2 * DVS <= 32 ? 32 : (2 * DVS <= 64 ? 64 : (2 * DVS <= 128 ? 128 : 256));
+    static constexpr uint32_t TMEM_COLS = 3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512);
+    static __host__ __device__ constexpr uint32_t d1col(int ci) { return (ci & 1) ? 2 * DVS : 0; }
 };
 
 template <int DV, int DVS>
@@ -749,6 +751,13 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         tmem_alloc(&tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
+    // B operand that copies 16 columns of an A operand into the accumulator: B[n][k] = (k % 16 == n)
+    for (int e = t; e < 16 * 64; e += C::NT) {
+        const int n = e >> 6, k = e & 63;
+        *reinterpret_cast<__nv_bfloat16*>(sm + C::IDN + sw128_offset(n, k, 16)) =
+            __float2bfloat16_rn((k & 15) == n ? 1.f : 0.f);
+    }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -763,14 +772,11 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 if (!mbar_wait(&empty[st], ((ci / NST) & 1) ^ 1, status)) break;
                 const uint8_t* pk = packets + static_cast<size_t>((lo + ci - win_lo) * H + h) * P::BYTES;
                 uint8_t* sb = sm + st * C::STAGE;
-                const uint32_t bytes = 32768 + 16384 + 512 + (trans ? 0u : DVS * 128 + C::OI_BYTES);
+                const uint32_t bytes = 32768 + 16384 + 512 + (trans ? 0u : C::UO_BYTES);
                 mbar_arrive_expect_tx(&full[st], bytes);
                 bulk_g2s(sb + C::AW, pk + P::AW, 32768, &full[st]);
                 bulk_g2s(sb + C::KD, pk + P::KD, 16384, &full[st]);
-                if (!trans) {
-                    bulk_g2s(sb + C::U, pk + P::U + (j0 / 8) * 1024, DVS * 128, &full[st]);
-                    bulk_g2s(sb + C::OI, pk + P::OI + (j0 / 64) * 8192, C::OI_BYTES, &full[st]);
-                }
+                if (!trans) bulk_g2s(sb + C::UO, pk + P::UO + (j0 / 64) * 16384, C::UO_BYTES, &full[st]);
                 bulk_g2s(sb + C::G, pk + P::G, 512, &full[st]);
                 issued = ci + 1;
             }
@@ -782,20 +788,36 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, DVS, false, C::MN);
-            const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP);
+            const uint32_t idesc16 = idesc_bf16(128, 16);
+            const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP), idn = smem_u32(sm + C::IDN);
+            // D1[ci] = [U; O_intra] of chunk ci: 16 columns per product against the copying B operand
+            // (exact: bf16 values times 1), so that product 1 adds [-W; P] S onto it in the accumulator
+            auto load_uo = [&](int ci) {
+                const uint32_t sb = smem_u32(sm + (ci % NST) * C::STAGE);
+                const int c_off = DVS >= 64 ? 0 : (j0 & 63);   // the slice's first column inside its atom
+#pragma unroll
+                for (int ks = 0; ks < DVS / 16; ++ks) {
+                    const int col = c_off + 16 * ks;
+                    const uint32_t kk = static_cast<uint32_t>((col & 63) >> 4) * 32;
+                    umma_f16(tm + C::d1col(ci) + 16 * ks, sdesc_k_sw128(sb + C::UO + (col >> 6) * 16384 + kk),
+                             sdesc_k_sw128(idn + kk), idesc16, false);
+                }
+            };
             for (int ci = 0; ci < nch; ++ci) {
                 const int st = ci % NST;
                 if (!mbar_wait(&s_ready, ci & 1, status)) break;
                 if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
                 tc_fence_after();
                 const uint32_t sb = smem_u32(sm + st * C::STAGE);
-                // D1 = [-W; P] S   (M = 128, N = DVS, K = 128)
+                if (ci == 0 && !trans) load_uo(0);
+                // D1 (+)= [-W; P] S   (M = 128, N = DVS, K = 128)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
                     const uint64_t bdesc = C::MN ? sdesc_mn_sw128(sop + ks * 2048, C::S_LBO)
                                                  : sdesc_k_sw128(sop + ka * (DVS * 128) + kb);
-                    umma_f16(tm, sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc, ks > 0);
+                    umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc,
+                             !trans || ks > 0);
                 }
                 umma_commit(&d1_full);
                 if (!mbar_wait(&up_ready, ci & 1, status)) break;
@@ -809,6 +831,13 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 }
                 umma_commit(&d2_full);
                 umma_commit(&empty[st]);
+                // the next chunk's [U; O_intra] into the other D1 buffer, read last by chunk ci - 1's
+                // epilogue (done: its warps arrived on s_ready for chunk ci)
+                if (!trans && ci + 1 < nch) {
+                    if (!mbar_wait(&full[(ci + 1) % NST], ((ci + 1) / NST) & 1, status)) break;
+                    tc_fence_after();
+                    load_uo(ci + 1);
+                }
             }
         }
     } else {
@@ -861,7 +890,8 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             tc_fence_after();
             float vv[NCW];   // D1 row i, columns jw .. jw + NCW: all loads in flight, one wait
 #pragma unroll
-            for (int cb = 0; cb < NCW; cb += 16) tmem_ld16(lane_base + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+            for (int cb = 0; cb < NCW; cb += 16)
+                tmem_ld16(lane_base + C::d1col(ci) + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
             tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
             for (int cb = 0; cb < NCW; cb += 16) {
@@ -869,20 +899,10 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {
                     const int cc = (jw + cb) / 8 + sub;   // 8-column chunk within the slice
-                    if (i < 64) {
+                    if (i < 64) {   // U' = U - W S (D1 was loaded with U before the product)
                         float u8[8];
-                        if (trans) {
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) u8[e] = 0.f;
-                        } else {
-                            unpack8(*reinterpret_cast<const uint4*>(sb + C::U + cc * 1024 + i * 16), u8);
-                        }
-#pragma unroll
-                        for (int e = 0; e < 8; e += 2) {
-                            const float2 a = __fadd2_rn(make_float2(u8[e], u8[e + 1]),
-                                                        make_float2(v[8 * sub + e], v[8 * sub + e + 1]));
-                            u8[e] = a.x; u8[e + 1] = a.y;
-                        }
+                        for (int e = 0; e < 8; ++e) u8[e] = v[8 * sub + e];
                         if constexpr (C::MN) {
                             *reinterpret_cast<uint4*>(sm + C::UOP + sw128_mn_offset(8 * cc, i, C::U_LBO)) = pack8(u8);
                         } else {
@@ -891,19 +911,14 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                                 *reinterpret_cast<__nv_bfloat16*>(sm + C::UOP + sw128_offset(8 * cc + e, i, DVS)) =
                                     __float2bfloat16_rn(u8[e]);
                         }
-                    } else if (!trans && i - 64 < n) {
+                    } else if (!trans && i - 64 < n) {   // O = O_intra + P S (D1 was loaded with O_intra)
                         const int r = i - 64;
                         const int col = j0 + 8 * cc;   // first column of this 8-column chunk
-                        uint8_t* ot = sb + C::OI + ((col >> 6) - (j0 >> 6)) * 8192 + r * 128 +
+                        uint8_t* ot = sb + C::UO + ((col >> 6) - (j0 >> 6)) * 16384 + (64 + r) * 128 +
                                       ((((col & 63) >> 3) ^ (r & 7)) << 4);
                         float o8[8];
-                        unpack8(*reinterpret_cast<const uint4*>(ot), o8);
 #pragma unroll
-                        for (int e = 0; e < 8; e += 2) {
-                            const float2 a = __fadd2_rn(make_float2(o8[e], o8[e + 1]),
-                                                        make_float2(v[8 * sub + e], v[8 * sub + e + 1]));
-                            o8[e] = a.x; o8[e + 1] = a.y;
-                        }
+                        for (int e = 0; e < 8; ++e) o8[e] = v[8 * sub + e];
                         if (full_tma) *reinterpret_cast<uint4*>(ot) = pack8(o8);
                         else *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + col) =
                                  pack8(o8);
@@ -921,7 +936,8 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 if (o_issuer) {
 #pragma unroll
                     for (int b = 0; b < DVS / 64; ++b)
-                        tma_store_3d(&map_o, j0 + 64 * b, h, static_cast<int>(seq_tok0 + c * 64), sb + C::OI + b * 8192);
+                        tma_store_3d(&map_o, j0 + 64 * b, h, static_cast<int>(seq_tok0 + c * 64),
+                                     sb + C::UO + b * 16384 + 8192);
                     bulk_commit();
                 }
             }
