@@ -846,14 +846,20 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         const int i = 32 * qw + lane;   // TMEM lane: row of D1 (token row / P row), channel of D2 and S
         const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
         float S[NCW];
+        {
+            const float* src = nullptr;
+            if (!first) src = carry + (sh * kDK + i) * CW + (trans ? DV : 0) + j0 + jw;
+            else if (!trans && initial_state) src = initial_state + (sh * kDK + i) * DV + j0 + jw;
 #pragma unroll
-        for (int j = 0; j < NCW; ++j) {
-            const int col = j0 + jw + j;
-            float x;
-            if (!first) x = carry[(sh * kDK + i) * CW + (trans ? DV : 0) + col];
-            else if (trans) x = (i == col) ? 1.f : 0.f;
-            else x = initial_state ? initial_state[(sh * kDK + i) * DV + col] : 0.f;
-            S[j] = x;
+            for (int e = 0; e < NCW / 4; ++e) {
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (src) x = reinterpret_cast<const float4*>(src)[e];
+                S[4 * e] = x.x; S[4 * e + 1] = x.y; S[4 * e + 2] = x.z; S[4 * e + 3] = x.w;
+            }
+            if (first && trans) {
+#pragma unroll
+                for (int j = 0; j < NCW; ++j) S[j] = (i == j0 + jw + j) ? 1.f : 0.f;
+            }
         }
         // S (and later U') as a B operand: MN-major rows are written 8 columns at a time
         auto write_sop = [&]() {
@@ -981,15 +987,18 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             if (lane == 0) mbar_arrive(&s_ready);
         }
         if (o_issuer) bulk_wait0();
+        // row i, columns j0 + jw .. + NCW: 16-byte stores (every row start and column offset is a multiple of 4)
+        float* dst = nullptr;
+        if (last) {
+            if (trans) dst = final_transition + (sh * kDK + i) * kDK + j0 + jw;
+            else if (final_state) dst = final_state + (sh * kDK + i) * DV + j0 + jw;
+        } else {
+            dst = carry + (sh * kDK + i) * CW + (trans ? DV : 0) + j0 + jw;
+        }
+        if (dst) {
 #pragma unroll
-        for (int j = 0; j < NCW; ++j) {
-            const int col = j0 + jw + j;
-            if (last) {
-                if (trans) final_transition[(sh * kDK + i) * kDK + col] = S[j];
-                else if (final_state) final_state[(sh * kDK + i) * DV + col] = S[j];
-            } else {
-                carry[(sh * kDK + i) * CW + (trans ? DV : 0) + col] = S[j];
-            }
+            for (int e = 0; e < NCW / 4; ++e)
+                reinterpret_cast<float4*>(dst)[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
         }
     }
     tc_fence_before();
