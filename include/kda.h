@@ -201,6 +201,56 @@ KDA_API kda_status_t kda_segment_compose(const float* transitions, const float* 
                                  float* start_states, float* end_states, kda_stream_t stream);
 
 /*
+ * Prefix reuse bookkeeping (orkas.ai "Kimi K3 architecture" post, section "비용은 서빙 스택에서
+ * 돌아옵니다", prefix-reuse item).  Half of the cache is per-token pages (full-attention layers) and half
+ * one fixed-size recurrent state per request (KDA layers); a cached prefix is usable only where both
+ * can be restored at the same boundary.  The granularities are decoupled: a hash every 512 tokens,
+ * allocation in units of 1024-6144 tokens, and recurrent-state checkpoints kept sparsely at some hash
+ * ends.  These host-only calls keep that directory; the checkpoint states themselves live in a device
+ * pool [n_slots, H, dk, dv] fp32 owned by the caller, filled from kda_chunk_fwd's checkpoints and
+ * passed back to it as initial_state when a request resumes.
+ *
+ * kda_prefix_block_hashes: chained 64-bit FNV-1a hashes of the full 512-token blocks of a token
+ *   sequence: hash[i] = FNV-1a over the 8 little-endian bytes of hash[i-1] (seed for i = 0) followed
+ *   by the 4 little-endian bytes of each token of block i, so hash[i] identifies tokens
+ *   [0, 512 (i+1)).  tokens: host int32 [n_tokens]; hashes: host uint64 [n_tokens / 512].  Returns
+ *   the number of full blocks (the partial tail block is not hashed), or -1 on a bad argument.
+ *
+ * kda_prefix_cache_create: a directory of at most max_blocks block hashes and n_slots checkpoint
+ *   slots; checkpoints are planned every unit_blocks blocks (2..12: 1024-6144 tokens) and at the last
+ *   full block of a request.  Least-recently-used entries are evicted (a block entry takes its slot
+ *   with it; a slot can also be taken from an older entry that keeps its hash).  Thread-safe.
+ *
+ * kda_prefix_cache_lookup: matched_blocks = the length of the request's leading run of cached
+ *   hashes; resume_blocks = the deepest block end <= matched_blocks whose state is checkpointed (0 if
+ *   none) and resume_slot its slot (-1 if none).  The request restarts at token 512 * resume_blocks
+ *   with the slot's state.  Touches the matched entries.
+ *
+ * kda_prefix_cache_plan: the block ends e (resume_blocks < e <= n_blocks, ascending) after which a
+ *   request should store its state: multiples of unit_blocks, and n_blocks itself.  Writes at most
+ *   max_out of them and returns how many there are (-1 on a bad argument).
+ *
+ * kda_prefix_cache_insert: records the request's n_blocks hashes and gives each planned end ends[i]
+ *   a slot out_slots[i] (the existing one if that hash already has a checkpoint, else a free slot,
+ *   else one taken from the least recently used checkpoint outside this request; -1 if none can be
+ *   freed).  The caller then copies the state after 512 * ends[i] tokens into that slot.
+ */
+#define KDA_PREFIX_BLOCK 512
+typedef struct kda_prefix_cache kda_prefix_cache;
+KDA_API int64_t kda_prefix_block_hashes(const int32_t* tokens, int64_t n_tokens, uint64_t seed, uint64_t* hashes);
+KDA_API kda_status_t kda_prefix_cache_create(int64_t max_blocks, int n_slots, int unit_blocks,
+                                     kda_prefix_cache** out);
+KDA_API void kda_prefix_cache_destroy(kda_prefix_cache* cache);
+KDA_API kda_status_t kda_prefix_cache_lookup(kda_prefix_cache* cache, const uint64_t* hashes, int64_t n_blocks,
+                                     int64_t* matched_blocks, int64_t* resume_blocks, int32_t* resume_slot);
+KDA_API int64_t kda_prefix_cache_plan(const kda_prefix_cache* cache, int64_t n_blocks, int64_t resume_blocks,
+                              int64_t* out_ends, int64_t max_out);
+KDA_API kda_status_t kda_prefix_cache_insert(kda_prefix_cache* cache, const uint64_t* hashes, int64_t n_blocks,
+                                     const int64_t* ends, int64_t n_ends, int32_t* out_slots);
+KDA_API kda_status_t kda_prefix_cache_stats(const kda_prefix_cache* cache, int64_t* n_blocks_cached,
+                                    int32_t* n_slots_used);
+
+/*
  * Host-only, pure: checkpoint offsets for kda_chunk_fwd.  host_ckpt_cu[0] = 0 and
  * host_ckpt_cu[i+1] = host_ckpt_cu[i] + floor(len_i / stride) with len_i from host_cu_seqlens
  * (host int32 [n+1]).  Returns KDA_ERR_ARG on a bad stride or a decreasing table.

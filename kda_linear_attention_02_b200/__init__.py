@@ -18,11 +18,14 @@ __all__ = [
     "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
     "kda_recurrent_step", "kda_decode_verify", "kda_decode_commit", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
     "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
-    "kda_selftest_umma",
+    "kda_selftest_umma", "KDA_PREFIX_BLOCK", "kda_prefix_block_hashes", "kda_prefix_cache_create",
+    "kda_prefix_cache_destroy", "kda_prefix_cache_lookup", "kda_prefix_cache_plan", "kda_prefix_cache_insert",
+    "kda_prefix_cache_stats",
 ]
 
 KDA_BF16 = 0
 KDA_F32 = 1
+KDA_PREFIX_BLOCK = 512
 KDA_CHUNK = 64
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -65,6 +68,21 @@ def _load():
     L.kda_decode_verify.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
     L.kda_decode_commit.restype = i32
     L.kda_decode_commit.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    u64, i64p = ctypes.c_uint64, ctypes.POINTER(ctypes.c_int64)
+    L.kda_prefix_block_hashes.restype = i64
+    L.kda_prefix_block_hashes.argtypes = [vp, i64, u64, vp]
+    L.kda_prefix_cache_create.restype = i32
+    L.kda_prefix_cache_create.argtypes = [i64, i32, i32, ctypes.POINTER(vp)]
+    L.kda_prefix_cache_destroy.restype = None
+    L.kda_prefix_cache_destroy.argtypes = [vp]
+    L.kda_prefix_cache_lookup.restype = i32
+    L.kda_prefix_cache_lookup.argtypes = [vp, vp, i64, i64p, i64p, ctypes.POINTER(i32)]
+    L.kda_prefix_cache_plan.restype = i64
+    L.kda_prefix_cache_plan.argtypes = [vp, i64, i64, vp, i64]
+    L.kda_prefix_cache_insert.restype = i32
+    L.kda_prefix_cache_insert.argtypes = [vp, vp, i64, vp, i64, vp]
+    L.kda_prefix_cache_stats.restype = i32
+    L.kda_prefix_cache_stats.argtypes = [vp, i64p, ctypes.POINTER(i32)]
     L.kda_segment_compose.restype = i32
     L.kda_segment_compose.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]
     L.kda_ckpt_offsets.restype = i32
@@ -356,3 +374,74 @@ def kda_selftest_umma(a, b, d, *, b_mn_major=False, stream=None):
     _check(_load().kda_selftest_umma(_p(a), _p(b), _p(d), n, int(bool(b_mn_major)), _stream(stream)),
            "kda_selftest_umma")
     return d
+
+
+# ---------------------------------------------------------------------------------------------- prefix reuse
+def _host_array(x, dtype):
+    import numpy as np
+    a = np.ascontiguousarray(x.cpu().numpy() if isinstance(x, torch.Tensor) else np.asarray(x), dtype=dtype)
+    return a
+
+
+def kda_prefix_block_hashes(tokens, seed=0):
+    """Chained FNV-1a hashes of the full 512-token blocks of `tokens` (C: kda_prefix_block_hashes).
+    Returns a numpy uint64 array of len(tokens) // 512 entries."""
+    import numpy as np
+    t = _host_array(tokens, np.int32)
+    out = np.zeros(max(len(t) // KDA_PREFIX_BLOCK, 1), dtype=np.uint64)
+    n = _load().kda_prefix_block_hashes(t.ctypes.data, len(t), int(seed) & (2 ** 64 - 1), out.ctypes.data)
+    if n < 0:
+        raise KDAError(-1, "kda_prefix_block_hashes")
+    return out[:n]
+
+
+def kda_prefix_cache_create(max_blocks, n_slots, unit_blocks):
+    """Opaque prefix-reuse directory handle (C: kda_prefix_cache_create); free it with kda_prefix_cache_destroy."""
+    h = ctypes.c_void_p()
+    _check(_load().kda_prefix_cache_create(int(max_blocks), int(n_slots), int(unit_blocks), ctypes.byref(h)),
+           "kda_prefix_cache_create")
+    return h
+
+
+def kda_prefix_cache_destroy(cache):
+    _load().kda_prefix_cache_destroy(cache)
+
+
+def kda_prefix_cache_lookup(cache, hashes):
+    """(matched_blocks, resume_blocks, resume_slot) for a request's block hashes (C: kda_prefix_cache_lookup)."""
+    import numpy as np
+    h = _host_array(hashes, np.uint64)
+    m, r, sl = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32()
+    _check(_load().kda_prefix_cache_lookup(cache, h.ctypes.data, len(h), ctypes.byref(m), ctypes.byref(r),
+                                           ctypes.byref(sl)), "kda_prefix_cache_lookup")
+    return m.value, r.value, sl.value
+
+
+def kda_prefix_cache_plan(cache, n_blocks, resume_blocks):
+    """Block ends after which a request stores its state (C: kda_prefix_cache_plan)."""
+    import numpy as np
+    n = _load().kda_prefix_cache_plan(cache, int(n_blocks), int(resume_blocks), None, 0)
+    if n < 0:
+        raise KDAError(-1, "kda_prefix_cache_plan")
+    out = np.zeros(max(n, 1), dtype=np.int64)
+    _load().kda_prefix_cache_plan(cache, int(n_blocks), int(resume_blocks), out.ctypes.data, n)
+    return out[:n].tolist()
+
+
+def kda_prefix_cache_insert(cache, hashes, ends):
+    """Record a processed request; returns the slot of each planned end, -1 where none could be freed
+    (C: kda_prefix_cache_insert)."""
+    import numpy as np
+    h = _host_array(hashes, np.uint64)
+    e = _host_array(ends, np.int64)
+    out = np.full(max(len(e), 1), -1, dtype=np.int32)
+    _check(_load().kda_prefix_cache_insert(cache, h.ctypes.data, len(h), e.ctypes.data, len(e), out.ctypes.data),
+           "kda_prefix_cache_insert")
+    return out[:len(e)].tolist()
+
+
+def kda_prefix_cache_stats(cache):
+    """(cached block hashes, slots in use) (C: kda_prefix_cache_stats)."""
+    nb, ns = ctypes.c_int64(), ctypes.c_int32()
+    _check(_load().kda_prefix_cache_stats(cache, ctypes.byref(nb), ctypes.byref(ns)), "kda_prefix_cache_stats")
+    return nb.value, ns.value

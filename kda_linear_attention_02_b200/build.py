@@ -2,8 +2,9 @@
 
     python -m kda_linear_attention_02_b200.build [--force]
 
-Each csrc/*.cu is compiled to an object under _build/ and linked into kda_linear_attention_02_b200/libkda.so
-(static CUDA runtime, position-independent).  Objects are rebuilt when their source or any header
+Each csrc/*.cu is compiled by nvcc, and each csrc/*.cpp (host-only code) by the host C++ compiler, to an
+object under _build/; all are linked into kda_linear_attention_02_b200/libkda.so (static CUDA runtime,
+position-independent).  Objects are rebuilt when their source or any header
 changed.
 """
 from __future__ import annotations
@@ -21,6 +22,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkda.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+CXX = os.environ.get("CXX", "g++")
+CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-fvisibility=hidden", "-Wall", "-I", INCLUDE]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -54,13 +57,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
         objs.append(obj)
         if force or _stale(obj, [src] + hdrs):
             jobs.append([NVCC, *NVCC_FLAGS, "-c", src, "-o", obj])
+    for src in sorted(glob.glob(os.path.join(CSRC, "*.cpp"))):
+        obj = os.path.join(BUILD, os.path.basename(src)[:-4] + ".host.o")
+        objs.append(obj)
+        if force or _stale(obj, [src] + hdrs):
+            jobs.append([CXX, *CXX_FLAGS, "-c", src, "-o", obj])
 
     def run(cmd):
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
-            raise RuntimeError(f"nvcc failed for {cmd[-3]}:\n{r.stdout}\n{r.stderr}")
+            raise RuntimeError(f"{os.path.basename(cmd[0])} failed for {cmd[-3]}:\n{r.stdout}\n{r.stderr}")
         return r.stderr
 
     with ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as ex:
