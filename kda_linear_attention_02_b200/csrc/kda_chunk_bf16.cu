@@ -163,8 +163,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tmem_alloc(&tmem_slot, 256);
         tmem_relinquish();
     }
-    // identity rows 0..63 of [I; Aqk] (rows 64..127 are rewritten for every item)
-    for (int e = t; e < 64 * 8; e += NT) {
+    // identity rows 0..63 of [I; Aqk]; rows 64..127 start at zero and every item rewrites only the columns of
+    // its row tile's variant (the Aqk entries past them are always zero)
+    for (int e = t; e < 128 * 8; e += NT) {
         const int r = e >> 3, sc = e & 7;
         uint4 z = make_uint4(0u, 0u, 0u, 0u);
         if ((r >> 3) == sc) {
@@ -355,35 +356,37 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         ph_mma ^= 1;
         tc_fence_after();
 
-        // ---------------- TMEM -> fp32 A (strict lower, beta rows) and bf16 Aqk (inclusive lower) into [I; Aqk]
-        if (w < 8) {
-            const int qw = w & 3, role = w >> 2;
-            const int vi = 2 * (qw & 1) + role;
-            const int nv = 16 * (vi + 1);
-            const int off = 8 * vi * (vi + 1);
+        // ---------------- TMEM -> fp32 A (strict lower, beta rows) and bf16 Aqk (inclusive lower) into [I; Aqk].
+        // Lane quarter qw holds the rows of tiles t0 = 2 (qw & 1) and t0 + 1 (K rows for qw < 2, Q rows
+        // otherwise).  Their variant columns form 2 t0 + 3 chunks of 16 (t0 + 1 of tile t0, t0 + 2 of tile
+        // t0 + 1), spread over the lane quarter's four warps, at most two per warp, loaded before one wait.
+        {
+            const int qw = w & 3, sub = w >> 2;
+            const int t0 = 2 * (qw & 1), nchunk = 2 * t0 + 3;
             const int r = (32 * qw + lane) & 63;
             const bool is_q = qw >= 2;
-            const bool mine = (lane >> 4) == role;
             const float br = bet[r];
+            float v2[32];
+            int tile_of[2], cb_of[2];
 #pragma unroll
-            for (int cb2 = 0; cb2 < 64; cb2 += 32) {
-                float v2[32];   // two 16-column loads in flight per wait
+            for (int hb = 0; hb < 2; ++hb) {
+                const int j = sub + 4 * hb;
+                tile_of[hb] = j < t0 + 1 ? t0 : t0 + 1;
+                cb_of[hb] = 16 * (j < t0 + 1 ? j : j - t0 - 1);
+                if (j < nchunk) {
+                    tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 8 * tile_of[hb] * (tile_of[hb] + 1) + cb_of[hb],
+                              *reinterpret_cast<float(*)[16]>(v2 + 16 * hb));
+                } else {
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    if (cb2 + 16 * hb < nv) {
-                        tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + off + cb2 + 16 * hb,
-                                  *reinterpret_cast<float(*)[16]>(v2 + 16 * hb));
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) v2[16 * hb + j] = 0.f;
-                    }
+                    for (int e = 0; e < 16; ++e) v2[16 * hb + e] = 0.f;
                 }
-                tmem_wait_ld_regs<32>(v2);
+            }
+            tmem_wait_ld_regs<32>(v2);
 #pragma unroll
-              for (int hb = 0; hb < 2; ++hb) {
-                const int cb = cb2 + 16 * hb;
+            for (int hb = 0; hb < 2; ++hb) {
+                const int cb = cb_of[hb];
                 const float* v = v2 + 16 * hb;
-                if (mine) {
+                if (sub + 4 * hb < nchunk && (r >> 4) == tile_of[hb]) {   // this lane's row belongs to the chunk's tile
                     if (is_q) {
                         float o8[8];
 #pragma unroll
@@ -399,14 +402,13 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                             const int s = cb + j;
                             if (s < r) AM[s * LDM + r] = br * v[j];
                         }
-                    } else if ((cb >> 4) < (r >> 4)) {    // off-diagonal block: row-major
+                    } else {                              // off-diagonal block: row-major
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4)
                             reinterpret_cast<float4*>(AM + r * LDM + cb)[q4] =
                                 make_float4(br * v[4 * q4], br * v[4 * q4 + 1], br * v[4 * q4 + 2], br * v[4 * q4 + 3]);
                     }
                 }
-              }
             }
         }
         tc_fence_before();
