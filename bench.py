@@ -259,26 +259,63 @@ def run_ours(args):
     hfs = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hla, hb))
     d2h = ho.numel() * ho.element_size() + hfs.numel() * hfs.element_size()
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e_steps = max(2, min(args.steps, 6))
+    # Pipelined through the public C ABI: step i's inputs go up on one stream while step i - 1 computes and
+    # its o and final state come down on a third; two device buffer sets alternate, ordered by events.
+    # Every step still uploads its own inputs and downloads its own results inside the timed region.
+    bufs = [(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, o, fs)]
+    bufs.append(tuple(torch.empty_like(t) for t in bufs[0]))
+    ws2 = ws
+    s_up, s_cmp, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {k_: [torch.cuda.Event() for _ in range(2)] for k_ in ("up", "cmp", "dn")}
+    ho2 = [ho, torch.empty_like(ho, pin_memory=True)]
+    hfs2 = [hfs, torch.empty_like(hfs, pin_memory=True)]
+    first_use = [True, True]
 
-    def e2e_step():
-        inp.q.copy_(hq, non_blocking=True); inp.k.copy_(hk, non_blocking=True); inp.v.copy_(hv, non_blocking=True)
-        inp.log_alpha.copy_(hla, non_blocking=True); inp.beta.copy_(hb, non_blocking=True)
-        step()
-        ho.copy_(o, non_blocking=True); hfs.copy_(fs, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        q_, k_, v_, la_, b_, o_, fs_ = bufs[b]
+        with torch.cuda.stream(s_up):
+            if not first_use[b]:
+                s_up.wait_event(ev["cmp"][b])          # step i - 2 has finished reading this input set
+            for d_, h_ in ((q_, hq), (k_, hk), (v_, hv), (la_, hla), (b_, hb)):
+                d_.copy_(h_, non_blocking=True)
+            ev["up"][b].record(s_up)
+        s_cmp.wait_event(ev["up"][b])
+        if not first_use[b]:
+            s_cmp.wait_event(ev["dn"][b])              # step i - 2's results have left this output set
+        kda.kda_chunk_fwd(q_, k_, v_, la_, b_, None, inp.cu_seqlens, o_, fs_, ckpt_stride=CKPT, checkpoints=ck,
+                          ckpt_cu=ckcu, workspace=ws2, stream=s_cmp)
+        ev["cmp"][b].record(s_cmp)
+        with torch.cuda.stream(s_dn):
+            s_dn.wait_event(ev["cmp"][b])
+            ho2[b].copy_(o_, non_blocking=True)
+            hfs2[b].copy_(fs_, non_blocking=True)
+            ev["dn"][b].record(s_dn)
+        first_use[b] = False
 
-    e2e_step()
-    torch.cuda.synchronize()
+    def drain():
+        for st in (s_up, s_cmp, s_dn):
+            st.synchronize()
+
+    for i in range(2):
+        e2e_step(i)
+    drain()
     barrier(world)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_cmp)
+    s_up.wait_event(e0)
+    s_dn.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    s_cmp.wait_stream(s_up)
+    s_cmp.wait_stream(s_dn)
+    e1.record(s_cmp)
+    drain()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     e2e = {"value": tokens_job / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
-    del hq, hk, hv, hla, hb, ho, hfs
+    del hq, hk, hv, hla, hb, ho, hfs, ho2, hfs2, bufs
 
     # ------------------------------------------------------------------ decode workload
     s0, dq, dk_, dv_, dla, db = synth.make_decode_inputs(DEC_N, H, D, D, dtype=torch.bfloat16, device=dev,
