@@ -160,7 +160,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         prefetch_tmap(&map_q); prefetch_tmap(&map_k); prefetch_tmap(&map_v); prefetch_tmap(&map_l);
     }
     if (w == 0) {
-        tmem_alloc(&tmem_slot, 256);
+        tmem_alloc(&tmem_slot, 512);   // one CTA per SM (its shared memory): all of the SM's TMEM
         tmem_relinquish();
     }
     // identity rows 0..63 of [I; Aqk]; rows 64..127 start at zero and every item rewrites only the columns of
@@ -300,7 +300,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                                pack2(__fmul2_rn(kF, make_float2(dvx[i], dvy[i]))));
                 // Q * gamma for the epilogue (P = Q gamma - ...)
                 st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2, pack2(__fmul2_rn(qf, G)));
-                const float2 tk2 = __fmul2_rn(__fmul2_rn(bt, kf), G);
+                const float2 tk2 = __fmul2_rn(__fmul2_rn(make_float2(-bt.x, -bt.y), kf), G);   // -beta K gamma
                 const float2 tv2 = __fmul2_rn(bt, vf);
                 const float2 td2 = __fmul2_rn(kF, ec2);
                 tk[0][j] = tk2.x; tk[1][j] = tk2.y;
@@ -448,11 +448,34 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
                 for (int r = 0; r < 16; ++r) XF[(o0 + r) * LDX + o0 + col] = x[r];
             }
-        } else {
-            for (int e = t - 128; e < 64 * 64; e += NT - 128) {   // the blocks above the diagonal are zero
+        } else if (w < 8) {
+            for (int e = t - 128; e < 64 * 64; e += 128) {   // the blocks above the diagonal are zero
                 const int r = e >> 6, c = e & 63;
                 if ((c >> 4) > (r >> 4)) XF[r * LDX + c] = 0.f;
             }
+        } else {
+            // meanwhile: product B's K-part accumulator (TMEM columns 0..127, free since the A epilogue)
+            // starts as [0; Q gamma], so that it ends as [-W; P] with P = Q gamma - Aqk W
+            const int qw = w & 3, half = (w - 8) >> 2;
+            const uint32_t base = tm + (static_cast<uint32_t>(32 * qw) << 16) + 64 * half;
+            const int r = 32 * qw + lane - 64;   // token row of the Q part (lane quarters 2 and 3)
+#pragma unroll
+            for (int c16 = 0; c16 < 4; ++c16) {
+                float x[16];
+                if (qw >= 2) {
+                    const int ch = (64 * half + 16 * c16) >> 3;   // first 8-channel chunk of the 16 columns
+                    float a8[8], b8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + ((ch ^ (r & 7)) << 4)), a8);
+                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + (((ch + 1) ^ (r & 7)) << 4)), b8);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) { x[j] = a8[j]; x[8 + j] = b8[j]; }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) x[j] = 0.f;
+                }
+                tmem_st16(base + 16 * c16, x);
+            }
+            // completion is waited for at the end of level 1, so the stores drain behind both levels
         }
         __syncthreads();
         // Levels 1 and 2 merge two inverted diagonal blocks: X_10 = -X_11 (A_10 X_00).  The products are
@@ -492,6 +515,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             xo[fg * LDX + 1] = -e[1];
             xo[(fg + 8) * LDX] = -e[2];
             xo[(fg + 8) * LDX + 1] = -e[3];
+        } else if (w >= 8) {   // the accumulator preload of level 0 has landed
+            tmem_wait_st();
+            tc_fence_before();
         }
         __syncthreads();
         if (w < 8) {   // level 2: 32 -> 64, row tile mt of 16 and column tile nt of 8
@@ -550,7 +576,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const uint32_t idesc = idesc_bf16(128, 64);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tm, sdesc_k_sw128(ia + ks * 32), sdesc_k_sw128(xt + ks * 32), idesc, ks > 0);
+                umma_f16(tm + 256, sdesc_k_sw128(ia + ks * 32), sdesc_k_sw128(xt + ks * 32), idesc, ks > 0);
             umma_commit(&bar_mma);
         }
         {
@@ -563,7 +589,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const int qw = w & 3, cg = w >> 2;
             const int m = 32 * qw + lane;
             float v[16];
-            tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 16 * cg, v);
+            tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 256 + 16 * cg, v);
             tmem_wait_ld_regs<16>(v);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -578,14 +604,18 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---------------- phase B: D[m, n] = [X; Y][m, :] . [beta K gamma | beta V]^T[n, :]  (N = 128 + DV, K = 64)
+        // ---------------- phase B: D[m, n] = [X; Y][m, :] . [-beta K gamma | beta V]^T[n, :]  (K = 64): the
+        // K part (N = 128) onto the preloaded [0; Q gamma], the V part (N = DV) from zero
         if (t == 0) {
             tc_fence_after();
             const uint32_t xa = smem_u32(sm + ps::XY), kb = smem_u32(sm + ps::BKV);
-            const uint32_t idesc = idesc_bf16(128, 128 + DV);
+            const uint32_t idk = idesc_bf16(128, 128), idv = idesc_bf16(128, DV);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tm, sdesc_k_sw128(xa + ks * 32), sdesc_k_sw128(kb + ks * 32), idesc, ks > 0);
+                umma_f16(tm, sdesc_k_sw128(xa + ks * 32), sdesc_k_sw128(kb + ks * 32), idk, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma_f16(tm + 128, sdesc_k_sw128(xa + ks * 32), sdesc_k_sw128(kb + 128 * 128 + ks * 32), idv, ks > 0);
             umma_commit(&bar_mma);
         }
         {
@@ -595,7 +625,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         ph_mma ^= 1;
         tc_fence_after();
 
-        // ---------------- epilogue: rows 0..63 -> -W | U, rows 64..127 -> P = Q gamma - Y bK gamma | O_intra
+        // ---------------- epilogue: rows 0..63 -> -W | U, rows 64..127 -> P | O_intra, all straight from TMEM
         {
             const int qw = w & 3, cg = w >> 2;   // 64-column group: 0,1 -> K part, 2,3 -> V part
             const int m = 32 * qw + lane;
@@ -613,16 +643,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         const int cc = 4 * c32 + sub;
                         const float* v = vv;
                         float o8[8];
-                        if (m < 64) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) o8[j] = -v[8 * sub + j];
-                        } else {
-                            const int r = m - 64;
-                            float q8[8];
-                            unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + ((cc ^ (r & 7)) << 4)), q8);
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) o8[j] = q8[j] - v[8 * sub + j];
-                        }
+                        for (int j = 0; j < 8; ++j) o8[j] = v[8 * sub + j];
                         *reinterpret_cast<uint4*>(sm + ps::AWS + (cc >> 3) * 16384 + m * 128 +
                                                   (((cc & 7) ^ (m & 7)) << 4)) = pack8(o8);
                     }
@@ -679,7 +701,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     }
     tc_fence_before();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tm, 256);
+    if (w == 0) tmem_dealloc(tm, 512);
 }
 
 // ------------------------------------------------------------------------------------------------
