@@ -40,7 +40,7 @@ struct DecodeTiling {
 // threads still read token t's values.
 template <int DK, int DV, int NT>
 struct DecodeSmem {
-    float a[2][DK], k[2][DK], q[2][DK], v[2][DV], u[2][DV], beta[2];
+    float a[2][DK], k[2][DK], q[2][DK], ak[2][DK], aq[2][DK], v[2][DV], u[2][DV], beta[2];
     float4 red[2][DecodeTiling<DK, DV, NT>::RG][DecodeTiling<DK, DV, NT>::CG];
     float kq;
 };
@@ -68,9 +68,14 @@ template <int DK, int DV, int NT, bool OUT>
 __device__ __forceinline__ void stage_token(DecodeSmem<DK, DV, NT>& sh, int par, const TokenIn& x) {
     const int t = threadIdx.x;
     if (t < DK) {
-        sh.a[par][t] = __expf(floor_log_decay(x.la));
+        const float a = __expf(floor_log_decay(x.la));
+        sh.a[par][t] = a;
         sh.k[par][t] = x.k;
-        if (OUT) sh.q[par][t] = x.q;
+        sh.ak[par][t] = a * x.k;   // the row weights of the two column sums, formed once per row
+        if (OUT) {
+            sh.q[par][t] = x.q;
+            sh.aq[par][t] = a * x.q;
+        }
     }
     if (t < DV) sh.v[par][t] = x.v;
     if (t == 0) sh.beta[par] = x.beta;
@@ -84,19 +89,22 @@ __device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>:
     using DT = DecodeTiling<DK, DV, NT>;
     constexpr int CG = DT::CG, RG = DT::RG, RPT = DT::RPT;
     const int t = threadIdx.x, cg = t % CG, rg = t / CG;
-    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+    // column sums against alpha k and alpha q, two lanes per packed fp32 FMA
+    float2 pk01 = make_float2(0.f, 0.f), pk23 = pk01, pq01 = pk01, pq23 = pk01;
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int i = rg + r * RG;
-        const float ak = sh.a[par][i] * sh.k[par][i];
-        pk.x = fmaf(ak, s[r].x, pk.x); pk.y = fmaf(ak, s[r].y, pk.y);
-        pk.z = fmaf(ak, s[r].z, pk.z); pk.w = fmaf(ak, s[r].w, pk.w);
+        const float ak = sh.ak[par][i];
+        pk01 = __ffma2_rn(make_float2(ak, ak), make_float2(s[r].x, s[r].y), pk01);
+        pk23 = __ffma2_rn(make_float2(ak, ak), make_float2(s[r].z, s[r].w), pk23);
         if (OUT) {
-            const float aq = sh.a[par][i] * sh.q[par][i];
-            pq.x = fmaf(aq, s[r].x, pq.x); pq.y = fmaf(aq, s[r].y, pq.y);
-            pq.z = fmaf(aq, s[r].z, pq.z); pq.w = fmaf(aq, s[r].w, pq.w);
+            const float aq = sh.aq[par][i];
+            pq01 = __ffma2_rn(make_float2(aq, aq), make_float2(s[r].x, s[r].y), pq01);
+            pq23 = __ffma2_rn(make_float2(aq, aq), make_float2(s[r].z, s[r].w), pq23);
         }
     }
+    const float4 pk = make_float4(pk01.x, pk01.y, pk23.x, pk23.y);
+    const float4 pq = make_float4(pq01.x, pq01.y, pq23.x, pq23.y);
     sh.red[0][rg][cg] = pk;
     if (OUT) {
         sh.red[1][rg][cg] = pq;
@@ -129,14 +137,15 @@ __device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>:
     __syncthreads();
 
     const float4 u4 = reinterpret_cast<const float4*>(sh.u[par])[cg];
+    const float2 u01 = make_float2(u4.x, u4.y), u23 = make_float2(u4.z, u4.w);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int i = rg + r * RG;
         const float a = sh.a[par][i], kk = sh.k[par][i];
-        s[r].x = fmaf(a, s[r].x, kk * u4.x);
-        s[r].y = fmaf(a, s[r].y, kk * u4.y);
-        s[r].z = fmaf(a, s[r].z, kk * u4.z);
-        s[r].w = fmaf(a, s[r].w, kk * u4.w);
+        const float2 a2 = make_float2(a, a), k2 = make_float2(kk, kk);
+        const float2 s01 = __ffma2_rn(a2, make_float2(s[r].x, s[r].y), __fmul2_rn(k2, u01));
+        const float2 s23 = __ffma2_rn(a2, make_float2(s[r].z, s[r].w), __fmul2_rn(k2, u23));
+        s[r] = make_float4(s01.x, s01.y, s23.x, s23.y);
     }
 }
 
