@@ -83,9 +83,10 @@ __device__ __forceinline__ void stage_token(DecodeSmem<DK, DV, NT>& sh, int par,
 
 // One token applied to the register-held state s (thread t holds rows rg + r RG, columns 4 cg ..),
 // its inputs staged in sh[par] and made visible by a barrier.  OUT: also o = S_t^T q for this token.
+// update = false skips the rank-1 update (the output needs only the column sums and u).
 template <typename T, int DK, int DV, int NT, bool OUT>
 __device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>::RPT], DecodeSmem<DK, DV, NT>& sh,
-                                           int par, T* __restrict__ o) {
+                                           int par, T* __restrict__ o, bool update = true) {
     using DT = DecodeTiling<DK, DV, NT>;
     constexpr int CG = DT::CG, RG = DT::RG, RPT = DT::RPT;
     const int t = threadIdx.x, cg = t % CG, rg = t / CG;
@@ -135,6 +136,7 @@ __device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>:
         }
     }
     __syncthreads();
+    if (!update) return;
 
     const float4 u4 = reinterpret_cast<const float4*>(sh.u[par])[cg];
     const float2 u01 = make_float2(u4.x, u4.y), u23 = make_float2(u4.z, u4.w);
@@ -225,7 +227,9 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
         const int par = d & 1;
         if (d + 1 < steps) load(x, d + 1);
         __syncthreads();   // token d staged (and every reader of the other half is past token d - 1)
-        token_step<T, DK, DVS, NT, VERIFY>(s, sh, par, VERIFY ? o + row_of(d) * DV + j0 : nullptr);
+        // verify discards the state: the last draft needs its output only
+        token_step<T, DK, DVS, NT, VERIFY>(s, sh, par, VERIFY ? o + row_of(d) * DV + j0 : nullptr,
+                                           !VERIFY || d + 1 < steps);
         if (d + 1 < steps) stage_token<DK, DVS, NT, VERIFY>(sh, par ^ 1, x);
     }
     if (!VERIFY) {
