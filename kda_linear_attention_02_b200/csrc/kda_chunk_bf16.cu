@@ -26,12 +26,16 @@
 //  prep_bf16_kernel   persistent, one (chunk, head) item at a time per CTA: TMA tensor loads of the
 //                     raw tiles (prefetched one item ahead), SIMT exponentials and operand
 //                     construction, tcgen05 products for A/Aqk (4 anchored variants), for
-//                     [X; Y] = [I; Aqk] X and for [X; Y] (beta K gamma | beta V), fp32 blocked
-//                     forward substitution for X, and a bulk TMA store of the MMA-ready packet.
+//                     [X; Y] = [I; Aqk] X and for [X; Y] (-beta K gamma | beta V) onto an
+//                     accumulator preloaded with [0; Q gamma] (so that it yields [-W; P]), X by
+//                     forward substitution of the four 16 x 16 diagonal blocks and two merge levels
+//                     on warp-level tf32 MMAs, and a bulk TMA store of the MMA-ready packet.
 //  state_bf16_kernel  one CTA per (sequence, head, dv-slice), warp-specialised: a producer warp
 //                     streams packets through a shared-memory ring with bulk TMA, one thread issues
-//                     the two tcgen05 products per chunk, 8 or 16 epilogue warps hold the fp32 state
-//                     in registers and feed bf16 copies of S and U' back as the next operands.
+//                     the tcgen05 products per chunk (copies of U and O_intra into a double-buffered
+//                     accumulator, then [-W; P] S onto them, then Kdec^T U'), 8 or 16 epilogue warps
+//                     hold the fp32 state in registers and feed bf16 copies of S and U' back as the
+//                     next operands.
 #include <cudaTypedefs.h>
 
 #include <cstring>
