@@ -418,6 +418,32 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tc_fence_before();
         __syncthreads();
 
+        // Meanwhile warps 8..15, idle in the solve, start product B's K-part accumulator (TMEM columns
+        // 0..127, free since the A epilogue) as [0; Q gamma], so that it ends as [-W; P] with
+        // P = Q gamma - Aqk W.  The TMEM stores are spread over the solve's first two levels and waited
+        // for in the third.
+        auto preload_qgamma = [&](int c_lo, int c_hi) {
+            const int qw = w & 3, half = (w - 8) >> 2;
+            const uint32_t base = tm + (static_cast<uint32_t>(32 * qw) << 16) + 64 * half;
+            const int r = 32 * qw + lane - 64;   // token row of the Q part (lane quarters 2 and 3)
+#pragma unroll
+            for (int c16 = 0; c16 < 4; ++c16) {
+                if (c16 < c_lo || c16 >= c_hi) continue;
+                float x[16];
+                if (qw >= 2) {
+                    const int ch = (64 * half + 16 * c16) >> 3;   // first 8-channel chunk of the 16 columns
+                    float a8[8], b8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + ((ch ^ (r & 7)) << 4)), a8);
+                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + (((ch + 1) ^ (r & 7)) << 4)), b8);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) { x[j] = a8[j]; x[8 + j] = b8[j]; }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) x[j] = 0.f;
+                }
+                tmem_st16(base + 16 * c16, x);
+            }
+        };
         // ---------------- X = (I + A)^-1 by blocked forward substitution over 16 x 16 tiles.
         // Level 0: each diagonal block by forward substitution, one warp per block, lane = column, the
         // column held in registers; a column of A comes as float4 broadcasts of a row of the transposed block.
@@ -458,28 +484,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 if ((c >> 4) > (r >> 4)) XF[r * LDX + c] = 0.f;
             }
         } else {
-            // meanwhile: product B's K-part accumulator (TMEM columns 0..127, free since the A epilogue)
-            // starts as [0; Q gamma], so that it ends as [-W; P] with P = Q gamma - Aqk W
-            const int qw = w & 3, half = (w - 8) >> 2;
-            const uint32_t base = tm + (static_cast<uint32_t>(32 * qw) << 16) + 64 * half;
-            const int r = 32 * qw + lane - 64;   // token row of the Q part (lane quarters 2 and 3)
-#pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16) {
-                float x[16];
-                if (qw >= 2) {
-                    const int ch = (64 * half + 16 * c16) >> 3;   // first 8-channel chunk of the 16 columns
-                    float a8[8], b8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + ((ch ^ (r & 7)) << 4)), a8);
-                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + (((ch + 1) ^ (r & 7)) << 4)), b8);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) { x[j] = a8[j]; x[8 + j] = b8[j]; }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) x[j] = 0.f;
-                }
-                tmem_st16(base + 16 * c16, x);
-            }
-            // completion is waited for at the end of level 1, so the stores drain behind both levels
+            preload_qgamma(0, 2);
         }
         __syncthreads();
         // Levels 1 and 2 merge two inverted diagonal blocks: X_10 = -X_11 (A_10 X_00).  The products are
@@ -519,9 +524,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             xo[fg * LDX + 1] = -e[1];
             xo[(fg + 8) * LDX] = -e[2];
             xo[(fg + 8) * LDX + 1] = -e[3];
-        } else if (w >= 8) {   // the accumulator preload of level 0 has landed
-            tmem_wait_st();
-            tc_fence_before();
+        } else if (w >= 8) {
+            preload_qgamma(2, 4);
         }
         __syncthreads();
         if (w < 8) {   // level 2: 32 -> 64, row tile mt of 16 and column tile nt of 8
@@ -560,6 +564,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             xo[fg * LDX + 1] = -e[1];
             xo[(fg + 8) * LDX] = -e[2];
             xo[(fg + 8) * LDX + 1] = -e[3];
+        } else {   // the accumulator preload has landed
+            tmem_wait_st();
+            tc_fence_before();
         }
         __syncthreads();
         // X^T as the bf16 B operand of the Y product: row m = column m of X, K = 64 rows of X
