@@ -1001,6 +1001,12 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);   // done with this stage's U, O_intra and gamma
             write_sop();
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_ready);
+            // the checkpoint leaves from registers after the next product has been released, so its
+            // stores drain while product 1 of the next chunk runs
             if (!trans && ckpt_stride > 0 && checkpoints && n == 64) {
                 const long long end = static_cast<long long>(c + 1) * 64;
                 if (end % ckpt_stride == 0) {
@@ -1016,10 +1022,6 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                     }
                 }
             }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_ready);
         }
         if (o_issuer) bulk_wait0();
         // row i, columns j0 + jw .. + NCW: 16-byte stores (every row start and column offset is a multiple of 4)
