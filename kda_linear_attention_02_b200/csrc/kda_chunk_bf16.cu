@@ -187,6 +187,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint32_t ph_load = 0, ph_mma = 0;
     bool load_pending = false;   // meaningful in thread 0 only
 
+    // everything above is private set-up; the chunk table and the inputs come from earlier launches
+    grid_dependency_wait();
     // chunk table entry {first token, valid tokens} of a window item (n = 0: past the last chunk)
     auto entry = [&](long long it) -> int2 { return it < n_items ? chunk_tab[it / H] : make_int2(0, 0); };
     long long item = blockIdx.x;
@@ -755,6 +757,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
     __shared__ __align__(8) uint64_t full[NST], empty[NST], d1_full, d2_full, s_ready, up_ready;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    grid_dependency_wait();   // the packets and the chunk index come from the launches before this one
     const int seq = blockIdx.x / H, h = blockIdx.x % H, slice = blockIdx.y;
     const bool trans = slice >= NSV;
     const int j0 = (trans ? slice - NSV : slice) * DVS;
@@ -1047,6 +1050,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
 // kernel finds any item with one load instead of a search.
 __global__ void chunk_table_kernel(const int32_t* __restrict__ cu_chunks, const int32_t* __restrict__ cu_seqlens,
                                    int n_seqs, long long win_lo, long long win_hi, int2* __restrict__ tab) {
+    grid_dependency_wait();   // the chunk index comes from the launch before this one
     const long long gc = win_lo + static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (gc >= win_hi) return;
     ChunkLoc loc;
@@ -1083,6 +1087,24 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch with programmatic stream serialization: the kernel's blocks may be scheduled while the
+// previous kernel of the stream drains, do their private set-up, and wait (grid_dependency_wait)
+// before touching anything an earlier launch produced.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 int num_sms() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -1102,11 +1124,10 @@ cudaError_t launch_state(const ChunkArgs& a, cudaStream_t s) {
     if (a.total_tokens > 0 &&
         !make_map(&mo, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, a.total_tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    state_bf16_kernel<DV, DVS><<<grid, C::NT, smem, s>>>(
-        static_cast<const uint8_t*>(a.packets), a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, a.win_hi,
-        a.initial_state, static_cast<__nv_bfloat16*>(a.o), mo, a.final_state, a.final_transition, a.ckpt_stride,
-        a.checkpoints, a.ckpt_cu, a.carry, a.status);
-    return cudaGetLastError();
+    return launch_pdl(state_bf16_kernel<DV, DVS>, grid, dim3(C::NT), smem, s, static_cast<const uint8_t*>(a.packets),
+                      a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, a.win_hi, a.initial_state,
+                      static_cast<__nv_bfloat16*>(a.o), mo, a.final_state, a.final_transition, a.ckpt_stride,
+                      a.checkpoints, a.ckpt_cu, a.carry, a.status);
 }
 
 template <int DV>
@@ -1124,14 +1145,12 @@ cudaError_t launch_bf16_t(const ChunkArgs& a, cudaStream_t s) {
         cudaError_t e = cudaFuncSetAttribute(prep_bf16_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         const long long wchunks = a.win_hi - a.win_lo;
-        chunk_table_kernel<<<static_cast<unsigned>((wchunks + 255) / 256), 256, 0, s>>>(
-            a.cu_chunks, a.cu_seqlens, a.n_seqs, a.win_lo, a.win_hi, a.chunk_tab);
-        e = cudaGetLastError();
+        e = launch_pdl(chunk_table_kernel, dim3(static_cast<unsigned>((wchunks + 255) / 256)), dim3(256), 0, s,
+                       a.cu_chunks, a.cu_seqlens, a.n_seqs, a.win_lo, a.win_hi, a.chunk_tab);
         if (e != cudaSuccess) return e;
         const long long grid = items < num_sms() ? items : num_sms();
-        prep_bf16_kernel<DV><<<static_cast<unsigned>(grid), ps::NT, smem, s>>>(
-            mq, mk, mv, ml, a.beta, a.chunk_tab, a.H, items, static_cast<uint8_t*>(a.packets), a.status);
-        e = cudaGetLastError();
+        e = launch_pdl(prep_bf16_kernel<DV>, dim3(static_cast<unsigned>(grid)), dim3(ps::NT), smem, s, mq, mk, mv, ml,
+                       a.beta, a.chunk_tab, a.H, items, static_cast<uint8_t*>(a.packets), a.status);
         if (e != cudaSuccess) return e;
     }
     if (a.events) cudaEventRecord(a.events->ev[2], s);

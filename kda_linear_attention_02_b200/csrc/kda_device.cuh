@@ -124,6 +124,11 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int c0, int
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may start
+// while the previous kernel of the stream is still finishing; this waits until that kernel has
+// completed and its memory is visible (a no-op for an ordinary launch).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
