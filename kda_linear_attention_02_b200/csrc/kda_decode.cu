@@ -158,6 +158,7 @@ decode_step_kernel(float* __restrict__ state, const T* __restrict__ q, const T* 
                    const float* __restrict__ beta, T* __restrict__ o) {
     using DT = DecodeTiling<DK, DV, 256>;
     __shared__ DecodeSmem<DK, DV, 256> sh;
+    grid_dependency_wait();   // the state (and inputs) come from earlier launches
     const int head = blockIdx.x;   // sequence * H + h
     const int t = threadIdx.x, cg = t % DT::CG, rg = t / DT::CG;
     float4* S = reinterpret_cast<float4*>(state + static_cast<size_t>(head) * DK * DV);
@@ -196,6 +197,7 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
     using DT = DecodeTiling<DK, DVS, NT>;
     static_assert(DT::RG == DecodeTiling<DK, DV, 256>::RG, "same row groups as the single step");
     __shared__ DecodeSmem<DK, DVS, NT> sh;
+    grid_dependency_wait();   // the state, counts and drafts come from earlier launches
     const int head = blockIdx.x;   // sequence * H + h
     const int seq = head / H, h = head % H, j0 = blockIdx.y * DVS;
     const int t = threadIdx.x, cg = t % DT::CG, rg = t / DT::CG;
@@ -238,12 +240,28 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
     }
 }
 
+// Consecutive decode launches are chained (programmatic stream serialization): the next kernel's
+// blocks may be scheduled while the previous one drains and wait (grid_dependency_wait) before any
+// memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 template <typename T, int DK, int DV>
 cudaError_t launch_decode_t(float* state, const void* q, const void* k, const void* v, const float* la,
                             const float* beta, void* o, int nh, cudaStream_t s) {
-    decode_step_kernel<T, DK, DV><<<nh, 256, 0, s>>>(state, static_cast<const T*>(q), static_cast<const T*>(k),
-                                                    static_cast<const T*>(v), la, beta, static_cast<T*>(o));
-    return cudaGetLastError();
+    return launch_chained(decode_step_kernel<T, DK, DV>, dim3(nh), dim3(256), s, state, static_cast<const T*>(q),
+                          static_cast<const T*>(k), static_cast<const T*>(v), la, beta, static_cast<T*>(o));
 }
 
 template <typename T, int DK, int DV>
@@ -253,14 +271,12 @@ cudaError_t launch_multi_t(float* state, const void* q, const void* k, const voi
     const T* qq = static_cast<const T*>(q);
     const T* kk = static_cast<const T*>(k);
     const T* vv = static_cast<const T*>(v);
-    const dim3 grid(n * H, DV / kSpecSlice);
+    const dim3 grid(n * H, DV / kSpecSlice), block(spec_threads<DV>());
     if (n_accept)
-        decode_multi_kernel<T, DK, DV, false><<<grid, spec_threads<DV>(), 0, s>>>(state, qq, kk, vv, la, beta, H, n_draft, n_accept,
-                                                                  nullptr, status);
-    else
-        decode_multi_kernel<T, DK, DV, true><<<grid, spec_threads<DV>(), 0, s>>>(state, qq, kk, vv, la, beta, H, n_draft, nullptr,
-                                                                 static_cast<T*>(o), status);
-    return cudaGetLastError();
+        return launch_chained(decode_multi_kernel<T, DK, DV, false>, grid, block, s, state, qq, kk, vv, la, beta, H,
+                              n_draft, n_accept, static_cast<T*>(nullptr), status);
+    return launch_chained(decode_multi_kernel<T, DK, DV, true>, grid, block, s, state, qq, kk, vv, la, beta, H,
+                          n_draft, static_cast<const int32_t*>(nullptr), static_cast<T*>(o), status);
 }
 
 }  // namespace
