@@ -25,9 +25,11 @@ namespace kda {
 
 namespace {
 
-// NT threads over a DK x DV state block: thread t holds float4 column group t % CG of rows
-// t / CG + r RG.  The column sums run over the same row groups in the same order whenever RG is the
-// same, so a 128-thread CTA over 64 columns reduces exactly like a 256-thread CTA over 128 columns.
+// NT threads over a DK x DV state block: thread t holds float4 column group t % CG of the RPT
+// consecutive rows (t / CG) RPT .. (t / CG) RPT + RPT - 1, so the per-row weights of a token come
+// as 16-byte shared loads.  The column sums run over the same row groups in the same order whenever RG
+// (and so RPT) is the same, so a 128-thread CTA over 64 columns reduces exactly like a 256-thread CTA
+// over 128 columns.
 template <int DK, int DV, int NT>
 struct DecodeTiling {
     static constexpr int CG = DV / 4;     // float4 column groups
@@ -94,7 +96,7 @@ __device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>:
     float2 pk01 = make_float2(0.f, 0.f), pk23 = pk01, pq01 = pk01, pq23 = pk01;
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
-        const int i = rg + r * RG;
+        const int i = rg * RPT + r;
         const float ak = sh.ak[par][i];
         pk01 = __ffma2_rn(make_float2(ak, ak), make_float2(s[r].x, s[r].y), pk01);
         pk23 = __ffma2_rn(make_float2(ak, ak), make_float2(s[r].z, s[r].w), pk23);
@@ -142,7 +144,7 @@ __device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>:
     const float2 u01 = make_float2(u4.x, u4.y), u23 = make_float2(u4.z, u4.w);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
-        const int i = rg + r * RG;
+        const int i = rg * RPT + r;
         const float a = sh.a[par][i], kk = sh.k[par][i];
         const float2 a2 = make_float2(a, a), k2 = make_float2(kk, kk);
         const float2 s01 = __ffma2_rn(a2, make_float2(s[r].x, s[r].y), __fmul2_rn(k2, u01));
@@ -164,7 +166,7 @@ decode_step_kernel(float* __restrict__ state, const T* __restrict__ q, const T* 
     float4* S = reinterpret_cast<float4*>(state + static_cast<size_t>(head) * DK * DV);
     float4 s[DT::RPT];
 #pragma unroll
-    for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg + r * DT::RG) * DT::CG + cg);
+    for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg * DT::RPT + r) * DT::CG + cg);
     const size_t hk = static_cast<size_t>(head) * DK, hv = static_cast<size_t>(head) * DV;
     TokenIn x;
     load_token<T, DK, DV, true>(x, q + hk, k + hk, v + hv, log_alpha + hk, beta + head);
@@ -172,7 +174,7 @@ decode_step_kernel(float* __restrict__ state, const T* __restrict__ q, const T* 
     __syncthreads();
     token_step<T, DK, DV, 256, true>(s, sh, 0, o + hv);
 #pragma unroll
-    for (int r = 0; r < DT::RPT; ++r) __stcs(S + (rg + r * DT::RG) * DT::CG + cg, s[r]);
+    for (int r = 0; r < DT::RPT; ++r) __stcs(S + (rg * DT::RPT + r) * DT::CG + cg, s[r]);
 }
 
 // Draft inputs are token-major per sequence: token (i, d) of sequence i at row i * n_draft + d of
@@ -214,7 +216,7 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
     float4* S = reinterpret_cast<float4*>(state + static_cast<size_t>(head) * DK * DV + j0);
     float4 s[DT::RPT];
 #pragma unroll
-    for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg + r * DT::RG) * (DV / 4) + cg);
+    for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg * DT::RPT + r) * (DV / 4) + cg);
     // token d + 1's inputs are loaded into registers while token d is applied, then staged
     auto row_of = [&](int d) { return (static_cast<size_t>(seq) * n_draft + d) * H + h; };
     auto load = [&](TokenIn& x, int d) {
@@ -236,7 +238,7 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
     }
     if (!VERIFY) {
 #pragma unroll
-        for (int r = 0; r < DT::RPT; ++r) __stcs(S + (rg + r * DT::RG) * (DV / 4) + cg, s[r]);
+        for (int r = 0; r < DT::RPT; ++r) __stcs(S + (rg * DT::RPT + r) * (DV / 4) + cg, s[r]);
     }
 }
 
