@@ -52,6 +52,13 @@ def _load():
         lib.oracle_segment_compose.argtypes = [
             ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_ubyte]
+        lib.oracle_e8m0_value.restype = ctypes.c_double
+        lib.oracle_e8m0_value.argtypes = [ctypes.c_ubyte]
+        lib.oracle_mxfp8_decode.restype = ctypes.c_int
+        lib.oracle_mxfp8_decode.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         del dp
         _lib = lib
     return _lib
@@ -109,6 +116,31 @@ def kda_seq(q, k, v, log_alpha, beta, s0=None, *, marks=None, want_o=True,
         out["marks"] = ms
     if want_transition:
         out["transition"] = tr
+    return out
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one FP8 E4M3 code (OCP MX v1.0 element type)."""
+    return _load().oracle_e4m3_value(int(code))
+
+
+def e8m0_value(code: int) -> float:
+    """Value of one E8M0 shared-scale code (OCP MX v1.0)."""
+    return _load().oracle_e8m0_value(int(code))
+
+
+def mxfp8_decode(codes, scales, block=32):
+    """MXFP8 -> float64: codes uint8 [..., d], scales uint8 [..., d / block] (one scale per `block`
+    consecutive elements of the last axis)."""
+    codes = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    scales = np.ascontiguousarray(np.asarray(scales, dtype=np.uint8))
+    d = codes.shape[-1]
+    n = codes.size // d if d else 0
+    if d % block or scales.shape[:-1] != codes.shape[:-1] or scales.shape[-1] != d // block:
+        raise ValueError("scales must be [..., d / block]")
+    out = np.empty(codes.shape, np.float64)
+    if out.size and _load().oracle_mxfp8_decode(n, d, block, _ptr(codes), _ptr(scales), _ptr(out)) != 0:
+        raise RuntimeError("oracle_mxfp8_decode failed")
     return out
 
 

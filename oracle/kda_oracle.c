@@ -168,3 +168,46 @@ int oracle_segment_compose(int nseg, int dk, int dv,
     free(X); free(Y);
     return 0;
 }
+
+/*
+ * MXFP8 inputs.  The til.kil9.dev "Kimi K3 기술 보고서" post (deployment paragraph) says the released
+ * model was trained quantisation-aware with MXFP8 activations, so q, k and v may arrive in that form.
+ * The format is the OCP Microscaling Formats (MX) v1.0 one: blocks of 32 consecutive elements share one
+ * E8M0 scale X, each element is an FP8 E4M3 number P_i, and the element's value is X * P_i.  Here the
+ * blocks run along the head dimension of each (token, head) row.
+ *
+ * E4M3: sign bit, 4 exponent bits (bias 7), 3 mantissa bits.  Exponent field 0 is subnormal,
+ * 2^-6 * m / 8; otherwise 2^(e - 7) * (1 + m / 8); exponent 15 with mantissa 7 is NaN (there are no
+ * infinities, and the largest finite magnitude is 448).
+ * E8M0: 8 exponent bits, no sign and no mantissa: 2^(e - 127); e = 255 is NaN.
+ */
+double oracle_e4m3_value(unsigned char b)
+{
+    const int s = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m / 8.0, -6);
+    else mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+double oracle_e8m0_value(unsigned char e)
+{
+    if (e == 255) return NAN;
+    return ldexp(1.0, (int)e - 127);
+}
+
+/*
+ * Decodes n rows of d MXFP8 elements: codes [n, d], scales [n, d / block] -> out [n, d] in double.
+ * Returns 0, or -1 on a bad argument (block must divide d).
+ */
+int oracle_mxfp8_decode(long n, int d, int block, const unsigned char* codes, const unsigned char* scales,
+                        double* out)
+{
+    if (n < 0 || d <= 0 || block <= 0 || d % block != 0) return -1;
+    const int nb = d / block;
+    for (long r = 0; r < n; ++r)
+        for (int i = 0; i < d; ++i)
+            out[r * d + i] = oracle_e8m0_value(scales[r * nb + i / block]) * oracle_e4m3_value(codes[r * d + i]);
+    return 0;
+}

@@ -39,6 +39,13 @@ MUTANTS = [
     ("compose with M transposed", "acc += Ms[(size_t)i * dk + m] * X[(size_t)m * dv + j];",
      "acc += Ms[(size_t)m * dk + i] * X[(size_t)m * dv + j];", 1),
     ("compose without the zero-start state", "double acc = Zs[(size_t)i * dv + j];", "double acc = 0.0;", 1),
+    ("E4M3 exponent bias 8", "else mag = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "else mag = ldexp(1.0 + (double)m / 8.0, e - 8);", 1),
+    ("E4M3 subnormals read as normals", "if (e == 0) mag = ldexp((double)m / 8.0, -6);",
+     "if (e == 0) mag = ldexp(1.0 + (double)m / 8.0, -7);", 1),
+    ("E4M3 max code read as NaN", "if (e == 15 && m == 7) return NAN;", "if (e == 15 && m >= 6) return NAN;", 1),
+    ("E8M0 bias 128", "return ldexp(1.0, (int)e - 127);", "return ldexp(1.0, (int)e - 128);", 1),
+    ("shared scale per 16 elements", "scales[r * nb + i / block]", "scales[r * nb + (i / (block / 2)) % nb]", 1),
 ]
 
 

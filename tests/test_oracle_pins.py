@@ -12,7 +12,10 @@ value axis instead of the key axis, o read from S_{t-1} instead of S_t, a wrong 
   * the decay floor facts printed on the orkas.ai page (tests/golden/decay_floor_facts.txt);
   * segment composition (transition + zero-start state, then a prefix scan) reproduces the unsplit
     run, while a plain sum of zero-start states does not;
-  * the fp64 chunk form (tests/chunk_reference.py) reproduces the sequential loop.
+  * the fp64 chunk form (tests/chunk_reference.py) reproduces the sequential loop;
+  * the MXFP8 input decode: every E4M3 and E8M0 code against torch's own float8 conversions (an
+    independent library routine), the format facts of the OCP MX v1.0 specification
+    (tests/golden/mxfp8_format_facts.txt), and the block structure of the shared scales.
 """
 import math
 import os
@@ -281,3 +284,58 @@ def test_tile_anchor_bound_at_the_floor():
         worst = max(worst, float(np.max(b - g[i0:i0 + 16])))
     assert abs(worst - (-16 * math.log(0.0067))) < 1e-9
     assert math.exp(worst) < torch.finfo(torch.bfloat16).max
+
+
+def test_e4m3_codes_match_library(oracle_mod):
+    codes = torch.arange(256, dtype=torch.uint8)
+    lib = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([oracle_mod.e4m3_value(c) for c in range(256)])
+    np.testing.assert_array_equal(np.isnan(mine), np.isnan(lib))
+    ok = ~np.isnan(lib)
+    np.testing.assert_array_equal(mine[ok], lib[ok])
+    np.testing.assert_array_equal(np.signbit(mine[ok]), np.signbit(lib[ok]))
+
+
+def test_e8m0_codes_match_library(oracle_mod):
+    codes = torch.arange(256, dtype=torch.uint8)
+    lib = codes.view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    mine = np.array([oracle_mod.e8m0_value(c) for c in range(256)])
+    np.testing.assert_array_equal(np.isnan(mine), np.isnan(lib))
+    ok = ~np.isnan(lib)
+    np.testing.assert_array_equal(mine[ok], lib[ok])
+
+
+def test_mxfp8_format_facts(oracle_mod):
+    block = None
+    for line in open(os.path.join(GOLDEN, "mxfp8_format_facts.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        kind, code, val = line.split()
+        if kind == "block":
+            block = int(val)
+            continue
+        got = (oracle_mod.e4m3_value if kind == "e4m3" else oracle_mod.e8m0_value)(int(code, 16))
+        want = float(val)
+        if math.isnan(want):
+            assert math.isnan(got), (kind, code)
+        else:
+            assert got == want and math.copysign(1, got) == math.copysign(1, want), (kind, code, got)
+    # one shared scale per 32 elements: a row of ones with four different scales decodes block by block
+    assert block == 32
+    codes = np.full((2, 128), 0x38, np.uint8)
+    scales = np.array([[127, 128, 126, 130], [0, 254, 127, 120]], np.uint8)
+    out = oracle_mod.mxfp8_decode(codes, scales, block)
+    for r in range(2):
+        for i in range(128):
+            assert out[r, i] == 2.0 ** (int(scales[r, i // block]) - 127)
+
+
+def test_mxfp8_decode_is_scale_times_element(oracle_mod):
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 256, (3, 7, 64)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3A           # no NaN codes
+    scales = rng.integers(100, 140, (3, 7, 2)).astype(np.uint8)
+    out = oracle_mod.mxfp8_decode(codes, scales)
+    elem = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    scl = torch.from_numpy(scales).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    np.testing.assert_array_equal(out, elem * np.repeat(scl, 32, axis=-1))
