@@ -9,7 +9,8 @@ H=32 heads, dk=dv=128, bf16 q/k/v, fp32 log_alpha/beta, zero initial state, fp32
 fp32 state checkpoints every 512 tokens): the per-chunk decay prep, the intra-chunk tcgen05 pass,
 the inter-chunk tcgen05 state pass and the checkpoint writes.  The decode workload (256 sequences x
 32 heads of 128 x 128 fp32 state, 1024 consecutive kda_recurrent_step calls) and a segment compose
-are timed alongside and reported under "decode" and "compose".  Inputs are seeded synthetic data
+are timed alongside and reported under "decode" and "compose", with speculative decoding under
+"speculative" and the prefill with MXFP8 q/k/v under "mxfp8".  Inputs are seeded synthetic data
 drawn on the device; every input and output set is larger than the 126 MB L2, so no flush is needed.
 
 Under torchrun (N > 1) every rank runs its own batch on its own GPU (weak scaling, no data-path
@@ -41,6 +42,8 @@ SPEC_ND, SPEC_POOL, SPEC_ROUNDS = 4, 16, 256   # drafts per round, distinct draf
 # (128 x 128 x 4 B / 512 = 128 B) and the final state (64 KiB per 4096 tokens = 16 B).
 PREFILL_READ_B = 3 * 256 + 512 + 4
 PREFILL_WRITE_B = 256 + 128 + 16
+# The same with MXFP8 q, k, v: 1-byte E4M3 codes plus one E8M0 scale byte per 32 channels.
+PREFILL_READ_MX_B = 3 * 128 + 3 * 4 + 512 + 4
 # Decode bytes per (sequence, head) step: state read + write (2 x 64 KiB), q/k/v bf16, log_alpha,
 # beta, o bf16.
 DECODE_B = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2
@@ -328,6 +331,45 @@ def run_ours(args):
            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
     del hq, hk, hv, hla, hb, ho, hfs, ho2, hfs2, bufs
 
+    # ------------------------------------------------------------------ the prefill with MXFP8 q, k, v
+    # The same workload, its q, k, v quantised to MXFP8 (E4M3 codes, one E8M0 scale per 32 channels).
+    mx = (*synth.mxfp8_quantize(inp.q), *synth.mxfp8_quantize(inp.k), *synth.mxfp8_quantize(inp.v))
+
+    def mx_step():
+        kda.kda_chunk_fwd_mxfp8(*mx, inp.log_alpha, inp.beta, None, inp.cu_seqlens, o, fs, ckpt_stride=CKPT,
+                                checkpoints=ck, ckpt_cu=ckcu, workspace=ws)
+
+    mx_steps = max(3, min(args.steps, 50))
+    for _ in range(3):
+        mx_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(mx_steps):
+        mx_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mx_ms = max_over_ranks(e0.elapsed_time(e1) / mx_steps, world)
+    kda.kda_profile_begin(mx_steps)
+    for _ in range(mx_steps):
+        mx_step()
+    torch.cuda.synchronize()
+    _, mx_prep, mx_state, mx_n = kda.kda_profile_end()
+    barrier(world)
+    mx_prep_ms = mx_prep / mx_n
+    mx_prep_gbs = PREFILL_READ_MX_B * th / (mx_prep_ms / 1e3) / 1e9
+    mxfp8 = {"workload": "the prefill workload with q, k, v in MXFP8 (E4M3 codes, E8M0 scale per 32 channels)",
+             "value": tokens_job / (mx_ms / 1e3), "unit": "tokens/s", "ms_per_step": round(mx_ms, 5),
+             "kernels": {"prep_bf16_kernel<MX>": {"ms": round(mx_prep_ms, 4)},
+                         "state_bf16_kernel": {"ms": round(mx_state / mx_n, 4)}},
+             "roofline": {"bound": "hbm", "kernel": "prep_bf16_kernel (MXFP8 inputs)",
+                          "achieved": round(mx_prep_gbs, 1), "peak": hbm, "unit": "GB/s",
+                          "frac": round(mx_prep_gbs / hbm, 4), "alg_bytes_per_launch": PREFILL_READ_MX_B * th}}
+    st = kda.kda_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {kda.kda_status_string(st)}")
+    del mx
+
     # ------------------------------------------------------------------ decode workload
     s0, dq, dk_, dv_, dla, db = synth.make_decode_inputs(DEC_N, H, D, D, dtype=torch.bfloat16, device=dev,
                                                          seed=100 + rank, steps=DEC_STEPS)
@@ -440,7 +482,7 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs and outputs larger than L2 (1.1 GB per step), no flush"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-            "gpu_launches": 4 * args.steps, "decode": decode, "speculative": speculative, "compose": compose,
+            "gpu_launches": 4 * args.steps, "decode": decode, "speculative": speculative, "compose": compose, "mxfp8": mxfp8,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

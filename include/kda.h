@@ -60,7 +60,8 @@ typedef enum {
     KDA_ERR_DEVICE_INPUT = -7  /* device: cu_seqlens / seg_cu / ckpt_cu inconsistent */
 } kda_status_t;
 
-typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype_t;
+/* KDA_MXFP8: MXFP8 q, k, v (kda_chunk_fwd_mxfp8 only; for the workspace queries it sizes like KDA_BF16). */
+typedef enum { KDA_BF16 = 0, KDA_F32 = 1, KDA_MXFP8 = 2 } kda_dtype_t;
 
 /* Token count of one chunk of the chunked form (fixed) and of the tiles inside it. */
 #define KDA_CHUNK 64
@@ -110,6 +111,36 @@ KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v,
                            const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
                            int H, int dk, int dv, kda_dtype_t dtype,
                            int ckpt_stride,
+                           void* o, float* final_state,
+                           float* checkpoints, const int32_t* ckpt_cu,
+                           float* final_transition,
+                           void* workspace, size_t ws_bytes, kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd with MXFP8 q, k and v.  The til.kil9.dev "Kimi K3 기술 보고서" post (deployment
+ * paragraph) says the model was trained quantisation-aware with MXFP8 activations, so the projections
+ * that feed KDA may arrive in that form.  The format is that of the OCP Microscaling Formats (MX) v1.0
+ * specification: each (token, head) row of q, k or v is cut into blocks of 32 consecutive channels; a
+ * block holds 32 FP8 E4M3 codes and one E8M0 shared scale X = 2^(e - 127), and element i is X * E4M3(i).
+ *
+ *   q, k        [T_tot,H,dk] uint8 E4M3 codes, 16-byte aligned      q_scale, k_scale  [T_tot,H,dk/32] uint8
+ *   v           [T_tot,H,dv] uint8 E4M3 codes, 16-byte aligned      v_scale           [T_tot,H,dv/32] uint8
+ *   the scale arrays are aligned to dk/32 (q_scale, k_scale) and dv/32 (v_scale) bytes.
+ *   o           [T_tot,H,dv] bf16.
+ * Everything else (log_alpha, beta, states, checkpoints, transition, workspace, window processing, errors)
+ * is as for kda_chunk_fwd with dtype KDA_BF16, and so are the supported sizes (dk = 128, dv in {64, 128}).
+ * The codes are decoded in the kernel that reads them; the values are exact (E4M3 has 4 significant bits)
+ * as long as X * E4M3 stays inside the fp32 range, so the results equal kda_chunk_fwd's on the decoded
+ * values given as bf16.  NaN inputs are outside the contract: a NaN code (E4M3 S.1111.111) is read as
+ * +-480 and a NaN scale (0xFF) gives NaN results.
+ */
+KDA_API kda_status_t kda_chunk_fwd_mxfp8(const uint8_t* q, const uint8_t* q_scale,
+                           const uint8_t* k, const uint8_t* k_scale,
+                           const uint8_t* v, const uint8_t* v_scale,
+                           const float* log_alpha, const float* beta,
+                           const float* initial_state,
+                           const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
+                           int H, int dk, int dv, int ckpt_stride,
                            void* o, float* final_state,
                            float* checkpoints, const int32_t* ckpt_cu,
                            float* final_transition,

@@ -14,8 +14,9 @@ import os
 import torch
 
 __all__ = [
-    "KDA_BF16", "KDA_F32", "KDA_CHUNK", "KDAError", "lib_path",
-    "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
+    "KDA_BF16", "KDA_F32", "KDA_MXFP8", "KDA_CHUNK", "KDAError", "lib_path",
+    "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd", "kda_chunk_fwd_mxfp8",
+    "kda_chunk_fwd_noalloc",
     "kda_recurrent_step", "kda_decode_verify", "kda_decode_commit", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
     "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
     "kda_selftest_umma", "KDA_PREFIX_BLOCK", "kda_prefix_block_hashes", "kda_prefix_cache_create",
@@ -25,6 +26,7 @@ __all__ = [
 
 KDA_BF16 = 0
 KDA_F32 = 1
+KDA_MXFP8 = 2
 KDA_PREFIX_BLOCK = 512
 KDA_CHUNK = 64
 
@@ -59,6 +61,9 @@ def _load():
     L.kda_chunk_fwd.restype = i32
     L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32,
                                 vp, vp, vp, vp, vp, vp, sz, vp]
+    L.kda_chunk_fwd_mxfp8.restype = i32
+    L.kda_chunk_fwd_mxfp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                      vp, vp, vp, vp, vp, vp, sz, vp]
     L.kda_chunk_fwd_noalloc.restype = i32
     L.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32,
                                         vp, vp, vp, vp, vp, vp]
@@ -202,6 +207,65 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, o, final_
                                _p(checkpoints if ckpt_stride else None), _p(ckpt_cu if ckpt_stride else None),
                                _p(final_transition), _p(workspace), workspace.numel(), _stream(stream))
     _check(st, "kda_chunk_fwd")
+    return o
+
+
+def _bytes_of(t, name, shape, dev, kinds):
+    """A uint8 (or same-size float8) tensor of the given shape, as raw bytes."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype not in kinds:
+        raise TypeError(f"{name}: expected one of {kinds}, got {t.dtype}")
+    _need(t, name, shape, None, dev)
+
+
+def kda_chunk_fwd_mxfp8(q, q_scale, k, k_scale, v, v_scale, log_alpha, beta, initial_state, cu_seqlens, o,
+                        final_state=None, *, ckpt_stride=0, checkpoints=None, ckpt_cu=None, final_transition=None,
+                        workspace=None, stream=None):
+    """Chunked KDA forward with MXFP8 q, k, v (C: kda_chunk_fwd_mxfp8).
+
+    q, k [T,H,dk] and v [T,H,dv]: E4M3 codes (uint8 or torch.float8_e4m3fn); q_scale, k_scale [T,H,dk/32]
+    and v_scale [T,H,dv/32]: E8M0 shared scales (uint8 or torch.float8_e8m0fnu), one per 32 channels.
+    o [T,H,dv] bf16.  Everything else as kda_chunk_fwd.
+    """
+    codes = (torch.uint8, torch.float8_e4m3fn)
+    scales = (torch.uint8, torch.float8_e8m0fnu)
+    if q is None:
+        raise ValueError("q is required")
+    dev = q.device
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = cu_seqlens.numel() - 1
+    _bytes_of(q, "q", (T, H, dk), dev, codes)
+    _bytes_of(k, "k", (T, H, dk), dev, codes)
+    _bytes_of(v, "v", (T, H, dv), dev, codes)
+    if dk % 32 or dv % 32:
+        raise ValueError("dk and dv must be multiples of the 32-channel scale block")
+    _bytes_of(q_scale, "q_scale", (T, H, dk // 32), dev, scales)
+    _bytes_of(k_scale, "k_scale", (T, H, dk // 32), dev, scales)
+    _bytes_of(v_scale, "v_scale", (T, H, dv // 32), dev, scales)
+    _need(o, "o", (T, H, dv), torch.bfloat16, dev)
+    _need(log_alpha, "log_alpha", (T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (T, H), torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", (n + 1,), torch.int32, dev)
+    _opt(initial_state, "initial_state", (n, H, dk, dv), torch.float32, dev)
+    _opt(final_state, "final_state", (n, H, dk, dv), torch.float32, dev)
+    _opt(final_transition, "final_transition", (n, H, dk, dk), torch.float32, dev)
+    if ckpt_stride:
+        _need(checkpoints, "checkpoints", None, torch.float32, dev)
+        if checkpoints.dim() != 4 or tuple(checkpoints.shape[1:]) != (H, dk, dv):
+            raise ValueError("checkpoints must be [n_ckpt, H, dk, dv]")
+        _need(ckpt_cu, "ckpt_cu", (n + 1,), torch.int32, dev)
+    if workspace is None:
+        nbytes = kda_chunk_fwd_workspace_bytes(T, n, H, dk, dv, KDA_MXFP8)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", None, torch.uint8, dev)
+    st = _load().kda_chunk_fwd_mxfp8(_p(q), _p(q_scale), _p(k), _p(k_scale), _p(v), _p(v_scale), _p(log_alpha),
+                                     _p(beta), _p(initial_state), _p(cu_seqlens), n, T, H, dk, dv, int(ckpt_stride),
+                                     _p(o), _p(final_state), _p(checkpoints if ckpt_stride else None),
+                                     _p(ckpt_cu if ckpt_stride else None), _p(final_transition), _p(workspace),
+                                     workspace.numel(), _stream(stream))
+    _check(st, "kda_chunk_fwd_mxfp8")
     return o
 
 

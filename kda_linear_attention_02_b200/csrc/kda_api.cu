@@ -116,7 +116,7 @@ bool supported(kda_dtype_t dt, int dk, int dv) {
     const bool dims = (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
     if (!dims) return false;
     if (dt == KDA_F32) return true;
-    if (dt == KDA_BF16) return dk == 128;
+    if (dt == KDA_BF16 || dt == KDA_MXFP8) return dk == 128;
     return false;
 }
 
@@ -180,14 +180,20 @@ size_t kda_chunk_fwd_min_workspace_bytes(int n_seqs, int H, int dk, int dv, kda_
     return index_bytes(n_seqs) + carry_bytes(n_seqs, H, dk, dv) + chunk_bytes(dt, H, dk, dv);
 }
 
-kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
-                           const float* initial_state, const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
-                           int H, int dk, int dv, kda_dtype_t dtype, int ckpt_stride, void* o, float* final_state,
-                           float* checkpoints, const int32_t* ckpt_cu, float* final_transition, void* workspace,
-                           size_t ws_bytes, kda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// kda_chunk_fwd and kda_chunk_fwd_mxfp8: dtype KDA_MXFP8 takes the shared-scale arrays (checked by the
+// caller) and writes a bf16 o; it uses the bf16 path's packets and workspace.
+kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v, const void* q_scale, const void* k_scale,
+                            const void* v_scale, const float* log_alpha, const float* beta,
+                            const float* initial_state, const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
+                            int H, int dk, int dv, kda_dtype_t dtype, int ckpt_stride, void* o, float* final_state,
+                            float* checkpoints, const int32_t* ckpt_cu, float* final_transition, void* workspace,
+                            size_t ws_bytes, kda_stream_t stream) {
     if (n_seqs < 0 || total_tokens < 0 || H <= 0 || ckpt_stride < 0) return KDA_ERR_ARG;
     if (total_tokens > 0x7fffffffLL) return KDA_ERR_ARG;   // cu_seqlens is int32
-    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_ARG;
     if (!supported(dtype, dk, dv)) return KDA_ERR_UNSUPPORTED;
     if (ckpt_stride > 0 && (ckpt_stride % kChunk != 0 || !checkpoints || !ckpt_cu)) return KDA_ERR_ARG;
     if (n_seqs == 0) return KDA_OK;
@@ -208,6 +214,7 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
     char* ws = static_cast<char*>(workspace);
     ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.initial_state = initial_state;
+    a.q_scale = q_scale; a.k_scale = k_scale; a.v_scale = v_scale; a.mx = dtype == KDA_MXFP8;
     a.cu_seqlens = cu_seqlens; a.cu_chunks = reinterpret_cast<int32_t*>(ws); a.n_seqs = n_seqs;
     a.total_tokens = total_tokens; a.H = H; a.dk = dk; a.dv = dv; a.ckpt_stride = ckpt_stride; a.o = o;
     a.final_state = final_state; a.checkpoints = checkpoints; a.ckpt_cu = ckpt_cu;
@@ -245,6 +252,39 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
         lo += win;
     } while (lo < ub);
     return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                           const float* initial_state, const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
+                           int H, int dk, int dv, kda_dtype_t dtype, int ckpt_stride, void* o, float* final_state,
+                           float* checkpoints, const int32_t* ckpt_cu, float* final_transition, void* workspace,
+                           size_t ws_bytes, kda_stream_t stream) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_ARG;   // MXFP8 needs its scales: kda_chunk_fwd_mxfp8
+    return chunk_fwd_impl(q, k, v, nullptr, nullptr, nullptr, log_alpha, beta, initial_state, cu_seqlens, n_seqs,
+                          total_tokens, H, dk, dv, dtype, ckpt_stride, o, final_state, checkpoints, ckpt_cu,
+                          final_transition, workspace, ws_bytes, stream);
+}
+
+kda_status_t kda_chunk_fwd_mxfp8(const uint8_t* q, const uint8_t* q_scale, const uint8_t* k, const uint8_t* k_scale,
+                                 const uint8_t* v, const uint8_t* v_scale, const float* log_alpha, const float* beta,
+                                 const float* initial_state, const int32_t* cu_seqlens, int n_seqs,
+                                 int64_t total_tokens, int H, int dk, int dv, int ckpt_stride, void* o,
+                                 float* final_state, float* checkpoints, const int32_t* ckpt_cu,
+                                 float* final_transition, void* workspace, size_t ws_bytes, kda_stream_t stream) {
+    if (!supported(KDA_MXFP8, dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if (n_seqs > 0 && total_tokens > 0) {
+        if (!q_scale || !k_scale || !v_scale) return KDA_ERR_ARG;
+        // one scale byte per 32 channels, read as whole rows: 4 bytes (128 channels) or 2 (64)
+        if (!aligned_to(q_scale, dk / 32) || !aligned_to(k_scale, dk / 32) || !aligned_to(v_scale, dv / 32))
+            return KDA_ERR_ALIGN;
+    }
+    return chunk_fwd_impl(q, k, v, q_scale, k_scale, v_scale, log_alpha, beta, initial_state, cu_seqlens, n_seqs,
+                          total_tokens, H, dk, dv, KDA_MXFP8, ckpt_stride, o, final_state, checkpoints, ckpt_cu,
+                          final_transition, workspace, ws_bytes, stream);
 }
 
 kda_status_t kda_recurrent_step(float* state, const void* q, const void* k, const void* v, const float* log_alpha,

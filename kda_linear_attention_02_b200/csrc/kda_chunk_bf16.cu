@@ -73,6 +73,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 constexpr float kLog2e = 1.4426950408889634f;
+// MXFP8 inputs (OCP Microscaling Formats v1.0).  Two E4M3 codes (the first in the low byte) -> 2^-120
+// times their values as fp32, with integer operations only: a code's 7 magnitude bits placed at bits
+// 20..26 of an fp32 make exponent field e and mantissa m << 20, which reads 2^(e - 127) (1 + m / 8) for
+// e > 0 and m 2^-129 (an fp32 subnormal) for e = 0 -- exactly 2^-120 times the E4M3 magnitude either way;
+// the sign moves to bit 31.  (The NaN codes S.1111.111 read as +-480.)  Multiplying by 2^120 and then by
+// the shared scale is exact unless the value leaves the fp32 range.
+__device__ __forceinline__ float2 e4m3x2_scaled(uint32_t u) {
+    const uint32_t lo = ((u << 20) & 0x07F00000u) | ((u << 24) & 0x80000000u);
+    const uint32_t hi = ((u << 12) & 0x07F00000u) | ((u << 16) & 0x80000000u);
+    return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+constexpr float kE4M3Unscale = 1.329227995784916e36f;   // 2^120
+// E8M0 shared scale -> 2^(e - 127) (code 0 is the fp32 subnormal 2^-127, code 255 is NaN)
+__device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
+    return e == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float(e ? e << 23 : 0x00400000u);
+}
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                       pack_bf16x2(f[6], f[7]));
@@ -102,42 +118,63 @@ constexpr uint32_t BVAR = 114688;    // key side: variants 0..3 stacked as rows 
                                      // of one 160-row B operand, [2 K atoms][160 rows][128 B]
 constexpr uint32_t QT = 155648;      // Q * gamma, [64][128] bf16, 16-byte chunks swizzled by row
 constexpr uint32_t BKV = 172032;     // [beta K gamma | beta V]^T: (128+DV) x 64 bf16 (B operand)
-constexpr uint32_t MISC = 204800;    // beta[64] fp32, half-tile totals [8][128] fp32
+constexpr uint32_t MISC = 204800;    // beta[64] fp32 (of even items for MXFP8 inputs), half-tile totals [8][128] fp32
+constexpr uint32_t BET1 = MISC + 4352;   // MXFP8 inputs: beta[64] fp32 of odd items (fetched during the previous one)
 constexpr uint32_t IAQ = 209920;     // [I; Aqk]: 128 x 64 bf16 (A operand of the Y product)
 // aliases of RALL/BVAR once phase A has completed
 constexpr uint32_t AM = 81920, XF = 99328, TT = 118016, XT = 124928, XY = 133120;   // solve
 constexpr uint32_t AWS = 81920, UOS = 114688;                                    // packet staging
 constexpr uint32_t BYTES = IAQ + 16384;
+constexpr uint32_t SCF = BYTES;      // MXFP8 inputs only: shared scales of the chunk's tokens, [q, k, v][64][4] fp32
+constexpr uint32_t SCW = SCF + 3 * 64 * 16;   // and their E8M0 code words as fetched, [2 items][q, k, v][64] u32
+constexpr uint32_t BYTES_MX = SCW + 2 * 3 * 64 * 4;
+static_assert(BYTES_MX + 1024 <= 232448, "shared memory of one CTA");
 constexpr int LDM = 68;              // fp32 row pitch of AM (float4-aligned rows; 4 rows apart = 16 banks)
 constexpr int LDX = 73;              // fp32 row pitch of X (odd: column reads of X^T spread over the banks)
 constexpr int LDTT = 40;             // fp32 row pitch of the product scratch (8 banks per row: B fragments clash-free)
 static_assert(XF + 64 * LDX * 4 <= TT && TT + 32 * LDTT * 4 <= XT && AM + 64 * LDM * 4 <= XF, "solve map");
+static_assert(BET1 + 256 <= IAQ, "beta buffers");
+
 constexpr int NT = 512;              // threads per CTA
 }  // namespace ps
 
-template <int DV>
+// One chunk's input tiles into the staging area.  bf16: q, k, v as 64-column boxes, [dk / 64][64 tokens][128 B];
+// MXFP8: one box of codes each, [64 tokens][dk or DV bytes].  log_alpha: 32-column boxes.
+template <int DV, bool MX>
 __device__ __forceinline__ void issue_tile_loads(uint8_t* sm, const CUtensorMap* mq, const CUtensorMap* mk,
                                                  const CUtensorMap* mv, const CUtensorMap* ml, uint64_t* bar,
                                                  int h, long long tok0) {
     const int tok = static_cast<int>(tok0);
-    mbar_arrive_expect_tx(bar, 2 * 16384 + DV * 128 + 32768);
+    if constexpr (MX) {
+        mbar_arrive_expect_tx(bar, 2 * 8192 + DV * 64 + 32768);
+        tma_load_3d(sm + ps::STG_Q, mq, 0, h, tok, bar);
+        tma_load_3d(sm + ps::STG_K, mk, 0, h, tok, bar);
+        tma_load_3d(sm + ps::STG_V, mv, 0, h, tok, bar);
+    } else {
+        mbar_arrive_expect_tx(bar, 2 * 16384 + DV * 128 + 32768);
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        tma_load_3d(sm + ps::STG_Q + hf * 8192, mq, hf * 64, h, tok, bar);
-        tma_load_3d(sm + ps::STG_K + hf * 8192, mk, hf * 64, h, tok, bar);
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_3d(sm + ps::STG_Q + hf * 8192, mq, hf * 64, h, tok, bar);
+            tma_load_3d(sm + ps::STG_K + hf * 8192, mk, hf * 64, h, tok, bar);
+        }
+#pragma unroll
+        for (int hf = 0; hf < DV / 64; ++hf) tma_load_3d(sm + ps::STG_V + hf * 8192, mv, hf * 64, h, tok, bar);
     }
-#pragma unroll
-    for (int hf = 0; hf < DV / 64; ++hf) tma_load_3d(sm + ps::STG_V + hf * 8192, mv, hf * 64, h, tok, bar);
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) tma_load_3d(sm + ps::STG_L + qq * 8192, ml, qq * 32, h, tok, bar);
 }
 
-template <int DV>
+// MX: q, k, v arrive as MXFP8 (E4M3 codes with one E8M0 scale per 32 channels of a (token, head) row;
+// q_scale/k_scale [T, H, 4] and v_scale [T, H, DV / 32] bytes) and are decoded exactly in the column pass;
+// everything after it is the bf16 path unchanged.
+template <int DV, bool MX>
 __global__ void __launch_bounds__(512, 1)
 prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_l,
-                 const float* __restrict__ beta, const int2* __restrict__ chunk_tab, int H, long long n_items,
-                 uint8_t* __restrict__ packets, int* status) {
+                 const float* __restrict__ beta, const uint8_t* __restrict__ q_scale,
+                 const uint8_t* __restrict__ k_scale, const uint8_t* __restrict__ v_scale,
+                 const int2* __restrict__ chunk_tab, int H, long long n_items, uint8_t* __restrict__ packets,
+                 int* status) {
     using P = Pk<DV>;
     constexpr int NT = ps::NT;
     constexpr int LDM = ps::LDM;
@@ -148,8 +185,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     __shared__ __align__(8) uint64_t bar_load, bar_mma;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-    float* bet = reinterpret_cast<float*>(sm + ps::MISC);
-    float* tot = bet + 64;   // [8 half-tiles][128 channels]
+    float* bet = reinterpret_cast<float*>(sm + ps::MISC);           // this item's beta (buffer of its parity)
+    float* tot = reinterpret_cast<float*>(sm + ps::MISC + 256);   // [8 half-tiles][128 channels]
     // AM holds the strictly lower A = beta_r (K e^g)_r . (K e^-g)_s in two forms that never overlap: the
     // off-diagonal 16 x 16 blocks row-major (AM[r][s], tile(s) < tile(r)), and each diagonal block
     // transposed into its upper triangle (AM[s][r] for s < r in the same tile)
@@ -187,6 +224,26 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint32_t ph_load = 0, ph_mma = 0;
     bool load_pending = false;   // meaningful in thread 0 only
 
+    // MXFP8 inputs: beta and the scale words of an item's 64 rows into the buffers of parity pb, by cp.async,
+    // so that they land while the previous item computes (rows past the item's n tokens read as zero), by
+    // warps 8..15, which never issue bulk copies.  (bf16 inputs load beta when the item starts: there an
+    // early fetch measured slower.)
+    auto fetch_rows = [&](int2 l, int hh, int pb) {
+        if constexpr (!MX) return;
+        const bool in = (t & 63) < l.y;
+        const size_t row = (static_cast<size_t>(l.x) + (t & 63)) * H + hh;
+        if (t >= 256 && t < 320) {
+            cp_async4(sm + (pb ? ps::BET1 : ps::MISC) + 4 * (t - 256), in ? beta + row : beta, in ? 4u : 0u);
+        } else if (t >= 320) {
+            const int which = (t - 320) >> 6;
+            const uint8_t* src = which == 0 ? q_scale : which == 1 ? k_scale : v_scale;
+            uint8_t* dst = sm + ps::SCW + pb * 768 + 4 * (t - 320);
+            if (which < 2 || DV == 128) cp_async4(dst, in ? src + 4 * row : src, in ? 4u : 0u);
+            else *reinterpret_cast<uint32_t*>(dst) =   // DV = 64: 2-byte rows, too small for cp.async
+                     0x7F7F0000u | (in ? reinterpret_cast<const uint16_t*>(v_scale)[row] : 0x7F7Fu);
+        }
+    };
+
     // everything above is private set-up; the chunk table and the inputs come from earlier launches
     grid_dependency_wait();
     // chunk table entry {first token, valid tokens} of a window item (n = 0: past the last chunk)
@@ -197,15 +254,31 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     bool valid = loc.y > 0;
     int2 nloc = entry(item + gridDim.x);   // one item ahead
     if (t == 0 && valid) {
-        issue_tile_loads<DV>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, h, loc.x);
+        issue_tile_loads<DV, MX>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, h, loc.x);
         load_pending = true;
     }
+    if (valid) fetch_rows(loc, h, 0);
+    int par = 0;   // parity of the item: its beta / scale-word buffers
 
     while (valid) {
         const int n = loc.y;
-        const long long tok0 = loc.x;
         uint8_t* pkt = packets + static_cast<size_t>(item) * P::BYTES;
-        if (t < 64) bet[t] = t < n ? beta[(static_cast<size_t>(tok0) + t) * H + h] : 0.f;
+        if constexpr (!MX) {
+            if (t < 64) bet[t] = t < n ? beta[(static_cast<size_t>(loc.x) + t) * H + h] : 0.f;
+        } else {
+            bet = reinterpret_cast<float*>(sm + (par ? ps::BET1 : ps::MISC));
+            if (t >= 256) cp_async_wait_all();   // this thread's fetches of the item's rows have landed
+        }
+        if constexpr (MX) {   // the shared scales of the chunk's tokens as fp32 (scale 1.0 past its end)
+            if (t >= 320) {
+                const uint32_t wv = (t & 63) < n ? *reinterpret_cast<const uint32_t*>(sm + ps::SCW + par * 768 +
+                                                                                       4 * (t - 320))
+                                                 : 0x7F7F7F7Fu;
+                reinterpret_cast<float4*>(sm + ps::SCF)[t - 320] =
+                    make_float4(e8m0_to_f32(wv & 0xFFu), e8m0_to_f32((wv >> 8) & 0xFFu),
+                                e8m0_to_f32((wv >> 16) & 0xFFu), e8m0_to_f32(wv >> 24));
+            }
+        }
         {
             const bool ok = mbar_wait(&bar_load, ph_load, status);
             if (__syncthreads_or(!ok)) break;
@@ -233,11 +306,17 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int r = 8 * q8 + j;
-                kb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
-                qb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
-                vb8[j] = c0 < DV ? *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 + r * 128 +
-                                                                       (c0 & 63) * 2)
-                                 : 0u;
+                if constexpr (MX) {   // two E4M3 codes per channel pair
+                    kb8[j] = *reinterpret_cast<const uint16_t*>(sm + ps::STG_K + r * 128 + c0);
+                    qb8[j] = *reinterpret_cast<const uint16_t*>(sm + ps::STG_Q + r * 128 + c0);
+                    vb8[j] = c0 < DV ? *reinterpret_cast<const uint16_t*>(sm + ps::STG_V + r * DV + c0) : 0u;
+                } else {
+                    kb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
+                    qb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
+                    vb8[j] = c0 < DV ? *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 + r * 128 +
+                                                                           (c0 & 63) * 2)
+                                     : 0u;
+                }
             }
             if (t == 0) bulk_wait_read0();   // the previous item's packet staging has been read out
             __syncthreads();
@@ -284,9 +363,18 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 // rows past the sequence end (n <= r) keep whatever the tile holds: their log-decay and beta are
                 // zero, so they add nothing to A, W, U, Kdec^T U' or the state, and their own P / O_intra rows
                 // are never stored as outputs
-                const float2 kf = bf2_to_f2(kb8[j]);
-                const float2 qf = bf2_to_f2(qb8[j]);
-                const float2 vf = bf2_to_f2(vb8[j]);
+                float2 kf, qf, vf;
+                if constexpr (MX) {   // code x shared scale of the 32-channel block holding c0
+                    const float* scf = reinterpret_cast<const float*>(sm + ps::SCF) + (c0 >> 5);
+                    const float2 un = f2(kE4M3Unscale);
+                    kf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(kb8[j]), un), f2(scf[4 * (64 + r)]));
+                    qf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(qb8[j]), un), f2(scf[4 * r]));
+                    vf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(vb8[j]), un), f2(scf[4 * (128 + r)]));
+                } else {
+                    kf = bf2_to_f2(kb8[j]);
+                    qf = bf2_to_f2(qb8[j]);
+                    vf = bf2_to_f2(vb8[j]);
+                }
                 const float2 pl = __fmul2_rn(p[j], f2(kLog2e));
                 const float2 E = make_float2(ex2_approx(pl.x), ex2_approx(pl.y));     // e^{g_r - b_t} <= 1
                 const float2 I = make_float2(ex2_approx(-pl.x), ex2_approx(-pl.y));   // e^{b_t - g_r} <= e^80.09
@@ -351,9 +439,10 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int nh = static_cast<int>(nitem % H);
         const bool nvalid = nloc.y > 0;
         if (t == 0 && nvalid) {
-            issue_tile_loads<DV>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.x);
+            issue_tile_loads<DV, MX>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.x);
             load_pending = true;
         }
+        if (nvalid) fetch_rows(nloc, nh, par ^ 1);
         const int2 nnloc = entry(nitem + gridDim.x);
         {
             const bool ok = mbar_wait(&bar_mma, ph_mma, status);
@@ -707,7 +796,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         nloc = nnloc;
         h = nh;
         valid = nvalid;
+        par ^= 1;
     }
+    if (MX && t >= 256) cp_async_wait_all();   // nor a fetch of rows
     if (t == 0) {
         if (load_pending) mbar_wait(&bar_load, ph_load, nullptr);   // never leave a TMA write in flight
         bulk_wait0();
@@ -1130,27 +1221,37 @@ cudaError_t launch_state(const ChunkArgs& a, cudaStream_t s) {
                       a.checkpoints, a.ckpt_cu, a.carry, a.status);
 }
 
+template <int DV, bool MX>
+cudaError_t launch_prep(const ChunkArgs& a, long long items, cudaStream_t s) {
+    CUtensorMap mq, mk, mv, ml;
+    const CUtensorMapDataType dt = MX ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int es = MX ? 1 : 2;
+    // bf16: 64-column boxes; MXFP8: the whole row of codes in one box
+    if (!make_map(&mq, a.q, dt, es, kDK, a.H, a.total_tokens, MX ? kDK : 64) ||
+        !make_map(&mk, a.k, dt, es, kDK, a.H, a.total_tokens, MX ? kDK : 64) ||
+        !make_map(&mv, a.v, dt, es, DV, a.H, a.total_tokens, MX ? DV : 64) ||
+        !make_map(&ml, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, a.H, a.total_tokens, 32))
+        return cudaErrorInvalidValue;
+    const int smem = static_cast<int>(MX ? ps::BYTES_MX : ps::BYTES) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(prep_bf16_kernel<DV, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const long long grid = items < num_sms() ? items : num_sms();
+    return launch_pdl(prep_bf16_kernel<DV, MX>, dim3(static_cast<unsigned>(grid)), dim3(ps::NT), smem, s, mq, mk, mv,
+                      ml, a.beta, static_cast<const uint8_t*>(a.q_scale), static_cast<const uint8_t*>(a.k_scale),
+                      static_cast<const uint8_t*>(a.v_scale), a.chunk_tab, a.H, items,
+                      static_cast<uint8_t*>(a.packets), a.status);
+}
+
 template <int DV>
 cudaError_t launch_bf16_t(const ChunkArgs& a, cudaStream_t s) {
     const long long items = (a.win_hi - a.win_lo) * a.H;
     if (a.events) cudaEventRecord(a.events->ev[1], s);
     if (a.total_tokens > 0 && items > 0) {
-        CUtensorMap mq, mk, mv, ml;
-        if (!make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, a.H, a.total_tokens, 64) ||
-            !make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, a.H, a.total_tokens, 64) ||
-            !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, a.total_tokens, 64) ||
-            !make_map(&ml, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, a.H, a.total_tokens, 32))
-            return cudaErrorInvalidValue;
-        const int smem = static_cast<int>(ps::BYTES) + 1024;
-        cudaError_t e = cudaFuncSetAttribute(prep_bf16_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
         const long long wchunks = a.win_hi - a.win_lo;
-        e = launch_pdl(chunk_table_kernel, dim3(static_cast<unsigned>((wchunks + 255) / 256)), dim3(256), 0, s,
-                       a.cu_chunks, a.cu_seqlens, a.n_seqs, a.win_lo, a.win_hi, a.chunk_tab);
+        cudaError_t e = launch_pdl(chunk_table_kernel, dim3(static_cast<unsigned>((wchunks + 255) / 256)), dim3(256),
+                                   0, s, a.cu_chunks, a.cu_seqlens, a.n_seqs, a.win_lo, a.win_hi, a.chunk_tab);
         if (e != cudaSuccess) return e;
-        const long long grid = items < num_sms() ? items : num_sms();
-        e = launch_pdl(prep_bf16_kernel<DV>, dim3(static_cast<unsigned>(grid)), dim3(ps::NT), smem, s, mq, mk, mv, ml,
-                       a.beta, a.chunk_tab, a.H, items, static_cast<uint8_t*>(a.packets), a.status);
+        e = a.mx ? launch_prep<DV, true>(a, items, s) : launch_prep<DV, false>(a, items, s);
         if (e != cudaSuccess) return e;
     }
     if (a.events) cudaEventRecord(a.events->ev[2], s);

@@ -100,6 +100,13 @@ __device__ __forceinline__ void bulk_s2g(void* dst, const void* src_smem, uint32
                  "r"(bytes)
                  : "memory");
 }
+// 4-byte asynchronous copy global -> shared in the calling thread's cp.async group; src_bytes = 0 writes
+// zeros and reads nothing.  cp_async_wait_all makes the thread's copies visible to that thread.
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst_smem)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }

@@ -33,6 +33,10 @@ struct ChunkArgs {
     const void* v;
     const float* log_alpha;
     const float* beta;
+    const void* q_scale;        // MXFP8 inputs only: E8M0 shared scales [T, H, dk / 32], [T, H, dv / 32]
+    const void* k_scale;
+    const void* v_scale;
+    bool mx;                    // q, k, v are MXFP8 codes (bf16 path with in-kernel decode)
     const float* initial_state;
     const int32_t* cu_seqlens;
     const int32_t* cu_chunks;   // device [N+1], filled by launch_chunk_index

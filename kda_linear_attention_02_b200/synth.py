@@ -127,3 +127,26 @@ def draft_layout(x):
     """[n_draft, n, H, ...] per-step decode inputs -> the token-major draft layout [n * n_draft, H, ...]
     (sequence i's drafts at rows i * n_draft ..) of kda_decode_verify / kda_decode_commit."""
     return x.transpose(0, 1).contiguous().reshape(x.shape[0] * x.shape[1], *x.shape[2:])
+
+
+def mxfp8_quantize(x: torch.Tensor, block: int = 32):
+    """Quantise x [..., d] to MXFP8 for use as an input: (E4M3 codes uint8 [..., d], E8M0 scales uint8
+    [..., d / block]).
+
+    The scale choice is the one the OCP Microscaling Formats v1.0 specification suggests: per block of
+    `block` consecutive elements, shared exponent floor(log2(amax)) - 8 (8 = largest exponent of E4M3),
+    elements divided by 2^shared and rounded to E4M3, saturating at +-448.  An all-zero block gets scale
+    1.0.  Rounding and the code bytes come from torch's float8 conversion.
+    """
+    xf = x.float()
+    d = xf.shape[-1]
+    if d % block:
+        raise ValueError("the last axis must be a multiple of the block")
+    xb = xf.reshape(*xf.shape[:-1], d // block, block)
+    amax = xb.abs().amax(dim=-1)
+    _, e = torch.frexp(amax)                   # amax = m 2^e, m in [0.5, 1): floor(log2 amax) = e - 1
+    shared = torch.where(amax > 0, e - 1 - 8, torch.zeros_like(e)).clamp(-127, 127)
+    elems = torch.ldexp(xb, -shared.unsqueeze(-1).to(xf.dtype)).clamp(-448.0, 448.0)
+    codes = elems.to(torch.float8_e4m3fn).view(torch.uint8).reshape(xf.shape)
+    scales = (shared + 127).to(torch.uint8)
+    return codes.contiguous(), scales.contiguous()

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 import torch
 
@@ -163,3 +164,61 @@ def test_binding_checks_shapes_on_cpu_tensors(lib):
     with pytest.raises(ValueError):
         kda.kda_chunk_fwd(q, q, q[:, :1], torch.zeros(64, 2, 128), torch.zeros(64, 2),
                           None, torch.tensor([0, 64], dtype=torch.int32), q)
+
+
+def _call_mx(lib, **over):
+    """kda_chunk_fwd_mxfp8 with fake (never dereferenced) pointers: all of these must fail on the host."""
+    a = dict(q=0x1000, qs=0x1100, k=0x2000, ks=0x2100, v=0x3000, vs=0x3100, la=0x4000, b=0x5000, s0=None,
+             cu=0x6000, n=2, T=100, H=4, dk=128, dv=128, stride=0, o=0x7000, fs=None, ck=None, ckcu=None, tr=None,
+             ws=0x10000, wsb=1 << 30)
+    a.update(over)
+    vp = ctypes.c_void_p
+    return lib.kda_chunk_fwd_mxfp8(vp(a["q"]), vp(a["qs"]), vp(a["k"]), vp(a["ks"]), vp(a["v"]), vp(a["vs"]),
+                                   vp(a["la"]), vp(a["b"]), vp(a["s0"]), vp(a["cu"]), a["n"], a["T"], a["H"],
+                                   a["dk"], a["dv"], a["stride"], vp(a["o"]), vp(a["fs"]), vp(a["ck"]),
+                                   vp(a["ckcu"]), vp(a["tr"]), vp(a["ws"]), a["wsb"], None)
+
+
+def test_mxfp8_chunk_fwd_host_argument_errors(lib):
+    assert _call_mx(lib, dk=64) == -3                     # dk = 128 only, as the bf16 path
+    assert _call_mx(lib, dv=96) == -3
+    assert _call_mx(lib, qs=None) == -1                   # every scale array is required
+    assert _call_mx(lib, vs=None) == -1
+    assert _call_mx(lib, ks=0x2102) == -2                 # q/k scales: whole 4-byte rows
+    assert _call_mx(lib, dv=64, vs=0x3101) == -2
+    assert _call_mx(lib, q=0x1008) == -2                  # codes move by TMA: 16-byte aligned
+    assert _call_mx(lib, H=0) == -1
+    assert _call_mx(lib, wsb=100) == -6
+    assert _call_mx(lib, n=0) == 0
+    # kda_chunk_fwd cannot take MXFP8 (no scales); the workspace queries size it like bf16
+    assert _call_chunk(lib, dt=2) == -1
+    assert kda.kda_chunk_fwd_workspace_bytes(4096, 1, 32, 128, 128, kda.KDA_MXFP8) == \
+        kda.kda_chunk_fwd_workspace_bytes(4096, 1, 32, 128, 128, kda.KDA_BF16)
+    assert kda.kda_chunk_fwd_workspace_bytes(4096, 1, 32, 64, 64, kda.KDA_MXFP8) == 0
+
+
+def test_mxfp8_quantizer_recipe():
+    import oracle
+    from kda_linear_attention_02_b200 import synth
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(7, 3, 128, generator=g) * torch.tensor([1e-3, 1.0, 40.0, 1e4]).repeat_interleave(32)
+    x[0, 0, 32:64] = 0.0
+    codes, scales = synth.mxfp8_quantize(x)
+    assert codes.dtype == torch.uint8 and scales.shape == (7, 3, 4)
+    assert int(scales[0, 0, 1]) == 127                    # an all-zero block gets scale 1.0
+    dec = oracle.mxfp8_decode(codes.numpy(), scales.numpy())
+    amax = x.reshape(7, 3, 4, 32).abs().amax(-1).numpy()
+    # the largest element of a block lands in [256, 448] (or saturates at 448) after its scale
+    X = 2.0 ** (scales.numpy().astype(np.int64) - 127)
+    top = amax / X
+    nz = amax > 0
+    assert np.all((top[nz] >= 256) & (top[nz] < 512))
+    # E4M3 rounding: relative error at most 2^-4 where the scaled value is a normal E4M3 number below
+    # the largest one; above 448 it saturates to 448
+    Xe = np.repeat(X, 32, axis=-1)
+    xs = np.abs(x.numpy()) / Xe
+    normal = (xs >= 2.0 ** -6) & (xs <= 448)
+    err = np.abs(dec - x.numpy())[normal] / np.abs(x.numpy())[normal]
+    assert err.max() <= 2.0 ** -4 + 1e-12
+    sat = xs > 448
+    assert np.all(np.abs(dec[sat]) == 448 * Xe[sat])
