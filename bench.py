@@ -47,6 +47,7 @@ PREFILL_READ_MX_B = 3 * 128 + 3 * 4 + 512 + 4
 # Decode bytes per (sequence, head) step: state read + write (2 x 64 KiB), q/k/v bf16, log_alpha,
 # beta, o bf16.
 DECODE_B = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2
+DECODE_MX_B = 2 * D * D * 4 + 3 * D + 3 * D // 32 + D * 4 + 4 + D * 2
 
 
 def peaks():
@@ -395,7 +396,28 @@ def run_ours(args):
               "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": round(dec_gbs, 1),
                            "peak": hbm, "unit": "GB/s", "frac": round(dec_gbs / hbm, 4),
                            "alg_bytes_per_launch": dec_bytes}}
-    del s0, dq, dk_, dv_, dla, db, state, do
+    # the same decode loop with MXFP8 q, k, v (1-byte codes + one scale byte per 32 channels)
+    mxd = (*synth.mxfp8_quantize(dq), *synth.mxfp8_quantize(dk_), *synth.mxfp8_quantize(dv_))
+    del dq, dk_, dv_
+    state.copy_(s0)
+    for t_ in range(3):
+        kda.kda_recurrent_step_mxfp8(state, *(x[t_] for x in mxd), dla[t_], db[t_], do)
+    state.copy_(s0)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for t_ in range(DEC_STEPS):
+        kda.kda_recurrent_step_mxfp8(state, *(x[t_] for x in mxd), dla[t_], db[t_], do)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mxd_ms = max_over_ranks(e0.elapsed_time(e1), world) / DEC_STEPS
+    mxd_bytes = DECODE_MX_B * DEC_N * H
+    decode["mxfp8"] = {"value": world / (mxd_ms / 1e3), "unit": "steps/s", "ms_per_step": round(mxd_ms, 5),
+                       "roofline": {"bound": "hbm", "kernel": "decode_step_kernel (MXFP8 inputs)",
+                                    "achieved": round(mxd_bytes / (mxd_ms / 1e3) / 1e9, 1), "peak": hbm,
+                                    "unit": "GB/s", "frac": round(mxd_bytes / (mxd_ms / 1e3) / 1e9 / hbm, 4),
+                                    "alg_bytes_per_launch": mxd_bytes}}
+    del s0, mxd, dla, db, state, do
 
     # ------------------------------------------------------------------ speculative decoding
     # The decode workload's 256 sequences x 32 heads; each round verifies 4 drafts per sequence

@@ -186,6 +186,18 @@ KDA_API kda_status_t kda_recurrent_step(float* state, const void* q, const void*
                                 void* o, kda_stream_t stream);
 
 /*
+ * kda_recurrent_step with MXFP8 q, k and v (the format of kda_chunk_fwd_mxfp8: E4M3 codes, one E8M0 scale
+ * per 32 consecutive channels of a (sequence, head) row).  q, k: [n,H,dk] uint8 codes with q_scale,
+ * k_scale [n,H,dk/32]; v: [n,H,dv] codes with v_scale [n,H,dv/32]; o: [n,H,dv] bf16; everything else and
+ * the supported sizes as kda_recurrent_step.  The codes are decoded exactly, so the results equal
+ * kda_recurrent_step's with the decoded values given as bf16.
+ */
+KDA_API kda_status_t kda_recurrent_step_mxfp8(float* state, const uint8_t* q, const uint8_t* q_scale,
+                           const uint8_t* k, const uint8_t* k_scale, const uint8_t* v,
+                           const uint8_t* v_scale, const float* log_alpha, const float* beta,
+                           int n, int H, int dk, int dv, void* o, kda_stream_t stream);
+
+/*
  * Speculative decoding (orkas.ai "Kimi K3 architecture" post, section "비용은 서빙 스택에서
  * 돌아옵니다", speculative-decoding item).  The recurrent state is updated in place, so a rejected
  * draft token cannot be rolled back.  Instead the caller keeps the drafts' projected inputs, which

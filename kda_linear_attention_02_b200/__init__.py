@@ -17,7 +17,7 @@ __all__ = [
     "KDA_BF16", "KDA_F32", "KDA_MXFP8", "KDA_CHUNK", "KDAError", "lib_path",
     "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_min_workspace_bytes", "kda_chunk_fwd", "kda_chunk_fwd_mxfp8",
     "kda_chunk_fwd_noalloc",
-    "kda_recurrent_step", "kda_decode_verify", "kda_decode_commit", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
+    "kda_recurrent_step", "kda_recurrent_step_mxfp8", "kda_decode_verify", "kda_decode_commit", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
     "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
     "kda_selftest_umma", "KDA_PREFIX_BLOCK", "kda_prefix_block_hashes", "kda_prefix_cache_create",
     "kda_prefix_cache_destroy", "kda_prefix_cache_lookup", "kda_prefix_cache_plan", "kda_prefix_cache_insert",
@@ -69,6 +69,8 @@ def _load():
                                         vp, vp, vp, vp, vp, vp]
     L.kda_recurrent_step.restype = i32
     L.kda_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
+    L.kda_recurrent_step_mxfp8.restype = i32
+    L.kda_recurrent_step_mxfp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]
     L.kda_decode_verify.restype = i32
     L.kda_decode_verify.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
     L.kda_decode_commit.restype = i32
@@ -322,6 +324,35 @@ def kda_recurrent_step(state, q, k, v, log_alpha, beta, o, *, stream=None):
     st = _load().kda_recurrent_step(_p(state), _p(q), _p(k), _p(v), _p(log_alpha), _p(beta), n, H, dk, dv, dt,
                                     _p(o), _stream(stream))
     _check(st, "kda_recurrent_step")
+    return o
+
+
+def kda_recurrent_step_mxfp8(state, q, q_scale, k, k_scale, v, v_scale, log_alpha, beta, o, *, stream=None):
+    """One decode step with MXFP8 q, k, v (C: kda_recurrent_step_mxfp8).
+
+    q, k [n,H,dk] and v [n,H,dv]: E4M3 codes (uint8 or torch.float8_e4m3fn); q_scale, k_scale [n,H,dk/32],
+    v_scale [n,H,dv/32]: E8M0 scales (uint8 or torch.float8_e8m0fnu); o [n,H,dv] bf16; state as
+    kda_recurrent_step.
+    """
+    _need(state, "state", None, torch.float32)
+    dev = state.device
+    n, H, dk, dv = state.shape
+    codes = (torch.uint8, torch.float8_e4m3fn)
+    scales = (torch.uint8, torch.float8_e8m0fnu)
+    if dk % 32 or dv % 32:
+        raise ValueError("dk and dv must be multiples of the 32-channel scale block")
+    _bytes_of(q, "q", (n, H, dk), dev, codes)
+    _bytes_of(k, "k", (n, H, dk), dev, codes)
+    _bytes_of(v, "v", (n, H, dv), dev, codes)
+    _bytes_of(q_scale, "q_scale", (n, H, dk // 32), dev, scales)
+    _bytes_of(k_scale, "k_scale", (n, H, dk // 32), dev, scales)
+    _bytes_of(v_scale, "v_scale", (n, H, dv // 32), dev, scales)
+    _need(o, "o", (n, H, dv), torch.bfloat16, dev)
+    _need(log_alpha, "log_alpha", (n, H, dk), torch.float32, dev)
+    _need(beta, "beta", (n, H), torch.float32, dev)
+    st = _load().kda_recurrent_step_mxfp8(_p(state), _p(q), _p(q_scale), _p(k), _p(k_scale), _p(v), _p(v_scale),
+                                          _p(log_alpha), _p(beta), n, H, dk, dv, _p(o), _stream(stream))
+    _check(st, "kda_recurrent_step_mxfp8")
     return o
 
 

@@ -305,6 +305,21 @@ kda_status_t kda_recurrent_step(float* state, const void* q, const void* k, cons
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
+kda_status_t kda_recurrent_step_mxfp8(float* state, const uint8_t* q, const uint8_t* q_scale, const uint8_t* k,
+                                      const uint8_t* k_scale, const uint8_t* v, const uint8_t* v_scale,
+                                      const float* log_alpha, const float* beta, int n, int H, int dk, int dv, void* o,
+                                      kda_stream_t stream) {
+    if (n < 0 || H <= 0) return KDA_ERR_ARG;
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+    if (n == 0) return KDA_OK;
+    if (!state || !q || !q_scale || !k || !k_scale || !v || !v_scale || !log_alpha || !beta || !o) return KDA_ERR_ARG;
+    // the state moves by 16-byte vectors; codes and scales are read byte by byte
+    if (!aligned16(state) || !aligned_to(o, 2) || !aligned4(log_alpha) || !aligned4(beta)) return KDA_ERR_ALIGN;
+    if (static_cast<long long>(n) * H > 0x7fffffffLL) return KDA_ERR_ARG;
+    return from_cuda(launch_decode_mx(state, q, q_scale, k, k_scale, v, v_scale, log_alpha, beta, o, n * H, dk, dv,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 // Shared argument checks of the two speculative-decoding calls.
 static kda_status_t check_multi(int n, int n_draft, int H, int dk, int dv, kda_dtype_t dtype) {
     if (n < 0 || H <= 0 || n_draft <= 0) return KDA_ERR_ARG;

@@ -73,22 +73,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 constexpr float kLog2e = 1.4426950408889634f;
-// MXFP8 inputs (OCP Microscaling Formats v1.0).  Two E4M3 codes (the first in the low byte) -> 2^-120
-// times their values as fp32, with integer operations only: a code's 7 magnitude bits placed at bits
-// 20..26 of an fp32 make exponent field e and mantissa m << 20, which reads 2^(e - 127) (1 + m / 8) for
-// e > 0 and m 2^-129 (an fp32 subnormal) for e = 0 -- exactly 2^-120 times the E4M3 magnitude either way;
-// the sign moves to bit 31.  (The NaN codes S.1111.111 read as +-480.)  Multiplying by 2^120 and then by
-// the shared scale is exact unless the value leaves the fp32 range.
-__device__ __forceinline__ float2 e4m3x2_scaled(uint32_t u) {
-    const uint32_t lo = ((u << 20) & 0x07F00000u) | ((u << 24) & 0x80000000u);
-    const uint32_t hi = ((u << 12) & 0x07F00000u) | ((u << 16) & 0x80000000u);
-    return make_float2(__uint_as_float(lo), __uint_as_float(hi));
-}
-constexpr float kE4M3Unscale = 1.329227995784916e36f;   // 2^120
-// E8M0 shared scale -> 2^(e - 127) (code 0 is the fp32 subnormal 2^-127, code 255 is NaN)
-__device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
-    return e == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float(e ? e << 23 : 0x00400000u);
-}
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                       pack_bf16x2(f[6], f[7]));

@@ -52,17 +52,32 @@ struct TokenIn {
     float la, k, q, v, beta;
 };
 
-template <typename T, int DK, int DV, bool OUT>
-__device__ __forceinline__ void load_token(TokenIn& x, const T* __restrict__ q, const T* __restrict__ k,
-                                           const T* __restrict__ v, const float* __restrict__ la,
-                                           const float* __restrict__ beta) {
+// Element i of a token vector: of type T, or (MX) an MXFP8 code with the scale of its 32-element block
+// (E4M3 codes, E8M0 scales: OCP Microscaling Formats v1.0), decoded exactly.
+template <typename T, bool MX>
+__device__ __forceinline__ float in_value(const void* __restrict__ p, const uint8_t* __restrict__ scale, int i) {
+    if constexpr (MX) return mx8_value(static_cast<const uint8_t*>(p)[i], scale[i >> 5]);
+    else return to_f32(static_cast<const T*>(p)[i]);
+}
+// p advanced by n elements (bytes for MX codes)
+template <typename T, bool MX>
+__device__ __forceinline__ const void* in_at(const void* p, size_t n) {
+    return static_cast<const char*>(p) + n * (MX ? 1 : sizeof(T));
+}
+
+template <typename T, int DK, int DV, bool OUT, bool MX = false>
+__device__ __forceinline__ void load_token(TokenIn& x, const void* __restrict__ q, const void* __restrict__ k,
+                                           const void* __restrict__ v, const float* __restrict__ la,
+                                           const float* __restrict__ beta, const uint8_t* __restrict__ qs = nullptr,
+                                           const uint8_t* __restrict__ ks = nullptr,
+                                           const uint8_t* __restrict__ vs = nullptr) {
     const int t = threadIdx.x;
     if (t < DK) {
         x.la = la[t];
-        x.k = to_f32(k[t]);
-        if (OUT) x.q = to_f32(q[t]);
+        x.k = in_value<T, MX>(k, ks, t);
+        if (OUT) x.q = in_value<T, MX>(q, qs, t);
     }
-    if (t < DV) x.v = to_f32(v[t]);
+    if (t < DV) x.v = in_value<T, MX>(v, vs, t);
     if (t == 0) x.beta = *beta;
 }
 
@@ -153,11 +168,14 @@ __device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>:
     }
 }
 
-template <typename T, int DK, int DV>
+// MX: q, k, v are MXFP8 codes with their scale arrays (q_scale, k_scale [n, H, dk / 32], v_scale
+// [n, H, dv / 32]) and T is the type of o (bf16).
+template <typename T, int DK, int DV, bool MX>
 __global__ void __launch_bounds__(256, 2)
-decode_step_kernel(float* __restrict__ state, const T* __restrict__ q, const T* __restrict__ k,
-                   const T* __restrict__ v, const float* __restrict__ log_alpha,
-                   const float* __restrict__ beta, T* __restrict__ o) {
+decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const void* __restrict__ k,
+                   const void* __restrict__ v, const uint8_t* __restrict__ q_scale,
+                   const uint8_t* __restrict__ k_scale, const uint8_t* __restrict__ v_scale,
+                   const float* __restrict__ log_alpha, const float* __restrict__ beta, T* __restrict__ o) {
     using DT = DecodeTiling<DK, DV, 256>;
     __shared__ DecodeSmem<DK, DV, 256> sh;
     grid_dependency_wait();   // the state (and inputs) come from earlier launches
@@ -169,7 +187,9 @@ decode_step_kernel(float* __restrict__ state, const T* __restrict__ q, const T* 
     for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg * DT::RPT + r) * DT::CG + cg);
     const size_t hk = static_cast<size_t>(head) * DK, hv = static_cast<size_t>(head) * DV;
     TokenIn x;
-    load_token<T, DK, DV, true>(x, q + hk, k + hk, v + hv, log_alpha + hk, beta + head);
+    load_token<T, DK, DV, true, MX>(x, in_at<T, MX>(q, hk), in_at<T, MX>(k, hk), in_at<T, MX>(v, hv), log_alpha + hk,
+                                    beta + head, MX ? q_scale + hk / 32 : nullptr, MX ? k_scale + hk / 32 : nullptr,
+                                    MX ? v_scale + hv / 32 : nullptr);
     stage_token<DK, DV, 256, true>(sh, 0, x);
     __syncthreads();
     token_step<T, DK, DV, 256, true>(s, sh, 0, o + hv);
@@ -259,11 +279,12 @@ cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, cuda
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, bool MX = false>
 cudaError_t launch_decode_t(float* state, const void* q, const void* k, const void* v, const float* la,
-                            const float* beta, void* o, int nh, cudaStream_t s) {
-    return launch_chained(decode_step_kernel<T, DK, DV>, dim3(nh), dim3(256), s, state, static_cast<const T*>(q),
-                          static_cast<const T*>(k), static_cast<const T*>(v), la, beta, static_cast<T*>(o));
+                            const float* beta, void* o, int nh, cudaStream_t s, const uint8_t* qs = nullptr,
+                            const uint8_t* ks = nullptr, const uint8_t* vs = nullptr) {
+    return launch_chained(decode_step_kernel<T, DK, DV, MX>, dim3(nh), dim3(256), s, state, q, k, v, qs, ks, vs, la,
+                          beta, static_cast<T*>(o));
 }
 
 template <typename T, int DK, int DV>
@@ -296,6 +317,18 @@ cudaError_t launch_decode(float* state, const void* q, const void* k, const void
         KDA_DECODE_CASE(float, 64, 128) KDA_DECODE_CASE(float, 64, 64)
     }
 #undef KDA_DECODE_CASE
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_mx(float* state, const void* q, const uint8_t* qs, const void* k, const uint8_t* ks,
+                             const void* v, const uint8_t* vs, const float* la, const float* beta, void* o, int nh,
+                             int dk, int dv, cudaStream_t s) {
+    if (nh == 0) return cudaSuccess;
+#define KDA_DECODE_MX_CASE(DK, DV) \
+    if (dk == DK && dv == DV)       \
+        return launch_decode_t<__nv_bfloat16, DK, DV, true>(state, q, k, v, la, beta, o, nh, s, qs, ks, vs);
+    KDA_DECODE_MX_CASE(128, 128) KDA_DECODE_MX_CASE(128, 64) KDA_DECODE_MX_CASE(64, 128) KDA_DECODE_MX_CASE(64, 64)
+#undef KDA_DECODE_MX_CASE
     return cudaErrorInvalidValue;
 }
 

@@ -11,6 +11,10 @@ namespace kda {
 // Decode step (kda_decode.cu).
 cudaError_t launch_decode(float* state, const void* q, const void* k, const void* v, const float* la,
                           const float* beta, void* o, int nh, int dk, int dv, bool bf16, cudaStream_t s);
+// Decode step with MXFP8 q, k, v (codes + E8M0 scale arrays), bf16 o (kda_decode.cu).
+cudaError_t launch_decode_mx(float* state, const void* q, const uint8_t* qs, const void* k, const uint8_t* ks,
+                             const void* v, const uint8_t* vs, const float* la, const float* beta, void* o, int nh,
+                             int dk, int dv, cudaStream_t s);
 // Speculative decoding (kda_decode.cu): n_accept == nullptr verifies (outputs of all n_draft drafts, state
 // read only); otherwise commits the first n_accept[i] drafts of every sequence into the state.
 cudaError_t launch_decode_multi(float* state, const void* q, const void* k, const void* v, const float* la,

@@ -222,3 +222,15 @@ def test_mxfp8_quantizer_recipe():
     assert err.max() <= 2.0 ** -4 + 1e-12
     sat = xs > 448
     assert np.all(np.abs(dec[sat]) == 448 * Xe[sat])
+
+
+def test_mxfp8_decode_host_argument_errors(lib):
+    vp = ctypes.c_void_p
+    st, q, qs, k, ks, v, vs, la, b, o = (vp(0x1000 * (i + 1)) for i in range(10))
+    call = lambda *a, **kw: lib.kda_recurrent_step_mxfp8(*a)
+    assert call(st, q, qs, k, ks, v, vs, la, b, 2, 0, 128, 128, o, None) == -1        # no heads
+    assert call(st, q, qs, k, ks, v, vs, la, b, 2, 4, 96, 128, o, None) == -3         # dk
+    assert call(st, q, None, k, ks, v, vs, la, b, 2, 4, 128, 128, o, None) == -1      # a scale array missing
+    assert call(vp(0x1004), q, qs, k, ks, v, vs, la, b, 2, 4, 128, 128, o, None) == -2
+    assert call(st, q, qs, k, ks, v, vs, la, b, 2, 4, 128, 128, vp(0xA001), None) == -2   # o is bf16
+    assert call(st, q, qs, k, ks, v, vs, la, b, 0, 4, 128, 128, o, None) == 0         # empty batch

@@ -160,3 +160,54 @@ def test_mxfp8_prefill_workload_sampled():
         for j in range(len(r["marks"])):
             agg.add("checkpoints", f32np(ck[ckcu[i] + j, h]), r["marks"][j], f"ckpt {j} seq {i} head {h}")
     agg.check()
+
+
+# ---------------------------------------------------------------------------- decode step with MXFP8 inputs
+
+def _mx_decode_inputs(n, H, dk, dv, steps, seed):
+    s0, q, k, v, la, b = synth.make_decode_inputs(n, H, dk, dv, dtype=BF, device=DEV, seed=seed, steps=steps)
+    f = [0.5, 1.0, 0.25, 0.125]
+    qs_ = _skew(q, [1.0, 4.0, 0.25, 2.0])
+    qs_ = qs_ / qs_.norm(dim=-1, keepdim=True).clamp_min(1e-6)
+    ks_ = _skew(k, [1.0, 2.0, 4.0, 8.0])
+    ks_ = ks_ / ks_.norm(dim=-1, keepdim=True).clamp_min(1e-6)
+    mx = (*synth.mxfp8_quantize(qs_), *synth.mxfp8_quantize(ks_), *synth.mxfp8_quantize(_skew(v, f)))
+    return s0, mx, la, b
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (128, 64), (64, 128), (64, 64)])
+def test_mxfp8_decode_steps_vs_oracle(dk, dv):
+    n, H, steps = 5, 3, 6
+    s0, mx, la, b = _mx_decode_inputs(n, H, dk, dv, steps, seed=31)
+    state = s0.clone()
+    outs = []
+    for t in range(steps):
+        o = torch.full((n, H, dv), float("nan"), dtype=BF, device=DEV)
+        kda.kda_recurrent_step_mxfp8(state, *(x[t] for x in mx), la[t], b[t], o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    dec = [oracle.mxfp8_decode(mx[j].cpu().numpy(), mx[j + 1].cpu().numpy()) for j in (0, 2, 4)]
+    agg = _Agg(BF)
+    for i in range(n):
+        for h in range(H):
+            r = oracle.kda_seq(dec[0][:, i, h], dec[1][:, i, h], dec[2][:, i, h], f32np(la[:, i, h]),
+                               f32np(b[:, i, h]), s0=s0[i, h].double().cpu().numpy())
+            o = np.stack([f32np(outs[t][i, h]) for t in range(steps)])
+            agg.add("o", o, r["o"], f"decode o seq {i} head {h}", per_slice_rel=False)
+            agg.add("state", f32np(state[i, h]), r["state"], f"decode state seq {i} head {h}")
+    agg.check()
+
+
+def test_mxfp8_decode_equals_bf16_decode_on_decoded_inputs():
+    n, H, dk, dv, steps = 7, 4, 128, 128, 4
+    s0, mx, la, b = _mx_decode_inputs(n, H, dk, dv, steps, seed=32)
+    q, k, v = _torch_decoded_bf16(mx)
+    sa, sb = s0.clone(), s0.clone()
+    for t in range(steps):
+        oa = torch.empty(n, H, dv, dtype=BF, device=DEV)
+        ob = torch.empty(n, H, dv, dtype=BF, device=DEV)
+        kda.kda_recurrent_step_mxfp8(sa, *(x[t] for x in mx), la[t], b[t], oa)
+        kda.kda_recurrent_step(sb, q[t], k[t], v[t], la[t], b[t], ob)
+        torch.cuda.synchronize()
+        assert torch.equal(oa, ob), f"step {t}: o differs from the bf16 decode on the decoded inputs"
+    assert torch.equal(sa, sb)
