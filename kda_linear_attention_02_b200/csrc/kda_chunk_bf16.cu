@@ -247,6 +247,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     while (valid) {
         const int n = loc.y;
         uint8_t* pkt = packets + static_cast<size_t>(item) * P::BYTES;
+        const long long nitem = item + gridDim.x;   // this CTA's next item
+        const int nh = static_cast<int>(nitem % H);
+        const bool nvalid = nloc.y > 0;
         if constexpr (!MX) {
             if (t < 64) bet[t] = t < n ? beta[(static_cast<size_t>(loc.x) + t) * H + h] : 0.f;
         } else {
@@ -302,8 +305,15 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                                      : 0u;
                 }
             }
+            // the staging tiles have been read into registers: after the fence and the barrier the next
+            // item's tiles may overwrite them (the TMA writes through the async proxy)
+            fence_proxy_async_smem();
             if (t == 0) bulk_wait_read0();   // the previous item's packet staging has been read out
             __syncthreads();
+            if (t == 0 && nvalid) {
+                issue_tile_loads<DV, MX>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.x);
+                load_pending = true;
+            }
             if (hh) {   // second half of the tile: add the first half's total
                 const float2 ob = *reinterpret_cast<const float2*>(tot + (q8 - 1) * 128 + c0);
 #pragma unroll
@@ -418,14 +428,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
             umma_commit(&bar_mma);
         }
-        // prefetch the next item's tiles into the (now free) staging area; look one more item ahead
-        const long long nitem = item + gridDim.x;
-        const int nh = static_cast<int>(nitem % H);
-        const bool nvalid = nloc.y > 0;
-        if (t == 0 && nvalid) {
-            issue_tile_loads<DV, MX>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.x);
-            load_pending = true;
-        }
+        // the next item's rows (MXFP8 inputs); look one more item ahead
         if (nvalid) fetch_rows(nloc, nh, par ^ 1);
         const int2 nnloc = entry(nitem + gridDim.x);
         {
