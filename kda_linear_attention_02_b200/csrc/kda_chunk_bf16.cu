@@ -314,6 +314,10 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 issue_tile_loads<DV, MX>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.x);
                 load_pending = true;
             }
+            if constexpr (!MX) {   // and the next item's beta rows into L2, for the load at its start
+                if (nvalid && t >= 256 && t - 256 < nloc.y)
+                    prefetch_l2(beta + (static_cast<size_t>(nloc.x) + (t - 256)) * H + nh);
+            }
             if (hh) {   // second half of the tile: add the first half's total
                 const float2 ob = *reinterpret_cast<const float2*>(tot + (q8 - 1) * 128 + c0);
 #pragma unroll

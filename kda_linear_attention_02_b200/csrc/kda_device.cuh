@@ -100,6 +100,8 @@ __device__ __forceinline__ void bulk_s2g(void* dst, const void* src_smem, uint32
                  "r"(bytes)
                  : "memory");
 }
+// Warm L2 with the line holding p (no data returned; nothing waits on it).
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 // 4-byte asynchronous copy global -> shared in the calling thread's cp.async group; src_bytes = 0 writes
 // zeros and reads nothing.  cp_async_wait_all makes the thread's copies visible to that thread.
 __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src, uint32_t src_bytes) {
