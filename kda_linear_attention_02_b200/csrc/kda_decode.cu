@@ -183,13 +183,41 @@ decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const 
     const int t = threadIdx.x, cg = t % DT::CG, rg = t / DT::CG;
     float4* S = reinterpret_cast<float4*>(state + static_cast<size_t>(head) * DK * DV);
     float4 s[DT::RPT];
-#pragma unroll
-    for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg * DT::RPT + r) * DT::CG + cg);
     const size_t hk = static_cast<size_t>(head) * DK, hv = static_cast<size_t>(head) * DV;
     TokenIn x;
-    load_token<T, DK, DV, true, MX>(x, in_at<T, MX>(q, hk), in_at<T, MX>(k, hk), in_at<T, MX>(v, hv), log_alpha + hk,
-                                    beta + head, MX ? q_scale + hk / 32 : nullptr, MX ? k_scale + hk / 32 : nullptr,
-                                    MX ? v_scale + hv / 32 : nullptr);
+    if constexpr (MX) {
+        // the token's bytes are loaded first, ahead of the 64 KiB state stream in the load queue, and
+        // decoded once the state loads have been issued
+        const uint8_t* qc = static_cast<const uint8_t*>(q) + hk;
+        const uint8_t* kc = static_cast<const uint8_t*>(k) + hk;
+        const uint8_t* vc = static_cast<const uint8_t*>(v) + hv;
+        uint32_t rq = 0, rk = 0, rqs = 0, rks = 0, rv = 0, rvs = 0;
+        if (t < DK) {
+            x.la = log_alpha[hk + t];
+            rk = kc[t];
+            rks = k_scale[hk / 32 + (t >> 5)];
+            rq = qc[t];
+            rqs = q_scale[hk / 32 + (t >> 5)];
+        }
+        if (t < DV) {
+            rv = vc[t];
+            rvs = v_scale[hv / 32 + (t >> 5)];
+        }
+        if (t == 0) x.beta = beta[head];
+        asm volatile("" ::: "memory");
+#pragma unroll
+        for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg * DT::RPT + r) * DT::CG + cg);
+        if (t < DK) {
+            x.k = mx8_value(rk, rks);
+            x.q = mx8_value(rq, rqs);
+        }
+        if (t < DV) x.v = mx8_value(rv, rvs);
+    } else {
+#pragma unroll
+        for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg * DT::RPT + r) * DT::CG + cg);
+        load_token<T, DK, DV, true>(x, in_at<T, false>(q, hk), in_at<T, false>(k, hk), in_at<T, false>(v, hv),
+                                    log_alpha + hk, beta + head);
+    }
     stage_token<DK, DV, 256, true>(sh, 0, x);
     __syncthreads();
     token_step<T, DK, DV, 256, true>(s, sh, 0, o + hv);
