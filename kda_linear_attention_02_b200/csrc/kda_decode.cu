@@ -260,20 +260,38 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
         }
         if (steps == 0) return;
     }
+    auto row_of = [&](int d) { return (static_cast<size_t>(seq) * n_draft + d) * H + h; };
+    // the first draft's inputs are loaded ahead of the state stream, so that they do not queue behind it,
+    // and converted once the state loads have been issued
+    TokenIn x;
+    T rq{}, rk{}, rv{};
+    {
+        const size_t row = row_of(0);
+        if (t < DK) {
+            x.la = log_alpha[row * DK + t];
+            rk = k[row * DK + t];
+            if (VERIFY) rq = q[row * DK + t];
+        }
+        if (t < DVS) rv = v[row * DV + j0 + t];
+        if (t == 0) x.beta = beta[row];
+    }
+    asm volatile("" ::: "memory");
     // state rows are DV wide; this CTA's float4 column groups start at j0
     float4* S = reinterpret_cast<float4*>(state + static_cast<size_t>(head) * DK * DV + j0);
     float4 s[DT::RPT];
 #pragma unroll
     for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg * DT::RPT + r) * (DV / 4) + cg);
+    if (t < DK) {
+        x.k = to_f32(rk);
+        if (VERIFY) x.q = to_f32(rq);
+    }
+    if (t < DVS) x.v = to_f32(rv);
     // token d + 1's inputs are loaded into registers while token d is applied, then staged
-    auto row_of = [&](int d) { return (static_cast<size_t>(seq) * n_draft + d) * H + h; };
     auto load = [&](TokenIn& x, int d) {
         const size_t row = row_of(d);
         load_token<T, DK, DVS, VERIFY>(x, VERIFY ? q + row * DK : nullptr, k + row * DK, v + row * DV + j0,
                                        log_alpha + row * DK, beta + row);
     };
-    TokenIn x;
-    load(x, 0);
     stage_token<DK, DVS, NT, VERIFY>(sh, 0, x);
     for (int d = 0; d < steps; ++d) {
         const int par = d & 1;
