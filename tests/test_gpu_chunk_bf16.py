@@ -12,7 +12,6 @@ import torch
 
 import kda_linear_attention_02_b200 as kda
 from kda_linear_attention_02_b200 import synth
-from kda_testlib import assert_close, f32np, oracle_slices
 from test_gpu_basic import _check_chunk, _run_chunk
 
 pytestmark = pytest.mark.gpu
