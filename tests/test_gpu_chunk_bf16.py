@@ -6,7 +6,6 @@ several tiles, checkpoints, transitions, windows); the full-size workloads are c
 """
 import math
 
-import numpy as np
 import pytest
 import torch
 
