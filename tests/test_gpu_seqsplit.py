@@ -7,7 +7,6 @@ is run from it. The concatenated outputs and the last segment's final state matc
 the unsplit run. The distributed wrapper is then run in a one-rank NCCL group, where its result must
 equal the plain run bit for bit.
 """
-import os
 import socket
 
 import numpy as np

@@ -10,7 +10,6 @@
 """
 import gc
 
-import numpy as np
 import pytest
 import torch
 
