@@ -339,3 +339,19 @@ def test_mxfp8_decode_is_scale_times_element(oracle_mod):
     elem = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
     scl = torch.from_numpy(scales).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
     np.testing.assert_array_equal(out, elem * np.repeat(scl, 32, axis=-1))
+
+
+def test_resuming_from_a_state_continues_the_sequence(oracle_mod):
+    # T tokens, then n more from the state they leave, is the run over T + n tokens: outputs, states and
+    # transition (the step map is applied token by token, so the split point changes nothing)
+    rng = np.random.default_rng(17)
+    T, n, dk, dv = 23, 9, 6, 5
+    q, k, v, la, b = _rand_inputs(rng, T + n, dk, dv)
+    s0 = rng.standard_normal((dk, dv))
+    full = oracle_mod.kda_seq(q, k, v, la, b, s0=s0, marks=[T], want_transition=True)
+    head = oracle_mod.kda_seq(q[:T], k[:T], v[:T], la[:T], b[:T], s0=s0, want_transition=True)
+    tail = oracle_mod.kda_seq(q[T:], k[T:], v[T:], la[T:], b[T:], s0=head["state"], want_transition=True)
+    np.testing.assert_array_equal(full["marks"][0], head["state"])
+    np.testing.assert_allclose(np.concatenate([head["o"], tail["o"]]), full["o"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(tail["state"], full["state"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(tail["transition"] @ head["transition"], full["transition"], rtol=0, atol=1e-12)
