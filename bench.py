@@ -186,6 +186,34 @@ def cpu_oracle_sample(inp, budget_s=12.0, max_slices=None):
                       f"{dt:.1f} s on {threads} threads; tokens/s = token-heads/s / {Hh}"}
 
 
+def cpu_oracle_decode_sample(s0, q, k, v, la, b, budget_s=6.0, max_slices=512):
+    """Times the fp64 oracle (as it stands) on the decode workload: whole (sequence, head) slices, each
+    one head's state carried through all the steps, as many as fit the time budget; steps/s of the whole
+    workload is extrapolated from the sample.  q, k, v, la: [steps, n, H, d]; b: [steps, n, H]."""
+    import oracle
+    steps, n, Hh = b.shape
+
+    def job(i, h):
+        f = lambda t: t.float().cpu().numpy()
+        return dict(q=f(q[:, i, h]), k=f(k[:, i, h]), v=f(v[:, i, h]), log_alpha=f(la[:, i, h]), beta=f(b[:, i, h]),
+                    s0=s0[i, h].double().cpu().numpy(), want_o=True)
+
+    threads = oracle.threads_used()
+    t0 = time.perf_counter()
+    oracle.kda_seq(**job(0, 0))
+    one = time.perf_counter() - t0
+    m = max(1, min(n * Hh, max_slices, int(budget_s * threads / max(one, 1e-3))))
+    keys = [(i, h) for i in range(n) for h in range(Hh)][:m]
+    jobs = [(key, job(*key)) for key in keys]
+    t0 = time.perf_counter()
+    oracle.run_slices(jobs, threads)
+    dt = time.perf_counter() - t0
+    whole_s = dt * (n * Hh) / m
+    return {"value": steps / whole_s, "unit": "steps/s", "cores": threads, "kind": "oracle",
+            "sample": f"{m} of {n * Hh} (sequence, head) slices x {steps} steps, fp64, {dt:.1f} s on {threads} "
+                      f"threads; steps/s of the whole workload extrapolated from the sample"}
+
+
 def run_ours(args):
     import torch
     import kda_linear_attention_02_b200 as kda
@@ -396,6 +424,8 @@ def run_ours(args):
               "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": round(dec_gbs, 1),
                            "peak": hbm, "unit": "GB/s", "frac": round(dec_gbs / hbm, 4),
                            "alg_bytes_per_launch": dec_bytes}}
+    # kept for the oracle's decode timing, which runs after the clock sampling has stopped
+    dec_in = (s0, dq, dk_, dv_, dla, db) if rank == 0 and world == 1 and not args.no_cpu_baseline else None
     # the same decode loop with MXFP8 q, k, v (1-byte codes + one scale byte per 32 channels)
     mxd = (*synth.mxfp8_quantize(dq), *synth.mxfp8_quantize(dk_), *synth.mxfp8_quantize(dv_))
     del dq, dk_, dv_
@@ -492,6 +522,9 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(inp)
+    if dec_in is not None:
+        decode["cpu_baseline"] = cpu_oracle_decode_sample(*dec_in)
+        dec_in = None
 
     if rank == 0:
         line = {
