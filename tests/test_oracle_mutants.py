@@ -39,6 +39,10 @@ MUTANTS = [
     ("compose with M transposed", "acc += Ms[(size_t)i * dk + m] * X[(size_t)m * dv + j];",
      "acc += Ms[(size_t)m * dk + i] * X[(size_t)m * dv + j];", 1),
     ("compose without the zero-start state", "double acc = Zs[(size_t)i * dv + j];", "double acc = 0.0;", 1),
+    ("initial state ignored", "    if (s0) memcpy(S, s0, sizeof(double) * (size_t)dk * dv);", "    (void)s0;", 1),
+    ("initial state read transposed", "    if (s0) memcpy(S, s0, sizeof(double) * (size_t)dk * dv);",
+     "    if (s0) for (int i = 0; i < dk; ++i) for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] = "
+     "s0[(size_t)(j % dk) * dv + (i % dv)];", 1),
     ("E4M3 exponent bias 8", "else mag = ldexp(1.0 + (double)m / 8.0, e - 7);",
      "else mag = ldexp(1.0 + (double)m / 8.0, e - 8);", 1),
     ("E4M3 subnormals read as normals", "if (e == 0) mag = ldexp((double)m / 8.0, -6);",
