@@ -2,7 +2,8 @@
 
   * long-context prefill: B=1, T=1,048,576, H=32, dk=dv=128, bf16, log_alpha = -5 sigmoid(N(2,1)) (near
     the floor), random fp32 initial state ~ N(0, 0.02), fp32 checkpoints every 512 tokens;
-  * decode: 256 sequences x 32 heads of 128 x 128 fp32 state, 1024 consecutive steps;
+  * decode: 256 sequences x 32 heads of 128 x 128 fp32 state, 1024 consecutive steps, with bf16 and with
+    MXFP8 q, k, v;
   * varlen: 64 sequences with lengths uniform in [1024, 65536] (seed 1) packed by cu_seqlens,
     processed through a windowed workspace; half the sequences resumed from a checkpoint at a
     512-token boundary; every sequence split into 8 segments whose transitions and zero-start states
@@ -83,6 +84,33 @@ def test_decode_256x32_1024_steps():
                            f32np(b[:, i, h]), s0=s0[i, h].double().cpu().numpy())
         agg.add("o", f32np(outs[:, pi]), r["o"], f"decode o ({i},{h})")
         agg.add("state", f32np(state[i, h]), r["state"], f"decode state ({i},{h})")
+    agg.check()
+    assert torch.isfinite(state).all()
+
+
+def test_decode_256x32_1024_steps_mxfp8():
+    # the decode workload with MXFP8 q, k, v, as the benchmark times it; the oracle decodes the same bytes
+    n, H, D, steps = 256, 32, 128, 1024
+    s0, q, k, v, la, b = synth.make_decode_inputs(n, H, D, D, dtype=BF, device=DEV, seed=4, steps=steps)
+    mx = (*synth.mxfp8_quantize(q), *synth.mxfp8_quantize(k), *synth.mxfp8_quantize(v))
+    del q, k, v
+    state = s0.clone()
+    pairs = [(0, 0), (91, 12), (255, 31)]
+    outs = torch.empty(steps, len(pairs), D, dtype=BF, device=DEV)
+    o = torch.empty(n, H, D, dtype=BF, device=DEV)
+    idx_n = torch.tensor([p[0] for p in pairs], device=DEV)
+    idx_h = torch.tensor([p[1] for p in pairs], device=DEV)
+    for t_ in range(steps):
+        kda.kda_recurrent_step_mxfp8(state, *(x[t_] for x in mx), la[t_], b[t_], o)
+        outs[t_] = o[idx_n, idx_h]
+    torch.cuda.synchronize()
+    agg = _Agg(BF)
+    for pi, (i, h) in enumerate(pairs):
+        dec = [oracle.mxfp8_decode(mx[j][:, i, h].cpu().numpy(), mx[j + 1][:, i, h].cpu().numpy()) for j in (0, 2, 4)]
+        r = oracle.kda_seq(dec[0], dec[1], dec[2], f32np(la[:, i, h]), f32np(b[:, i, h]),
+                           s0=s0[i, h].double().cpu().numpy())
+        agg.add("o", f32np(outs[:, pi]), r["o"], f"MXFP8 decode o ({i},{h})")
+        agg.add("state", f32np(state[i, h]), r["state"], f"MXFP8 decode state ({i},{h})")
     agg.check()
     assert torch.isfinite(state).all()
 
