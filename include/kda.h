@@ -23,13 +23,15 @@
  *    decode state must be 16-byte aligned (TMA tiles and 16-byte vectors); beta, the int32 tables and
  *    the decode step's per-token inputs need only their natural alignment.  The workspace must be
  *    256-byte aligned.
- *  - dtype (kda_dtype_t) is the element type of q, k, v and o.  log_alpha, beta and all states are
- *    fp32 always.
+ *  - dtype (kda_dtype_t) is the element type of q, k, v and o (KDA_BF16, KDA_F32).  The *_mxfp8 entry
+ *    points take q, k, v as MXFP8 codes with their scale arrays and write a bf16 o.  log_alpha, beta
+ *    and all states are fp32 always.
  *  - Calls are asynchronous on `stream`.  Argument errors that the host can see are returned before
  *    anything is launched.  Errors that only the device can see (a bad cu_seqlens table, a bounded
  *    wait that ran out) are recorded in the per-device status word and read with
  *    kda_get_device_status; the kernels never trap.
- *  - Supported sizes: dk, dv in {64, 128} for KDA_F32; dk = 128 and dv in {64, 128} for KDA_BF16.
+ *  - Supported sizes: dk, dv in {64, 128} for KDA_F32; dk = 128 and dv in {64, 128} for KDA_BF16 and
+ *    for kda_chunk_fwd_mxfp8; dk, dv in {64, 128} for the decode calls of every type.
  */
 #ifndef KDA_H_
 #define KDA_H_
