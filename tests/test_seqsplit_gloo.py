@@ -1,4 +1,4 @@
-"""Sequence split, exchange step on CPU: two gloo ranks all-gather their fixed-size (transition,
+"""Sequence split, exchange step on CPU: two or four gloo ranks all-gather their fixed-size (transition,
 zero-start state) summaries; every rank must receive all summaries in rank order, bit for bit."""
 import os
 import socket
@@ -39,9 +39,9 @@ def _worker(rank, world, port, H, dk, dv, q):
             dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128)])
-def test_gather_segment_summaries_two_ranks(dk, dv):
-    world, H = 2, 3
+@pytest.mark.parametrize("world,dk,dv", [(2, 128, 128), (2, 64, 128), (4, 128, 64)])
+def test_gather_segment_summaries(world, dk, dv):
+    H = 3
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -51,4 +51,4 @@ def test_gather_segment_summaries_two_ranks(dk, dv):
     res = dict(q.get(timeout=120) for _ in range(world))
     for p in procs:
         p.join(timeout=60)
-    assert res == {0: True, 1: True}
+    assert res == {r: True for r in range(world)}
