@@ -154,9 +154,10 @@ def barrier(world):
         dist.barrier()
 
 
-def cpu_oracle_sample(inp, budget_s=12.0, max_slices=None):
+def cpu_oracle_sample(inp, budget_s=12.0, max_slices=None, ckpt=CKPT):
     """Times the fp64 oracle (as it stands) on whole (sequence, head) slices of the workload,
-    as many as fit the time budget (estimated from one calibration slice)."""
+    as many as fit the time budget (estimated from one calibration slice).  Like the GPU step it
+    produces the outputs, the final state and the state after every `ckpt` tokens (0 = none)."""
     import oracle
     cu = inp.cu_seqlens.cpu().tolist()
     nseq = len(cu) - 1
@@ -165,8 +166,11 @@ def cpu_oracle_sample(inp, budget_s=12.0, max_slices=None):
     def job(i, h):
         a, b = cu[i], cu[i + 1]
         f = lambda t: t.float().cpu().numpy()
+        marks = list(range(ckpt, b - a + 1, ckpt)) if ckpt else None
+        s0 = None if inp.state0 is None else inp.state0[i, h].double().cpu().numpy()
         return dict(q=f(inp.q[a:b, h]), k=f(inp.k[a:b, h]), v=f(inp.v[a:b, h]),
-                    log_alpha=f(inp.log_alpha[a:b, h]), beta=f(inp.beta[a:b, h]), want_o=True)
+                    log_alpha=f(inp.log_alpha[a:b, h]), beta=f(inp.beta[a:b, h]), s0=s0, marks=marks,
+                    want_o=True)
 
     threads = oracle.threads_used()
     t0 = time.perf_counter()
@@ -568,8 +572,9 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "KDA prefill B=4 T=4096 H=32 dk=dv=128 bf16 inputs, zero initial state",
-                       "global_batch": B, "seq_len": T, "heads": H},
+            "config": {"workload": "KDA prefill B=4 T=4096 H=32 dk=dv=128 bf16, zero initial state, fp32 final "
+                                   "state, fp32 checkpoints every 512 tokens",
+                       "global_batch": B, "seq_len": T, "heads": H, "dk": D, "dv": D, "ckpt_stride": CKPT},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": samples[0]["cores"], "kind": "oracle",
                              "sample": f"each step: {per_step_slices} (sequence, head) slices x {T} tokens"},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

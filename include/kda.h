@@ -10,12 +10,16 @@
  *
  * with alpha_t = exp(max(log_alpha_t, ln 0.0067)): every step keeps at least 0.67 % of what it held
  * (orkas.ai "Kimi K3 architecture" post, section "GPU 코드 경로 하나를 없앤 하한").  There is no scale
- * on q.  A NaN log-decay is treated as the floor (fmaxf semantics).
+ * on q.  A NaN log-decay is treated as the floor (fmaxf semantics).  Precondition: log_alpha <= 0 (a
+ * decay in (0, 1], i.e. forgetting).  The bf16 chunk path relies on it for the in-tile bound e^80.09 of
+ * the floor section; a positive log-decay is outside the contract and can give inf or NaN there with
+ * no status code.
  *
  * Conventions for every entry point:
  *  - Pointers are DEVICE pointers unless the argument says "host".  The caller owns every buffer; the
- *    library never allocates device memory and keeps no state between calls apart from one status
- *    word per device (see kda_get_device_status).
+ *    library never allocates device memory.  Between calls it keeps one status word per device (see
+ *    kda_get_device_status) and one fixed scratch array per device that only kda_chunk_fwd_noalloc
+ *    uses (KDA_NOALLOC_SCRATCH_BYTES, compiled into the library; see that entry point).
  *  - Layouts are dense row-major, token-major with heads interleaved:
  *        q, k, log_alpha: [T_tot, H, dk]     v, o: [T_tot, H, dv]     beta: [T_tot, H]
  *        states: [N, H, dk, dv] fp32 (dv contiguous)
@@ -264,23 +268,43 @@ KDA_API kda_status_t kda_segment_compose(const float* transitions, const float* 
  * kda_prefix_cache_create: a directory of at most max_blocks block hashes and n_slots checkpoint
  *   slots; checkpoints are planned every unit_blocks blocks (2..12: 1024-6144 tokens) and at the last
  *   full block of a request.  Least-recently-used entries are evicted (a block entry takes its slot
- *   with it; a slot can also be taken from an older entry that keeps its hash).  Thread-safe.
+ *   with it; a slot can also be taken from an older entry that keeps its hash).  Every call takes one
+ *   lock, so several host threads may share a directory.
+ *
+ * A slot is in one of three states: free, PENDING (handed out by kda_prefix_cache_insert, its state
+ *   not yet copied) or COMMITTED (kda_prefix_cache_commit was called after the copy).  Independently a
+ *   slot is PINNED while a lookup that named it has not been released.  Lookups only return committed
+ *   slots; eviction and slot reuse only touch committed, unpinned slots.  So a resume point is never a
+ *   slot whose copy may still be in flight, and a slot never changes under a request that resumes from
+ *   it.  The copies themselves are asynchronous GPU work: commit a slot once the copy is ordered before
+ *   every later reader (e.g. after synchronising its stream, or when all work runs on one stream), and
+ *   release a pin once the kernel that read the slot is done with it (same rule).
  *
  * kda_prefix_cache_lookup: matched_blocks = the length of the request's leading run of cached
- *   hashes; resume_blocks = the deepest block end <= matched_blocks whose state is checkpointed (0 if
+ *   hashes; resume_blocks = the deepest block end <= matched_blocks whose state is committed (0 if
  *   none) and resume_slot its slot (-1 if none).  The request restarts at token 512 * resume_blocks
- *   with the slot's state.  Touches the matched entries.
+ *   with the slot's state.  Touches the matched entries and pins resume_slot (if any) until
+ *   kda_prefix_cache_release.
  *
  * kda_prefix_cache_plan: the block ends e (resume_blocks < e <= n_blocks, ascending) after which a
  *   request should store its state: multiples of unit_blocks, and n_blocks itself.  Writes at most
  *   max_out of them and returns how many there are (-1 on a bad argument).
  *
- * kda_prefix_cache_insert: records the request's n_blocks hashes and gives each planned end ends[i]
- *   a slot out_slots[i] (the existing one if that hash already has a checkpoint, else a free slot,
- *   else one taken from the least recently used checkpoint outside this request; -1 if none can be
- *   freed).  The caller then copies the state after 512 * ends[i] tokens into that slot.
+ * kda_prefix_cache_insert: records the request's n_blocks hashes and, for each planned end ends[i],
+ *   writes out_slots[i]: a slot (>= 0, now PENDING) into which the caller copies the state after
+ *   512 * ends[i] tokens and then commits; KDA_PREFIX_STORED if that block end already has a
+ *   checkpoint slot (nothing to copy); KDA_PREFIX_NO_SLOT if every slot is busy or was used by this
+ *   request.  A new slot is a free one, else one taken from the least recently used committed,
+ *   unpinned checkpoint outside this request.
+ *
+ * kda_prefix_cache_commit: marks the given slots (out_slots of an insert; negative entries are
+ *   skipped) as holding their states.  kda_prefix_cache_abort gives pending slots back instead (their
+ *   copies will not happen; committed slots in the list are left alone).  kda_prefix_cache_release
+ *   ends one pin of a slot returned by a lookup (a negative slot is accepted and ignored).
  */
 #define KDA_PREFIX_BLOCK 512
+#define KDA_PREFIX_NO_SLOT (-1)
+#define KDA_PREFIX_STORED (-2)
 typedef struct kda_prefix_cache kda_prefix_cache;
 KDA_API int64_t kda_prefix_block_hashes(const int32_t* tokens, int64_t n_tokens, uint64_t seed, uint64_t* hashes);
 KDA_API kda_status_t kda_prefix_cache_create(int64_t max_blocks, int n_slots, int unit_blocks,
@@ -292,11 +316,17 @@ KDA_API int64_t kda_prefix_cache_plan(const kda_prefix_cache* cache, int64_t n_b
                               int64_t* out_ends, int64_t max_out);
 KDA_API kda_status_t kda_prefix_cache_insert(kda_prefix_cache* cache, const uint64_t* hashes, int64_t n_blocks,
                                      const int64_t* ends, int64_t n_ends, int32_t* out_slots);
+KDA_API kda_status_t kda_prefix_cache_commit(kda_prefix_cache* cache, const int32_t* slots, int64_t n);
+KDA_API kda_status_t kda_prefix_cache_abort(kda_prefix_cache* cache, const int32_t* slots, int64_t n);
+KDA_API kda_status_t kda_prefix_cache_release(kda_prefix_cache* cache, int32_t slot);
 KDA_API kda_status_t kda_prefix_cache_stats(const kda_prefix_cache* cache, int64_t* n_blocks_cached,
                                     int32_t* n_slots_used);
 
 /*
- * Host-only, pure: checkpoint offsets for kda_chunk_fwd.  host_ckpt_cu[0] = 0 and
+ * Host-only, pure: checkpoint offsets for kda_chunk_fwd's sparse state checkpoints (orkas.ai "Kimi K3
+ * architecture" post, section "비용은 서빙 스택에서 돌아옵니다", prefix-reuse item: states are kept
+ * only at some 512-token hash ends, so each sequence stores floor(len / stride) of them and the
+ * sequences' checkpoints are packed one after another).  host_ckpt_cu[0] = 0 and
  * host_ckpt_cu[i+1] = host_ckpt_cu[i] + floor(len_i / stride) with len_i from host_cu_seqlens
  * (host int32 [n+1]).  Returns KDA_ERR_ARG on a bad stride or a decreasing table.
  */

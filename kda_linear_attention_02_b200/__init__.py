@@ -21,13 +21,16 @@ __all__ = [
     "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
     "kda_selftest_umma", "KDA_PREFIX_BLOCK", "kda_prefix_block_hashes", "kda_prefix_cache_create",
     "kda_prefix_cache_destroy", "kda_prefix_cache_lookup", "kda_prefix_cache_plan", "kda_prefix_cache_insert",
-    "kda_prefix_cache_stats",
+    "kda_prefix_cache_commit", "kda_prefix_cache_abort", "kda_prefix_cache_release", "kda_prefix_cache_stats",
+    "KDA_PREFIX_NO_SLOT", "KDA_PREFIX_STORED",
 ]
 
 KDA_BF16 = 0
 KDA_F32 = 1
 KDA_MXFP8 = 2
 KDA_PREFIX_BLOCK = 512
+KDA_PREFIX_NO_SLOT = -1     # kda_prefix_cache_insert: no slot could be given for that block end
+KDA_PREFIX_STORED = -2      # kda_prefix_cache_insert: that block end already has a checkpoint slot
 KDA_CHUNK = 64
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -88,6 +91,11 @@ def _load():
     L.kda_prefix_cache_plan.argtypes = [vp, i64, i64, vp, i64]
     L.kda_prefix_cache_insert.restype = i32
     L.kda_prefix_cache_insert.argtypes = [vp, vp, i64, vp, i64, vp]
+    for name in ("kda_prefix_cache_commit", "kda_prefix_cache_abort"):
+        getattr(L, name).restype = i32
+        getattr(L, name).argtypes = [vp, vp, i64]
+    L.kda_prefix_cache_release.restype = i32
+    L.kda_prefix_cache_release.argtypes = [vp, i32]
     L.kda_prefix_cache_stats.restype = i32
     L.kda_prefix_cache_stats.argtypes = [vp, i64p, ctypes.POINTER(i32)]
     L.kda_segment_compose.restype = i32
@@ -533,6 +541,30 @@ def kda_prefix_cache_insert(cache, hashes, ends):
     _check(_load().kda_prefix_cache_insert(cache, h.ctypes.data, len(h), e.ctypes.data, len(e), out.ctypes.data),
            "kda_prefix_cache_insert")
     return out[:len(e)].tolist()
+
+
+def _slot_array(slots):
+    import numpy as np
+    return np.ascontiguousarray(np.asarray(list(slots), dtype=np.int32))
+
+
+def kda_prefix_cache_commit(cache, slots):
+    """Mark the slots handed out by an insert as holding their copied states (C: kda_prefix_cache_commit)."""
+    a = _slot_array(slots)
+    _check(_load().kda_prefix_cache_commit(cache, a.ctypes.data if a.size else None, a.size),
+           "kda_prefix_cache_commit")
+
+
+def kda_prefix_cache_abort(cache, slots):
+    """Give pending slots back when their copies will not happen (C: kda_prefix_cache_abort)."""
+    a = _slot_array(slots)
+    _check(_load().kda_prefix_cache_abort(cache, a.ctypes.data if a.size else None, a.size),
+           "kda_prefix_cache_abort")
+
+
+def kda_prefix_cache_release(cache, slot):
+    """End the pin that a lookup put on its resume slot (C: kda_prefix_cache_release)."""
+    _check(_load().kda_prefix_cache_release(cache, int(slot)), "kda_prefix_cache_release")
 
 
 def kda_prefix_cache_stats(cache):

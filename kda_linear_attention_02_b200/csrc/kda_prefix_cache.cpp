@@ -51,8 +51,15 @@ struct kda_prefix_cache {
     std::set<std::pair<uint64_t, uint64_t>> lru;         // (last_use, hash) of every entry
     std::set<std::pair<uint64_t, uint64_t>> lru_slots;   // (last_use, hash) of entries holding a slot
     std::vector<int32_t> free_slots;
+    // Per slot: handed out by an insert whose state copy has not been committed yet, and the number
+    // of lookups that named it as a resume point and have not released it.  A slot in either state is
+    // never returned by a lookup (pending) nor handed to another entry (pending or pinned).
+    std::vector<uint8_t> pending;
+    std::vector<int32_t> pins;
+    std::vector<uint64_t> owner;   // hash of the entry holding each slot (meaningful while it is held)
     mutable std::mutex mu;
 
+    bool slot_busy(int32_t s) const { return s >= 0 && (pending[s] || pins[s] > 0); }
     void touch(uint64_t h, Entry& e) {
         lru.erase({e.last_use, h});
         if (e.slot >= 0) lru_slots.erase({e.last_use, h});
@@ -64,15 +71,34 @@ struct kda_prefix_cache {
         if (e.slot < 0) return;
         lru_slots.erase({e.last_use, h});
         free_slots.push_back(e.slot);
+        pending[e.slot] = 0;
         e.slot = -1;
     }
-    void evict_block() {   // the least recently used entry, with its slot
-        const auto it = lru.begin();
-        const uint64_t h = it->second;
-        Entry& e = blocks[h];
-        drop_slot(h, e);
-        lru.erase(it);
-        blocks.erase(h);
+    // Evicts the least recently used entry that was last used before `start` and whose slot (if any)
+    // is neither pending nor pinned, together with its slot.  False if there is none.
+    bool evict_block(uint64_t start) {
+        for (auto it = lru.begin(); it != lru.end() && it->first <= start; ++it) {
+            const uint64_t h = it->second;
+            Entry& e = blocks[h];
+            if (slot_busy(e.slot)) continue;
+            drop_slot(h, e);
+            lru.erase(it);
+            blocks.erase(h);
+            return true;
+        }
+        return false;
+    }
+    // Frees the slot of the least recently used slot-holding entry last used before `start` whose slot
+    // is committed and unpinned (the entry keeps its hash).  False if there is none.
+    bool free_lru_slot(uint64_t start) {
+        for (auto it = lru_slots.begin(); it != lru_slots.end() && it->first <= start; ++it) {
+            const uint64_t h = it->second;
+            Entry& e = blocks[h];
+            if (slot_busy(e.slot)) continue;
+            drop_slot(h, e);
+            return true;
+        }
+        return false;
     }
 };
 
@@ -104,6 +130,9 @@ kda_status_t kda_prefix_cache_create(int64_t max_blocks, int n_slots, int unit_b
     c->n_slots = n_slots;
     c->unit_blocks = unit_blocks;
     c->free_slots.reserve(n_slots);
+    c->pending.assign(static_cast<size_t>(n_slots), 0);
+    c->pins.assign(static_cast<size_t>(n_slots), 0);
+    c->owner.assign(static_cast<size_t>(n_slots), 0);
     for (int s = n_slots - 1; s >= 0; --s) c->free_slots.push_back(s);   // slot 0 handed out first
     *out = c;
     return KDA_OK;
@@ -122,11 +151,13 @@ kda_status_t kda_prefix_cache_lookup(kda_prefix_cache* c, const uint64_t* hashes
         auto it = c->blocks.find(hashes[m]);
         if (it == c->blocks.end()) break;
         c->touch(it->first, it->second);
-        if (it->second.slot >= 0) {
+        const int32_t sl = it->second.slot;
+        if (sl >= 0 && !c->pending[sl]) {   // only a checkpoint whose state has been committed
             r = m + 1;
-            slot = it->second.slot;
+            slot = sl;
         }
     }
+    if (slot >= 0) ++c->pins[slot];          // held until kda_prefix_cache_release
     *matched_blocks = m;
     *resume_blocks = r;
     *resume_slot = slot;
@@ -160,31 +191,64 @@ kda_status_t kda_prefix_cache_insert(kda_prefix_cache* c, const uint64_t* hashes
     for (int64_t b = 0; b < n_blocks; ++b) {
         auto it = c->blocks.find(hashes[b]);
         if (it == c->blocks.end()) {
-            while (static_cast<int64_t>(c->blocks.size()) >= c->max_blocks && !c->lru.empty() &&
-                   c->lru.begin()->first <= start)
-                c->evict_block();
+            while (static_cast<int64_t>(c->blocks.size()) >= c->max_blocks && c->evict_block(start)) {
+            }
             if (static_cast<int64_t>(c->blocks.size()) >= c->max_blocks) break;   // this request fills the cache
             it = c->blocks.emplace(hashes[b], Entry{}).first;
         }
         c->touch(it->first, it->second);
     }
     for (int64_t i = 0; i < n_ends; ++i) {
-        out_slots[i] = -1;
+        out_slots[i] = KDA_PREFIX_NO_SLOT;
         auto it = c->blocks.find(hashes[ends[i] - 1]);
         if (it == c->blocks.end()) continue;
         Entry& e = it->second;
-        if (e.slot < 0) {
-            if (c->free_slots.empty() && !c->lru_slots.empty() && c->lru_slots.begin()->first <= start) {
-                const uint64_t victim = c->lru_slots.begin()->second;
-                c->drop_slot(victim, c->blocks[victim]);
-            }
-            if (c->free_slots.empty()) continue;
-            e.slot = c->free_slots.back();
-            c->free_slots.pop_back();
-            c->lru_slots.insert({e.last_use, it->first});
+        if (e.slot >= 0) {                     // stored already (or being stored): nothing to copy
+            out_slots[i] = KDA_PREFIX_STORED;
+            continue;
         }
+        if (c->free_slots.empty()) c->free_lru_slot(start);
+        if (c->free_slots.empty()) continue;
+        e.slot = c->free_slots.back();
+        c->free_slots.pop_back();
+        c->pending[e.slot] = 1;                // until the caller commits the copied state
+        c->owner[e.slot] = it->first;
+        c->lru_slots.insert({e.last_use, it->first});
         out_slots[i] = e.slot;
     }
+    return KDA_OK;
+}
+
+kda_status_t kda_prefix_cache_commit(kda_prefix_cache* c, const int32_t* slots, int64_t n) {
+    if (!c || n < 0 || (n > 0 && !slots)) return KDA_ERR_ARG;
+    std::lock_guard<std::mutex> lock(c->mu);
+    for (int64_t i = 0; i < n; ++i)
+        if (slots[i] >= c->n_slots) return KDA_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i)
+        if (slots[i] >= 0) c->pending[slots[i]] = 0;   // negative entries (no slot, stored) are skipped
+    return KDA_OK;
+}
+
+kda_status_t kda_prefix_cache_abort(kda_prefix_cache* c, const int32_t* slots, int64_t n) {
+    if (!c || n < 0 || (n > 0 && !slots)) return KDA_ERR_ARG;
+    std::lock_guard<std::mutex> lock(c->mu);
+    for (int64_t i = 0; i < n; ++i)
+        if (slots[i] >= c->n_slots) return KDA_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i) {
+        const int32_t s = slots[i];
+        if (s < 0 || !c->pending[s]) continue;   // only slots still waiting for their state
+        auto it = c->blocks.find(c->owner[s]);
+        if (it != c->blocks.end() && it->second.slot == s) c->drop_slot(it->first, it->second);
+    }
+    return KDA_OK;
+}
+
+kda_status_t kda_prefix_cache_release(kda_prefix_cache* c, int32_t slot) {
+    if (!c) return KDA_ERR_ARG;
+    if (slot < 0) return KDA_OK;               // a lookup that named no slot holds nothing
+    std::lock_guard<std::mutex> lock(c->mu);
+    if (slot >= c->n_slots || c->pins[slot] <= 0) return KDA_ERR_ARG;
+    --c->pins[slot];
     return KDA_OK;
 }
 

@@ -110,10 +110,12 @@ def test_bf16_empty_and_zero_token_batches():
 
 
 @pytest.mark.slow
-def test_bf16_prefill_b4_t4096_h32_sampled():
-    # KDA prefill, B=4, T=4096, H=32, dk=dv=128, bf16, zero initial state, seed 0
+def test_bf16_prefill_b4_t4096_h32_every_slice():
+    # KDA prefill, B=4, T=4096, H=32, dk=dv=128, bf16, zero initial state, seed 0, fp32 checkpoints every
+    # 512 tokens: the launch the benchmark times.  Every one of the 128 (sequence, head) slices -- outputs,
+    # checkpoints and final states -- against the oracle (about a second of fp64 work on the host).
     inp = synth.make_inputs([4096] * 4, 32, 128, 128, dtype=BF, device=DEV, seed=0)
-    outs = _run_chunk(inp, BF, init=False)
-    _check_chunk(inp, BF, outs, [0, 3], [0, 13, 31], )
+    outs = _run_chunk(inp, BF, init=False, ckpt_stride=512)
+    _check_chunk(inp, BF, outs, range(4), range(32), ckpt_stride=512)
     o = outs[0]
     assert torch.isfinite(o.float()).all()

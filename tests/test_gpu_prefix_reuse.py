@@ -64,6 +64,8 @@ def test_resume_from_looked_up_checkpoint_is_bit_exact():
         pool = torch.empty(8, H, D, D, device=DEV)
         for e, s in zip(ends, slots):
             pool[s] = ck1[e - 1]                      # checkpoint j holds the state after (j + 1) * 512 tokens
+        # the copies run on the current stream, before every later reader: the slots may be committed
+        kda.kda_prefix_cache_commit(cache, slots)
 
         # request 2: 9 full blocks are shared; the deepest checkpoint inside them ends block 8
         h2 = kda.kda_prefix_block_hashes(tok2)
@@ -76,5 +78,6 @@ def test_resume_from_looked_up_checkpoint_is_bit_exact():
         assert kda.kda_get_device_status() == 0
         assert torch.equal(o_sub, o_full[start:])
         assert torch.equal(fs_sub, fs_full)
+        kda.kda_prefix_cache_release(cache, s)        # the resumed prefill has read the slot
     finally:
         kda.kda_prefix_cache_destroy(cache)

@@ -80,8 +80,25 @@ def test_distributed_wrapper_single_rank_nccl_is_the_plain_run():
         fs = torch.empty(H, D, D, device=DEV)
         seqsplit.sequence_split_prefill(*f, o, fs, inp.state0[0])
         torch.cuda.synchronize()
+        # the same on a side stream: every step (library calls, torch copies, the collective) runs there,
+        # while the current stream is kept busy with unrelated work
+        side = torch.cuda.Stream(DEV)
+        side.wait_stream(torch.cuda.current_stream())
+        o2 = torch.full_like(o, float("nan"))
+        fs2 = torch.full_like(fs, float("nan"))
+        busy = torch.randn(4096, 4096, device=DEV)
+        for _ in range(8):
+            busy = busy @ busy.T / 4096.0
+        seqsplit.sequence_split_prefill(*f, o2, fs2, inp.state0[0], stream=side)
+        M, Z = seqsplit.segment_summary(*f, stream=side)
+        side.synchronize()
+        torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
     o_ref, fs_ref = _plain(f, inp.state0[0])
     assert torch.equal(o, o_ref)
     assert torch.equal(fs, fs_ref)
+    assert torch.equal(o2, o_ref)
+    assert torch.equal(fs2, fs_ref)
+    M0, Z0 = seqsplit.segment_summary(*f)
+    assert torch.equal(M, M0) and torch.equal(Z, Z0)

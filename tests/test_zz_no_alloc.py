@@ -3,15 +3,16 @@
 A serving engine that hands all device memory to its own pool, or a program with a fixed
 device-memory budget, cannot give kda_chunk_fwd a workspace; the no-allocation entry point keeps its
 scratch in a fixed array inside the library instead.  This test calls it twice in a row through the
-C ABI and compares every output with kda_chunk_fwd given an ordinary workspace, within the bf16
-tolerances the other tests use.  It sits in a file of its own that pytest collects last.
+C ABI and compares every output with kda_chunk_fwd given an ordinary workspace.  Both run the same
+kernels on the same chunk grid (windowed and single-pass workspaces give identical bits), so the
+comparison is exact: any difference would point at the windowing over the fixed array.  It sits in a
+file of its own that pytest collects last.
 """
 import pytest
 import torch
 
 import kda_linear_attention_02_b200 as kda
 from kda_linear_attention_02_b200 import synth
-from kda_testlib import assert_close, f32np
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -45,7 +46,34 @@ def test_noalloc_matches_workspace_entry_point_twice():
         torch.cuda.synchronize()
         assert kda.kda_get_device_status() == 0
         for name, a, b in zip(("o", "final_state", "checkpoints", "transition"), got, ref):
-            assert_close(f32np(a), f32np(b), BF, f"no-alloc call {call}: {name}")
+            assert torch.equal(a, b), f"no-alloc call {call}: {name} differs from kda_chunk_fwd"
+
+
+def test_noalloc_windows_over_the_fixed_array():
+    # one 4096-token sequence at H=32: the full scratch (~172 MB of packets) exceeds the 64 MiB array while
+    # its minimum (carried state + one chunk of packets) fits, so the call runs window by window and carries
+    # the states across windows inside the array
+    H, D, S = 32, 128, 512
+    lengths = [4096]
+    assert kda.kda_chunk_fwd_workspace_bytes(4096, 1, H, D, D) > (64 << 20)
+    assert kda.kda_chunk_fwd_min_workspace_bytes(1, H, D, D) <= (64 << 20)
+    inp = synth.make_inputs(lengths, H, D, D, dtype=BF, device=DEV, seed=22, with_state0=True)
+    ckcu = kda.kda_ckpt_offsets(inp.cu_seqlens.cpu(), S)
+    ckcu_d = ckcu.to(DEV)
+    ref = _outputs(inp, H, D, ckcu)
+    kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.state0, inp.cu_seqlens, ref[0], ref[1],
+                      ckpt_stride=S, checkpoints=ref[2], ckpt_cu=ckcu_d, final_transition=ref[3])
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    for call in range(2):
+        got = _outputs(inp, H, D, ckcu)
+        kda.kda_chunk_fwd_noalloc(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.state0, inp.cu_seqlens,
+                                  got[0], got[1], ckpt_stride=S, checkpoints=got[2], ckpt_cu=ckcu_d,
+                                  final_transition=got[3])
+        torch.cuda.synchronize()
+        assert kda.kda_get_device_status() == 0
+        for name, a, b in zip(("o", "final_state", "checkpoints", "transition"), got, ref):
+            assert torch.equal(a, b), f"windowed no-alloc call {call}: {name} differs from kda_chunk_fwd"
 
 
 def test_noalloc_refuses_batches_beyond_its_scratch():
