@@ -218,6 +218,209 @@ def cpu_oracle_decode_sample(s0, q, k, v, la, b, budget_s=6.0, max_slices=512):
                       f"threads; steps/s of the whole workload extrapolated from the sample"}
 
 
+def host_slices(inp, keys, ckpt=0, tok_limit=None):
+    """Host copies of whole (sequence, head) slices of a device workload, as oracle jobs (taken before
+    the device inputs are freed, timed later).  tok_limit keeps only each slice's first tokens."""
+    cu = inp.cu_seqlens.cpu().tolist()
+    jobs = []
+    for i, h in keys:
+        a, b = cu[i], cu[i + 1]
+        if tok_limit is not None:
+            b = min(b, a + tok_limit)
+        f = lambda t: t.float().cpu().numpy()
+        marks = list(range(ckpt, b - a + 1, ckpt)) if ckpt else None
+        s0 = None if inp.state0 is None else inp.state0[i, h].double().cpu().numpy()
+        jobs.append(((i, h), dict(q=f(inp.q[a:b, h]), k=f(inp.k[a:b, h]), v=f(inp.v[a:b, h]),
+                                  log_alpha=f(inp.log_alpha[a:b, h]), beta=f(inp.beta[a:b, h]), s0=s0,
+                                  marks=marks, want_o=True)))
+    return jobs
+
+
+def cpu_oracle_jobs(jobs, heads, total_token_heads, what):
+    """Times the fp64 oracle (as it stands) on prepared slice jobs and extrapolates the workload's
+    tokens/s (token-heads/s of the sample / heads)."""
+    import oracle
+    threads = oracle.threads_used()
+    t0 = time.perf_counter()
+    oracle.run_slices(jobs, threads)
+    dt = time.perf_counter() - t0
+    th = sum(j[1]["q"].shape[0] for j in jobs)
+    return {"value": th / dt / heads, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{what}: {len(jobs)} (sequence, head) slices, {th} token-heads of {total_token_heads} "
+                      f"({100.0 * th / total_token_heads:.3g} %), fp64, {dt:.1f} s on {threads} threads; "
+                      f"tokens/s = token-heads/s / {heads}, extrapolated from the sample"}
+
+
+def timed_calls(fn, steps, warmup, stream):
+    """Average device time (ms) of `steps` calls of fn after `warmup` calls, CUDA events on `stream`."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def prefill_roofline(token_heads, ms, hbm, extra_bytes=0, read_b=PREFILL_READ_B, out_b=256):
+    """HBM roofline of one chunked-prefill call: q, k, v, log_alpha, beta in, o out (per token-head),
+    plus `extra_bytes` (checkpoints, initial and final states) per call."""
+    alg = (read_b + out_b) * token_heads + extra_bytes
+    gbs = alg / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": "kda_chunk_fwd (whole call)", "achieved": round(gbs, 1), "peak": hbm,
+            "unit": "GB/s", "frac": round(gbs / hbm, 4), "alg_bytes_per_launch": int(alg),
+            "ideal_ms": round(alg / (hbm * 1e9) * 1e3, 4)}
+
+
+def run_workload_legs(kda, synth, dev, stream, hbm, want_cpu):
+    """The other configurations of the operator, each timed as whole kda_chunk_fwd calls: the fp32
+    workload (B=1, T=256, H=2, dk=dv=64), the long-context prefill (B=1, T=2^20, H=32, checkpoints every
+    512, initial state) and the varlen batch (64 sequences, lengths U[1024, 65536] seed 1, checkpoints,
+    a resumed batch, 8 segments per sequence composed).  Returns (legs, oracle jobs for later timing)."""
+    import gc
+    import torch
+    legs, cpu_jobs = {}, {}
+    Dd = D
+
+    # ---------------- fp32: B=1, T=256, H=2, dk=dv=64, zero initial state, seed 0
+    inp = synth.make_inputs([256], 2, 64, 64, dtype=torch.float32, device=dev, seed=0)
+    o = torch.empty(256, 2, 64, device=dev)
+    fs = torch.empty(1, 2, 64, 64, device=dev)
+    ws = torch.empty(kda.kda_chunk_fwd_workspace_bytes(256, 1, 2, 64, 64, kda.KDA_F32), dtype=torch.uint8,
+                     device=dev)
+    f = lambda: kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, inp.cu_seqlens, o, fs,
+                                  workspace=ws)
+    ms = timed_calls(f, 200, 20, stream)
+    # fp32 q, k, v (3 x 64 x 4 B), log_alpha (64 x 4 B), beta, o (64 x 4 B); final state 16 KiB per head
+    rl = prefill_roofline(512, ms, hbm, extra_bytes=2 * 64 * 64 * 4, read_b=3 * 256 + 256 + 4, out_b=256)
+    rl["note"] = "512 token-heads per call: launch- and latency-bound, far below any bandwidth limit"
+    legs["fp32"] = {"workload": "KDA chunked forward B=1 T=256 H=2 dk=dv=64 fp32, zero initial state, seed 0",
+                    "value": 256 / (ms / 1e3), "unit": "tokens/s", "ms_per_call": round(ms, 5), "dtype": "f32",
+                    "roofline": rl}
+    if want_cpu:
+        cpu_jobs["fp32"] = (host_slices(inp, [(0, 0), (0, 1)]), 2, 512, "the whole workload")
+    del inp, o, fs, ws
+
+    # ---------------- long context: B=1, T=2^20, H=32, bf16, log_alpha = -5 sigmoid(N(2, 1)), state ~ N(0, 0.02)
+    TL = 1 << 20
+    inp = synth.make_inputs([TL], H, Dd, Dd, dtype=torch.bfloat16, device=dev, seed=0, alpha_mu=2.0, alpha_sd=1.0,
+                            with_state0=True)
+    ckcu_h = kda.kda_ckpt_offsets(inp.cu_seqlens.cpu(), CKPT)
+    ck = torch.empty(int(ckcu_h[-1]), H, Dd, Dd, device=dev)
+    ckcu = ckcu_h.to(dev)
+    o = torch.empty(TL, H, Dd, dtype=torch.bfloat16, device=dev)
+    fs = torch.empty(1, H, Dd, Dd, device=dev)
+    ws = torch.empty(kda.kda_chunk_fwd_workspace_bytes(TL, 1, H, Dd, Dd, kda.KDA_BF16), dtype=torch.uint8, device=dev)
+    f = lambda: kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.state0, inp.cu_seqlens, o, fs,
+                                  ckpt_stride=CKPT, checkpoints=ck, ckpt_cu=ckcu, workspace=ws)
+    ms = timed_calls(f, 3, 3, stream)
+    kda.kda_profile_begin(2)
+    for _ in range(2):
+        f()
+    torch.cuda.synchronize()
+    _, lp, ls, ln = kda.kda_profile_end()
+    th = TL * H
+    st_b = Dd * Dd * 4 * H
+    rl = prefill_roofline(th, ms, hbm, extra_bytes=int(ckcu_h[-1]) * st_b + 2 * st_b)
+    legs["long_context"] = {
+        "workload": "KDA prefill B=1 T=1048576 H=32 dk=dv=128 bf16, log_alpha = -5 sigmoid(N(2,1)), initial state "
+                    "~ N(0, 0.02), fp32 checkpoints every 512 tokens, full workspace",
+        "value": TL / (ms / 1e3), "unit": "tokens/s", "ms_per_call": round(ms, 4), "dtype": "bf16",
+        "roofline": rl, "kernels": {"prep_bf16_kernel": {"ms": round(lp / ln, 4)},
+                                    "state_bf16_kernel": {"ms": round(ls / ln, 4)}}}
+    if want_cpu:
+        keys = [(0, h) for h in range(0, H, 2)]
+        cpu_jobs["long_context"] = (host_slices(inp, keys, ckpt=CKPT, tok_limit=1 << 15), H, th,
+                                    "first 32768 tokens of every second head, with the 512-token checkpoints")
+    del inp, o, fs, ws, ck, ckcu, f
+    gc.collect()
+    torch.cuda.empty_cache()
+
+    # ---------------- varlen: 64 sequences, lengths U[1024, 65536] (seed 1), H=32, bf16, checkpoints every 512
+    lengths = synth.varlen_lengths(64, 1024, 65536, 1)
+    N = len(lengths)
+    inp = synth.make_inputs(lengths, H, Dd, Dd, dtype=torch.bfloat16, device=dev, seed=0)
+    TV = inp.total_tokens
+    ckcu_h = kda.kda_ckpt_offsets(inp.cu_seqlens.cpu(), CKPT)
+    ck = torch.empty(int(ckcu_h[-1]), H, Dd, Dd, device=dev)
+    ckcu = ckcu_h.to(dev)
+    o = torch.empty(TV, H, Dd, dtype=torch.bfloat16, device=dev)
+    fs = torch.empty(N, H, Dd, Dd, device=dev)
+    full_ws = kda.kda_chunk_fwd_workspace_bytes(TV, N, H, Dd, Dd, kda.KDA_BF16)
+    free_b, _ = torch.cuda.mem_get_info(dev)
+    ws_b = int(min(full_ws, max(kda.kda_chunk_fwd_min_workspace_bytes(N, H, Dd, Dd), free_b - (16 << 30))))
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=dev)
+    f = lambda: kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, inp.cu_seqlens, o, fs,
+                                  ckpt_stride=CKPT, checkpoints=ck, ckpt_cu=ckcu, workspace=ws)
+    ms = timed_calls(f, 3, 3, stream)
+    th = TV * H
+    rl = prefill_roofline(th, ms, hbm, extra_bytes=int(ckcu_h[-1]) * st_b + N * st_b)
+    varlen = {"workload": f"KDA varlen prefill: 64 sequences, lengths U[1024, 65536] (seed 1, {TV} tokens), packed, "
+                          "H=32 dk=dv=128 bf16, zero initial state, fp32 checkpoints every 512 tokens",
+              "value": TV / (ms / 1e3), "unit": "tokens/s", "ms_per_call": round(ms, 4), "dtype": "bf16",
+              "workspace_bytes": ws_b, "windowed": ws_b < full_ws, "roofline": rl}
+    if want_cpu:
+        keys = [(i, h) for i in range(0, N, 8) for h in (0, 16)]
+        cpu_jobs["varlen"] = (host_slices(inp, keys, ckpt=CKPT), H, th,
+                              "whole sequences 0, 8, .., 56 at heads 0 and 16, with the 512-token checkpoints")
+    # 8 segments per sequence (b_s = 64 floor(s len / 512)) from a zero state with their transitions, then the
+    # prefix scan over the segments' (transition, zero-start state)
+    seg_len = []
+    for L in lengths:
+        bb = [64 * ((s_ * L) // 512) for s_ in range(8)] + [L]
+        seg_len += [bb[s_ + 1] - bb[s_] for s_ in range(8)]
+    seg_cu = synth.cu_from_lengths(seg_len, dev)
+    Zs = torch.empty(len(seg_len), H, Dd, Dd, device=dev)
+    Ms = torch.empty(len(seg_len), H, Dd, Dd, device=dev)
+    g = lambda: kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, seg_cu, o, Zs,
+                                  final_transition=Ms, workspace=ws)
+    seg_ms = timed_calls(g, 2, 1, stream)
+    starts = torch.empty_like(Zs)
+    ends = torch.empty(N, H, Dd, Dd, device=dev)
+    scu = synth.cu_from_lengths([8] * N, dev)
+    h_ = lambda: kda.kda_segment_compose(Ms, Zs, scu, None, starts, ends)
+    comp_ms = timed_calls(h_, 3, 1, stream)
+    varlen["segments"] = {"what": "kda_chunk_fwd over the 512 segments from zero with their transitions, then "
+                                  "kda_segment_compose", "chunk_fwd_ms": round(seg_ms, 4),
+                          "compose_ms": round(comp_ms, 4)}
+    # resumed batch: the even sequences restart at b_i = 512 floor(len_i / 1024) from their stored checkpoint, the
+    # odd ones run whole (their token inputs drawn afresh with those lengths; the states come from the run above)
+    even = list(range(0, N, 2))
+    b_res = {i: CKPT * (lengths[i] // 1024) for i in even}
+    init = torch.zeros(N, H, Dd, Dd, device=dev)
+    for i in even:
+        if b_res[i] > 0:
+            init[i] = ck[int(ckcu_h[i]) + b_res[i] // CKPT - 1]
+    rlen = [lengths[i] - b_res.get(i, 0) for i in range(N)]
+    del inp, o, fs, ck, ckcu, Zs, Ms, starts, ends, f, g, h_
+    gc.collect()
+    torch.cuda.empty_cache()
+    rin = synth.make_inputs(rlen, H, Dd, Dd, dtype=torch.bfloat16, device=dev, seed=1)
+    TR = rin.total_tokens
+    rck_h = kda.kda_ckpt_offsets(rin.cu_seqlens.cpu(), CKPT)
+    rck = torch.empty(max(1, int(rck_h[-1])), H, Dd, Dd, device=dev)
+    rckcu = rck_h.to(dev)
+    ro = torch.empty(TR, H, Dd, dtype=torch.bfloat16, device=dev)
+    rfs = torch.empty(N, H, Dd, Dd, device=dev)
+    f = lambda: kda.kda_chunk_fwd(rin.q, rin.k, rin.v, rin.log_alpha, rin.beta, init, rin.cu_seqlens, ro, rfs,
+                                  ckpt_stride=CKPT, checkpoints=rck, ckpt_cu=rckcu, workspace=ws)
+    rms = timed_calls(f, 3, 3, stream)
+    varlen["resume"] = {"what": "the batch with the even sequences resumed at 512 floor(len / 1024) from their "
+                                "checkpoints (odd ones whole)", "tokens": TR, "ms_per_call": round(rms, 4),
+                        "value": TR / (rms / 1e3), "unit": "tokens/s",
+                        "roofline": prefill_roofline(TR * H, rms, hbm,
+                                                     extra_bytes=int(rck_h[-1]) * st_b + 2 * N * st_b)}
+    legs["varlen"] = varlen
+    del rin, ro, rfs, rck, rckcu, init, ws, f
+    gc.collect()
+    torch.cuda.empty_cache()
+    return legs, cpu_jobs
+
+
 def run_ours(args):
     import torch
     import kda_linear_attention_02_b200 as kda
@@ -521,6 +724,10 @@ def run_ours(args):
     compose = {"workload": "64 sequences x 8 segments x H=32, dk=dv=128 fp32", "ms": round(comp_ms, 4),
                "achieved_gbs": round(comp_bytes / (comp_ms / 1e3) / 1e9, 1)}
     del M, Z, starts, ends
+    legs, leg_jobs = {}, {}
+    if not args.no_workloads:
+        legs, leg_jobs = run_workload_legs(kda, synth, dev, stream, hbm,
+                                           rank == 0 and world == 1 and not args.no_cpu_baseline)
     clk = clocks.stop()
 
     cpu = None
@@ -529,6 +736,9 @@ def run_ours(args):
     if dec_in is not None:
         decode["cpu_baseline"] = cpu_oracle_decode_sample(*dec_in)
         dec_in = None
+    for name, (jobs, heads, total, what) in leg_jobs.items():
+        legs[name]["cpu_baseline"] = cpu_oracle_jobs(jobs, heads, total, what)
+    leg_jobs = None
 
     if rank == 0:
         line = {
@@ -543,6 +753,7 @@ def run_ours(args):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
             "gpu_launches": 4 * args.steps, "decode": decode, "speculative": speculative, "compose": compose, "mxfp8": mxfp8,
         }
+        line.update(legs)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -588,6 +799,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the fp32, long-context and varlen workloads (timed after the headline)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
