@@ -276,6 +276,43 @@ def prefill_roofline(token_heads, ms, hbm, extra_bytes=0, read_b=PREFILL_READ_B,
             "ideal_ms": round(alg / (hbm * 1e9) * 1e3, 4)}
 
 
+# The tcgen05 products of one (chunk, head) item and one chunk step, as the kernels issue them:
+# (phase, N, K, B MN-major, products of that shape per unit).  M = 128 throughout.
+MMA_PHASES = [
+    ("prep A: [K e^(g-b); Q e^(g-b)] x 160 anchored key rows, per 64-channel half", 160, 64, False, 2),
+    ("prep Y: [I; Aqk] X", 64, 64, False, 1),
+    ("prep B, K part: [X; Y] diag(beta) x -(K gamma)^T onto [0; Q gamma]", 128, 64, False, 1),
+    ("prep B, V part: [X; Y] diag(beta) x V (MN-major)", 128, 64, True, 1),
+    ("state 1: [U; O_intra] + [-W; P] S (S MN-major)", 128, 128, True, 1),
+    ("state 2: Kdec^T U' (U' MN-major)", 128, 64, True, 1),
+]
+
+
+def mma_phase_rates(kda, tc_tflops, n_sms, sm_mhz):
+    """SM cycles per product for each tcgen05 phase shape, back to back and one at a time, as FLOP per
+    cycle per SM and as a fraction of the measured bf16 peak expressed per SM cycle."""
+    import torch
+    peak_fc = tc_tflops * 1e12 / (n_sms * sm_mhz * 1e6)
+    rows = []
+    for name, n, k, mn, per_unit in MMA_PHASES:
+        cyc = kda.kda_selftest_mma_rate(n, k, b_mn_major=mn, reps=512)
+        torch.cuda.synchronize()
+        c = cyc.cpu()
+        ok = c[:, 0] > 0
+        b2b, single = float(c[ok, 0].mean()), float(c[ok, 1].mean())
+        fl = 2.0 * 128 * n * k
+        rows.append({"phase": name, "M": 128, "N": n, "K": k, "b_mn_major": mn, "per_unit": per_unit,
+                     "cycles_back_to_back": round(b2b, 1), "cycles_single": round(single, 1),
+                     "flop_per_cycle_sm_back_to_back": round(fl / b2b, 1),
+                     "flop_per_cycle_sm_single": round(fl / single, 1),
+                     "frac_back_to_back": round(fl / b2b / peak_fc, 4), "frac_single": round(fl / single / peak_fc, 4)})
+    return {"peak_flop_per_cycle_sm": round(peak_fc, 1),
+            "peak_basis": f"measured bf16 peak {tc_tflops} TFLOP/s / {n_sms} SMs / {sm_mhz} MHz",
+            "how": "kda_selftest_mma_rate: one CTA per SM, 512 products of each shape timed with the SM clock, "
+                   "back to back (one commit at the end) and one at a time (commit and wait per product)",
+            "phases": rows}
+
+
 def run_workload_legs(kda, synth, dev, stream, hbm, want_cpu):
     """The other configurations of the operator, each timed as whole kda_chunk_fwd calls: the fp32
     workload (B=1, T=256, H=2, dk=dv=64), the long-context prefill (B=1, T=2^20, H=32, checkpoints every
@@ -724,6 +761,8 @@ def run_ours(args):
     compose = {"workload": "64 sequences x 8 segments x H=32, dk=dv=128 fp32", "ms": round(comp_ms, 4),
                "achieved_gbs": round(comp_bytes / (comp_ms / 1e3) / 1e9, 1)}
     del M, Z, starts, ends
+    props = torch.cuda.get_device_properties(dev)
+    mma = mma_phase_rates(kda, tc, props.multi_processor_count, 1965.0)
     legs, leg_jobs = {}, {}
     if not args.no_workloads:
         legs, leg_jobs = run_workload_legs(kda, synth, dev, stream, hbm,
@@ -751,7 +790,7 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs and outputs larger than L2 (1.1 GB per step), no flush"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-            "gpu_launches": 4 * args.steps, "decode": decode, "speculative": speculative, "compose": compose, "mxfp8": mxfp8,
+            "gpu_launches": 4 * args.steps, "mma_phases": mma, "decode": decode, "speculative": speculative, "compose": compose, "mxfp8": mxfp8,
         }
         line.update(legs)
         print(json.dumps(line), flush=True)

@@ -365,6 +365,17 @@ KDA_API kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_
  *  row-major (device), d [128,n] fp32 (device); n in {16, 32, ..., 256}.  b_mn_major != 0 stages B
  *  MN-major instead of K-major (then n must be a multiple of 64).
  */
+/*
+ *  kda_selftest_mma_rate: the tensor-core rate of one product shape as the chunk kernels issue it:
+ *  128 x n x k bf16 (k in {64, 128}, n in {16, ..., 256}; B K-major, or MN-major when b_mn_major, then
+ *  n a multiple of 64), fp32 accumulator in TMEM.  `grid` CTAs (one per SM when grid <= the SM count),
+ *  each with one issuing thread, time `reps` products back to back and then `reps` products each
+ *  waited for before the next, with the SM clock.  cycles (device, [grid][2] fp32) receives the SM
+ *  cycles per product in the two modes (-1 if a bounded wait ran out).  FLOP per cycle per SM of a
+ *  mode is 2 * 128 * n * k / cycles.
+ */
+KDA_API kda_status_t kda_selftest_mma_rate(int n, int k, int b_mn_major, int reps, float* cycles, int grid,
+                                           kda_stream_t stream);
 KDA_API kda_status_t kda_selftest_wait_timeout(int limit_us, kda_stream_t stream);
 KDA_API kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, int b_mn_major,
                                        kda_stream_t stream);

@@ -19,7 +19,7 @@ __all__ = [
     "kda_chunk_fwd_noalloc",
     "kda_recurrent_step", "kda_recurrent_step_mxfp8", "kda_decode_verify", "kda_decode_commit", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
     "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
-    "kda_selftest_umma", "KDA_PREFIX_BLOCK", "kda_prefix_block_hashes", "kda_prefix_cache_create",
+    "kda_selftest_umma", "kda_selftest_mma_rate", "KDA_PREFIX_BLOCK", "kda_prefix_block_hashes", "kda_prefix_cache_create",
     "kda_prefix_cache_destroy", "kda_prefix_cache_lookup", "kda_prefix_cache_plan", "kda_prefix_cache_insert",
     "kda_prefix_cache_commit", "kda_prefix_cache_abort", "kda_prefix_cache_release", "kda_prefix_cache_stats",
     "KDA_PREFIX_NO_SLOT", "KDA_PREFIX_STORED",
@@ -114,6 +114,8 @@ def _load():
     L.kda_profile_end.argtypes = [vp, vp, vp, vp]
     L.kda_selftest_wait_timeout.restype = i32
     L.kda_selftest_wait_timeout.argtypes = [i32, vp]
+    L.kda_selftest_mma_rate.restype = i32
+    L.kda_selftest_mma_rate.argtypes = [i32, i32, i32, i32, vp, i32, vp]
     L.kda_selftest_umma.restype = i32
     L.kda_selftest_umma.argtypes = [vp, vp, vp, i32, i32, vp]
     _lib = L
@@ -467,6 +469,18 @@ def kda_profile_end():
 
 def kda_selftest_wait_timeout(limit_us: int = 2000, stream=None) -> int:
     return int(_load().kda_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def kda_selftest_mma_rate(n, k, *, b_mn_major=False, reps=256, grid=None, stream=None):
+    """SM cycles per 128 x n x k bf16 tensor-core product, back to back and one at a time
+    (C: kda_selftest_mma_rate): a float32 tensor [grid, 2] on the current device."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if grid is None:
+        grid = torch.cuda.get_device_properties(dev).multi_processor_count
+    cyc = torch.empty(grid, 2, dtype=torch.float32, device=dev)
+    _check(_load().kda_selftest_mma_rate(int(n), int(k), int(bool(b_mn_major)), int(reps), _p(cyc), int(grid),
+                                         _stream(stream)), "kda_selftest_mma_rate")
+    return cyc
 
 
 def kda_selftest_umma(a, b, d, *, b_mn_major=False, stream=None):

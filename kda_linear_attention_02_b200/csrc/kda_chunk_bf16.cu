@@ -94,68 +94,58 @@ struct Pk {
 };
 
 // ------------------------------------------------------------------------------------------------
-// prep kernel shared memory (bytes from a 1024-aligned base)
+// prep kernel: two CTAs share an SM, so one (chunk, head) item's working set fits in about 110 KB of
+// shared memory and 256 TMEM columns; while one CTA waits on a tensor-core product, a barrier or its
+// loads, the other computes.  Shared memory (bytes from a 1024-aligned base), reused phase by phase:
+//   OPB   column pass, per 64-channel half: the row side [K e^(g-b); Q e^(g-b)] (128 x 64 bf16) at +0 and
+//         the key side (4 anchored variants stacked into 160 rows, 160 x 64 bf16) at +16384, K-major with
+//         the 128B swizzle (the operands of one K half of product A);
+//         solve: A (fp32, pitch LDM) at +0 and X (fp32, pitch LDX) at +17408;
+//         then [X; Y] diag(beta) (bf16, product B's A operand) at +0;
+//         epilogue: the packet's [-W; P] (two 64-column atoms) at +0 .. +32768
+//   QG    Q gamma [64 tokens][128 ch] bf16 (the accumulator preload), then X^T (product Y's B operand),
+//         then atom 0 of the packet's [U; O_intra]
+//   KG    -(K gamma)^T [128 ch][64 tokens] bf16, K-major (product B's B operand, K part), then atom 1 of
+//         [U; O_intra] (QG and KG are adjacent, so [U; O_intra] leaves in one bulk copy)
+//   VOP   V [DV/64][64 tokens][128 B] bf16, MN-major with the 128B swizzle (product B's B operand, V
+//         part): a TMA tile for bf16 inputs, written by the column pass for MXFP8 inputs
+//   IAQ   [I; Aqk] 128 x 64 bf16 (product Y's A operand)
+//   MISC  beta[64]; then the tile half-totals [8][64] fp32 (column pass) or the merge scratch (solve)
+//   SCF   MXFP8 inputs only: the shared scales as fp32, [q, k, v][64 tokens][4 blocks]
+// TMEM (256 columns): product A at [0, 160); then the preload [0; Q gamma] at [0, 128); product Y at
+// [128, 192); product B: the K part at [0, 128) onto the preload, the V part at [128, 128 + DV).
 namespace ps {
-constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_V = 32768, STG_L = 49152;   // raw TMA tiles
-constexpr uint32_t RALL = 81920;     // row side [K e^(g-b); Q e^(g-b)]: 128 x 128 bf16 (A operand)
-constexpr uint32_t BVAR = 114688;    // key side: variants 0..3 stacked as rows [0,16) [16,48) [48,96) [96,160)
-                                     // of one 160-row B operand, [2 K atoms][160 rows][128 B]
-constexpr uint32_t QT = 155648;      // Q * gamma, [64][128] bf16, 16-byte chunks swizzled by row
-constexpr uint32_t BKV = 172032;     // [beta K gamma | beta V]^T: (128+DV) x 64 bf16 (B operand)
-constexpr uint32_t MISC = 204800;    // beta[64] fp32 (of even items for MXFP8 inputs), half-tile totals [8][128] fp32
-constexpr uint32_t BET1 = MISC + 4352;   // MXFP8 inputs: beta[64] fp32 of odd items (fetched during the previous one)
-constexpr uint32_t IAQ = 209920;     // [I; Aqk]: 128 x 64 bf16 (A operand of the Y product)
-// aliases of RALL/BVAR once phase A has completed
-constexpr uint32_t AM = 81920, XF = 99328, TT = 118016, XT = 124928, XY = 133120;   // solve
-constexpr uint32_t AWS = 81920, UOS = 114688;                                    // packet staging
-constexpr uint32_t BYTES = IAQ + 16384;
-constexpr uint32_t SCF = BYTES;      // MXFP8 inputs only: shared scales of the chunk's tokens, [q, k, v][64][4] fp32
-constexpr uint32_t SCW = SCF + 3 * 64 * 16;   // and their E8M0 code words as fetched, [2 items][q, k, v][64] u32
-constexpr uint32_t BYTES_MX = SCW + 2 * 3 * 64 * 4;
-static_assert(BYTES_MX + 1024 <= 232448, "shared memory of one CTA");
+constexpr uint32_t OPB = 0;
+constexpr uint32_t BVAR = 16384;                 // key side, inside OPB
+constexpr uint32_t AM = 0, XF = 17408;           // solve, inside OPB
+constexpr uint32_t QG = 36864;
+constexpr uint32_t KG = QG + 16384;
+constexpr uint32_t VOP = KG + 16384;
+constexpr uint32_t IAQ = VOP + 16384;
+constexpr uint32_t MISC = IAQ + 16384;           // beta[64] fp32
+constexpr uint32_t TOT = MISC + 256;             // [8][64] fp32 (column pass) | [32][LDTT] fp32 (solve)
+constexpr uint32_t BYTES = TOT + 5120;
+constexpr uint32_t SCF = BYTES;                  // MXFP8 inputs only
+constexpr uint32_t BYTES_MX = SCF + 3 * 64 * 16;
 constexpr int LDM = 68;              // fp32 row pitch of AM (float4-aligned rows; 4 rows apart = 16 banks)
 constexpr int LDX = 73;              // fp32 row pitch of X (odd: column reads of X^T spread over the banks)
 constexpr int LDTT = 40;             // fp32 row pitch of the product scratch (8 banks per row: B fragments clash-free)
-static_assert(XF + 64 * LDX * 4 <= TT && TT + 32 * LDTT * 4 <= XT && AM + 64 * LDM * 4 <= XF, "solve map");
-static_assert(BET1 + 256 <= IAQ, "beta buffers");
-
-constexpr int NT = 512;              // threads per CTA
+static_assert(AM + 64 * LDM * 4 <= XF && XF + 64 * LDX * 4 <= QG, "solve scratch inside the operand buffer");
+static_assert(32 * LDTT * 4 <= 5120 && 8 * 64 * 4 <= 5120, "column-pass totals and merge scratch share MISC");
+constexpr int NT = 256;              // threads per CTA
+// two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2 per CTA, with the 1024-byte alignment slack
+static_assert(BYTES_MX + 1024 + 128 <= 115712, "two CTAs per SM");
 }  // namespace ps
-
-// One chunk's input tiles into the staging area.  bf16: q, k, v as 64-column boxes, [dk / 64][64 tokens][128 B];
-// MXFP8: one box of codes each, [64 tokens][dk or DV bytes].  log_alpha: 32-column boxes.
-template <int DV, bool MX>
-__device__ __forceinline__ void issue_tile_loads(uint8_t* sm, const CUtensorMap* mq, const CUtensorMap* mk,
-                                                 const CUtensorMap* mv, const CUtensorMap* ml, uint64_t* bar,
-                                                 int h, long long tok0) {
-    const int tok = static_cast<int>(tok0);
-    if constexpr (MX) {
-        mbar_arrive_expect_tx(bar, 2 * 8192 + DV * 64 + 32768);
-        tma_load_3d(sm + ps::STG_Q, mq, 0, h, tok, bar);
-        tma_load_3d(sm + ps::STG_K, mk, 0, h, tok, bar);
-        tma_load_3d(sm + ps::STG_V, mv, 0, h, tok, bar);
-    } else {
-        mbar_arrive_expect_tx(bar, 2 * 16384 + DV * 128 + 32768);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            tma_load_3d(sm + ps::STG_Q + hf * 8192, mq, hf * 64, h, tok, bar);
-            tma_load_3d(sm + ps::STG_K + hf * 8192, mk, hf * 64, h, tok, bar);
-        }
-#pragma unroll
-        for (int hf = 0; hf < DV / 64; ++hf) tma_load_3d(sm + ps::STG_V + hf * 8192, mv, hf * 64, h, tok, bar);
-    }
-#pragma unroll
-    for (int qq = 0; qq < 4; ++qq) tma_load_3d(sm + ps::STG_L + qq * 8192, ml, qq * 32, h, tok, bar);
-}
 
 // MX: q, k, v arrive as MXFP8 (E4M3 codes with one E8M0 scale per 32 channels of a (token, head) row;
 // q_scale/k_scale [T, H, 4] and v_scale [T, H, DV / 32] bytes) and are decoded exactly in the column pass;
 // everything after it is the bf16 path unchanged.
 template <int DV, bool MX>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(256, 2)
 prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_l,
-                 const float* __restrict__ beta, const uint8_t* __restrict__ q_scale,
+                 const uint8_t* __restrict__ qg, const uint8_t* __restrict__ kg, const uint8_t* __restrict__ vg,
+                 const float* __restrict__ lag, const float* __restrict__ beta, const uint8_t* __restrict__ q_scale,
                  const uint8_t* __restrict__ k_scale, const uint8_t* __restrict__ v_scale,
                  const int2* __restrict__ chunk_tab, int H, long long n_items, uint8_t* __restrict__ packets,
                  int* status) {
@@ -164,28 +154,29 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     constexpr int LDM = ps::LDM;
     constexpr int LDX = ps::LDX;
     constexpr int LDTT = ps::LDTT;
+    constexpr int ES = MX ? 1 : 2;   // bytes per q/k/v element
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    __shared__ __align__(8) uint64_t bar_load, bar_mma;
+    __shared__ __align__(8) uint64_t bar_v, bar_mma;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-    float* bet = reinterpret_cast<float*>(sm + ps::MISC);           // this item's beta (buffer of its parity)
-    float* tot = reinterpret_cast<float*>(sm + ps::MISC + 256);   // [8 half-tiles][128 channels]
+    float* bet = reinterpret_cast<float*>(sm + ps::MISC);
+    float* tot = reinterpret_cast<float*>(sm + ps::TOT);   // [8 half tiles][64 channels of the current half]
     // AM holds the strictly lower A = beta_r (K e^g)_r . (K e^-g)_s in two forms that never overlap: the
     // off-diagonal 16 x 16 blocks row-major (AM[r][s], tile(s) < tile(r)), and each diagonal block
     // transposed into its upper triangle (AM[s][r] for s < r in the same tile)
     float* AM = reinterpret_cast<float*>(sm + ps::AM);
     float* XF = reinterpret_cast<float*>(sm + ps::XF);    // X = (I + A)^-1, fp32, pitch LDX
-    float* TT = reinterpret_cast<float*>(sm + ps::TT);    // T = A_10 X_00 of a merge, pitch LDTT
+    float* TT = reinterpret_cast<float*>(sm + ps::TOT);   // T = A_10 X_00 of a merge, pitch LDTT
 
     if (t == 0) {
-        mbar_init(&bar_load, 1);
+        mbar_init(&bar_v, 1);
         mbar_init(&bar_mma, 1);
         fence_barrier_init();
         prefetch_tmap(&map_q); prefetch_tmap(&map_k); prefetch_tmap(&map_v); prefetch_tmap(&map_l);
     }
     if (w == 0) {
-        tmem_alloc(&tmem_slot, 512);   // one CTA per SM (its shared memory): all of the SM's TMEM
+        tmem_alloc(&tmem_slot, 256);   // two CTAs per SM: half of the SM's TMEM each
         tmem_relinquish();
     }
     // identity rows 0..63 of [I; Aqk]; rows 64..127 start at zero and every item rewrites only the columns of
@@ -205,26 +196,34 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tmem_slot;
-    uint32_t ph_load = 0, ph_mma = 0;
-    bool load_pending = false;   // meaningful in thread 0 only
+    uint32_t ph_v = 0, ph_mma = 0;
+    bool v_pending = false;   // meaningful in thread 0 only
 
-    // MXFP8 inputs: beta and the scale words of an item's 64 rows into the buffers of parity pb, by cp.async,
-    // so that they land while the previous item computes (rows past the item's n tokens read as zero), by
-    // warps 8..15, which never issue bulk copies.  (bf16 inputs load beta when the item starts: there an
-    // early fetch measured slower.)
-    auto fetch_rows = [&](int2 l, int hh, int pb) {
-        if constexpr (!MX) return;
-        const bool in = (t & 63) < l.y;
-        const size_t row = (static_cast<size_t>(l.x) + (t & 63)) * H + hh;
-        if (t >= 256 && t < 320) {
-            cp_async4(sm + (pb ? ps::BET1 : ps::MISC) + 4 * (t - 256), in ? beta + row : beta, in ? 4u : 0u);
-        } else if (t >= 320) {
-            const int which = (t - 320) >> 6;
-            const uint8_t* src = which == 0 ? q_scale : which == 1 ? k_scale : v_scale;
-            uint8_t* dst = sm + ps::SCW + pb * 768 + 4 * (t - 320);
-            if (which < 2 || DV == 128) cp_async4(dst, in ? src + 4 * row : src, in ? 4u : 0u);
-            else *reinterpret_cast<uint32_t*>(dst) =   // DV = 64: 2-byte rows, too small for cp.async
-                     0x7F7F0000u | (in ? reinterpret_cast<const uint16_t*>(v_scale)[row] : 0x7F7Fu);
+    // V of an item as product B's MN-major B operand (bf16 inputs; thread 0)
+    auto issue_v = [&](long long tok0, int hh) {
+        if constexpr (!MX) {
+            mbar_arrive_expect_tx(&bar_v, DV * 128);
+#pragma unroll
+            for (int b = 0; b < DV / 64; ++b)
+                tma_load_3d(sm + ps::VOP + b * 8192, &map_v, 64 * b, hh, static_cast<int>(tok0), &bar_v);
+            v_pending = true;
+        }
+    };
+    // an item's inputs that the column pass reads with plain loads, into L2 ahead of time (thread 0)
+    auto prefetch_inputs = [&](long long tok0, int hh) {
+        const int tk = static_cast<int>(tok0);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) tma_prefetch_3d(&map_l, 32 * qq, hh, tk);
+        if constexpr (MX) {
+            tma_prefetch_3d(&map_q, 0, hh, tk);
+            tma_prefetch_3d(&map_k, 0, hh, tk);
+            tma_prefetch_3d(&map_v, 0, hh, tk);
+        } else {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                tma_prefetch_3d(&map_q, 64 * b, hh, tk);
+                tma_prefetch_3d(&map_k, 64 * b, hh, tk);
+            }
         }
     };
 
@@ -236,90 +235,83 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     int2 loc = entry(item);
     int h = static_cast<int>(item % H);
     bool valid = loc.y > 0;
-    int2 nloc = entry(item + gridDim.x);   // one item ahead
     if (t == 0 && valid) {
-        issue_tile_loads<DV, MX>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, h, loc.x);
-        load_pending = true;
+        issue_v(loc.x, h);
+        prefetch_inputs(loc.x, h);
     }
-    if (valid) fetch_rows(loc, h, 0);
-    int par = 0;   // parity of the item: its beta / scale-word buffers
 
     while (valid) {
         const int n = loc.y;
         uint8_t* pkt = packets + static_cast<size_t>(item) * P::BYTES;
         const long long nitem = item + gridDim.x;   // this CTA's next item
+        const int2 nloc = entry(nitem);
         const int nh = static_cast<int>(nitem % H);
         const bool nvalid = nloc.y > 0;
-        if constexpr (!MX) {
-            if (t < 64) bet[t] = t < n ? beta[(static_cast<size_t>(loc.x) + t) * H + h] : 0.f;
-        } else {
-            bet = reinterpret_cast<float*>(sm + (par ? ps::BET1 : ps::MISC));
-            if (t >= 256) cp_async_wait_all();   // this thread's fetches of the item's rows have landed
+        if (t == 0 && nvalid) prefetch_inputs(nloc.x, nh);
+        if (t < 64) {
+            bet[t] = t < n ? beta[(static_cast<size_t>(loc.x) + t) * H + h] : 0.f;
+            if (nvalid && t < nloc.y) prefetch_l2(beta + (static_cast<size_t>(nloc.x) + t) * H + nh);
         }
         if constexpr (MX) {   // the shared scales of the chunk's tokens as fp32 (scale 1.0 past its end)
-            if (t >= 320) {
-                const uint32_t wv = (t & 63) < n ? *reinterpret_cast<const uint32_t*>(sm + ps::SCW + par * 768 +
-                                                                                       4 * (t - 320))
-                                                 : 0x7F7F7F7Fu;
-                reinterpret_cast<float4*>(sm + ps::SCF)[t - 320] =
+            if (t >= 64) {
+                const int which = (t - 64) >> 6, rr = (t - 64) & 63;
+                const size_t row = (static_cast<size_t>(loc.x) + rr) * H + h;
+                uint32_t wv = 0x7F7F7F7Fu;
+                if (rr < n) {
+                    if (which == 0) wv = ld_once_u32(q_scale + 4 * row);
+                    else if (which == 1) wv = ld_once_u32(k_scale + 4 * row);
+                    else wv = DV == 128 ? ld_once_u32(v_scale + 4 * row) : (0x7F7F0000u | ld_once_u16(v_scale + 2 * row));
+                }
+                reinterpret_cast<float4*>(sm + ps::SCF)[which * 64 + rr] =
                     make_float4(e8m0_to_f32(wv & 0xFFu), e8m0_to_f32((wv >> 8) & 0xFFu),
                                 e8m0_to_f32((wv >> 16) & 0xFFu), e8m0_to_f32(wv >> 24));
             }
         }
-        {
-            const bool ok = mbar_wait(&bar_load, ph_load, status);
-            if (__syncthreads_or(!ok)) break;
-        }
-        ph_load ^= 1;
-        if (t == 0) load_pending = false;
+        // the previous item's packet staging (OPB, QG, KG) must have been read out before this column
+        // pass writes there; the first barrier below publishes the wait
+        if (t == 0) bulk_wait_read0();
 
-        // ---------------- column pass: thread = (channel pair, 8-token half tile)
-        uint4 kd_pk[2];
-        {
-            const int cp = t & 63, q8 = t >> 6, tq = q8 >> 1, hh = q8 & 1, c0 = 2 * cp;
+        // ---------------- column pass, one 64-channel half at a time: thread = (channel pair, the 8 tokens
+        // of its warp); each half ends with its share of product A (K = 64 channels)
+        bool fail = false;
+        const size_t row0 = static_cast<size_t>(loc.x) * H + h;   // (token, head) row of the chunk's first token
+        for (int hf = 0; hf < 2; ++hf) {
+            const int c0 = 64 * hf + 2 * lane, tq = w >> 1;
             float2 p[8];
+            uint32_t kb8[8], qb8[8], vb8[8];
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const int r = 8 * q8 + j;
-                const float2 la =
-                    *reinterpret_cast<const float2*>(sm + ps::STG_L + (c0 >> 5) * 8192 + r * 128 + (c0 & 31) * 4);
-                if (r < n) acc = __fadd2_rn(acc, make_float2(floor_log_decay(la.x), floor_log_decay(la.y)));
-                p[j] = acc;
-            }
-            *reinterpret_cast<float2*>(tot + q8 * 128 + c0) = acc;
-            // the 8 tokens' inputs, loaded before the barrier (the staging tiles are not part of the packet)
-            uint32_t kb8[8], qb8[8], vb8[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = 8 * q8 + j;
-                if constexpr (MX) {   // two E4M3 codes per channel pair
-                    kb8[j] = *reinterpret_cast<const uint16_t*>(sm + ps::STG_K + r * 128 + c0);
-                    qb8[j] = *reinterpret_cast<const uint16_t*>(sm + ps::STG_Q + r * 128 + c0);
-                    vb8[j] = c0 < DV ? *reinterpret_cast<const uint16_t*>(sm + ps::STG_V + r * DV + c0) : 0u;
-                } else {
-                    kb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_K + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
-                    qb8[j] = *reinterpret_cast<const uint32_t*>(sm + ps::STG_Q + (c0 >> 6) * 8192 + r * 128 + (c0 & 63) * 2);
-                    vb8[j] = c0 < DV ? *reinterpret_cast<const uint32_t*>(sm + ps::STG_V + (c0 >> 6) * 8192 + r * 128 +
-                                                                           (c0 & 63) * 2)
-                                     : 0u;
+                const int r = 8 * w + j;
+                kb8[j] = qb8[j] = vb8[j] = 0u;
+                p[j] = make_float2(0.f, 0.f);
+                if (r < n) {
+                    const size_t rr = row0 + static_cast<size_t>(r) * H;
+                    p[j] = ld_once_f2(lag + rr * kDK + c0);
+                    if constexpr (MX) {
+                        kb8[j] = ld_once_u16(kg + rr * kDK + c0);
+                        qb8[j] = ld_once_u16(qg + rr * kDK + c0);
+                        if (c0 < DV) vb8[j] = ld_once_u16(vg + rr * DV + c0);
+                    } else {
+                        kb8[j] = ld_once_u32(kg + (rr * kDK + c0) * ES);
+                        qb8[j] = ld_once_u32(qg + (rr * kDK + c0) * ES);
+                    }
                 }
             }
-            // the staging tiles have been read into registers: after the fence and the barrier the next
-            // item's tiles may overwrite them (the TMA writes through the async proxy)
-            fence_proxy_async_smem();
-            if (t == 0) bulk_wait_read0();   // the previous item's packet staging has been read out
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (8 * w + j < n) acc = __fadd2_rn(acc, make_float2(floor_log_decay(p[j].x), floor_log_decay(p[j].y)));
+                p[j] = acc;
+            }
+            *reinterpret_cast<float2*>(tot + w * 64 + 2 * lane) = acc;
             __syncthreads();
-            if (t == 0 && nvalid) {
-                issue_tile_loads<DV, MX>(sm, &map_q, &map_k, &map_v, &map_l, &bar_load, nh, nloc.x);
-                load_pending = true;
+            if (hf == 1) {   // product A's first half has finished reading OPB
+                const bool ok = mbar_wait(&bar_mma, ph_mma, status);
+                ph_mma ^= 1;
+                if (__syncthreads_or(!ok)) { fail = true; break; }
             }
-            if constexpr (!MX) {   // and the next item's beta rows into L2, for the load at its start
-                if (nvalid && t >= 256 && t - 256 < nloc.y)
-                    prefetch_l2(beta + (static_cast<size_t>(nloc.x) + (t - 256)) * H + nh);
-            }
-            if (hh) {   // second half of the tile: add the first half's total
-                const float2 ob = *reinterpret_cast<const float2*>(tot + (q8 - 1) * 128 + c0);
+            if (w & 1) {   // second half of the tile: add the first half's total
+                const float2 ob = *reinterpret_cast<const float2*>(tot + (w - 1) * 64 + 2 * lane);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) { p[j].x += ob.x; p[j].y += ob.y; }
             }
@@ -328,8 +320,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             bx[0] = 0.f; by[0] = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float2 t0 = *reinterpret_cast<const float2*>(tot + (2 * i) * 128 + c0);
-                const float2 t1 = *reinterpret_cast<const float2*>(tot + (2 * i + 1) * 128 + c0);
+                const float2 t0 = *reinterpret_cast<const float2*>(tot + (2 * i) * 64 + 2 * lane);
+                const float2 t1 = *reinterpret_cast<const float2*>(tot + (2 * i + 1) * 64 + 2 * lane);
                 bx[i + 1] = bx[i] + t0.x + t1.x;
                 by[i + 1] = by[i] + t0.y + t1.y;
             }
@@ -347,94 +339,98 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 dvx[i] = i > tq ? __expf(bx[i] - bnx) : 0.f;
                 dvy[i] = i > tq ? __expf(by[i] - bny) : 0.f;
             }
-            if (q8 == 7)
+            if (w == 7)
                 *reinterpret_cast<float2*>(pkt + P::G + c0 * 4) = make_float2(__expf(bx[4]), __expf(by[4]));
-            float bt8[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) bt8[j] = bet[8 * q8 + j];
 
-            float tk[2][8], tv[2][8], td[2][8];   // beta K gamma, beta V, Kdec along the 8 tokens
+            // -K gamma and Kdec along the 8 tokens, packed to bf16 pairs of consecutive tokens as they are made
+            uint32_t tkw[2][4], tdw[2][4];
+            float2 tkp = make_float2(0.f, 0.f), tdp = make_float2(0.f, 0.f);
             const float2 ft2 = make_float2(ftx, fty), eb2 = make_float2(ebx, eby), ec2 = make_float2(ecx, ecy);
+            const uint32_t kk = static_cast<uint32_t>((c0 & 63) >> 3), kb = static_cast<uint32_t>(c0 & 7) * 2;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const int r = 8 * q8 + j;
-                // rows past the sequence end (n <= r) keep whatever the tile holds: their log-decay and beta are
-                // zero, so they add nothing to A, W, U, Kdec^T U' or the state, and their own P / O_intra rows
-                // are never stored as outputs
-                float2 kf, qf, vf;
+                const int r = 8 * w + j;
+                // rows past the sequence end (n <= r) hold zero inputs: their log-decay and beta are zero, so
+                // they add nothing to A, W, U, Kdec^T U' or the state, and their own P / O_intra rows are never
+                // stored as outputs
+                float2 kf, qf;
                 if constexpr (MX) {   // code x shared scale of the 32-channel block holding c0
                     const float* scf = reinterpret_cast<const float*>(sm + ps::SCF) + (c0 >> 5);
                     const float2 un = f2(kE4M3Unscale);
                     kf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(kb8[j]), un), f2(scf[4 * (64 + r)]));
                     qf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(qb8[j]), un), f2(scf[4 * r]));
-                    vf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(vb8[j]), un), f2(scf[4 * (128 + r)]));
+                    if (c0 < DV) {   // V as product B's MN-major operand
+                        const float2 vf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(vb8[j]), un), f2(scf[4 * (128 + r)]));
+                        st_b32(sm + ps::VOP + (c0 >> 6) * 8192 + (r >> 3) * 1024 + (r & 7) * 128 +
+                                   ((kk ^ static_cast<uint32_t>(r & 7)) << 4) + kb,
+                               pack2(vf));
+                    }
                 } else {
                     kf = bf2_to_f2(kb8[j]);
                     qf = bf2_to_f2(qb8[j]);
-                    vf = bf2_to_f2(vb8[j]);
                 }
                 const float2 pl = __fmul2_rn(p[j], f2(kLog2e));
                 const float2 E = make_float2(ex2_approx(pl.x), ex2_approx(pl.y));     // e^{g_r - b_t} <= 1
                 const float2 I = make_float2(ex2_approx(-pl.x), ex2_approx(-pl.y));   // e^{b_t - g_r} <= e^80.09
                 const float2 F = __fmul2_rn(ft2, I);                                  // e^{b_{t+1} - g_r} <= 1
                 const float2 G = __fmul2_rn(eb2, E);                                  // e^{g_r}
-                const float2 bt = f2(bt8[j]);
-                // row side of A / Aqk
-                st_b32(sm + ps::RALL + sw128_offset(r, c0, 128), pack2(__fmul2_rn(kf, E)));
-                st_b32(sm + ps::RALL + sw128_offset(64 + r, c0, 128), pack2(__fmul2_rn(qf, E)));
+                const uint32_t sw = ((kk ^ static_cast<uint32_t>(r & 7)) << 4) + kb;  // row r, rows 8 apart agree
+                // row side of A / Aqk (this half's K atom)
+                st_b32(sm + ps::OPB + r * 128 + sw, pack2(__fmul2_rn(kf, E)));
+                st_b32(sm + ps::OPB + (64 + r) * 128 + sw, pack2(__fmul2_rn(qf, E)));
                 // key side: own tile (diagonal) and the variants of later row tiles (variant i: rows 8 i (i+1) + r)
-                st_b32(sm + ps::BVAR + sw128_offset(8 * tq * (tq + 1) + r, c0, 160), pack2(__fmul2_rn(kf, I)));
+                st_b32(sm + ps::BVAR + (8 * tq * (tq + 1) + r) * 128 + sw, pack2(__fmul2_rn(kf, I)));
                 const float2 kF = __fmul2_rn(kf, F);
 #pragma unroll
                 for (int i = 1; i < 4; ++i)
                     if (i > tq)
-                        st_b32(sm + ps::BVAR + sw128_offset(8 * i * (i + 1) + r, c0, 160),
+                        st_b32(sm + ps::BVAR + (8 * i * (i + 1) + r) * 128 + sw,
                                pack2(__fmul2_rn(kF, make_float2(dvx[i], dvy[i]))));
-                // Q * gamma for the epilogue (P = Q gamma - ...)
-                st_b32(sm + ps::QT + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + (c0 & 7) * 2, pack2(__fmul2_rn(qf, G)));
-                const float2 tk2 = __fmul2_rn(__fmul2_rn(make_float2(-bt.x, -bt.y), kf), G);   // -beta K gamma
-                const float2 tv2 = __fmul2_rn(bt, vf);
-                const float2 td2 = __fmul2_rn(kF, ec2);
-                tk[0][j] = tk2.x; tk[1][j] = tk2.y;
-                tv[0][j] = tv2.x; tv[1][j] = tv2.y;
-                td[0][j] = td2.x; td[1][j] = td2.y;
+                // Q * gamma for the accumulator preload (P = Q gamma - ...)
+                st_b32(sm + ps::QG + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + kb, pack2(__fmul2_rn(qf, G)));
+                const float2 tk2 = __fmul2_rn(make_float2(-kf.x, -kf.y), G);   // -K gamma
+                const float2 td2 = __fmul2_rn(kF, ec2);                        // Kdec = K e^{g_C - g}
+                if (j & 1) {
+                    tkw[0][j >> 1] = pack_bf16x2(tkp.x, tk2.x); tkw[1][j >> 1] = pack_bf16x2(tkp.y, tk2.y);
+                    tdw[0][j >> 1] = pack_bf16x2(tdp.x, td2.x); tdw[1][j >> 1] = pack_bf16x2(tdp.y, td2.y);
+                } else {
+                    tkp = tk2;
+                    tdp = td2;
+                }
             }
-            // rows c of the transposed operands: lanes 4..7 of each quarter warp take their odd channel first,
-            // so that the 8 lanes of a quarter warp hit 8 different 16-byte bank groups
-            const bool odd_first = (cp >> 2) & 1;
+            // rows c of the transposed operands (8 tokens = one 16-byte chunk): lanes 4..7 of each quarter warp
+            // take their odd channel first, so that the 8 lanes of a quarter warp hit 8 different bank groups.
+            // -(K gamma)^T goes to KG; Kdec^T leaves for the packet straight from registers.
             {
-                const uint4 k0 = pack8(tk[0]), k1 = pack8(tk[1]), v0 = pack8(tv[0]), v1 = pack8(tv[1]);
+                const bool odd_first = (lane >> 2) & 1;
+                const uint4 k0 = make_uint4(tkw[0][0], tkw[0][1], tkw[0][2], tkw[0][3]);
+                const uint4 k1 = make_uint4(tkw[1][0], tkw[1][1], tkw[1][2], tkw[1][3]);
+                const uint4 d0 = make_uint4(tdw[0][0], tdw[0][1], tdw[0][2], tdw[0][3]);
+                const uint4 d1 = make_uint4(tdw[1][0], tdw[1][1], tdw[1][2], tdw[1][3]);
 #pragma unroll
                 for (int it = 0; it < 2; ++it) {
                     const int ch = it ^ static_cast<int>(odd_first);
                     const int c = c0 + ch;
-                    const uint32_t sw = static_cast<uint32_t>((q8 ^ (c & 7)) << 4);   // 8-token chunk q8 of row c
-                    *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + sw) = (ch ? k1 : k0);
-                    if (c < DV) *reinterpret_cast<uint4*>(sm + ps::BKV + (128 + c) * 128 + sw) = (ch ? v1 : v0);
+                    const uint32_t sw = static_cast<uint32_t>((w ^ (c & 7)) << 4);   // 8-token chunk w of row c
+                    *reinterpret_cast<uint4*>(sm + ps::KG + c * 128 + sw) = (ch ? k1 : k0);
+                    st_global_v4(pkt + P::KD + c * 128 + sw, ch ? d1 : d0);
                 }
             }
-            kd_pk[0] = pack8(td[0]);   // Kdec^T chunks: staged for the packet store after phase B
-            kd_pk[1] = pack8(td[1]);
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---------------- phase A: D[m, n] = RALL[m, :] . BVAR[n, :]  (M = 128, N = 160, K = 128); the
-        // columns of variant i (row tile i's key side) are [8 i (i+1), 8 (i+1)(i+2))
-        if (t == 0) {
-            tc_fence_after();
-            const uint32_t ra = smem_u32(sm + ps::RALL), bv = smem_u32(sm + ps::BVAR);
-            const uint32_t idesc = idesc_bf16(128, 160);
+            fence_proxy_async_smem();
+            __syncthreads();
+            // ---------------- product A, this half: D[m, n] += RALL[m, :] . BVAR[n, :]  (M = 128, N = 160,
+            // K = 64); the columns of variant i (row tile i's key side) are [8 i (i+1), 8 (i+1)(i+2))
+            if (t == 0) {
+                tc_fence_after();
+                const uint32_t ra = smem_u32(sm + ps::OPB), bv = smem_u32(sm + ps::BVAR);
+                const uint32_t idesc = idesc_bf16(128, 160);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
-                umma_f16(tm, sdesc_k_sw128(ra + ka * 16384 + kb), sdesc_k_sw128(bv + ka * 160 * 128 + kb), idesc, ks > 0);
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tm, sdesc_k_sw128(ra + ks * 32), sdesc_k_sw128(bv + ks * 32), idesc, hf > 0 || ks > 0);
+                umma_commit(&bar_mma);
             }
-            umma_commit(&bar_mma);
         }
-        // the next item's rows (MXFP8 inputs); look one more item ahead
-        if (nvalid) fetch_rows(nloc, nh, par ^ 1);
-        const int2 nnloc = entry(nitem + gridDim.x);
+        if (fail) break;
         {
             const bool ok = mbar_wait(&bar_mma, ph_mma, status);
             if (__syncthreads_or(!ok)) break;
@@ -445,54 +441,59 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // ---------------- TMEM -> fp32 A (strict lower, beta rows) and bf16 Aqk (inclusive lower) into [I; Aqk].
         // Lane quarter qw holds the rows of tiles t0 = 2 (qw & 1) and t0 + 1 (K rows for qw < 2, Q rows
         // otherwise).  Their variant columns form 2 t0 + 3 chunks of 16 (t0 + 1 of tile t0, t0 + 2 of tile
-        // t0 + 1), spread over the lane quarter's four warps, at most two per warp, loaded before one wait.
+        // t0 + 1), spread over the lane quarter's two warps, at most four per warp, in two rounds of two.
         {
             const int qw = w & 3, sub = w >> 2;
             const int t0 = 2 * (qw & 1), nchunk = 2 * t0 + 3;
             const int r = (32 * qw + lane) & 63;
             const bool is_q = qw >= 2;
             const float br = bet[r];
-            float v2[32];
-            int tile_of[2], cb_of[2];
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                const int j = sub + 4 * hb;
-                tile_of[hb] = j < t0 + 1 ? t0 : t0 + 1;
-                cb_of[hb] = 16 * (j < t0 + 1 ? j : j - t0 - 1);
-                if (j < nchunk) {
-                    tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 8 * tile_of[hb] * (tile_of[hb] + 1) + cb_of[hb],
-                              *reinterpret_cast<float(*)[16]>(v2 + 16 * hb));
-                } else {
+            for (int rd = 0; rd < 2; ++rd) {   // two rounds of two 16-column chunks: loads in flight, one wait
+                float v4[32];
+                int tile_of[2], cb_of[2];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v2[16 * hb + e] = 0.f;
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int j = sub + 2 * (2 * rd + hh);
+                    tile_of[hh] = j < t0 + 1 ? t0 : t0 + 1;
+                    cb_of[hh] = 16 * (j < t0 + 1 ? j : j - t0 - 1);
+                    if (j < nchunk) {
+                        tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 8 * tile_of[hh] * (tile_of[hh] + 1) +
+                                      cb_of[hh],
+                                  *reinterpret_cast<float(*)[16]>(v4 + 16 * hh));
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v4[16 * hh + e] = 0.f;
+                    }
                 }
-            }
-            tmem_wait_ld_regs<32>(v2);
+                tmem_wait_ld_regs<32>(v4);
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                const int cb = cb_of[hb];
-                const float* v = v2 + 16 * hb;
-                if (sub + 4 * hb < nchunk && (r >> 4) == tile_of[hb]) {   // this lane's row belongs to the chunk's tile
-                    if (is_q) {
-                        float o8[8];
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int cb = cb_of[hh];
+                    const float* v = v4 + 16 * hh;
+                    if (sub + 2 * (2 * rd + hh) < nchunk && (r >> 4) == tile_of[hh]) {   // the lane's row is in the tile
+                        if (is_q) {
+                            float o8[8];
 #pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
+                            for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) o8[j] = (cb + 8 * hf + j <= r) ? v[8 * hf + j] : 0.f;
-                            const int sc = (cb >> 3) + hf;
-                            *reinterpret_cast<uint4*>(sm + ps::IAQ + (64 + r) * 128 + ((sc ^ (r & 7)) << 4)) = pack8(o8);
+                                for (int j = 0; j < 8; ++j) o8[j] = (cb + 8 * hf + j <= r) ? v[8 * hf + j] : 0.f;
+                                const int sc = (cb >> 3) + hf;
+                                *reinterpret_cast<uint4*>(sm + ps::IAQ + (64 + r) * 128 + ((sc ^ (r & 7)) << 4)) =
+                                    pack8(o8);
+                            }
+                        } else if ((cb >> 4) == (r >> 4)) {   // diagonal block: transposed, strict lower part only
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int s2 = cb + j;
+                                if (s2 < r) AM[s2 * LDM + r] = br * v[j];
+                            }
+                        } else {                              // off-diagonal block: row-major
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                reinterpret_cast<float4*>(AM + r * LDM + cb)[q4] = make_float4(
+                                    br * v[4 * q4], br * v[4 * q4 + 1], br * v[4 * q4 + 2], br * v[4 * q4 + 3]);
                         }
-                    } else if ((cb >> 4) == (r >> 4)) {   // diagonal block: transposed, strict lower part only
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int s = cb + j;
-                            if (s < r) AM[s * LDM + r] = br * v[j];
-                        }
-                    } else {                              // off-diagonal block: row-major
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            reinterpret_cast<float4*>(AM + r * LDM + cb)[q4] =
-                                make_float4(br * v[4 * q4], br * v[4 * q4 + 1], br * v[4 * q4 + 2], br * v[4 * q4 + 3]);
                     }
                 }
             }
@@ -500,23 +501,24 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tc_fence_before();
         __syncthreads();
 
-        // Meanwhile warps 8..15, idle in the solve, start product B's K-part accumulator (TMEM columns
-        // 0..127, free since the A epilogue) as [0; Q gamma], so that it ends as [-W; P] with
-        // P = Q gamma - Aqk W.  The TMEM stores are spread over the solve's first two levels and waited
-        // for in the third.
+        // Meanwhile warps 4..7, idle in the first two solve levels, start product B's K-part accumulator
+        // (TMEM columns 0..127, free since the A epilogue) as [0; Q gamma], so that it ends as [-W; P] with
+        // P = Q gamma - Aqk W.  Warp w writes the 128 columns of lane quarter w & 3, 64 per level, and waits
+        // for its stores before the third level.
         auto preload_qgamma = [&](int c_lo, int c_hi) {
-            const int qw = w & 3, half = (w - 8) >> 2;
-            const uint32_t base = tm + (static_cast<uint32_t>(32 * qw) << 16) + 64 * half;
+            tc_fence_after();   // after the A epilogue's TMEM loads of these columns (barrier in between)
+            const int qw = w & 3;
+            const uint32_t base = tm + (static_cast<uint32_t>(32 * qw) << 16);
             const int r = 32 * qw + lane - 64;   // token row of the Q part (lane quarters 2 and 3)
 #pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16) {
+            for (int c16 = 0; c16 < 8; ++c16) {
                 if (c16 < c_lo || c16 >= c_hi) continue;
                 float x[16];
                 if (qw >= 2) {
-                    const int ch = (64 * half + 16 * c16) >> 3;   // first 8-channel chunk of the 16 columns
+                    const int ch = 2 * c16;   // first 8-channel chunk of the 16 columns
                     float a8[8], b8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + ((ch ^ (r & 7)) << 4)), a8);
-                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QT + r * 256 + (((ch + 1) ^ (r & 7)) << 4)), b8);
+                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QG + r * 256 + ((ch ^ (r & 7)) << 4)), a8);
+                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QG + r * 256 + (((ch + 1) ^ (r & 7)) << 4)), b8);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) { x[j] = a8[j]; x[8 + j] = b8[j]; }
                 } else {
@@ -560,13 +562,12 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
                 for (int r = 0; r < 16; ++r) XF[(o0 + r) * LDX + o0 + col] = x[r];
             }
-        } else if (w < 8) {
+        } else {
             for (int e = t - 128; e < 64 * 64; e += 128) {   // the blocks above the diagonal are zero
                 const int r = e >> 6, c = e & 63;
                 if ((c >> 4) > (r >> 4)) XF[r * LDX + c] = 0.f;
             }
-        } else {
-            preload_qgamma(0, 2);
+            preload_qgamma(0, 4);
         }
         __syncthreads();
         // Levels 1 and 2 merge two inverted diagonal blocks: X_10 = -X_11 (A_10 X_00).  The products are
@@ -606,11 +607,13 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             xo[fg * LDX + 1] = -e[1];
             xo[(fg + 8) * LDX] = -e[2];
             xo[(fg + 8) * LDX + 1] = -e[3];
-        } else if (w >= 8) {
-            preload_qgamma(2, 4);
+        } else {
+            preload_qgamma(4, 8);
+            tmem_wait_st();   // the accumulator preload has landed (published by the barriers before product B)
+            tc_fence_before();
         }
         __syncthreads();
-        if (w < 8) {   // level 2: 32 -> 64, row tile mt of 16 and column tile nt of 8
+        {   // level 2: 32 -> 64, row tile mt of 16 and column tile nt of 8
             const int nt = w & 3, mt = w >> 2;
             float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -646,18 +649,17 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             xo[fg * LDX + 1] = -e[1];
             xo[(fg + 8) * LDX] = -e[2];
             xo[(fg + 8) * LDX + 1] = -e[3];
-        } else {   // the accumulator preload has landed
-            tmem_wait_st();
-            tc_fence_before();
         }
         __syncthreads();
-        // X^T as the bf16 B operand of the Y product: row m = column m of X, K = 64 rows of X
-        {
-            const int m = t >> 3, uc = t & 7;
+        // X^T as the bf16 B operand of the Y product (row m = column m of X, K = 64 rows of X), over Q gamma
+        // (consumed by the preload)
+#pragma unroll
+        for (int e = t; e < 64 * 8; e += NT) {
+            const int m = e >> 3, uc = e & 7;
             float v[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) v[j] = XF[(8 * uc + j) * LDX + m];
-            *reinterpret_cast<uint4*>(sm + ps::XT + m * 128 + ((uc ^ (m & 7)) << 4)) = pack8(v);
+            *reinterpret_cast<uint4*>(sm + ps::QG + m * 128 + ((uc ^ (m & 7)) << 4)) = pack8(v);
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -665,11 +667,11 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // ---------------- phase Y: [X; Y] = [I; Aqk] X   (M = 128, N = 64, K = 64)
         if (t == 0) {
             tc_fence_after();
-            const uint32_t ia = smem_u32(sm + ps::IAQ), xt = smem_u32(sm + ps::XT);
+            const uint32_t ia = smem_u32(sm + ps::IAQ), xt = smem_u32(sm + ps::QG);
             const uint32_t idesc = idesc_bf16(128, 64);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tm + 256, sdesc_k_sw128(ia + ks * 32), sdesc_k_sw128(xt + ks * 32), idesc, ks > 0);
+                umma_f16(tm + 128, sdesc_k_sw128(ia + ks * 32), sdesc_k_sw128(xt + ks * 32), idesc, ks > 0);
             umma_commit(&bar_mma);
         }
         {
@@ -678,37 +680,47 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
         ph_mma ^= 1;
         tc_fence_after();
-        {   // 16 warps: lane quarter qw, 16-column group cg
+        {   // [X; Y] diag(beta) as product B's A operand (K = 64 tokens): lane quarter qw, 32-column group cg
             const int qw = w & 3, cg = w >> 2;
             const int m = 32 * qw + lane;
-            float v[16];
-            tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 256 + 16 * cg, v);
-            tmem_wait_ld_regs<16>(v);
+            float v[32];
+            tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 128 + 32 * cg, *reinterpret_cast<float(*)[16]>(v));
+            tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 128 + 32 * cg + 16,
+                      *reinterpret_cast<float(*)[16]>(v + 16));
+            tmem_wait_ld_regs<32>(v);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            for (int hf = 0; hf < 4; ++hf) {
                 float o8[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) o8[j] = v[8 * hf + j];
-                const int sc = 2 * cg + hf;
-                *reinterpret_cast<uint4*>(sm + ps::XY + m * 128 + ((sc ^ (m & 7)) << 4)) = pack8(o8);
+                for (int j = 0; j < 8; ++j) o8[j] = v[8 * hf + j] * bet[32 * cg + 8 * hf + j];
+                const int sc = 4 * cg + hf;
+                *reinterpret_cast<uint4*>(sm + ps::OPB + m * 128 + ((sc ^ (m & 7)) << 4)) = pack8(o8);
             }
         }
         tc_fence_before();
         fence_proxy_async_smem();
-        __syncthreads();
+        {   // V of this item has landed (bf16 inputs: its TMA tile)
+            bool ok = true;
+            if (!MX && t == 0) {
+                ok = mbar_wait(&bar_v, ph_v, status);
+                v_pending = false;
+            }
+            ph_v ^= 1;
+            if (__syncthreads_or(!ok)) break;
+        }
 
-        // ---------------- phase B: D[m, n] = [X; Y][m, :] . [-beta K gamma | beta V]^T[n, :]  (K = 64): the
-        // K part (N = 128) onto the preloaded [0; Q gamma], the V part (N = DV) from zero
+        // ---------------- phase B: D[m, n] = [X; Y] diag(beta) [m, :] . B[n, :]  (K = 64 tokens): the K part
+        // (N = 128, B = -(K gamma)^T) onto the preloaded [0; Q gamma], the V part (N = DV, B = V MN-major) from zero
         if (t == 0) {
             tc_fence_after();
-            const uint32_t xa = smem_u32(sm + ps::XY), kb = smem_u32(sm + ps::BKV);
-            const uint32_t idk = idesc_bf16(128, 128), idv = idesc_bf16(128, DV);
+            const uint32_t xa = smem_u32(sm + ps::OPB), kb = smem_u32(sm + ps::KG), vb = smem_u32(sm + ps::VOP);
+            const uint32_t idk = idesc_bf16(128, 128), idv = idesc_bf16(128, DV, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 umma_f16(tm, sdesc_k_sw128(xa + ks * 32), sdesc_k_sw128(kb + ks * 32), idk, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tm + 128, sdesc_k_sw128(xa + ks * 32), sdesc_k_sw128(kb + 128 * 128 + ks * 32), idv, ks > 0);
+                umma_f16(tm + 128, sdesc_k_sw128(xa + ks * 32), sdesc_mn_sw128(vb + ks * 2048, 8192), idv, ks > 0);
             umma_commit(&bar_mma);
         }
         {
@@ -717,86 +729,54 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
         ph_mma ^= 1;
         tc_fence_after();
+        // product B has read VOP: the next item's V may land there now
+        if (t == 0 && nvalid) issue_v(nloc.x, nh);
 
-        // ---------------- epilogue: rows 0..63 -> -W | U, rows 64..127 -> P | O_intra, all straight from TMEM
+        // ---------------- epilogue: rows 0..63 -> -W | U, rows 64..127 -> P | O_intra, straight from TMEM into
+        // the packet staging ([-W; P] over OPB, [U; O_intra] over QG and KG)
         {
-            const int qw = w & 3, cg = w >> 2;   // 64-column group: 0,1 -> K part, 2,3 -> V part
+            const int qw = w & 3, cg = w >> 2;   // cg 0: K part, cg 1: V part
             const int m = 32 * qw + lane;
-            const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
-            if (cg < 2) {
-                {   // the group's 64 columns: four loads in flight, one wait
-                    const int c32 = 2 * cg;
-                    float vv[64];
+            const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16) + 128 * cg;
+            uint8_t* dst0 = sm + (cg == 0 ? ps::OPB : ps::QG);
+            const int natoms = cg == 0 ? 2 : DV / 64;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        tmem_ld16(lane_base + 32 * c32 + 16 * i, *reinterpret_cast<float(*)[16]>(vv + 16 * i));
-                    tmem_wait_ld_regs<64>(vv);
+            for (int a = 0; a < 2; ++a) {
+                if (a >= natoms) break;
+                float vv[64];
 #pragma unroll
-                    for (int sub = 0; sub < 8; ++sub) {
-                        const int cc = 4 * c32 + sub;
-                        const float* v = vv;
-                        float o8[8];
+                for (int i = 0; i < 4; ++i) tmem_ld16(lane_base + 64 * a + 16 * i, *reinterpret_cast<float(*)[16]>(vv + 16 * i));
+                tmem_wait_ld_regs<64>(vv);
+                uint8_t* dst = dst0 + a * 16384 + m * 128;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) o8[j] = v[8 * sub + j];
-                        *reinterpret_cast<uint4*>(sm + ps::AWS + (cc >> 3) * 16384 + m * 128 +
-                                                  (((cc & 7) ^ (m & 7)) << 4)) = pack8(o8);
-                    }
+                for (int sub = 0; sub < 8; ++sub) {
+                    float o8[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) o8[j] = vv[8 * sub + j];
+                    *reinterpret_cast<uint4*>(dst + ((sub ^ (m & 7)) << 4)) = pack8(o8);
                 }
-            } else if (64 * (cg - 2) < DV) {
-                {
-                    const int c32 = 2 * (cg - 2);
-                    float vv[64];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        tmem_ld16(lane_base + 128 + 32 * c32 + 16 * i, *reinterpret_cast<float(*)[16]>(vv + 16 * i));
-                    tmem_wait_ld_regs<64>(vv);
-#pragma unroll
-                    for (int sub = 0; sub < 8; ++sub) {
-                        const int cc = 4 * c32 + sub;
-                        const float* v = vv;
-                        float o8[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) o8[j] = v[8 * sub + j];
-                        *reinterpret_cast<uint4*>(sm + ps::UOS + (cc >> 3) * 16384 + m * 128 +
-                                                  (((cc & 7) ^ (m & 7)) << 4)) = pack8(o8);
-                    }
-                }
-            }
-        }
-        {   // Kdec^T (held in registers since the column pass) into the B operand area phase B has released
-            const int cp = t & 63, c0 = 2 * cp, q8 = t >> 6;
-            const int odd_first = (cp >> 2) & 1;
-#pragma unroll
-            for (int it = 0; it < 2; ++it) {
-                const int ch = it ^ odd_first;
-                const int c = c0 + ch;
-                *reinterpret_cast<uint4*>(sm + ps::BKV + c * 128 + ((q8 ^ (c & 7)) << 4)) = ch ? kd_pk[1] : kd_pk[0];
             }
         }
         tc_fence_before();
         fence_proxy_async_smem();
         __syncthreads();
         if (t == 0) {
-            bulk_s2g(pkt + P::AW, sm + ps::AWS, 32768);
-            bulk_s2g(pkt + P::KD, sm + ps::BKV, 16384);
-            bulk_s2g(pkt + P::UO, sm + ps::UOS, DV * 256);
+            bulk_s2g(pkt + P::AW, sm + ps::OPB, 32768);
+            bulk_s2g(pkt + P::UO, sm + ps::QG, DV * 256);
             bulk_commit();   // the next column pass waits for the read-out before reusing the staging
         }
         item = nitem;
         loc = nloc;
-        nloc = nnloc;
         h = nh;
         valid = nvalid;
-        par ^= 1;
     }
-    if (MX && t >= 256) cp_async_wait_all();   // nor a fetch of rows
     if (t == 0) {
-        if (load_pending) mbar_wait(&bar_load, ph_load, nullptr);   // never leave a TMA write in flight
+        if (v_pending) mbar_wait(&bar_v, ph_v, nullptr);   // never leave a TMA write in flight
         bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tm, 512);
+    if (w == 0) tmem_dealloc(tm, 256);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -1217,20 +1197,29 @@ cudaError_t launch_prep(const ChunkArgs& a, long long items, cudaStream_t s) {
     CUtensorMap mq, mk, mv, ml;
     const CUtensorMapDataType dt = MX ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int es = MX ? 1 : 2;
-    // bf16: 64-column boxes; MXFP8: the whole row of codes in one box
+    // q, k (and MXFP8 v codes) are read with plain loads: their maps only prefetch boxes into L2 (bf16: 64-column
+    // boxes; MXFP8: the whole row of codes).  bf16 v is loaded as product B's operand: 64-column x 64-token boxes
+    // with the 128-byte swizzle, the MN-major layout of the tensor-core descriptor.
     if (!make_map(&mq, a.q, dt, es, kDK, a.H, a.total_tokens, MX ? kDK : 64) ||
         !make_map(&mk, a.k, dt, es, kDK, a.H, a.total_tokens, MX ? kDK : 64) ||
-        !make_map(&mv, a.v, dt, es, DV, a.H, a.total_tokens, MX ? DV : 64) ||
+        !make_map(&mv, a.v, dt, es, DV, a.H, a.total_tokens, MX ? DV : 64,
+                  MX ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&ml, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, a.H, a.total_tokens, 32))
         return cudaErrorInvalidValue;
     const int smem = static_cast<int>(MX ? ps::BYTES_MX : ps::BYTES) + 1024;
     cudaError_t e = cudaFuncSetAttribute(prep_bf16_kernel<DV, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const long long grid = items < num_sms() ? items : num_sms();
+    // all of the SM's unified L1 / shared storage as shared memory, so that two CTAs fit side by side
+    e = cudaFuncSetAttribute(prep_bf16_kernel<DV, MX>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    const long long slots = 2LL * num_sms();   // two CTAs per SM
+    const long long grid = items < slots ? items : slots;
     return launch_pdl(prep_bf16_kernel<DV, MX>, dim3(static_cast<unsigned>(grid)), dim3(ps::NT), smem, s, mq, mk, mv,
-                      ml, a.beta, static_cast<const uint8_t*>(a.q_scale), static_cast<const uint8_t*>(a.k_scale),
-                      static_cast<const uint8_t*>(a.v_scale), a.chunk_tab, a.H, items,
-                      static_cast<uint8_t*>(a.packets), a.status);
+                      ml, static_cast<const uint8_t*>(a.q), static_cast<const uint8_t*>(a.k),
+                      static_cast<const uint8_t*>(a.v), a.log_alpha, a.beta, static_cast<const uint8_t*>(a.q_scale),
+                      static_cast<const uint8_t*>(a.k_scale), static_cast<const uint8_t*>(a.v_scale), a.chunk_tab,
+                      a.H, items, static_cast<uint8_t*>(a.packets), a.status);
 }
 
 template <int DV>

@@ -1,6 +1,8 @@
-// kda_umma_selftest.cu -- diagnostic: one tcgen05 bf16 product through the same shared-memory
-// descriptors (128-byte swizzle; B K-major or MN-major), TMEM allocation, commit and TMEM-load path
-// that the chunk kernels use.  D[128, n] = A[128, 64] * B[n, 64]^T.  No KDA arithmetic.
+// kda_umma_selftest.cu -- diagnostics of the tcgen05 path the chunk kernels use, no KDA arithmetic:
+//  * one bf16 product through the same shared-memory descriptors (128-byte swizzle; B K-major or
+//    MN-major), TMEM allocation, commit and TMEM-load path: D[128, n] = A[128, 64] * B[n, 64]^T;
+//  * the tensor-core rate of a product shape as the kernels issue it (M = 128 x N x K, one CTA per SM,
+//    timed with the SM clock): back to back, and one product at a time waited for before the next.
 #include "kda_device.cuh"
 #include "kda_internal.h"
 
@@ -73,6 +75,80 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
     tc_fence_before();
     __syncthreads();
     if (w == 0) tmem_dealloc(tm, 256);
+}
+
+// One CTA per SM; thread 0 times `reps` products of shape 128 x n x k (operands zero: only the timing
+// matters) issued back to back with one commit at the end, then `reps` products each committed and waited
+// for before the next.  cycles[2 * blockIdx.x + {0, 1}] = SM cycles per product in the two modes.
+__global__ void __launch_bounds__(128) selftest_mma_rate_kernel(int n, int k, int b_mn, int reps, float* cycles,
+                                                                int* status) {
+    extern __shared__ __align__(1024) uint8_t raw[];
+    uint8_t* base = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+    uint8_t* sA = base;                          // [k / 64 atoms][128 rows][128 B]
+    uint8_t* sB = base + (k / 64) * 16384;       // K-major [k / 64][n][128 B] or MN-major [n / 64][k][128 B]
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t tbase;
+    const int t = threadIdx.x, w = t >> 5;
+    const int words = ((k / 64) * 16384 + n * k * 2) / 16;
+    for (int e = t; e < words; e += 128) reinterpret_cast<uint4*>(base)[e] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+    if (t == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    if (w == 0) {
+        tmem_alloc(&tbase, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tbase;
+    if (t == 0) {
+        const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0);
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+        auto product = [&]() {
+            for (int ks = 0; ks < k / 16; ++ks) {
+                const uint32_t ka = (ks >> 2) * 16384 + (ks & 3) * 32;
+                const uint64_t db = b_mn ? sdesc_mn_sw128(b0 + ks * 2048, static_cast<uint32_t>(k) * 128)
+                                         : sdesc_k_sw128(b0 + (ks >> 2) * n * 128 + (ks & 3) * 32);
+                umma_f16(tm, sdesc_k_sw128(a0 + ka), db, idesc, ks > 0);
+            }
+        };
+        uint32_t ph = 0;
+        bool ok = true;
+        product();                               // warm-up
+        umma_commit(&bar);
+        ok = ok && mbar_wait(&bar, ph, status);
+        ph ^= 1;
+        const long long t0 = clock64();
+        for (int r = 0; r < reps; ++r) product();
+        umma_commit(&bar);
+        ok = ok && mbar_wait(&bar, ph, status);
+        ph ^= 1;
+        const long long t1 = clock64();
+        for (int r = 0; r < reps && ok; ++r) {
+            product();
+            umma_commit(&bar);
+            ok = mbar_wait(&bar, ph, status);
+            ph ^= 1;
+        }
+        const long long t2 = clock64();
+        cycles[2 * blockIdx.x] = ok ? static_cast<float>(t1 - t0) / reps : -1.f;
+        cycles[2 * blockIdx.x + 1] = ok ? static_cast<float>(t2 - t1) / reps : -1.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tm, 256);
+}
+
+cudaError_t launch_selftest_mma_rate(int n, int k, int b_mn, int reps, float* cycles, int grid, int* status,
+                                     cudaStream_t s) {
+    const int smem = 1024 + (k / 64) * 16384 + n * k * 2;
+    cudaError_t e = cudaFuncSetAttribute(selftest_mma_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    selftest_mma_rate_kernel<<<grid, 128, smem, s>>>(n, k, b_mn, reps, cycles, status);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int b_mn, int* status,
