@@ -154,10 +154,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     constexpr int LDM = ps::LDM;
     constexpr int LDX = ps::LDX;
     constexpr int LDTT = ps::LDTT;
-    constexpr int ES = MX ? 1 : 2;   // bytes per q/k/v element
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    __shared__ __align__(8) uint64_t bar_v, bar_mma;
+    __shared__ __align__(8) uint64_t bar_in, bar_mma;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     float* bet = reinterpret_cast<float*>(sm + ps::MISC);
@@ -170,7 +169,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     float* TT = reinterpret_cast<float*>(sm + ps::TOT);   // T = A_10 X_00 of a merge, pitch LDTT
 
     if (t == 0) {
-        mbar_init(&bar_v, 1);
+        mbar_init(&bar_in, 1);
         mbar_init(&bar_mma, 1);
         fence_barrier_init();
         prefetch_tmap(&map_q); prefetch_tmap(&map_k); prefetch_tmap(&map_v); prefetch_tmap(&map_l);
@@ -196,34 +195,47 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tmem_slot;
-    uint32_t ph_v = 0, ph_mma = 0;
-    bool v_pending = false;   // meaningful in thread 0 only
+    uint32_t ph_in = 0, ph_mma = 0;
+    bool in_pending = false;   // a TMA load into VOP is in flight (meaningful in thread 0 only)
 
-    // V of an item as product B's MN-major B operand (bf16 inputs; thread 0)
-    auto issue_v = [&](long long tok0, int hh) {
+    // bf16 inputs (thread 0): VOP takes, in turn, the k and q tiles of the first 64-channel half of an item
+    // ([64 tokens][128 B] each, read by the column pass), those of the second half, and finally V as product
+    // B's MN-major operand; each load completes one phase of bar_in.
+    auto issue_kq = [&](long long tok0, int hh, int hf) {
         if constexpr (!MX) {
-            mbar_arrive_expect_tx(&bar_v, DV * 128);
-#pragma unroll
-            for (int b = 0; b < DV / 64; ++b)
-                tma_load_3d(sm + ps::VOP + b * 8192, &map_v, 64 * b, hh, static_cast<int>(tok0), &bar_v);
-            v_pending = true;
+            mbar_arrive_expect_tx(&bar_in, 2 * 8192);
+            tma_load_3d(sm + ps::VOP, &map_k, 64 * hf, hh, static_cast<int>(tok0), &bar_in);
+            tma_load_3d(sm + ps::VOP + 8192, &map_q, 64 * hf, hh, static_cast<int>(tok0), &bar_in);
+            in_pending = true;
         }
     };
-    // an item's inputs that the column pass reads with plain loads, into L2 ahead of time (thread 0)
-    auto prefetch_inputs = [&](long long tok0, int hh) {
-        const int tk = static_cast<int>(tok0);
+    auto issue_v = [&](long long tok0, int hh) {
+        if constexpr (!MX) {
+            mbar_arrive_expect_tx(&bar_in, DV * 128);
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) tma_prefetch_3d(&map_l, 32 * qq, hh, tk);
-        if constexpr (MX) {
-            tma_prefetch_3d(&map_q, 0, hh, tk);
-            tma_prefetch_3d(&map_k, 0, hh, tk);
-            tma_prefetch_3d(&map_v, 0, hh, tk);
-        } else {
+            for (int b = 0; b < DV / 64; ++b)
+                tma_load_3d(sm + ps::VOP + b * 8192, &map_v, 64 * b, hh, static_cast<int>(tok0), &bar_in);
+            in_pending = true;
+        }
+    };
+    // bounded wait for the load into VOP issued last (all threads; bf16 inputs only)
+    auto wait_in = [&]() -> bool {
+        if constexpr (MX) return true;
+        const bool ok = mbar_wait(&bar_in, ph_in, status);
+        ph_in ^= 1;
+        if (t == 0) in_pending = false;
+        return ok;
+    };
+    // this thread's log_alpha pairs (channels c0, c0 + 1; the 8 tokens of its warp) of one 64-channel half,
+    // loaded one half ahead of their use (zero past the item's n tokens)
+    float2 nla[8];
+    auto load_la_half = [&](int2 l, int hh, int hf) {
+        const size_t row0 = static_cast<size_t>(l.x) * H + hh;
+        const int c0 = 64 * hf + 2 * lane;
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                tma_prefetch_3d(&map_q, 64 * b, hh, tk);
-                tma_prefetch_3d(&map_k, 64 * b, hh, tk);
-            }
+        for (int j = 0; j < 8; ++j) {
+            const int r = 8 * w + j;
+            nla[j] = r < l.y ? ld_once_f2(lag + (row0 + static_cast<size_t>(r) * H) * kDK + c0) : make_float2(0.f, 0.f);
         }
     };
 
@@ -235,9 +247,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     int2 loc = entry(item);
     int h = static_cast<int>(item % H);
     bool valid = loc.y > 0;
-    if (t == 0 && valid) {
-        issue_v(loc.x, h);
-        prefetch_inputs(loc.x, h);
+    if (valid && !MX) {
+        if (t == 0) issue_kq(loc.x, h, 0);
+        load_la_half(loc, h, 0);
     }
 
     while (valid) {
@@ -247,29 +259,24 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int2 nloc = entry(nitem);
         const int nh = static_cast<int>(nitem % H);
         const bool nvalid = nloc.y > 0;
-        if (t == 0 && nvalid) prefetch_inputs(nloc.x, nh);
+        // beta (threads 0..63) and the MXFP8 scale words (threads 64..255) of the chunk's rows go to shared
+        // memory only later in the column pass, so that no thread waits for these loads before its first barrier
+        float beta_r = 0.f;
+        uint32_t scale_w = 0x7F7F7F7Fu;   // scale 1.0 past the item's end
         if (t < 64) {
-            bet[t] = t < n ? beta[(static_cast<size_t>(loc.x) + t) * H + h] : 0.f;
+            if (t < n) beta_r = beta[(static_cast<size_t>(loc.x) + t) * H + h];
             if (nvalid && t < nloc.y) prefetch_l2(beta + (static_cast<size_t>(nloc.x) + t) * H + nh);
-        }
-        if constexpr (MX) {   // the shared scales of the chunk's tokens as fp32 (scale 1.0 past its end)
-            if (t >= 64) {
-                const int which = (t - 64) >> 6, rr = (t - 64) & 63;
-                const size_t row = (static_cast<size_t>(loc.x) + rr) * H + h;
-                uint32_t wv = 0x7F7F7F7Fu;
-                if (rr < n) {
-                    if (which == 0) wv = ld_once_u32(q_scale + 4 * row);
-                    else if (which == 1) wv = ld_once_u32(k_scale + 4 * row);
-                    else wv = DV == 128 ? ld_once_u32(v_scale + 4 * row) : (0x7F7F0000u | ld_once_u16(v_scale + 2 * row));
-                }
-                reinterpret_cast<float4*>(sm + ps::SCF)[which * 64 + rr] =
-                    make_float4(e8m0_to_f32(wv & 0xFFu), e8m0_to_f32((wv >> 8) & 0xFFu),
-                                e8m0_to_f32((wv >> 16) & 0xFFu), e8m0_to_f32(wv >> 24));
+        } else if constexpr (MX) {
+            const int which = (t - 64) >> 6, rr = (t - 64) & 63;
+            const size_t row = (static_cast<size_t>(loc.x) + rr) * H + h;
+            if (rr < n) {
+                if (which == 0) scale_w = ld_once_u32(q_scale + 4 * row);
+                else if (which == 1) scale_w = ld_once_u32(k_scale + 4 * row);
+                else scale_w = DV == 128 ? ld_once_u32(v_scale + 4 * row) : (0x7F7F0000u | ld_once_u16(v_scale + 2 * row));
             }
         }
-        // the previous item's packet staging (OPB, QG, KG) must have been read out before this column
-        // pass writes there; the first barrier below publishes the wait
-        if (t == 0) bulk_wait_read0();
+        // the previous item's packet staging (OPB, QG, KG) must have been read out before this column pass
+        // writes there: each warp's lane 0 waits for the bulk copies it issued, before the first barrier below
 
         // ---------------- column pass, one 64-channel half at a time: thread = (channel pair, the 8 tokens
         // of its warp); each half ends with its share of product A (K = 64 channels)
@@ -284,30 +291,40 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             for (int j = 0; j < 8; ++j) {
                 const int r = 8 * w + j;
                 kb8[j] = qb8[j] = vb8[j] = 0u;
-                p[j] = make_float2(0.f, 0.f);
-                if (r < n) {
-                    const size_t rr = row0 + static_cast<size_t>(r) * H;
-                    p[j] = ld_once_f2(lag + rr * kDK + c0);
-                    if constexpr (MX) {
+                if constexpr (MX) {   // MXFP8: log_alpha and the codes of this half with plain loads
+                    p[j] = make_float2(0.f, 0.f);
+                    if (r < n) {
+                        const size_t rr = row0 + static_cast<size_t>(r) * H;
+                        p[j] = ld_once_f2(lag + rr * kDK + c0);
                         kb8[j] = ld_once_u16(kg + rr * kDK + c0);
                         qb8[j] = ld_once_u16(qg + rr * kDK + c0);
                         if (c0 < DV) vb8[j] = ld_once_u16(vg + rr * DV + c0);
-                    } else {
-                        kb8[j] = ld_once_u32(kg + (rr * kDK + c0) * ES);
-                        qb8[j] = ld_once_u32(qg + (rr * kDK + c0) * ES);
                     }
+                } else {              // bf16: log_alpha loaded one half ahead; k, q are the TMA tiles in VOP
+                    p[j] = nla[j];
                 }
             }
+            if (!MX && hf == 0) load_la_half(loc, h, 1);   // lands while this half's operands are made
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 if (8 * w + j < n) acc = __fadd2_rn(acc, make_float2(floor_log_decay(p[j].x), floor_log_decay(p[j].y)));
                 p[j] = acc;
             }
             *reinterpret_cast<float2*>(tot + w * 64 + 2 * lane) = acc;
-            __syncthreads();
-            if (hf == 1) {   // product A's first half has finished reading OPB
-                const bool ok = mbar_wait(&bar_mma, ph_mma, status);
-                ph_mma ^= 1;
+            if constexpr (MX) {   // the shared scales of the chunk's tokens as fp32, needed from here on
+                if (hf == 0 && t >= 64)
+                    reinterpret_cast<float4*>(sm + ps::SCF)[t - 64] =
+                        make_float4(e8m0_to_f32(scale_w & 0xFFu), e8m0_to_f32((scale_w >> 8) & 0xFFu),
+                                    e8m0_to_f32((scale_w >> 16) & 0xFFu), e8m0_to_f32(scale_w >> 24));
+            }
+            if (hf == 0 && lane == 0) bulk_wait_read0();
+            {   // this half's k and q tiles have landed (bf16), and product A's first half has finished reading
+                // OPB (second half)
+                bool ok = wait_in();
+                if (hf == 1) {
+                    ok = mbar_wait(&bar_mma, ph_mma, status) && ok;
+                    ph_mma ^= 1;
+                }
                 if (__syncthreads_or(!ok)) { fail = true; break; }
             }
             if (w & 1) {   // second half of the tile: add the first half's total
@@ -365,9 +382,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                                    ((kk ^ static_cast<uint32_t>(r & 7)) << 4) + kb,
                                pack2(vf));
                     }
-                } else {
-                    kf = bf2_to_f2(kb8[j]);
-                    qf = bf2_to_f2(qb8[j]);
+                } else {   // rows past n hold other tokens' (finite) values, which nothing below lets through
+                    kf = bf2_to_f2(*reinterpret_cast<const uint32_t*>(sm + ps::VOP + r * 128 + (c0 & 63) * 2));
+                    qf = bf2_to_f2(*reinterpret_cast<const uint32_t*>(sm + ps::VOP + 8192 + r * 128 + (c0 & 63) * 2));
                 }
                 const float2 pl = __fmul2_rn(p[j], f2(kLog2e));
                 const float2 E = make_float2(ex2_approx(pl.x), ex2_approx(pl.y));     // e^{g_r - b_t} <= 1
@@ -416,6 +433,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     st_global_v4(pkt + P::KD + c * 128 + sw, ch ? d1 : d0);
                 }
             }
+            if (hf == 0 && t < 64) bet[t] = beta_r;   // first read by the A epilogue
             fence_proxy_async_smem();
             __syncthreads();
             // ---------------- product A, this half: D[m, n] += RALL[m, :] . BVAR[n, :]  (M = 128, N = 160,
@@ -428,6 +446,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 for (int ks = 0; ks < 4; ++ks)
                     umma_f16(tm, sdesc_k_sw128(ra + ks * 32), sdesc_k_sw128(bv + ks * 32), idesc, hf > 0 || ks > 0);
                 umma_commit(&bar_mma);
+                // VOP has been read: the second half's k and q tiles, then V (product B's operand)
+                if (hf == 0) issue_kq(loc.x, h, 1);
+                else issue_v(loc.x, h);
             }
         }
         if (fail) break;
@@ -700,12 +721,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tc_fence_before();
         fence_proxy_async_smem();
         {   // V of this item has landed (bf16 inputs: its TMA tile)
-            bool ok = true;
-            if (!MX && t == 0) {
-                ok = mbar_wait(&bar_v, ph_v, status);
-                v_pending = false;
-            }
-            ph_v ^= 1;
+            const bool ok = wait_in();
             if (__syncthreads_or(!ok)) break;
         }
 
@@ -729,11 +745,16 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
         ph_mma ^= 1;
         tc_fence_after();
-        // product B has read VOP: the next item's V may land there now
-        if (t == 0 && nvalid) issue_v(nloc.x, nh);
+        // product B has read VOP
+        if (!MX && nvalid) {   // VOP is free again: the next item's first k, q tiles; and its first log_alpha half
+            if (t == 0) issue_kq(nloc.x, nh, 0);
+            load_la_half(nloc, nh, 0);
+        }
 
         // ---------------- epilogue: rows 0..63 -> -W | U, rows 64..127 -> P | O_intra, straight from TMEM into
-        // the packet staging ([-W; P] over OPB, [U; O_intra] over QG and KG)
+        // the packet staging ([-W; P] over OPB, [U; O_intra] over QG and KG).  Each warp stages the 32 rows of
+        // its lane quarter (4 KB of each atom it covers) and sends them with its own bulk copies at once, so no
+        // CTA barrier precedes the packet store.
         {
             const int qw = w & 3, cg = w >> 2;   // cg 0: K part, cg 1: V part
             const int m = 32 * qw + lane;
@@ -756,24 +777,23 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     *reinterpret_cast<uint4*>(dst + ((sub ^ (m & 7)) << 4)) = pack8(o8);
                 }
             }
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (t == 0) {
-            bulk_s2g(pkt + P::AW, sm + ps::OPB, 32768);
-            bulk_s2g(pkt + P::UO, sm + ps::QG, DV * 256);
-            bulk_commit();   // the next column pass waits for the read-out before reusing the staging
+            tc_fence_before();   // this warp's TMEM loads precede the next item's products (barriers in between)
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                uint8_t* gdst = pkt + (cg == 0 ? P::AW : P::UO) + 32 * qw * 128;
+                for (int a = 0; a < natoms; ++a)
+                    bulk_s2g(gdst + a * 16384, dst0 + a * 16384 + 32 * qw * 128, 4096);
+                bulk_commit();   // waited for (read out) before the next column pass's first barrier
+            }
         }
         item = nitem;
         loc = nloc;
         h = nh;
         valid = nvalid;
     }
-    if (t == 0) {
-        if (v_pending) mbar_wait(&bar_v, ph_v, nullptr);   // never leave a TMA write in flight
-        bulk_wait0();
-    }
+    if (t == 0 && in_pending) mbar_wait(&bar_in, ph_in, nullptr);   // never leave a TMA write in flight
+    if (lane == 0) bulk_wait0();                                    // nor a packet store
     tc_fence_before();
     __syncthreads();
     if (w == 0) tmem_dealloc(tm, 256);
