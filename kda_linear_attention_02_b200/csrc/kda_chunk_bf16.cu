@@ -198,16 +198,18 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint32_t ph_in = 0, ph_mma = 0;
     bool in_pending = false;   // a TMA load into VOP is in flight (meaningful in thread 0 only)
 
-    // bf16 inputs (thread 0): VOP takes, in turn, the k and q tiles of the first 64-channel half of an item
-    // ([64 tokens][128 B] each, read by the column pass), those of the second half, and finally V as product
-    // B's MN-major operand; each load completes one phase of bar_in.
+    // The k and q tiles of each 64-channel half of an item are staged by TMA (thread 0 issues; each load
+    // completes one phase of bar_in).  bf16: VOP takes, in turn, the k and q tiles of the first half
+    // ([64 tokens][128 B] each), those of the second half, and finally V as product B's MN-major operand.
+    // MXFP8: the code tiles ([64 tokens][64 B] each) go to the Aqk rows of [I; Aqk], free from product Y of
+    // the previous item until this item's A epilogue (VOP holds the V the column pass decodes).
+    uint8_t* const kq_stage = sm + (MX ? ps::IAQ + 8192 : ps::VOP);
+    constexpr uint32_t kKQ = MX ? 4096 : 8192;   // bytes of one half-tile
     auto issue_kq = [&](long long tok0, int hh, int hf) {
-        if constexpr (!MX) {
-            mbar_arrive_expect_tx(&bar_in, 2 * 8192);
-            tma_load_3d(sm + ps::VOP, &map_k, 64 * hf, hh, static_cast<int>(tok0), &bar_in);
-            tma_load_3d(sm + ps::VOP + 8192, &map_q, 64 * hf, hh, static_cast<int>(tok0), &bar_in);
-            in_pending = true;
-        }
+        mbar_arrive_expect_tx(&bar_in, 2 * kKQ);
+        tma_load_3d(kq_stage, &map_k, 64 * hf, hh, static_cast<int>(tok0), &bar_in);
+        tma_load_3d(kq_stage + kKQ, &map_q, 64 * hf, hh, static_cast<int>(tok0), &bar_in);
+        in_pending = true;
     };
     auto issue_v = [&](long long tok0, int hh) {
         if constexpr (!MX) {
@@ -218,9 +220,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             in_pending = true;
         }
     };
-    // bounded wait for the load into VOP issued last (all threads; bf16 inputs only)
+    // bounded wait for the staging load issued last (all threads)
     auto wait_in = [&]() -> bool {
-        if constexpr (MX) return true;
         const bool ok = mbar_wait(&bar_in, ph_in, status);
         ph_in ^= 1;
         if (t == 0) in_pending = false;
@@ -247,9 +248,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     int2 loc = entry(item);
     int h = static_cast<int>(item % H);
     bool valid = loc.y > 0;
-    if (valid && !MX) {
+    if (valid) {
         if (t == 0) issue_kq(loc.x, h, 0);
-        load_la_half(loc, h, 0);
+        if (!MX) load_la_half(loc, h, 0);
     }
 
     while (valid) {
@@ -291,13 +292,11 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             for (int j = 0; j < 8; ++j) {
                 const int r = 8 * w + j;
                 kb8[j] = qb8[j] = vb8[j] = 0u;
-                if constexpr (MX) {   // MXFP8: log_alpha and the codes of this half with plain loads
+                if constexpr (MX) {   // MXFP8: log_alpha and the v codes of this half with plain loads
                     p[j] = make_float2(0.f, 0.f);
                     if (r < n) {
                         const size_t rr = row0 + static_cast<size_t>(r) * H;
                         p[j] = ld_once_f2(lag + rr * kDK + c0);
-                        kb8[j] = ld_once_u16(kg + rr * kDK + c0);
-                        qb8[j] = ld_once_u16(qg + rr * kDK + c0);
                         if (c0 < DV) vb8[j] = ld_once_u16(vg + rr * DV + c0);
                     }
                 } else {              // bf16: log_alpha loaded one half ahead; k, q are the TMA tiles in VOP
@@ -374,8 +373,11 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 if constexpr (MX) {   // code x shared scale of the 32-channel block holding c0
                     const float* scf = reinterpret_cast<const float*>(sm + ps::SCF) + (c0 >> 5);
                     const float2 un = f2(kE4M3Unscale);
-                    kf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(kb8[j]), un), f2(scf[4 * (64 + r)]));
-                    qf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(qb8[j]), un), f2(scf[4 * r]));
+                    // rows past n hold other tokens' (finite) codes, which nothing below lets through
+                    const uint32_t kc = *reinterpret_cast<const uint16_t*>(kq_stage + r * 64 + (c0 & 63));
+                    const uint32_t qc = *reinterpret_cast<const uint16_t*>(kq_stage + kKQ + r * 64 + (c0 & 63));
+                    kf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(kc), un), f2(scf[4 * (64 + r)]));
+                    qf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(qc), un), f2(scf[4 * r]));
                     if (c0 < DV) {   // V as product B's MN-major operand
                         const float2 vf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(vb8[j]), un), f2(scf[4 * (128 + r)]));
                         st_b32(sm + ps::VOP + (c0 >> 6) * 8192 + (r >> 3) * 1024 + (r & 7) * 128 +
@@ -517,6 +519,12 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         }
                     }
                 }
+            }
+            if (MX && is_q && sub == 0) {   // the Aqk row's chunks past its tile's key columns held staged codes:
+                                            // zero them (bf16 inputs keep them zero from the start)
+                for (int sc = 2 * ((r >> 4) + 1); sc < 8; ++sc)
+                    *reinterpret_cast<uint4*>(sm + ps::IAQ + (64 + r) * 128 + ((sc ^ (r & 7)) << 4)) =
+                        make_uint4(0u, 0u, 0u, 0u);
             }
         }
         tc_fence_before();
@@ -701,6 +709,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
         ph_mma ^= 1;
         tc_fence_after();
+        // MXFP8: product Y has read the Aqk rows, which now take the next item's first code tiles
+        if (MX && nvalid && t == 0) issue_kq(nloc.x, nh, 0);
         {   // [X; Y] diag(beta) as product B's A operand (K = 64 tokens): lane quarter qw, 32-column group cg
             const int qw = w & 3, cg = w >> 2;
             const int m = 32 * qw + lane;
@@ -721,7 +731,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tc_fence_before();
         fence_proxy_async_smem();
         {   // V of this item has landed (bf16 inputs: its TMA tile)
-            const bool ok = wait_in();
+            const bool ok = MX || wait_in();
             if (__syncthreads_or(!ok)) break;
         }
 
@@ -1217,11 +1227,11 @@ cudaError_t launch_prep(const ChunkArgs& a, long long items, cudaStream_t s) {
     CUtensorMap mq, mk, mv, ml;
     const CUtensorMapDataType dt = MX ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int es = MX ? 1 : 2;
-    // q, k (and MXFP8 v codes) are read with plain loads: their maps only prefetch boxes into L2 (bf16: 64-column
-    // boxes; MXFP8: the whole row of codes).  bf16 v is loaded as product B's operand: 64-column x 64-token boxes
-    // with the 128-byte swizzle, the MN-major layout of the tensor-core descriptor.
-    if (!make_map(&mq, a.q, dt, es, kDK, a.H, a.total_tokens, MX ? kDK : 64) ||
-        !make_map(&mk, a.k, dt, es, kDK, a.H, a.total_tokens, MX ? kDK : 64) ||
+    // q, k: 64-channel half-tiles staged by TMA for the column pass (MXFP8 v codes are read with plain loads).
+    // bf16 v is loaded as product B's operand: 64-column x 64-token boxes with the 128-byte swizzle, the
+    // MN-major layout of the tensor-core descriptor.  log_alpha is read with plain loads (its map is unused).
+    if (!make_map(&mq, a.q, dt, es, kDK, a.H, a.total_tokens, 64) ||
+        !make_map(&mk, a.k, dt, es, kDK, a.H, a.total_tokens, 64) ||
         !make_map(&mv, a.v, dt, es, DV, a.H, a.total_tokens, MX ? DV : 64,
                   MX ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&ml, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, a.H, a.total_tokens, 32))
