@@ -750,13 +750,7 @@ def run_ours(args):
     seg_cu = synth.cu_from_lengths([nseg] * 64, dev)
     starts = torch.empty_like(Z)
     ends = torch.empty(64, H, D, D, device=dev)
-    kda.kda_segment_compose(M, Z, seg_cu, None, starts, ends)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    kda.kda_segment_compose(M, Z, seg_cu, None, starts, ends)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    comp_ms = e0.elapsed_time(e1)
+    comp_ms = timed_calls(lambda: kda.kda_segment_compose(M, Z, seg_cu, None, starts, ends), 5, 3, stream)
     comp_bytes = 64 * nseg * H * 3 * D * D * 4
     compose = {"workload": "64 sequences x 8 segments x H=32, dk=dv=128 fp32", "ms": round(comp_ms, 4),
                "achieved_gbs": round(comp_bytes / (comp_ms / 1e3) / 1e9, 1)}

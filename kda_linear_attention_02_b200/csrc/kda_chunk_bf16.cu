@@ -250,7 +250,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     bool valid = loc.y > 0;
     if (valid) {
         if (t == 0) issue_kq(loc.x, h, 0);
-        if (!MX) load_la_half(loc, h, 0);
+        load_la_half(loc, h, 0);
     }
 
     while (valid) {
@@ -282,7 +282,6 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // ---------------- column pass, one 64-channel half at a time: thread = (channel pair, the 8 tokens
         // of its warp); each half ends with its share of product A (K = 64 channels)
         bool fail = false;
-        const size_t row0 = static_cast<size_t>(loc.x) * H + h;   // (token, head) row of the chunk's first token
         for (int hf = 0; hf < 2; ++hf) {
             const int c0 = 64 * hf + 2 * lane, tq = w >> 1;
             float2 p[8];
@@ -292,18 +291,13 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             for (int j = 0; j < 8; ++j) {
                 const int r = 8 * w + j;
                 kb8[j] = qb8[j] = vb8[j] = 0u;
-                if constexpr (MX) {   // MXFP8: log_alpha and the v codes of this half with plain loads
-                    p[j] = make_float2(0.f, 0.f);
-                    if (r < n) {
-                        const size_t rr = row0 + static_cast<size_t>(r) * H;
-                        p[j] = ld_once_f2(lag + rr * kDK + c0);
-                        if (c0 < DV) vb8[j] = ld_once_u16(vg + rr * DV + c0);
-                    }
-                } else {              // bf16: log_alpha loaded one half ahead; k, q are the TMA tiles in VOP
-                    p[j] = nla[j];
+                p[j] = nla[j];   // log_alpha, loaded one half ahead (k, q: the staged TMA tiles)
+                if constexpr (MX) {   // MXFP8 v codes of this half with plain loads
+                    const size_t rr = (static_cast<size_t>(loc.x) + r) * H + h;   // (token, head) row
+                    if (r < n && c0 < DV) vb8[j] = ld_once_u16(vg + rr * DV + c0);
                 }
             }
-            if (!MX && hf == 0) load_la_half(loc, h, 1);   // lands while this half's operands are made
+            if (hf == 0) load_la_half(loc, h, 1);   // lands while this half's operands are made
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 if (8 * w + j < n) acc = __fadd2_rn(acc, make_float2(floor_log_decay(p[j].x), floor_log_decay(p[j].y)));
@@ -756,8 +750,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         ph_mma ^= 1;
         tc_fence_after();
         // product B has read VOP
-        if (!MX && nvalid) {   // VOP is free again: the next item's first k, q tiles; and its first log_alpha half
-            if (t == 0) issue_kq(nloc.x, nh, 0);
+        if (nvalid) {   // bf16: VOP is free again for the next item's first k, q tiles; and its first log_alpha half
+            if (!MX && t == 0) issue_kq(nloc.x, nh, 0);
             load_la_half(nloc, nh, 0);
         }
 

@@ -193,6 +193,28 @@ compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, cons
     uint32_t ph = 0;
     for (int s = s0; s < s1; ++s) {
         const size_t bs = static_cast<size_t>(s) * H + h;
+        {   // the accumulator starts as Z_s (TMEM stores from the rows' loads): lane quarter w & 3 holds rows
+            // 32 (w & 3) .., warp w >> 2 a half of the columns
+            const int qw = w & 3, i = 32 * qw + lane, jh = (w >> 2) * (DV / 2);
+            const float* zr = Z + (bs * DK + i) * DV + jh;
+            if (s + 1 < s1) {   // the next segment's rows of Z into L2 meanwhile
+#pragma unroll
+                for (int l = 0; l < DV / 2; l += 32) prefetch_l2(Z + ((bs + H) * DK + i) * DV + jh + l);
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int jb = 0; jb < DV / 2; jb += 16) {
+                float z[16];
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(zr + jb + e);
+                    z[e] = v4.x; z[e + 1] = v4.y; z[e + 2] = v4.z; z[e + 3] = v4.w;
+                }
+                tmem_st16(tm + (static_cast<uint32_t>(32 * qw) << 16) + jh + jb, z);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+        }
         {   // M_s as three K-major A operand pieces: thread = (row i, 64-column half)
             const int i = t >> 1, m0 = (t & 1) * 64;
             const float* src = M + (bs * DK + i) * DK + m0;
@@ -222,7 +244,7 @@ compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, cons
         }
         fence_proxy_async_smem();
         __syncthreads();
-        // D = sum over the six piece pairs (a, b) of A_a X_b  (M = 128, N = DV, K = 128)
+        // D = Z_s + sum over the six piece pairs (a, b) of A_a X_b  (M = 128, N = DV, K = 128)
         if (t == 0) {
             tc_fence_after();
             const uint32_t a0 = smem_u32(sm + C::A0), b0 = smem_u32(sm + C::B0);
@@ -233,16 +255,15 @@ compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, cons
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     umma_f16(tm, sdesc_k_sw128(a0 + pa[p] * C::A_PIECE + (ks >> 2) * 16384 + (ks & 3) * 32),
-                             sdesc_mn_sw128(b0 + pb[p] * C::B_PIECE + ks * 2048, C::LBO), idesc, p > 0 || ks > 0);
+                             sdesc_mn_sw128(b0 + pb[p] * C::B_PIECE + ks * 2048, C::LBO), idesc, 1u);
             umma_commit(&bar);
         }
         const bool ok = mbar_wait(&bar, ph, status);
         ph ^= 1;
         if (__syncthreads_or(!ok)) break;
         tc_fence_after();
-        {   // X_{s+1} = D + Z_s: lane quarter w & 3 holds rows 32 (w & 3) .., warp w >> 2 a half of the columns
+        {   // X_{s+1} = D: lane quarter w & 3 holds rows 32 (w & 3) .., warp w >> 2 a half of the columns
             const int qw = w & 3, i = 32 * qw + lane, jh = (w >> 2) * (DV / 2);
-            const float* zr = Z + (bs * DK + i) * DV;
             float* dst = s + 1 < s1 ? starts + (((bs + H) * DK) + i) * DV : (ends ? ends + (sh0 * DK + i) * DV : nullptr);
 #pragma unroll
             for (int jb = 0; jb < DV / 2; jb += 16) {
@@ -250,11 +271,8 @@ compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, cons
                 tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + jh + jb, d);
                 tmem_wait_ld_regs<16>(d);
 #pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    const float4 z = *reinterpret_cast<const float4*>(zr + jh + jb + e);
-                    d[e] += z.x; d[e + 1] += z.y; d[e + 2] += z.z; d[e + 3] += z.w;
+                for (int e = 0; e < 16; e += 4)
                     if (dst) *reinterpret_cast<float4*>(dst + jh + jb + e) = make_float4(d[e], d[e + 1], d[e + 2], d[e + 3]);
-                }
                 if (s + 1 < s1) {   // the next product's B operand
                     float x8[8];
 #pragma unroll
