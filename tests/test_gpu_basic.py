@@ -31,6 +31,22 @@ def test_selftest_umma_matches_matmul(n, mn):
     np.testing.assert_allclose(d.cpu().numpy(), ref.numpy(), rtol=1e-4, atol=1e-4)
 
 
+
+@pytest.mark.parametrize("n,k,mn", [(160, 64, False), (64, 64, False), (128, 128, True)])
+def test_selftest_mma_rate_is_plausible(n, k, mn):
+    # one CTA per SM times the product shape; the rate must lie between a small fraction and about the
+    # hardware's dense bf16 rate (8192 FLOP per cycle per SM), and products one at a time never beat
+    # products back to back
+    cyc = kda.kda_selftest_mma_rate(n, k, b_mn_major=mn, reps=64)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    c = cyc.cpu()
+    assert bool((c > 0).all()), "a bounded wait ran out"
+    flop = 2.0 * 128 * n * k
+    rate = flop / c[:, 0]
+    assert float(rate.max()) <= 8192 * 1.05 and float(rate.min()) >= 200
+    assert bool((c[:, 1] >= 0.9 * c[:, 0]).all())
+
 def test_bounded_wait_times_out_cleanly():
     st = kda.kda_selftest_wait_timeout(2000)
     assert kda.kda_status_string(st) == "KDA_ERR_TIMEOUT"
