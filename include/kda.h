@@ -163,7 +163,7 @@ KDA_API kda_status_t kda_chunk_fwd_mxfp8(const uint8_t* q, const uint8_t* q_scal
  * holds it until the process exits.  The chunks are processed in windows sized to that array.
  * A batch whose minimum scratch (kda_chunk_fwd_min_workspace_bytes: chunk index, the carried state
  * of every (sequence, head), one chunk of packets) exceeds it is refused with KDA_ERR_WORKSPACE;
- * at dk = dv = 128 that allows up to 491 (sequence, head) pairs, e.g. 15 sequences of 32 heads.
+ * at dk = dv = 128 and H = 32 that allows up to 493 (sequence, head) pairs, e.g. 15 sequences of 32 heads.
  * The first call on each device looks the array's device address up (with that device current)
  * and keeps it; make that first call before any stream capture.  All calls share the one array and
  * it keeps the last call's contents (nothing in it needs to start at zero): calls that may overlap

@@ -3,13 +3,12 @@
 // The chunk algebra (per chunk of C = 64 tokens, positions r; lambda = max(log_alpha, ln 0.0067),
 // g = chunk-local inclusive cumsum of lambda, gamma = exp(g)):
 //   A[r,s]   = beta_r sum_c k_rc k_sc exp(g_rc - g_sc)   (s < r),     Aqk[r,s] = sum_c q_rc k_sc exp(..)  (s <= r)
-//   X = (I + A)^-1 (blocked forward substitution over 16 x 16 tiles),  Y = Aqk X
+//   X = (I + A)^-1 (blocked forward substitution over 16 x 16 tiles)
 //   W = X diag(beta) (K * gamma),  U = X diag(beta) V
-//   P = Q * gamma - Y diag(beta) (K * gamma)  (= Q gamma - Aqk W),   O_intra = Y diag(beta) V  (= Aqk U)
 // and across chunks, with the fp32 state S:
-//   U' = U - W S,   O = P S + O_intra,   S <- Diag(gamma_C) S + (K * exp(g_C - g))^T U'.
-// Folding Aqk into P and O_intra takes the output off the chunk-to-chunk critical path: the
-// inter-chunk step is two dependent products ([-W; P] S, then Kdec^T U').
+//   U' = U - W S,   O = (Q * gamma) S + Aqk U',   S <- Diag(gamma_C) S + (K * exp(g_C - g))^T U'.
+// The inter-chunk step has two dependent products ([-W; Q gamma] S, then Kdec^T U'); the output's
+// Aqk U' is a third product beside Kdec^T U', off the chunk-to-chunk critical path.
 //
 // Decay floor (orkas.ai "Kimi K3 architecture" post, section "GPU 코드 경로 하나를 없앤 하한"): with
 // lambda >= ln 0.0067 the cumulative log-decay of a 16-token tile lies in [-80.09, 0], so with the
@@ -25,15 +24,14 @@
 // Kernels:
 //  prep_bf16_kernel   persistent, one (chunk, head) item at a time per CTA: TMA tensor loads of the
 //                     raw tiles (prefetched one item ahead), SIMT exponentials and operand
-//                     construction, tcgen05 products for A/Aqk (4 anchored variants), for
-//                     [X; Y] = [I; Aqk] X and for [X; Y] (-beta K gamma | beta V) onto an
-//                     accumulator preloaded with [0; Q gamma] (so that it yields [-W; P]), X by
-//                     forward substitution of the four 16 x 16 diagonal blocks and two merge levels
-//                     on warp-level tf32 MMAs, and a bulk TMA store of the MMA-ready packet.
+//                     construction, tcgen05 products for A/Aqk (4 anchored variants) and for
+//                     X diag(beta) (-K gamma | V) (which yields -W and U), X by forward substitution
+//                     of the four 16 x 16 diagonal blocks and two merge levels on warp-level tf32
+//                     MMAs, and bulk TMA stores of the MMA-ready packet.
 //  state_bf16_kernel  one CTA per (sequence, head, dv-slice), warp-specialised: a producer warp
 //                     streams packets through a shared-memory ring with bulk TMA, one thread issues
-//                     the tcgen05 products per chunk (copies of U and O_intra into a double-buffered
-//                     accumulator, then [-W; P] S onto them, then Kdec^T U'), 8 or 16 epilogue warps
+//                     the tcgen05 products per chunk ([I; 0] U into a double-buffered accumulator,
+//                     [-W; Q gamma] S onto it, then Kdec^T U' and Aqk U'), 8 or 16 epilogue warps
 //                     hold the fp32 state in registers and feed bf16 copies of S and U' back as the
 //                     next operands.
 #include <cudaTypedefs.h>
@@ -60,10 +58,6 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
     __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
     return __bfloat1622float2(h);
 }
-__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
-    const float2 a = bf2_to_f2(u.x), b = bf2_to_f2(u.y), c = bf2_to_f2(u.z), d = bf2_to_f2(u.w);
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
-}
 __device__ __forceinline__ uint32_t pack2(float2 f) { return pack_bf16x2(f.x, f.y); }
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 // 2^x by the ex2.approx instruction; e^x is taken as 2^(x log2 e) with the scaling done two lanes at a time
@@ -83,13 +77,17 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 // shared-memory stage so that it moves with plain bulk copies.
 template <int DV>
 struct Pk {
-    static constexpr uint32_t AW = 0;                 // [-W; P]: 128 x 128 bf16, K-major, 128B swizzle, 2 K atoms
-    static constexpr uint32_t KD = 32768;             // Kdec^T:  128 x 64 bf16, K-major, 128B swizzle
-    // [U; O_intra] per 64-column atom: [DV/64][128 rows: U rows 0..63, O_intra rows 64..127][128 B],
-    // 16-byte chunks ^ (row % 8) -- the K-major 128B-swizzle A operand that loads them into the state
-    // pass's accumulator, and the layout of the O tensor store
-    static constexpr uint32_t UO = 49152;
-    static constexpr uint32_t G = UO + DV * 256;      // gamma_C: [128] fp32
+    // [-W; Q gamma]: 128 x 128 bf16, K-major, 128B swizzle, 2 K atoms of [128 rows][128 B] (16-byte
+    // chunks ^ (row % 8)): rows 0..63 -W, rows 64..127 Q gamma
+    static constexpr uint32_t AW = 0;
+    static constexpr uint32_t KD = 32768;             // Kdec^T: 128 x 64 bf16, K-major, 128B swizzle
+    // Aqk (inclusive lower, zero above): 64 x 64 bf16, K-major, 128B swizzle; it follows Kdec^T, so that the
+    // 128-row operand starting 64 rows into Kdec^T has Aqk as its rows 64..127
+    static constexpr uint32_t AQ = 49152;
+    // U per 64-column atom: [DV/64][64 tokens][128 B], 16-byte chunks ^ (token % 8) -- the MN-major
+    // 128B-swizzle B operand of the state pass's copy product, and the layout of the O tensor store
+    static constexpr uint32_t U = 57344;
+    static constexpr uint32_t G = U + DV * 128;       // gamma_C: [128] fp32
     static constexpr uint32_t BYTES = ((G + 512 + 1023) / 1024) * 1024;
 };
 
@@ -101,19 +99,17 @@ struct Pk {
 //         the key side (4 anchored variants stacked into 160 rows, 160 x 64 bf16) at +16384, K-major with
 //         the 128B swizzle (the operands of one K half of product A);
 //         solve: A (fp32, pitch LDM) at +0 and X (fp32, pitch LDX) at +17408;
-//         then [X; Y] diag(beta) (bf16, product B's A operand) at +0;
-//         epilogue: the packet's [-W; P] (two 64-column atoms) at +0 .. +32768
-//   QG    Q gamma [64 tokens][128 ch] bf16 (the accumulator preload), then X^T (product Y's B operand),
-//         then atom 0 of the packet's [U; O_intra]
-//   KG    -(K gamma)^T [128 ch][64 tokens] bf16, K-major (product B's B operand, K part), then atom 1 of
-//         [U; O_intra] (QG and KG are adjacent, so [U; O_intra] leaves in one bulk copy)
+//         then [X; X] diag(beta) (bf16, product B's A operand: rows 64..127 repeat rows 0..63) at +0;
+//         epilogue: the packet's -W (two 64-column atoms of 64 rows) at +0, U at +16384
+//   QG    Q gamma in the packet's layout, [2 atoms][64 tokens][128 B] bf16 (rows 64..127 of [-W; Q gamma])
+//   KG    -(K gamma)^T [128 ch][64 tokens] bf16, K-major (product B's B operand, K part)
 //   VOP   V [DV/64][64 tokens][128 B] bf16, MN-major with the 128B swizzle (product B's B operand, V
 //         part): a TMA tile for bf16 inputs, written by the column pass for MXFP8 inputs
-//   IAQ   [I; Aqk] 128 x 64 bf16 (product Y's A operand)
+//   IAQ   MXFP8 inputs: the staged q and k code half-tiles at +0; Aqk (64 x 64 bf16, the packet's layout) at +8192
 //   MISC  beta[64]; then the tile half-totals [8][64] fp32 (column pass) or the merge scratch (solve)
 //   SCF   MXFP8 inputs only: the shared scales as fp32, [q, k, v][64 tokens][4 blocks]
-// TMEM (256 columns): product A at [0, 160); then the preload [0; Q gamma] at [0, 128); product Y at
-// [128, 192); product B: the K part at [0, 128) onto the preload, the V part at [128, 128 + DV).
+// TMEM (256 columns): product A at [0, 160); then product B: the K part at [0, 128), the V part at
+// [128, 128 + DV).
 namespace ps {
 constexpr uint32_t OPB = 0;
 constexpr uint32_t BVAR = 16384;                 // key side, inside OPB
@@ -178,18 +174,10 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tmem_alloc(&tmem_slot, 256);   // two CTAs per SM: half of the SM's TMEM each
         tmem_relinquish();
     }
-    // identity rows 0..63 of [I; Aqk]; rows 64..127 start at zero and every item rewrites only the columns of
-    // its row tile's variant (the Aqk entries past them are always zero)
-    for (int e = t; e < 128 * 8; e += NT) {
-        const int r = e >> 3, sc = e & 7;
-        uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        if ((r >> 3) == sc) {
-            const uint32_t one = 0x3F80u << (16 * (r & 1));   // bf16 1.0 in the low or high half
-            const int word = (r & 7) >> 1;
-            if (word == 0) z.x = one; else if (word == 1) z.y = one; else if (word == 2) z.z = one; else z.w = one;
-        }
-        *reinterpret_cast<uint4*>(sm + ps::IAQ + r * 128 + ((sc ^ (r & 7)) << 4)) = z;
-    }
+    // Aqk starts at zero: every item rewrites only the columns of its row tile's variant (the entries past
+    // them are always zero)
+    for (int e = t; e < 64 * 8; e += NT)
+        *reinterpret_cast<uint4*>(sm + ps::IAQ + 8192 + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -201,9 +189,9 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // The k and q tiles of each 64-channel half of an item are staged by TMA (thread 0 issues; each load
     // completes one phase of bar_in).  bf16: VOP takes, in turn, the k and q tiles of the first half
     // ([64 tokens][128 B] each), those of the second half, and finally V as product B's MN-major operand.
-    // MXFP8: the code tiles ([64 tokens][64 B] each) go to the Aqk rows of [I; Aqk], free from product Y of
-    // the previous item until this item's A epilogue (VOP holds the V the column pass decodes).
-    uint8_t* const kq_stage = sm + (MX ? ps::IAQ + 8192 : ps::VOP);
+    // MXFP8: the code tiles ([64 tokens][64 B] each) go to IAQ + 0, the next item's first half as soon as
+    // this item's second half has been read (VOP holds the V the column pass decodes).
+    uint8_t* const kq_stage = sm + (MX ? ps::IAQ : ps::VOP);
     constexpr uint32_t kKQ = MX ? 4096 : 8192;   // bytes of one half-tile
     auto issue_kq = [&](long long tok0, int hh, int hf) {
         mbar_arrive_expect_tx(&bar_in, 2 * kKQ);
@@ -361,7 +349,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             for (int j = 0; j < 8; ++j) {
                 const int r = 8 * w + j;
                 // rows past the sequence end (n <= r) hold zero inputs: their log-decay and beta are zero, so
-                // they add nothing to A, W, U, Kdec^T U' or the state, and their own P / O_intra rows are never
+                // they add nothing to A, W, U, Kdec^T U' or the state, and their own Q gamma / Aqk rows are never
                 // stored as outputs
                 float2 kf, qf;
                 if constexpr (MX) {   // code x shared scale of the 32-channel block holding c0
@@ -399,8 +387,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     if (i > tq)
                         st_b32(sm + ps::BVAR + (8 * i * (i + 1) + r) * 128 + sw,
                                pack2(__fmul2_rn(kF, make_float2(dvx[i], dvy[i]))));
-                // Q * gamma for the accumulator preload (P = Q gamma - ...)
-                st_b32(sm + ps::QG + r * 256 + ((((c0 >> 3) ^ (r & 7))) << 4) + kb, pack2(__fmul2_rn(qf, G)));
+                // Q * gamma, rows 64..127 of the packet's [-W; Q gamma] (atom hf)
+                st_b32(sm + ps::QG + hf * 8192 + r * 128 + sw, pack2(__fmul2_rn(qf, G)));
                 const float2 tk2 = __fmul2_rn(make_float2(-kf.x, -kf.y), G);   // -K gamma
                 const float2 td2 = __fmul2_rn(kF, ec2);                        // Kdec = K e^{g_C - g}
                 if (j & 1) {
@@ -442,9 +430,11 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 for (int ks = 0; ks < 4; ++ks)
                     umma_f16(tm, sdesc_k_sw128(ra + ks * 32), sdesc_k_sw128(bv + ks * 32), idesc, hf > 0 || ks > 0);
                 umma_commit(&bar_mma);
-                // VOP has been read: the second half's k and q tiles, then V (product B's operand)
+                // VOP has been read: the second half's k and q tiles, then V (product B's operand); MXFP8: the
+                // second half's code tiles have been read, so the next item's first ones follow
                 if (hf == 0) issue_kq(loc.x, h, 1);
-                else issue_v(loc.x, h);
+                else if (!MX) issue_v(loc.x, h);
+                else if (nvalid) issue_kq(nloc.x, nh, 0);
             }
         }
         if (fail) break;
@@ -455,7 +445,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         ph_mma ^= 1;
         tc_fence_after();
 
-        // ---------------- TMEM -> fp32 A (strict lower, beta rows) and bf16 Aqk (inclusive lower) into [I; Aqk].
+        // ---------------- TMEM -> fp32 A (strict lower, beta rows) and bf16 Aqk (inclusive lower, the packet's layout).
         // Lane quarter qw holds the rows of tiles t0 = 2 (qw & 1) and t0 + 1 (K rows for qw < 2, Q rows
         // otherwise).  Their variant columns form 2 t0 + 3 chunks of 16 (t0 + 1 of tile t0, t0 + 2 of tile
         // t0 + 1), spread over the lane quarter's two warps, at most four per warp, in two rounds of two.
@@ -514,43 +504,18 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
             }
-            if (MX && is_q && sub == 0) {   // the Aqk row's chunks past its tile's key columns held staged codes:
-                                            // zero them (bf16 inputs keep them zero from the start)
-                for (int sc = 2 * ((r >> 4) + 1); sc < 8; ++sc)
-                    *reinterpret_cast<uint4*>(sm + ps::IAQ + (64 + r) * 128 + ((sc ^ (r & 7)) << 4)) =
-                        make_uint4(0u, 0u, 0u, 0u);
-            }
         }
         tc_fence_before();
+        fence_proxy_async_smem();   // Aqk leaves by a bulk copy
         __syncthreads();
+        // Aqk and Q gamma are final: warp 4 sends them to the packet (waited for before the next column pass)
+        if (t == 128) {
+            bulk_s2g(pkt + P::AQ, sm + ps::IAQ + 8192, 8192);
+            bulk_s2g(pkt + P::AW + 8192, sm + ps::QG, 8192);
+            bulk_s2g(pkt + P::AW + 16384 + 8192, sm + ps::QG + 8192, 8192);
+            bulk_commit();
+        }
 
-        // Meanwhile warps 4..7, idle in the first two solve levels, start product B's K-part accumulator
-        // (TMEM columns 0..127, free since the A epilogue) as [0; Q gamma], so that it ends as [-W; P] with
-        // P = Q gamma - Aqk W.  Warp w writes the 128 columns of lane quarter w & 3, 64 per level, and waits
-        // for its stores before the third level.
-        auto preload_qgamma = [&](int c_lo, int c_hi) {
-            tc_fence_after();   // after the A epilogue's TMEM loads of these columns (barrier in between)
-            const int qw = w & 3;
-            const uint32_t base = tm + (static_cast<uint32_t>(32 * qw) << 16);
-            const int r = 32 * qw + lane - 64;   // token row of the Q part (lane quarters 2 and 3)
-#pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
-                if (c16 < c_lo || c16 >= c_hi) continue;
-                float x[16];
-                if (qw >= 2) {
-                    const int ch = 2 * c16;   // first 8-channel chunk of the 16 columns
-                    float a8[8], b8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QG + r * 256 + ((ch ^ (r & 7)) << 4)), a8);
-                    unpack8(*reinterpret_cast<const uint4*>(sm + ps::QG + r * 256 + (((ch + 1) ^ (r & 7)) << 4)), b8);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) { x[j] = a8[j]; x[8 + j] = b8[j]; }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) x[j] = 0.f;
-                }
-                tmem_st16(base + 16 * c16, x);
-            }
-        };
         // ---------------- X = (I + A)^-1 by blocked forward substitution over 16 x 16 tiles.
         // Level 0: each diagonal block by forward substitution, one warp per block, lane = column, the
         // column held in registers; a column of A comes as float4 broadcasts of a row of the transposed block.
@@ -590,7 +555,6 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 const int r = e >> 6, c = e & 63;
                 if ((c >> 4) > (r >> 4)) XF[r * LDX + c] = 0.f;
             }
-            preload_qgamma(0, 4);
         }
         __syncthreads();
         // Levels 1 and 2 merge two inverted diagonal blocks: X_10 = -X_11 (A_10 X_00).  The products are
@@ -630,10 +594,6 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             xo[fg * LDX + 1] = -e[1];
             xo[(fg + 8) * LDX] = -e[2];
             xo[(fg + 8) * LDX + 1] = -e[3];
-        } else {
-            preload_qgamma(4, 8);
-            tmem_wait_st();   // the accumulator preload has landed (published by the barriers before product B)
-            tc_fence_before();
         }
         __syncthreads();
         {   // level 2: 32 -> 64, row tile mt of 16 and column tile nt of 8
@@ -674,70 +634,34 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             xo[(fg + 8) * LDX + 1] = -e[3];
         }
         __syncthreads();
-        // X^T as the bf16 B operand of the Y product (row m = column m of X, K = 64 rows of X), over Q gamma
-        // (consumed by the preload)
+        // [X; X] diag(beta) as product B's A operand (K = 64 tokens, K-major): rows 64..127 repeat rows 0..63, so
+        // that the lanes of all four TMEM quarters hold -W and U rows for the epilogue
 #pragma unroll
         for (int e = t; e < 64 * 8; e += NT) {
             const int m = e >> 3, uc = e & 7;
             float v[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = XF[(8 * uc + j) * LDX + m];
-            *reinterpret_cast<uint4*>(sm + ps::QG + m * 128 + ((uc ^ (m & 7)) << 4)) = pack8(v);
+            for (int j = 0; j < 8; ++j) v[j] = XF[m * LDX + 8 * uc + j] * bet[8 * uc + j];
+            const uint4 pk8 = pack8(v);
+            const uint32_t off = static_cast<uint32_t>(m * 128 + ((uc ^ (m & 7)) << 4));
+            *reinterpret_cast<uint4*>(sm + ps::OPB + off) = pk8;
+            *reinterpret_cast<uint4*>(sm + ps::OPB + 8192 + off) = pk8;
         }
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---------------- phase Y: [X; Y] = [I; Aqk] X   (M = 128, N = 64, K = 64)
-        if (t == 0) {
-            tc_fence_after();
-            const uint32_t ia = smem_u32(sm + ps::IAQ), xt = smem_u32(sm + ps::QG);
-            const uint32_t idesc = idesc_bf16(128, 64);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tm + 128, sdesc_k_sw128(ia + ks * 32), sdesc_k_sw128(xt + ks * 32), idesc, ks > 0);
-            umma_commit(&bar_mma);
-        }
-        {
-            const bool ok = mbar_wait(&bar_mma, ph_mma, status);
-            if (__syncthreads_or(!ok)) break;
-        }
-        ph_mma ^= 1;
-        tc_fence_after();
-        // MXFP8: product Y has read the Aqk rows, which now take the next item's first code tiles
-        if (MX && nvalid && t == 0) issue_kq(nloc.x, nh, 0);
-        {   // [X; Y] diag(beta) as product B's A operand (K = 64 tokens): lane quarter qw, 32-column group cg
-            const int qw = w & 3, cg = w >> 2;
-            const int m = 32 * qw + lane;
-            float v[32];
-            tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 128 + 32 * cg, *reinterpret_cast<float(*)[16]>(v));
-            tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + 128 + 32 * cg + 16,
-                      *reinterpret_cast<float(*)[16]>(v + 16));
-            tmem_wait_ld_regs<32>(v);
-#pragma unroll
-            for (int hf = 0; hf < 4; ++hf) {
-                float o8[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) o8[j] = v[8 * hf + j] * bet[32 * cg + 8 * hf + j];
-                const int sc = 4 * cg + hf;
-                *reinterpret_cast<uint4*>(sm + ps::OPB + m * 128 + ((sc ^ (m & 7)) << 4)) = pack8(o8);
-            }
-        }
-        tc_fence_before();
         fence_proxy_async_smem();
         {   // V of this item has landed (bf16 inputs: its TMA tile)
             const bool ok = MX || wait_in();
             if (__syncthreads_or(!ok)) break;
         }
+        tc_fence_after();
 
-        // ---------------- phase B: D[m, n] = [X; Y] diag(beta) [m, :] . B[n, :]  (K = 64 tokens): the K part
-        // (N = 128, B = -(K gamma)^T) onto the preloaded [0; Q gamma], the V part (N = DV, B = V MN-major) from zero
+        // ---------------- phase B: D[m, n] = [X; X] diag(beta) [m, :] . B[n, :]  (K = 64 tokens): the K part
+        // (N = 128, B = -(K gamma)^T) gives -W, the V part (N = DV, B = V MN-major) gives U
         if (t == 0) {
-            tc_fence_after();
             const uint32_t xa = smem_u32(sm + ps::OPB), kb = smem_u32(sm + ps::KG), vb = smem_u32(sm + ps::VOP);
             const uint32_t idk = idesc_bf16(128, 128), idv = idesc_bf16(128, DV, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tm, sdesc_k_sw128(xa + ks * 32), sdesc_k_sw128(kb + ks * 32), idk, true);
+                umma_f16(tm, sdesc_k_sw128(xa + ks * 32), sdesc_k_sw128(kb + ks * 32), idk, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 umma_f16(tm + 128, sdesc_k_sw128(xa + ks * 32), sdesc_mn_sw128(vb + ks * 2048, 8192), idv, ks > 0);
@@ -755,40 +679,41 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             load_la_half(nloc, nh, 0);
         }
 
-        // ---------------- epilogue: rows 0..63 -> -W | U, rows 64..127 -> P | O_intra, straight from TMEM into
-        // the packet staging ([-W; P] over OPB, [U; O_intra] over QG and KG).  Each warp stages the 32 rows of
-        // its lane quarter (4 KB of each atom it covers) and sends them with its own bulk copies at once, so no
-        // CTA barrier precedes the packet store.
+        // ---------------- epilogue: -W (lane quarters 0, 1) and U (lane quarters 2, 3, the repeated rows), straight
+        // from TMEM into the packet staging (-W over OPB, U at OPB + 16384).  Each warp stages the 32 rows of its
+        // lane quarter in one 64-column atom (4 KB) and sends them with its own bulk copy at once, so no CTA
+        // barrier precedes the packet store.
         {
-            const int qw = w & 3, cg = w >> 2;   // cg 0: K part, cg 1: V part
-            const int m = 32 * qw + lane;
-            const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16) + 128 * cg;
-            uint8_t* dst0 = sm + (cg == 0 ? ps::OPB : ps::QG);
-            const int natoms = cg == 0 ? 2 : DV / 64;
+            const int qw = w & 3, cg = w >> 2;   // qw 0, 1: -W atom cg; qw 2, 3: U atom cg
+            const bool upart = qw >= 2;
+            const int m = (32 * qw + lane) & 63;   // token row
+            if (!upart || cg < DV / 64) {
+                const uint32_t col = upart ? 128 + 64 * cg : 64 * cg;
+                const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16) + col;
+                uint8_t* const stg = sm + ps::OPB + (upart ? 16384 : 0) + cg * 8192;
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                if (a >= natoms) break;
-                float vv[64];
+                for (int hq = 0; hq < 2; ++hq) {
+                    float vv[32];
+                    tmem_ld16(lane_base + 32 * hq, *reinterpret_cast<float(*)[16]>(vv));
+                    tmem_ld16(lane_base + 32 * hq + 16, *reinterpret_cast<float(*)[16]>(vv + 16));
+                    tmem_wait_ld_regs<32>(vv);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) tmem_ld16(lane_base + 64 * a + 16 * i, *reinterpret_cast<float(*)[16]>(vv + 16 * i));
-                tmem_wait_ld_regs<64>(vv);
-                uint8_t* dst = dst0 + a * 16384 + m * 128;
+                    for (int sub = 0; sub < 4; ++sub) {
+                        float o8[8];
 #pragma unroll
-                for (int sub = 0; sub < 8; ++sub) {
-                    float o8[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) o8[j] = vv[8 * sub + j];
-                    *reinterpret_cast<uint4*>(dst + ((sub ^ (m & 7)) << 4)) = pack8(o8);
+                        for (int j = 0; j < 8; ++j) o8[j] = vv[8 * sub + j];
+                        *reinterpret_cast<uint4*>(stg + m * 128 + (((4 * hq + sub) ^ (m & 7)) << 4)) = pack8(o8);
+                    }
                 }
-            }
-            tc_fence_before();   // this warp's TMEM loads precede the next item's products (barriers in between)
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                uint8_t* gdst = pkt + (cg == 0 ? P::AW : P::UO) + 32 * qw * 128;
-                for (int a = 0; a < natoms; ++a)
-                    bulk_s2g(gdst + a * 16384, dst0 + a * 16384 + 32 * qw * 128, 4096);
-                bulk_commit();   // waited for (read out) before the next column pass's first barrier
+                tc_fence_before();   // this warp's TMEM loads precede the next item's products (barriers in between)
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int r0 = 32 * (qw & 1);   // first token row of this warp
+                    uint8_t* gdst = pkt + (upart ? P::U + cg * 8192 : P::AW + cg * 16384) + r0 * 128;
+                    bulk_s2g(gdst, stg + r0 * 128, 4096);
+                    bulk_commit();   // waited for (read out) before the next column pass's first barrier
+                }
             }
         }
         item = nitem;
@@ -811,19 +736,24 @@ struct SCfg {
     static constexpr int NCW = DVS * 4 / NEW;              // state columns per epilogue warp (>= 16)
     static constexpr int NT = 32 * (NEW + 2);              // + producer warp + MMA warp
     static constexpr bool MN = DVS >= 64;                  // S and U' staged MN-major (row = channel / token)
-    static constexpr int NST = DVS == 128 ? 2 : 3;
-    static constexpr uint32_t UO_BYTES = DVS >= 64 ? DVS * 256 : 16384;   // whole 64-column atoms of [U; O_intra]
-    static constexpr uint32_t AW = 0, KD = 32768, UO = 49152, G = UO + UO_BYTES;
+    static constexpr int NST = DVS == 32 ? 3 : 2;
+    static constexpr int NCP = DVS >= 64 ? DVS : 64;       // columns of U copied into D1: whole 64-column atoms
+    static constexpr uint32_t U_BYTES = NCP * 128;
+    // stage: the packet's parts for this slice (Aqk right after Kdec^T, as in the packet)
+    static constexpr uint32_t AW = 0, KD = 32768, AQ = 49152, U = 57344, G = U + U_BYTES;
     static constexpr uint32_t STAGE = ((G + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SOP = NST * STAGE;      // S as B operand (N = DVS, K = 128)
     static constexpr uint32_t UOP = SOP + DVS * 256;  // U' as B operand (N = DVS, K = 64)
-    static constexpr uint32_t IDN = UOP + DVS * 128;  // 16 x 64 bf16 B operand, row n = 1 where k % 16 == n
-    static constexpr uint32_t BYTES = IDN + 2048;
-    // TMEM: D1 double-buffered at columns [0, DVS) and [2 DVS, 3 DVS), D2 at [DVS, 2 DVS)
+    static constexpr uint32_t IZ = UOP + DVS * 128;   // [I; 0]: 128 x 64 bf16 K-major A operand of the U copy
+    static constexpr uint32_t BYTES = IZ + 16384;
+    // TMEM: D1 double-buffered at columns [0, NCP) and [NCP + DVS, 2 NCP + DVS), D2 at [NCP, NCP + DVS);
+    // the slice's columns of D1 start at c_off = j0 % 64 when a slice is narrower than an atom
     static constexpr uint32_t S_LBO = 128 * 128;      // MN-major: 64 columns x 128 K rows per block
     static constexpr uint32_t U_LBO = 64 * 128;       // MN-major: 64 columns x 64 K rows per block
-    static constexpr uint32_t TMEM_COLS = 3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512);
-    static __host__ __device__ constexpr uint32_t d1col(int ci) { return (ci & 1) ? 2 * DVS : 0; }
+    static constexpr uint32_t TMEM_COLS = 2 * NCP + DVS <= 128 ? 128 : (2 * NCP + DVS <= 256 ? 256 : 512);
+    static __host__ __device__ constexpr uint32_t d1col(int ci) { return (ci & 1) ? NCP + DVS : 0; }
+    static_assert(BYTES + 1024 <= 232448, "one CTA per SM");
+    static_assert(IZ % 1024 == 0 && STAGE % 1024 == 0 && SOP % 1024 == 0, "128B-swizzle operands on 1024-byte atoms");
 };
 
 template <int DV, int DVS>
@@ -831,7 +761,6 @@ __global__ void __launch_bounds__(SCfg<DV, DVS>::NT, 1)
 state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict__ cu_seqlens,
                   const int32_t* __restrict__ cu_chunks, int n_seqs, int H, long long win_lo, long long win_hi,
                   const float* __restrict__ initial_state, __nv_bfloat16* __restrict__ o,
-                  const __grid_constant__ CUtensorMap map_o,
                   float* __restrict__ final_state, float* __restrict__ final_transition, int ckpt_stride,
                   float* __restrict__ checkpoints, const int32_t* __restrict__ ckpt_cu, float* __restrict__ carry,
                   int* status) {
@@ -840,7 +769,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
     constexpr int NST = C::NST, NCW = C::NCW, NEW = C::NEW, NSV = DV / DVS, CW = DV + kDK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    __shared__ __align__(8) uint64_t full[NST], empty[NST], d1_full, d2_full, s_ready, up_ready;
+    __shared__ __align__(8) uint64_t full[NST], empty[NST], d1_full, d2_full, o_full, s_ready, up_ready, o_done;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     grid_dependency_wait();   // the packets and the chunk index come from the launches before this one
@@ -867,19 +796,27 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         }
         mbar_init(&d1_full, 1);
         mbar_init(&d2_full, 1);
+        mbar_init(&o_full, 1);
         mbar_init(&s_ready, NEW);
         mbar_init(&up_ready, NEW / 2);   // only the warps that produce U' (TMEM lanes 0..63)
+        mbar_init(&o_done, NEW / 2);     // only the warps that read O (TMEM lanes 64..127)
         fence_barrier_init();
     }
     if (w == 0) {
         tmem_alloc(&tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
-    // B operand that copies 16 columns of an A operand into the accumulator: B[n][k] = (k % 16 == n)
-    for (int e = t; e < 16 * 64; e += C::NT) {
-        const int n = e >> 6, k = e & 63;
-        *reinterpret_cast<__nv_bfloat16*>(sm + C::IDN + sw128_offset(n, k, 16)) =
-            __float2bfloat16_rn((k & 15) == n ? 1.f : 0.f);
+    // [I; 0] (rows 0..63 the identity, rows 64..127 zero): [I; 0] U puts U into D1 rows 0..63 and zero into
+    // rows 64..127, exactly (bf16 values times 1)
+    for (int e = t; e < 128 * 8; e += C::NT) {
+        const int r = e >> 3, sc = e & 7;
+        uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        if (r < 64 && (r >> 3) == sc) {
+            const uint32_t one = 0x3F80u << (16 * (r & 1));   // bf16 1.0 in the low or high half
+            const int word = (r & 7) >> 1;
+            if (word == 0) z.x = one; else if (word == 1) z.y = one; else if (word == 2) z.z = one; else z.w = one;
+        }
+        *reinterpret_cast<uint4*>(sm + C::IZ + r * 128 + ((sc ^ (r & 7)) << 4)) = z;
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -896,11 +833,14 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 if (!mbar_wait(&empty[st], ((ci / NST) & 1) ^ 1, status)) break;
                 const uint8_t* pk = packets + static_cast<size_t>((lo + ci - win_lo) * H + h) * P::BYTES;
                 uint8_t* sb = sm + st * C::STAGE;
-                const uint32_t bytes = 32768 + 16384 + 512 + (trans ? 0u : C::UO_BYTES);
+                const uint32_t bytes = 32768 + 16384 + 512 + (trans ? 0u : 8192u + C::U_BYTES);
                 mbar_arrive_expect_tx(&full[st], bytes);
                 bulk_g2s(sb + C::AW, pk + P::AW, 32768, &full[st]);
                 bulk_g2s(sb + C::KD, pk + P::KD, 16384, &full[st]);
-                if (!trans) bulk_g2s(sb + C::UO, pk + P::UO + (j0 / 64) * 16384, C::UO_BYTES, &full[st]);
+                if (!trans) {
+                    bulk_g2s(sb + C::AQ, pk + P::AQ, 8192, &full[st]);
+                    bulk_g2s(sb + C::U, pk + P::U + (j0 / 64) * 8192, C::U_BYTES, &full[st]);
+                }
                 bulk_g2s(sb + C::G, pk + P::G, 512, &full[st]);
                 issued = ci + 1;
             }
@@ -912,20 +852,20 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, DVS, false, C::MN);
-            const uint32_t idesc16 = idesc_bf16(128, 16);
-            const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP), idn = smem_u32(sm + C::IDN);
-            // D1[ci] = [U; O_intra] of chunk ci: 16 columns per product against the copying B operand
-            // (exact: bf16 values times 1), so that product 1 adds [-W; P] S onto it in the accumulator
-            auto load_uo = [&](int ci) {
+            const uint32_t idcp = idesc_bf16(128, C::NCP, false, true);
+            const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP), iz = smem_u32(sm + C::IZ);
+            const uint32_t c_off = DVS >= 64 ? 0u : static_cast<uint32_t>(j0 & 63);
+            // D1[ci] = [I; 0] U of chunk ci (U MN-major, K = 64 tokens): U in rows 0..63, zero in rows 64..127,
+            // so that product 1 adds [-W; Q gamma] S onto it
+            auto load_u = [&](int ci) {
                 const uint32_t sb = smem_u32(sm + (ci % NST) * C::STAGE);
-                const int c_off = DVS >= 64 ? 0 : (j0 & 63);   // the slice's first column inside its atom
 #pragma unroll
-                for (int ks = 0; ks < DVS / 16; ++ks) {
-                    const int col = c_off + 16 * ks;
-                    const uint32_t kk = static_cast<uint32_t>((col & 63) >> 4) * 32;
-                    umma_f16(tm + C::d1col(ci) + 16 * ks, sdesc_k_sw128(sb + C::UO + (col >> 6) * 16384 + kk),
-                             sdesc_k_sw128(idn + kk), idesc16, false);
-                }
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tm + C::d1col(ci), sdesc_k_sw128(iz + ks * 32), sdesc_mn_sw128(sb + C::U + ks * 2048, 8192),
+                             idcp, ks > 0);
+            };
+            auto ubdesc = [&](int ks) -> uint64_t {   // U' as the B operand (K = 64 tokens)
+                return C::MN ? sdesc_mn_sw128(uop + ks * 2048, C::U_LBO) : sdesc_k_sw128(uop + ks * 32);
             };
             for (int ci = 0; ci < nch; ++ci) {
                 const int st = ci % NST;
@@ -933,14 +873,14 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
                 tc_fence_after();
                 const uint32_t sb = smem_u32(sm + st * C::STAGE);
-                if (ci == 0 && !trans) load_uo(0);
-                // D1 (+)= [-W; P] S   (M = 128, N = DVS, K = 128)
+                if (ci == 0 && !trans) load_u(0);
+                // D1 (+)= [-W; Q gamma] S   (M = 128, N = DVS, K = 128)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
                     const uint64_t bdesc = C::MN ? sdesc_mn_sw128(sop + ks * 2048, C::S_LBO)
                                                  : sdesc_k_sw128(sop + ka * (DVS * 128) + kb);
-                    umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc,
+                    umma_f16(tm + C::d1col(ci) + c_off, sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc,
                              !trans || ks > 0);
                 }
                 umma_commit(&d1_full);
@@ -948,19 +888,26 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 tc_fence_after();
                 // D2 = Kdec^T U'   (M = 128, N = DVS, K = 64)
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t bdesc = C::MN ? sdesc_mn_sw128(uop + ks * 2048, C::U_LBO)
-                                                 : sdesc_k_sw128(uop + ks * 32);
-                    umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), bdesc, idesc, ks > 0);
-                }
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tm + C::NCP, sdesc_k_sw128(sb + C::KD + ks * 32), ubdesc(ks), idesc, ks > 0);
                 umma_commit(&d2_full);
+                if (!trans) {
+                    // the O warps have read chunk ci - 1's O (its D1 buffer takes chunk ci + 1's U below)
+                    if (ci > 0 && !mbar_wait(&o_done, (ci - 1) & 1, status)) break;
+                    // D1 rows 64..127 += Aqk U' (O = Q gamma S + Aqk U'): the A operand starts 64 rows into Kdec^T,
+                    // so its rows 64..127 are Aqk; what it adds to rows 0..63 (U', already read) is never used
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_f16(tm + C::d1col(ci) + c_off, sdesc_k_sw128(sb + C::KD + 8192 + ks * 32), ubdesc(ks),
+                                 idesc, true);
+                    umma_commit(&o_full);
+                }
                 umma_commit(&empty[st]);
-                // the next chunk's [U; O_intra] into the other D1 buffer, read last by chunk ci - 1's
-                // epilogue (done: its warps arrived on s_ready for chunk ci)
+                // the next chunk's U into the other D1 buffer (chunk ci - 1's, whose O has been read)
                 if (!trans && ci + 1 < nch) {
                     if (!mbar_wait(&full[(ci + 1) % NST], ((ci + 1) / NST) & 1, status)) break;
                     tc_fence_after();
-                    load_uo(ci + 1);
+                    load_u(ci + 1);
                 }
             }
         }
@@ -1006,33 +953,30 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_ready);
-        // full chunks leave through a TMA tensor store of the O tile, written in place over O_intra
-        const bool o_issuer = (w == 2) && lane == 0;
+        const uint32_t c_off = DVS >= 64 ? 0u : static_cast<uint32_t>(j0 & 63);
         for (int ci = 0; ci < nch; ++ci) {
             const int st = ci % NST;
             uint8_t* sb = sm + st * C::STAGE;
             const int c = static_cast<int>(lo + ci - ch_lo);
             const long long rem = seq_len - static_cast<long long>(c) * 64;
             const int n = rem < 64 ? static_cast<int>(rem) : 64;
-            const bool full_tma = C::MN && !trans && n == 64;
             if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
-            if (!mbar_wait(&d1_full, ci & 1, status)) break;
-            tc_fence_after();
-            float vv[NCW];   // D1 row i, columns jw .. jw + NCW: all loads in flight, one wait
+            if (qw < 2) {   // U' = U - W S: D1 rows 0..63 (loaded with U before the product)
+                if (!mbar_wait(&d1_full, ci & 1, status)) break;
+                tc_fence_after();
+                float vv[NCW];   // D1 row i, columns jw .. jw + NCW: all loads in flight, one wait
 #pragma unroll
-            for (int cb = 0; cb < NCW; cb += 16)
-                tmem_ld16(lane_base + C::d1col(ci) + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
-            tmem_wait_ld_regs<NCW>(vv);
+                for (int cb = 0; cb < NCW; cb += 16)
+                    tmem_ld16(lane_base + C::d1col(ci) + c_off + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+                tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
-            for (int cb = 0; cb < NCW; cb += 16) {
-                const float* v = vv + cb;
+                for (int cb = 0; cb < NCW; cb += 16) {
 #pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    const int cc = (jw + cb) / 8 + sub;   // 8-column chunk within the slice
-                    if (i < 64) {   // U' = U - W S (D1 was loaded with U before the product)
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const int cc = (jw + cb) / 8 + sub;   // 8-column chunk within the slice
                         float u8[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) u8[e] = v[8 * sub + e];
+                        for (int e = 0; e < 8; ++e) u8[e] = vv[cb + 8 * sub + e];
                         if constexpr (C::MN) {
                             *reinterpret_cast<uint4*>(sm + C::UOP + sw128_mn_offset(8 * cc, i, C::U_LBO)) = pack8(u8);
                         } else {
@@ -1041,35 +985,12 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                                 *reinterpret_cast<__nv_bfloat16*>(sm + C::UOP + sw128_offset(8 * cc + e, i, DVS)) =
                                     __float2bfloat16_rn(u8[e]);
                         }
-                    } else if (!trans && i - 64 < n) {   // O = O_intra + P S (D1 was loaded with O_intra)
-                        const int r = i - 64;
-                        const int col = j0 + 8 * cc;   // first column of this 8-column chunk
-                        uint8_t* ot = sb + C::UO + ((col >> 6) - (j0 >> 6)) * 16384 + (64 + r) * 128 +
-                                      ((((col & 63) >> 3) ^ (r & 7)) << 4);
-                        float o8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) o8[e] = v[8 * sub + e];
-                        if (full_tma) *reinterpret_cast<uint4*>(ot) = pack8(o8);
-                        else *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + col) =
-                                 pack8(o8);
                     }
                 }
-            }
-            tc_fence_before();
-            if (qw < 2) {
+                tc_fence_before();
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&up_ready);
-            } else if (full_tma) {
-                fence_proxy_async_smem();
-                named_bar_sync(1, 32 * NEW / 2);   // every O warp has written its rows of the tile
-                if (o_issuer) {
-#pragma unroll
-                    for (int b = 0; b < DVS / 64; ++b)
-                        tma_store_3d(&map_o, j0 + 64 * b, h, static_cast<int>(seq_tok0 + c * 64),
-                                     sb + C::UO + b * 16384 + 8192);
-                    bulk_commit();
-                }
             }
             if (!mbar_wait(&d2_full, ci & 1, status)) break;
             tc_fence_after();
@@ -1078,7 +999,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 float vv[NCW];
 #pragma unroll
                 for (int cb = 0; cb < NCW; cb += 16)
-                    tmem_ld16(lane_base + DVS + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+                    tmem_ld16(lane_base + C::NCP + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
                 tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
                 for (int e = 0; e < NCW; e += 2) {
@@ -1086,14 +1007,36 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                     S[e] = a.x; S[e + 1] = a.y;
                 }
             }
-            if (o_issuer) bulk_wait_read0();   // the O tile has been read out of this stage
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);   // done with this stage's U, O_intra and gamma
+            if (lane == 0) mbar_arrive(&empty[st]);   // done with this stage
             write_sop();
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_ready);
+            if (qw >= 2 && !trans) {   // O = Q gamma S + Aqk U': D1 rows 64..127, read while the next product 1 runs
+                if (!mbar_wait(&o_full, ci & 1, status)) break;
+                tc_fence_after();
+                float vv[NCW];
+#pragma unroll
+                for (int cb = 0; cb < NCW; cb += 16)
+                    tmem_ld16(lane_base + C::d1col(ci) + c_off + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+                tmem_wait_ld_regs<NCW>(vv);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&o_done);   // this D1 buffer may take chunk ci + 2's U
+                const int r = i - 64;   // token row: NCW columns (a multiple of 16) of o leave as 16-byte stores
+                if (r < n) {
+                    __nv_bfloat16* orow = o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + j0 + jw;
+#pragma unroll
+                    for (int e8 = 0; e8 < NCW / 8; ++e8) {
+                        float o8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o8[e] = vv[8 * e8 + e];
+                        reinterpret_cast<uint4*>(orow)[e8] = pack8(o8);
+                    }
+                }
+            }
             // the checkpoint leaves from registers after the next product has been released, so its
             // stores drain while product 1 of the next chunk runs
             if (!trans && ckpt_stride > 0 && checkpoints && n == 64) {
@@ -1112,7 +1055,6 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 }
             }
         }
-        if (o_issuer) bulk_wait0();
         // row i, columns j0 + jw .. + NCW: 16-byte stores (every row start and column offset is a multiple of 4)
         float* dst = nullptr;
         if (last) {
@@ -1205,14 +1147,9 @@ cudaError_t launch_state(const ChunkArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int slices = DV / DVS + (a.final_transition ? kDK / DVS : 0);
     dim3 grid(a.n_seqs * a.H, slices);
-    CUtensorMap mo;   // o [T, H, DV]: 64-column x 64-token boxes with the 128-byte swizzle
-    memset(&mo, 0, sizeof(mo));
-    if (a.total_tokens > 0 &&
-        !make_map(&mo, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, a.total_tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
     return launch_pdl(state_bf16_kernel<DV, DVS>, grid, dim3(C::NT), smem, s, static_cast<const uint8_t*>(a.packets),
                       a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, a.win_hi, a.initial_state,
-                      static_cast<__nv_bfloat16*>(a.o), mo, a.final_state, a.final_transition, a.ckpt_stride,
+                      static_cast<__nv_bfloat16*>(a.o), a.final_state, a.final_transition, a.ckpt_stride,
                       a.checkpoints, a.ckpt_cu, a.carry, a.status);
 }
 
