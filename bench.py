@@ -282,8 +282,7 @@ MMA_PHASES = [
     ("prep A: [K e^(g-b); Q e^(g-b)] x 160 anchored key rows, per 64-channel half", 160, 64, False, 2),
     ("prep B, K part: [X; X] diag(beta) x -(K gamma)^T", 128, 64, False, 1),
     ("prep B, V part: [X; X] diag(beta) x V (MN-major)", 128, 64, True, 1),
-    ("state 0: [I; 0] U (U MN-major)", 128, 64, True, 1),
-    ("state 1: [-W; Q gamma] S onto [U; 0] (S MN-major)", 128, 128, True, 1),
+    ("state 1: [-W; Q gamma] S (S MN-major)", 128, 128, True, 1),
     ("state 2: Kdec^T U' (U' MN-major)", 128, 64, True, 1),
     ("state 3: Aqk U' (U' MN-major)", 128, 64, True, 1),
 ]

@@ -30,8 +30,8 @@
 //                     MMAs, and bulk TMA stores of the MMA-ready packet.
 //  state_bf16_kernel  one CTA per (sequence, head, dv-slice), warp-specialised: a producer warp
 //                     streams packets through a shared-memory ring with bulk TMA, one thread issues
-//                     the tcgen05 products per chunk ([I; 0] U into a double-buffered accumulator,
-//                     [-W; Q gamma] S onto it, then Kdec^T U' and Aqk U'), 8 or 16 epilogue warps
+//                     the tcgen05 products per chunk ([-W; Q gamma] S into a double-buffered
+//                     accumulator, then Kdec^T U' and Aqk U'), 8 or 16 epilogue warps
 //                     hold the fp32 state in registers and feed bf16 copies of S and U' back as the
 //                     next operands.
 #include <cudaTypedefs.h>
@@ -57,6 +57,10 @@ __device__ __forceinline__ void st_b32(uint8_t* p, uint32_t v) { *reinterpret_ca
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
     __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
     return __bfloat1622float2(h);
+}
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+    const float2 a = bf2_to_f2(u.x), b = bf2_to_f2(u.y), c = bf2_to_f2(u.z), d = bf2_to_f2(u.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
 }
 __device__ __forceinline__ uint32_t pack2(float2 f) { return pack_bf16x2(f.x, f.y); }
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
@@ -737,23 +741,24 @@ struct SCfg {
     static constexpr int NT = 32 * (NEW + 2);              // + producer warp + MMA warp
     static constexpr bool MN = DVS >= 64;                  // S and U' staged MN-major (row = channel / token)
     static constexpr int NST = DVS == 32 ? 3 : 2;
-    static constexpr int NCP = DVS >= 64 ? DVS : 64;       // columns of U copied into D1: whole 64-column atoms
-    static constexpr uint32_t U_BYTES = NCP * 128;
+    static constexpr uint32_t U_BYTES = DVS >= 64 ? DVS * 128 : 8192;   // whole 64-column atoms of U
     // stage: the packet's parts for this slice (Aqk right after Kdec^T, as in the packet)
     static constexpr uint32_t AW = 0, KD = 32768, AQ = 49152, U = 57344, G = U + U_BYTES;
     static constexpr uint32_t STAGE = ((G + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SOP = NST * STAGE;      // S as B operand (N = DVS, K = 128)
     static constexpr uint32_t UOP = SOP + DVS * 256;  // U' as B operand (N = DVS, K = 64)
-    static constexpr uint32_t IZ = UOP + DVS * 128;   // [I; 0]: 128 x 64 bf16 K-major A operand of the U copy
-    static constexpr uint32_t BYTES = IZ + 16384;
-    // TMEM: D1 double-buffered at columns [0, NCP) and [NCP + DVS, 2 NCP + DVS), D2 at [NCP, NCP + DVS);
-    // the slice's columns of D1 start at c_off = j0 % 64 when a slice is narrower than an atom
+    // O tile staging for the tensor store, [DVS/64][64 tokens][128 B] with the 128B swizzle (slices of whole
+    // 64-column atoms only; narrower slices store O from registers)
+    static constexpr uint32_t OST = UOP + DVS * 128;
+    static constexpr uint32_t BYTES = OST + (MN ? DVS * 128 : 0);
+    // TMEM: D1 double-buffered at columns [0, DVS) and [2 DVS, 3 DVS), D2 at [DVS, 2 DVS)
     static constexpr uint32_t S_LBO = 128 * 128;      // MN-major: 64 columns x 128 K rows per block
     static constexpr uint32_t U_LBO = 64 * 128;       // MN-major: 64 columns x 64 K rows per block
-    static constexpr uint32_t TMEM_COLS = 2 * NCP + DVS <= 128 ? 128 : (2 * NCP + DVS <= 256 ? 256 : 512);
-    static __host__ __device__ constexpr uint32_t d1col(int ci) { return (ci & 1) ? NCP + DVS : 0; }
+    static constexpr uint32_t TMEM_COLS = 3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512);
+    static __host__ __device__ constexpr uint32_t d1col(int ci) { return (ci & 1) ? 2 * DVS : 0; }
     static_assert(BYTES + 1024 <= 232448, "one CTA per SM");
-    static_assert(IZ % 1024 == 0 && STAGE % 1024 == 0 && SOP % 1024 == 0, "128B-swizzle operands on 1024-byte atoms");
+    static_assert(STAGE % 1024 == 0 && SOP % 1024 == 0 && UOP % 1024 == 0 && OST % 1024 == 0,
+                  "128B-swizzle operands and tiles on 1024-byte atoms");
 };
 
 template <int DV, int DVS>
@@ -761,6 +766,7 @@ __global__ void __launch_bounds__(SCfg<DV, DVS>::NT, 1)
 state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict__ cu_seqlens,
                   const int32_t* __restrict__ cu_chunks, int n_seqs, int H, long long win_lo, long long win_hi,
                   const float* __restrict__ initial_state, __nv_bfloat16* __restrict__ o,
+                  const __grid_constant__ CUtensorMap map_o,
                   float* __restrict__ final_state, float* __restrict__ final_transition, int ckpt_stride,
                   float* __restrict__ checkpoints, const int32_t* __restrict__ ckpt_cu, float* __restrict__ carry,
                   int* status) {
@@ -769,7 +775,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
     constexpr int NST = C::NST, NCW = C::NCW, NEW = C::NEW, NSV = DV / DVS, CW = DV + kDK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    __shared__ __align__(8) uint64_t full[NST], empty[NST], d1_full, d2_full, o_full, s_ready, up_ready, o_done;
+    __shared__ __align__(8) uint64_t full[NST], empty[NST], d1_full, d2_full, o_full, s_ready, up_ready;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     grid_dependency_wait();   // the packets and the chunk index come from the launches before this one
@@ -799,26 +805,12 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         mbar_init(&o_full, 1);
         mbar_init(&s_ready, NEW);
         mbar_init(&up_ready, NEW / 2);   // only the warps that produce U' (TMEM lanes 0..63)
-        mbar_init(&o_done, NEW / 2);     // only the warps that read O (TMEM lanes 64..127)
         fence_barrier_init();
     }
     if (w == 0) {
         tmem_alloc(&tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
-    // [I; 0] (rows 0..63 the identity, rows 64..127 zero): [I; 0] U puts U into D1 rows 0..63 and zero into
-    // rows 64..127, exactly (bf16 values times 1)
-    for (int e = t; e < 128 * 8; e += C::NT) {
-        const int r = e >> 3, sc = e & 7;
-        uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        if (r < 64 && (r >> 3) == sc) {
-            const uint32_t one = 0x3F80u << (16 * (r & 1));   // bf16 1.0 in the low or high half
-            const int word = (r & 7) >> 1;
-            if (word == 0) z.x = one; else if (word == 1) z.y = one; else if (word == 2) z.z = one; else z.w = one;
-        }
-        *reinterpret_cast<uint4*>(sm + C::IZ + r * 128 + ((sc ^ (r & 7)) << 4)) = z;
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -852,18 +844,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, DVS, false, C::MN);
-            const uint32_t idcp = idesc_bf16(128, C::NCP, false, true);
-            const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP), iz = smem_u32(sm + C::IZ);
-            const uint32_t c_off = DVS >= 64 ? 0u : static_cast<uint32_t>(j0 & 63);
-            // D1[ci] = [I; 0] U of chunk ci (U MN-major, K = 64 tokens): U in rows 0..63, zero in rows 64..127,
-            // so that product 1 adds [-W; Q gamma] S onto it
-            auto load_u = [&](int ci) {
-                const uint32_t sb = smem_u32(sm + (ci % NST) * C::STAGE);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tm + C::d1col(ci), sdesc_k_sw128(iz + ks * 32), sdesc_mn_sw128(sb + C::U + ks * 2048, 8192),
-                             idcp, ks > 0);
-            };
+            const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP);
             auto ubdesc = [&](int ks) -> uint64_t {   // U' as the B operand (K = 64 tokens)
                 return C::MN ? sdesc_mn_sw128(uop + ks * 2048, C::U_LBO) : sdesc_k_sw128(uop + ks * 32);
             };
@@ -873,15 +854,14 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
                 tc_fence_after();
                 const uint32_t sb = smem_u32(sm + st * C::STAGE);
-                if (ci == 0 && !trans) load_u(0);
-                // D1 (+)= [-W; Q gamma] S   (M = 128, N = DVS, K = 128)
+                // D1 = [-W; Q gamma] S   (M = 128, N = DVS, K = 128).  D1[ci] was last read as chunk ci - 2's O,
+                // before the O warps' s_ready arrival for chunk ci - 1.
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
                     const uint64_t bdesc = C::MN ? sdesc_mn_sw128(sop + ks * 2048, C::S_LBO)
                                                  : sdesc_k_sw128(sop + ka * (DVS * 128) + kb);
-                    umma_f16(tm + C::d1col(ci) + c_off, sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc,
-                             !trans || ks > 0);
+                    umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc, ks > 0);
                 }
                 umma_commit(&d1_full);
                 if (!mbar_wait(&up_ready, ci & 1, status)) break;
@@ -889,26 +869,17 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 // D2 = Kdec^T U'   (M = 128, N = DVS, K = 64)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tm + C::NCP, sdesc_k_sw128(sb + C::KD + ks * 32), ubdesc(ks), idesc, ks > 0);
+                    umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), ubdesc(ks), idesc, ks > 0);
                 umma_commit(&d2_full);
                 if (!trans) {
-                    // the O warps have read chunk ci - 1's O (its D1 buffer takes chunk ci + 1's U below)
-                    if (ci > 0 && !mbar_wait(&o_done, (ci - 1) & 1, status)) break;
                     // D1 rows 64..127 += Aqk U' (O = Q gamma S + Aqk U'): the A operand starts 64 rows into Kdec^T,
                     // so its rows 64..127 are Aqk; what it adds to rows 0..63 (U', already read) is never used
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        umma_f16(tm + C::d1col(ci) + c_off, sdesc_k_sw128(sb + C::KD + 8192 + ks * 32), ubdesc(ks),
-                                 idesc, true);
+                        umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::KD + 8192 + ks * 32), ubdesc(ks), idesc, true);
                     umma_commit(&o_full);
                 }
                 umma_commit(&empty[st]);
-                // the next chunk's U into the other D1 buffer (chunk ci - 1's, whose O has been read)
-                if (!trans && ci + 1 < nch) {
-                    if (!mbar_wait(&full[(ci + 1) % NST], ((ci + 1) / NST) & 1, status)) break;
-                    tc_fence_after();
-                    load_u(ci + 1);
-                }
             }
         }
     } else {
@@ -953,38 +924,47 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_ready);
-        const uint32_t c_off = DVS >= 64 ? 0u : static_cast<uint32_t>(j0 & 63);
+        const int ucol = (DVS >= 64 ? 0 : (j0 & 63)) + jw;   // this warp's first column inside the stage's U atoms
+        // full chunks of whole-atom slices leave through a TMA tensor store of the O tile staged in OST
+        const bool o_issuer = (w == 2) && lane == 0;
         for (int ci = 0; ci < nch; ++ci) {
             const int st = ci % NST;
-            uint8_t* sb = sm + st * C::STAGE;
+            const uint8_t* sb = sm + st * C::STAGE;
             const int c = static_cast<int>(lo + ci - ch_lo);
             const long long rem = seq_len - static_cast<long long>(c) * 64;
             const int n = rem < 64 ? static_cast<int>(rem) : 64;
+            const bool full_tma = C::MN && !trans && n == 64;
             if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
-            if (qw < 2) {   // U' = U - W S: D1 rows 0..63 (loaded with U before the product)
+            if (qw < 2) {   // U' = U - W S: U row i from the stage, -W S from D1 rows 0..63
+                uint4 ur[NCW / 8];
+#pragma unroll
+                for (int e8 = 0; e8 < NCW / 8; ++e8) {
+                    const int col = ucol + 8 * e8;
+                    ur[e8] = trans ? make_uint4(0u, 0u, 0u, 0u)
+                                   : *reinterpret_cast<const uint4*>(sb + C::U + (col >> 6) * 8192 + i * 128 +
+                                                                     ((((col & 63) >> 3) ^ (i & 7)) << 4));
+                }
                 if (!mbar_wait(&d1_full, ci & 1, status)) break;
                 tc_fence_after();
                 float vv[NCW];   // D1 row i, columns jw .. jw + NCW: all loads in flight, one wait
 #pragma unroll
                 for (int cb = 0; cb < NCW; cb += 16)
-                    tmem_ld16(lane_base + C::d1col(ci) + c_off + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+                    tmem_ld16(lane_base + C::d1col(ci) + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
                 tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
-                for (int cb = 0; cb < NCW; cb += 16) {
+                for (int e8 = 0; e8 < NCW / 8; ++e8) {
+                    const int cc = jw / 8 + e8;   // 8-column chunk within the slice
+                    float u8[8];
+                    unpack8(ur[e8], u8);
 #pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
-                        const int cc = (jw + cb) / 8 + sub;   // 8-column chunk within the slice
-                        float u8[8];
+                    for (int e = 0; e < 8; ++e) u8[e] += vv[8 * e8 + e];
+                    if constexpr (C::MN) {
+                        *reinterpret_cast<uint4*>(sm + C::UOP + sw128_mn_offset(8 * cc, i, C::U_LBO)) = pack8(u8);
+                    } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) u8[e] = vv[cb + 8 * sub + e];
-                        if constexpr (C::MN) {
-                            *reinterpret_cast<uint4*>(sm + C::UOP + sw128_mn_offset(8 * cc, i, C::U_LBO)) = pack8(u8);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                *reinterpret_cast<__nv_bfloat16*>(sm + C::UOP + sw128_offset(8 * cc + e, i, DVS)) =
-                                    __float2bfloat16_rn(u8[e]);
-                        }
+                        for (int e = 0; e < 8; ++e)
+                            *reinterpret_cast<__nv_bfloat16*>(sm + C::UOP + sw128_offset(8 * cc + e, i, DVS)) =
+                                __float2bfloat16_rn(u8[e]);
                     }
                 }
                 tc_fence_before();
@@ -999,7 +979,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 float vv[NCW];
 #pragma unroll
                 for (int cb = 0; cb < NCW; cb += 16)
-                    tmem_ld16(lane_base + C::NCP + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+                    tmem_ld16(lane_base + DVS + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
                 tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
                 for (int e = 0; e < NCW; e += 2) {
@@ -1020,13 +1000,31 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 float vv[NCW];
 #pragma unroll
                 for (int cb = 0; cb < NCW; cb += 16)
-                    tmem_ld16(lane_base + C::d1col(ci) + c_off + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+                    tmem_ld16(lane_base + C::d1col(ci) + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
                 tmem_wait_ld_regs<NCW>(vv);
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&o_done);   // this D1 buffer may take chunk ci + 2's U
-                const int r = i - 64;   // token row: NCW columns (a multiple of 16) of o leave as 16-byte stores
-                if (r < n) {
+                const int r = i - 64;   // token row
+                if (full_tma) {
+                    if (o_issuer) bulk_wait_read0();   // the previous tile has left OST
+                    named_bar_sync(2, 32 * NEW / 2);
+#pragma unroll
+                    for (int e8 = 0; e8 < NCW / 8; ++e8) {
+                        const int col = jw + 8 * e8;   // column within the slice
+                        float o8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o8[e] = vv[8 * e8 + e];
+                        *reinterpret_cast<uint4*>(sm + C::OST + (col >> 6) * 8192 + r * 128 +
+                                                  ((((col & 63) >> 3) ^ (r & 7)) << 4)) = pack8(o8);
+                    }
+                    fence_proxy_async_smem();
+                    named_bar_sync(1, 32 * NEW / 2);   // every O warp has written its rows of the tile
+                    if (o_issuer) {
+#pragma unroll
+                        for (int b = 0; b < DVS / 64; ++b)
+                            tma_store_3d(&map_o, j0 + 64 * b, h, static_cast<int>(seq_tok0 + c * 64), sm + C::OST + b * 8192);
+                        bulk_commit();
+                    }
+                } else if (r < n) {   // NCW columns (a multiple of 16) of row r as 16-byte stores
                     __nv_bfloat16* orow = o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + j0 + jw;
 #pragma unroll
                     for (int e8 = 0; e8 < NCW / 8; ++e8) {
@@ -1055,6 +1053,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 }
             }
         }
+        if (o_issuer) bulk_wait0();
         // row i, columns j0 + jw .. + NCW: 16-byte stores (every row start and column offset is a multiple of 4)
         float* dst = nullptr;
         if (last) {
@@ -1147,9 +1146,14 @@ cudaError_t launch_state(const ChunkArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int slices = DV / DVS + (a.final_transition ? kDK / DVS : 0);
     dim3 grid(a.n_seqs * a.H, slices);
+    CUtensorMap mo;   // o [T, H, DV]: 64-column x 64-token boxes with the 128-byte swizzle
+    memset(&mo, 0, sizeof(mo));
+    if (a.total_tokens > 0 &&
+        !make_map(&mo, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, a.total_tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
     return launch_pdl(state_bf16_kernel<DV, DVS>, grid, dim3(C::NT), smem, s, static_cast<const uint8_t*>(a.packets),
                       a.cu_seqlens, a.cu_chunks, a.n_seqs, a.H, a.win_lo, a.win_hi, a.initial_state,
-                      static_cast<__nv_bfloat16*>(a.o), a.final_state, a.final_transition, a.ckpt_stride,
+                      static_cast<__nv_bfloat16*>(a.o), mo, a.final_state, a.final_transition, a.ckpt_stride,
                       a.checkpoints, a.ckpt_cu, a.carry, a.status);
 }
 
