@@ -427,6 +427,12 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             // ---------------- product A, this half: D[m, n] += RALL[m, :] . BVAR[n, :]  (M = 128, N = 160,
             // K = 64); the columns of variant i (row tile i's key side) are [8 i (i+1), 8 (i+1)(i+2))
             if (t == 0) {
+                // VOP has been read: the second half's k and q tiles, then V (product B's operand); MXFP8: the
+                // second half's code tiles have been read, so the next item's first ones follow.  The loads go
+                // first: issuing the products holds this thread for several hundred cycles.
+                if (hf == 0) issue_kq(loc.x, h, 1);
+                else if (!MX) issue_v(loc.x, h);
+                else if (nvalid) issue_kq(nloc.x, nh, 0);
                 tc_fence_after();
                 const uint32_t ra = smem_u32(sm + ps::OPB), bv = smem_u32(sm + ps::BVAR);
                 const uint32_t idesc = idesc_bf16(128, 160);
@@ -434,11 +440,6 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 for (int ks = 0; ks < 4; ++ks)
                     umma_f16(tm, sdesc_k_sw128(ra + ks * 32), sdesc_k_sw128(bv + ks * 32), idesc, hf > 0 || ks > 0);
                 umma_commit(&bar_mma);
-                // VOP has been read: the second half's k and q tiles, then V (product B's operand); MXFP8: the
-                // second half's code tiles have been read, so the next item's first ones follow
-                if (hf == 0) issue_kq(loc.x, h, 1);
-                else if (!MX) issue_v(loc.x, h);
-                else if (nvalid) issue_kq(nloc.x, nh, 0);
             }
         }
         if (fail) break;
