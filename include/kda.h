@@ -362,9 +362,13 @@ KDA_API kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_
  *  kernels' waits end without a fault.
  *  kda_selftest_umma: one 128 x n x 64 bf16 tcgen05 product D = A B^T through the same shared-memory
  *  descriptors, TMEM allocation and load path the chunk kernels use. a [128,64], b [n,64] bf16
- *  row-major (device), d [128,n] fp32 (device); n in {16, 32, ..., 256}.  b_mn_major != 0 stages B
- *  MN-major instead of K-major (then n must be a multiple of 64).
+ *  row-major (device), d [128,n] fp32 (device); n in {16, 32, ..., 256}.  flags: KDA_SELFTEST_B_MN_MAJOR
+ *  stages B MN-major instead of K-major (then n must be a multiple of 64); KDA_SELFTEST_A_TMEM reads A
+ *  from tensor memory (row m in lane m, two bf16 per 32-bit column), the operand form the segment
+ *  compose uses, instead of shared memory.  Other flag bits: KDA_ERR_ARG.
  */
+#define KDA_SELFTEST_B_MN_MAJOR 1
+#define KDA_SELFTEST_A_TMEM 2
 /*
  *  kda_selftest_mma_rate: the tensor-core rate of one product shape as the chunk kernels issue it:
  *  128 x n x k bf16 (k in {64, 128}, n in {16, ..., 256}; B K-major, or MN-major when b_mn_major, then
@@ -377,7 +381,7 @@ KDA_API kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_
 KDA_API kda_status_t kda_selftest_mma_rate(int n, int k, int b_mn_major, int reps, float* cycles, int grid,
                                            kda_stream_t stream);
 KDA_API kda_status_t kda_selftest_wait_timeout(int limit_us, kda_stream_t stream);
-KDA_API kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, int b_mn_major,
+KDA_API kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, int flags,
                                        kda_stream_t stream);
 
 #ifdef __cplusplus

@@ -19,7 +19,7 @@ __all__ = [
     "kda_chunk_fwd_noalloc",
     "kda_recurrent_step", "kda_recurrent_step_mxfp8", "kda_decode_verify", "kda_decode_commit", "kda_segment_compose", "kda_ckpt_offsets", "kda_get_device_status",
     "kda_status_string", "kda_version", "kda_profile_begin", "kda_profile_end", "kda_selftest_wait_timeout",
-    "kda_selftest_umma", "kda_selftest_mma_rate", "KDA_PREFIX_BLOCK", "kda_prefix_block_hashes", "kda_prefix_cache_create",
+    "kda_selftest_umma", "KDA_SELFTEST_B_MN_MAJOR", "KDA_SELFTEST_A_TMEM", "kda_selftest_mma_rate", "KDA_PREFIX_BLOCK", "kda_prefix_block_hashes", "kda_prefix_cache_create",
     "kda_prefix_cache_destroy", "kda_prefix_cache_lookup", "kda_prefix_cache_plan", "kda_prefix_cache_insert",
     "kda_prefix_cache_commit", "kda_prefix_cache_abort", "kda_prefix_cache_release", "kda_prefix_cache_stats",
     "KDA_PREFIX_NO_SLOT", "KDA_PREFIX_STORED",
@@ -483,13 +483,17 @@ def kda_selftest_mma_rate(n, k, *, b_mn_major=False, reps=256, grid=None, stream
     return cyc
 
 
-def kda_selftest_umma(a, b, d, *, b_mn_major=False, stream=None):
+KDA_SELFTEST_B_MN_MAJOR = 1
+KDA_SELFTEST_A_TMEM = 2
+
+
+def kda_selftest_umma(a, b, d, *, b_mn_major=False, a_tmem=False, stream=None):
     n = b.shape[0]
     _need(a, "a", (128, 64), torch.bfloat16)
     _need(b, "b", (n, 64), torch.bfloat16, a.device)
     _need(d, "d", (128, n), torch.float32, a.device)
-    _check(_load().kda_selftest_umma(_p(a), _p(b), _p(d), n, int(bool(b_mn_major)), _stream(stream)),
-           "kda_selftest_umma")
+    flags = (KDA_SELFTEST_B_MN_MAJOR if b_mn_major else 0) | (KDA_SELFTEST_A_TMEM if a_tmem else 0)
+    _check(_load().kda_selftest_umma(_p(a), _p(b), _p(d), n, flags, _stream(stream)), "kda_selftest_umma")
     return d
 
 

@@ -1,6 +1,7 @@
 // kda_umma_selftest.cu -- diagnostics of the tcgen05 path the chunk kernels use, no KDA arithmetic:
 //  * one bf16 product through the same shared-memory descriptors (128-byte swizzle; B K-major or
-//    MN-major), TMEM allocation, commit and TMEM-load path: D[128, n] = A[128, 64] * B[n, 64]^T;
+//    MN-major), TMEM allocation, commit and TMEM-load path: D[128, n] = A[128, 64] * B[n, 64]^T, with A
+//    from shared memory or from tensor memory (row m in lane m, two bf16 per 32-bit column);
 //  * the tensor-core rate of a product shape as the kernels issue it (M = 128 x N x K, one CTA per SM,
 //    timed with the SM clock): back to back, and one product at a time waited for before the next.
 #include "kda_device.cuh"
@@ -10,7 +11,8 @@ namespace kda {
 
 __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16* __restrict__ a,
                                                             const __nv_bfloat16* __restrict__ b,
-                                                            float* __restrict__ d, int n, int b_mn, int* status) {
+                                                            float* __restrict__ d, int n, int flags, int* status) {
+    const int b_mn = flags & 1, a_tmem = flags & 2;
     extern __shared__ __align__(1024) uint8_t raw[];
     uint8_t* base = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);   // stays a shared-memory pointer
     uint8_t* sA = base;                 // 128 rows x 128 B
@@ -44,20 +46,32 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
         fence_barrier_init();
     }
     if (w == 0) {
-        tmem_alloc(&tbase, 256);
+        tmem_alloc(&tbase, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tbase;
+    if (a_tmem) {   // row 32 w + lane of A into TMEM columns [256, 288) of this warp's lanes
+        const uint32_t* ar = reinterpret_cast<const uint32_t*>(a + (32 * w + lane) * 64);
+        for (int c0 = 0; c0 < 32; c0 += 16) {
+            float x[16];
+            for (int j = 0; j < 16; ++j) x[j] = __uint_as_float(ar[c0 + j]);
+            tmem_st16(tm + (static_cast<uint32_t>(32 * w) << 16) + 256 + c0, x);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
     if (t == 0) {
         const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0);
         for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t da = sdesc_k_sw128(smem_u32(sA) + kk * 32);
             const uint64_t db = b_mn ? sdesc_mn_sw128(smem_u32(sB) + kk * 2048, lbo)
                                      : sdesc_k_sw128(smem_u32(sB) + kk * 32);
-            umma_f16(tm, da, db, idesc, kk > 0);
+            if (a_tmem) umma_f16_ts(tm, tm + 256 + kk * 8, db, idesc, kk > 0);
+            else umma_f16(tm, sdesc_k_sw128(smem_u32(sA) + kk * 32), db, idesc, kk > 0);
         }
         umma_commit(&bar);
     }
@@ -74,7 +88,7 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
     }
     tc_fence_before();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tm, 256);
+    if (w == 0) tmem_dealloc(tm, 512);
 }
 
 // One CTA per SM; thread 0 times `reps` products of shape 128 x n x k (operands zero: only the timing
@@ -151,13 +165,13 @@ cudaError_t launch_selftest_mma_rate(int n, int k, int b_mn, int reps, float* cy
     return cudaGetLastError();
 }
 
-cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int b_mn, int* status,
+cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int flags, int* status,
                                  cudaStream_t s) {
     const int smem = 1024 + 128 * 128 + ((n + 63) / 64) * 64 * 128;
     cudaError_t e = cudaFuncSetAttribute(selftest_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     selftest_umma_kernel<<<1, 128, smem, s>>>(static_cast<const __nv_bfloat16*>(a),
-                                              static_cast<const __nv_bfloat16*>(b), d, n, b_mn, status);
+                                              static_cast<const __nv_bfloat16*>(b), d, n, flags, status);
     return cudaGetLastError();
 }
 

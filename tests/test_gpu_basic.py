@@ -20,13 +20,16 @@ def _clear_status():
     assert kda.kda_get_device_status() == 0, "a kernel recorded an error in the status word"
 
 
-@pytest.mark.parametrize("n,mn", [(16, False), (64, False), (128, False), (256, False), (64, True), (128, True)])
-def test_selftest_umma_matches_matmul(n, mn):
+@pytest.mark.parametrize("n,mn,at", [(16, False, False), (64, False, False), (128, False, False), (256, False, False),
+                                     (64, True, False), (128, True, False),
+                                     (64, False, True), (128, True, True), (256, False, True)])
+def test_selftest_umma_matches_matmul(n, mn, at):
+    # at: A read from tensor memory (row m in lane m, two bf16 per 32-bit column), as the compose issues it
     g = torch.Generator(DEV).manual_seed(n)
     a = torch.randn(128, 64, device=DEV, generator=g).to(torch.bfloat16)
     b = torch.randn(n, 64, device=DEV, generator=g).to(torch.bfloat16)
     d = torch.full((128, n), float("nan"), device=DEV)
-    kda.kda_selftest_umma(a, b, d, b_mn_major=mn)
+    kda.kda_selftest_umma(a, b, d, b_mn_major=mn, a_tmem=at)
     ref = a.double().cpu() @ b.double().cpu().T
     np.testing.assert_allclose(d.cpu().numpy(), ref.numpy(), rtol=1e-4, atol=1e-4)
 
