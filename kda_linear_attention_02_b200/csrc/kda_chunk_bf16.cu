@@ -1088,23 +1088,10 @@ __global__ void chunk_table_kernel(const int32_t* __restrict__ cu_chunks, const 
 
 // ------------------------------------------------------------------------------------------------
 // host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, []() {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
 // 3D map over a [T, H, d] tensor (d innermost), box {box_d, 1, 64 tokens}, no swizzle.
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int d, int H, long long T,
               int box_d, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
-    auto enc = get_encode();
+    auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize, static_cast<cuuint64_t>(H) * d * esize};
@@ -1213,6 +1200,19 @@ cudaError_t launch_bf16_t(const ChunkArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
 
 size_t chunk_packet_bytes_bf16(int dk, int dv) { return dv == 64 ? Pk<64>::BYTES : Pk<128>::BYTES; }
 

@@ -6,15 +6,18 @@
 // cumulative transition M_s and its zero-start state Z_s, and a prefix scan recovers every segment's
 // start state:  X_0 = init,  X_{s+1} = M_s X_s + Z_s.
 //
-// dk = 128 (compose_tc_kernel): one CTA per (sequence, head) walks the sequence's segments in order
+// dk = 128 (compose_ts_kernel): one CTA per (sequence, head) walks the sequence's segments in order
 // and forms M_s X_s on the tensor cores.  fp32 accuracy comes from splitting every fp32 operand value
 // into three bf16 pieces x = x1 + x2 + x3 (x1 = bf16(x), x2 = bf16(x - x1), x3 = bf16(x - x1 - x2): 24
 // significant bits) and summing the six products x1 y1 + x1 y2 + x2 y1 + x1 y3 + x3 y1 + x2 y2 in the
-// fp32 accumulator; the terms left out are below 2^-24 of |M| |X|.  M_s is a K-major operand (rows i,
-// K = m), X_s an MN-major one (K rows m, N = dv columns j), both with the 128-byte swizzle.
+// fp32 accumulator; the terms left out are below 2^-24 of |M| |X|.  M_s's pieces are the A operand in
+// tensor memory (row i in lane i, K = m), X_s's the MN-major B operand in shared memory (K rows m, N = dv
+// columns j, 128-byte swizzle).  The next segment's M and Z arrive by TMA while this one's products run.
 // dk = 64 (compose_kernel): the dv columns of X evolve independently, so a CTA owns one (sequence,
 // head, 32-column slice) and walks the segments in order, staging M_s^T in shared memory and forming
 // the 64 x 32 product with 4 x 4 register blocking in fp32.
+#include <cstring>
+
 #include "kda_device.cuh"
 #include "kda_internal.h"
 
@@ -112,25 +115,32 @@ __device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
 }
 
 template <int DV>
-struct ComposeTc {
+struct ComposeTs {
     static constexpr int NT = 256;
-    static constexpr uint32_t A_PIECE = 128 * 128 * 2;      // M_s piece: [2 K atoms][128 rows][128 B]
-    static constexpr uint32_t B_PIECE = DV * 128 * 2;       // X_s piece: [DV / 64 blocks][128 K rows][128 B]
-    static constexpr uint32_t A0 = 0, B0 = 3 * A_PIECE;
-    static constexpr uint32_t BYTES = B0 + 3 * B_PIECE;
+    static constexpr uint32_t B_PIECE = DV * 128 * 2;      // X_s piece: [DV / 64 blocks][128 K rows][128 B]
+    static constexpr uint32_t B0 = 0;
+    // M_s and Z_s staged by TMA as fp32 boxes of [128 rows][32 columns] with the 128-byte swizzle (16 KB each)
+    static constexpr uint32_t MS = B0 + 3 * B_PIECE;
+    static constexpr uint32_t ZS = MS + 4 * 16384;
+    static constexpr uint32_t BYTES = ZS + (DV / 32) * 16384;
     static constexpr uint32_t LBO = 128 * 128;             // MN-major: 64 columns x 128 K rows per block
+    // TMEM (512 columns): the accumulator at [0, DV); piece p of M_s (A operand, row i in lane i, two bf16
+    // of K per column) at [TA + 64 p, TA + 64 p + 64)
+    static constexpr uint32_t TA = 256;
+    static_assert(MS % 1024 == 0 && ZS % 1024 == 0, "TMA boxes with the 128-byte swizzle on 1024-byte boundaries");
+    static_assert(BYTES + 1024 <= 232448, "one CTA per SM");
 };
 
 template <int DV>
 __global__ void __launch_bounds__(256, 1)
-compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, const int32_t* __restrict__ seg_cu,
-                  const float* __restrict__ init, int n_seqs, int n_segs, int H, float* __restrict__ starts,
-                  float* __restrict__ ends, int* status) {
-    using C = ComposeTc<DV>;
+compose_ts_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_z,
+                  const int32_t* __restrict__ seg_cu, const float* __restrict__ init, int n_seqs, int n_segs, int H,
+                  float* __restrict__ starts, float* __restrict__ ends, int* status) {
+    using C = ComposeTs<DV>;
     constexpr int DK = 128;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar;
+    __shared__ __align__(8) uint64_t bar_ld, bar_mma;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     const int seq = blockIdx.x / H, h = blockIdx.x % H;
@@ -140,15 +150,30 @@ compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, cons
         return;
     }
     if (t == 0) {
-        mbar_init(&bar, 1);
+        mbar_init(&bar_ld, 1);
+        mbar_init(&bar_mma, 1);
         fence_barrier_init();
+        prefetch_tmap(&map_m);
+        prefetch_tmap(&map_z);
     }
     if (w == 0) {
-        tmem_alloc(&tmem_slot, 128);
+        tmem_alloc(&tmem_slot, 512);
         tmem_relinquish();
     }
-    // X as the MN-major B operand pieces: thread = (row i = t >> 1, half of the DV columns), 8 columns per
-    // 16-byte chunk of each piece
+    __syncthreads();   // the barriers are initialised before the first load completes on one
+    // M_s and Z_s of this head into MS and ZS (thread 0; one phase of bar_ld)
+    bool ld_pending = false;
+    auto issue_ld = [&](int s) {
+        const int row = (s * H + h) * DK;
+        mbar_arrive_expect_tx(&bar_ld, (4 + DV / 32) * 16384);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(sm + C::MS + b * 16384, &map_m, 32 * b, row, &bar_ld);
+#pragma unroll
+        for (int b = 0; b < DV / 32; ++b) tma_load_2d(sm + C::ZS + b * 16384, &map_z, 32 * b, row, &bar_ld);
+        ld_pending = true;
+    };
+    if (t == 0 && s1 > s0) issue_ld(s0);
+    // X as the MN-major B operand pieces, 8 columns per 16-byte chunk of each piece
     auto put_x_row8 = [&](int i, int j, const float (&x)[8]) {
         float a[8], b[8], c[8];
 #pragma unroll
@@ -162,7 +187,7 @@ compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, cons
             make_uint4(pack_bf16x2(c[0], c[1]), pack_bf16x2(c[2], c[3]), pack_bf16x2(c[4], c[5]), pack_bf16x2(c[6], c[7]));
     };
     const size_t sh0 = static_cast<size_t>(seq) * H + h;
-    {   // X_0 = init (or zero): pieces, and the first segment's start state
+    {   // X_0 = init (or zero): pieces, and the first segment's start state; thread = (row i = t >> 1, half)
         const int i = t >> 1, j0 = (t & 1) * (DV / 2);
         const float* src = init ? init + (sh0 * DK + i) * DV : nullptr;
         float* dst = s1 > s0 ? starts + ((static_cast<size_t>(s0) * H + h) * DK + i) * DV : nullptr;
@@ -186,94 +211,99 @@ compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, cons
                     src ? *reinterpret_cast<const float4*>(src + j0 + jj) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tmem_slot;
-    uint32_t ph = 0;
+    // TMEM lane quarter w & 3 holds rows 32 (w & 3) ..; warp w >> 2 takes a half of the columns
+    const int qw = w & 3, hh = w >> 2, i = 32 * qw + lane;
+    const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
+    uint32_t ph_ld = 0, ph_mma = 0;
     for (int s = s0; s < s1; ++s) {
         const size_t bs = static_cast<size_t>(s) * H + h;
-        {   // the accumulator starts as Z_s (TMEM stores from the rows' loads): lane quarter w & 3 holds rows
-            // 32 (w & 3) .., warp w >> 2 a half of the columns
-            const int qw = w & 3, i = 32 * qw + lane, jh = (w >> 2) * (DV / 2);
-            const float* zr = Z + (bs * DK + i) * DV + jh;
-            if (s + 1 < s1) {   // the next segment's rows of Z into L2 meanwhile
-#pragma unroll
-                for (int l = 0; l < DV / 2; l += 32) prefetch_l2(Z + ((bs + H) * DK + i) * DV + jh + l);
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int jb = 0; jb < DV / 2; jb += 16) {
-                float z[16];
-#pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    const float4 v4 = *reinterpret_cast<const float4*>(zr + jb + e);
-                    z[e] = v4.x; z[e + 1] = v4.y; z[e + 2] = v4.z; z[e + 3] = v4.w;
-                }
-                tmem_st16(tm + (static_cast<uint32_t>(32 * qw) << 16) + jh + jb, z);
-            }
-            tmem_wait_st();
-            tc_fence_before();
+        {   // M_s and Z_s have landed
+            const bool ok = mbar_wait(&bar_ld, ph_ld, status);
+            ph_ld ^= 1;
+            if (t == 0) ld_pending = false;
+            if (__syncthreads_or(!ok)) break;
         }
-        {   // M_s as three K-major A operand pieces: thread = (row i, 64-column half)
-            const int i = t >> 1, m0 = (t & 1) * 64;
-            const float* src = M + (bs * DK + i) * DK + m0;
-            if (s + 1 < s1) {   // the next segment's rows into L2 meanwhile
-                const float* nx = M + ((bs + H) * DK + i) * DK + m0;
-                prefetch_l2(nx);
-                prefetch_l2(nx + 32);
-            }
+        // row i of M_s, columns [64 hh, 64 hh + 64): its three bf16 pieces into TMEM, 32 columns per box
 #pragma unroll
-            for (int mm = 0; mm < 64; mm += 8) {
-                const float4 u = *reinterpret_cast<const float4*>(src + mm);
-                const float4 v = *reinterpret_cast<const float4*>(src + mm + 4);
-                const float x[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
-                float a[8], b[8], c[8];
+        for (int q = 0; q < 2; ++q) {
+            const uint8_t* rowp = sm + C::MS + (2 * hh + q) * 16384 + i * 128;
+            float x[32];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) split3(x[e], a[e], b[e], c[e]);
-                const uint32_t off = C::A0 + sw128_offset(i, m0 + mm, 128);
-                *reinterpret_cast<uint4*>(sm + off) = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
-                                                                 pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
-                *reinterpret_cast<uint4*>(sm + off + C::A_PIECE) =
-                    make_uint4(pack_bf16x2(b[0], b[1]), pack_bf16x2(b[2], b[3]), pack_bf16x2(b[4], b[5]),
-                               pack_bf16x2(b[6], b[7]));
-                *reinterpret_cast<uint4*>(sm + off + 2 * C::A_PIECE) =
-                    make_uint4(pack_bf16x2(c[0], c[1]), pack_bf16x2(c[2], c[3]), pack_bf16x2(c[4], c[5]),
-                               pack_bf16x2(c[6], c[7]));
+            for (int c = 0; c < 8; ++c) {
+                const float4 v = *reinterpret_cast<const float4*>(rowp + ((c ^ (i & 7)) << 4));
+                x[4 * c] = v.x; x[4 * c + 1] = v.y; x[4 * c + 2] = v.z; x[4 * c + 3] = v.w;
             }
+            float p0[16], p1[16], p2[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                float a0, b0, c0, a1, b1, c1;
+                split3(x[2 * e], a0, b0, c0);
+                split3(x[2 * e + 1], a1, b1, c1);
+                p0[e] = __uint_as_float(pack_bf16x2(a0, a1));
+                p1[e] = __uint_as_float(pack_bf16x2(b0, b1));
+                p2[e] = __uint_as_float(pack_bf16x2(c0, c1));
+            }
+            const uint32_t col = C::TA + 32 * hh + 16 * q;
+            tmem_st16(lane_base + col, p0);
+            tmem_st16(lane_base + col + 64, p1);
+            tmem_st16(lane_base + col + 128, p2);
         }
-        fence_proxy_async_smem();
+        // row i of Z_s, columns [hh DV / 2, (hh + 1) DV / 2): the accumulator's start
+#pragma unroll
+        for (int q = 0; q < DV / 64; ++q) {
+            const uint8_t* rowp = sm + C::ZS + (hh * (DV / 64) + q) * 16384 + i * 128;
+            float z[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 v = *reinterpret_cast<const float4*>(rowp + ((c ^ (i & 7)) << 4));
+                z[4 * c] = v.x; z[4 * c + 1] = v.y; z[4 * c + 2] = v.z; z[4 * c + 3] = v.w;
+            }
+            tmem_st16(lane_base + hh * (DV / 2) + 32 * q, *reinterpret_cast<float(*)[16]>(z));
+            tmem_st16(lane_base + hh * (DV / 2) + 32 * q + 16, *reinterpret_cast<float(*)[16]>(z + 16));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        fence_proxy_async_smem();   // MS and ZS have been read: the next segment's loads may overwrite them
         __syncthreads();
-        // D = Z_s + sum over the six piece pairs (a, b) of A_a X_b  (M = 128, N = DV, K = 128)
+        // D = Z_s + sum over the six piece pairs (a, b) of A_a X_b  (M = 128, N = DV, K = 128); the next
+        // segment's M and Z load meanwhile (issued first: issuing the products holds the thread)
         if (t == 0) {
+            if (s + 1 < s1) issue_ld(s + 1);
             tc_fence_after();
-            const uint32_t a0 = smem_u32(sm + C::A0), b0 = smem_u32(sm + C::B0);
+            const uint32_t b0 = smem_u32(sm + C::B0);
             const uint32_t idesc = idesc_bf16(128, DV, false, true);
             constexpr int pa[6] = {0, 0, 1, 0, 2, 1}, pb[6] = {0, 1, 0, 2, 0, 1};
 #pragma unroll
             for (int p = 0; p < 6; ++p)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    umma_f16(tm, sdesc_k_sw128(a0 + pa[p] * C::A_PIECE + (ks >> 2) * 16384 + (ks & 3) * 32),
-                             sdesc_mn_sw128(b0 + pb[p] * C::B_PIECE + ks * 2048, C::LBO), idesc, 1u);
-            umma_commit(&bar);
+                    umma_f16_ts(tm, tm + C::TA + 64 * pa[p] + 8 * ks,
+                                sdesc_mn_sw128(b0 + pb[p] * C::B_PIECE + ks * 2048, C::LBO), idesc, 1u);
+            umma_commit(&bar_mma);
         }
-        const bool ok = mbar_wait(&bar, ph, status);
-        ph ^= 1;
-        if (__syncthreads_or(!ok)) break;
+        {
+            const bool ok = mbar_wait(&bar_mma, ph_mma, status);
+            ph_mma ^= 1;
+            if (__syncthreads_or(!ok)) break;
+        }
         tc_fence_after();
-        {   // X_{s+1} = D: lane quarter w & 3 holds rows 32 (w & 3) .., warp w >> 2 a half of the columns
-            const int qw = w & 3, i = 32 * qw + lane, jh = (w >> 2) * (DV / 2);
+        {   // X_{s+1} = D: the next start state (or the end state), and the next product's B operand
+            const int jh = hh * (DV / 2);
             float* dst = s + 1 < s1 ? starts + (((bs + H) * DK) + i) * DV : (ends ? ends + (sh0 * DK + i) * DV : nullptr);
 #pragma unroll
             for (int jb = 0; jb < DV / 2; jb += 16) {
                 float d[16];
-                tmem_ld16(tm + (static_cast<uint32_t>(32 * qw) << 16) + jh + jb, d);
+                tmem_ld16(lane_base + jh + jb, d);
                 tmem_wait_ld_regs<16>(d);
 #pragma unroll
                 for (int e = 0; e < 16; e += 4)
                     if (dst) *reinterpret_cast<float4*>(dst + jh + jb + e) = make_float4(d[e], d[e + 1], d[e + 2], d[e + 3]);
-                if (s + 1 < s1) {   // the next product's B operand
+                if (s + 1 < s1) {
                     float x8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) x8[e] = d[e];
@@ -288,19 +318,40 @@ compose_tc_kernel(const float* __restrict__ M, const float* __restrict__ Z, cons
         fence_proxy_async_smem();
         __syncthreads();
     }
+    if (t == 0 && ld_pending) mbar_wait(&bar_ld, ph_ld, nullptr);   // never leave a TMA write in flight
     tc_fence_before();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tm, 128);
+    if (w == 0) tmem_dealloc(tm, 512);
+}
+
+// 2D map over a row-major fp32 matrix [rows][cols]: boxes of 32 columns x 128 rows with the 128-byte swizzle
+static bool make_map_f32_rows(CUtensorMap* m, const float* base, int cols, long long rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * sizeof(float)};
+    const cuuint32_t box[2] = {32u, 128u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int DV>
-static cudaError_t launch_compose_tc(const float* M, const float* Z, const int32_t* seg_cu, const float* init,
+static cudaError_t launch_compose_ts(const float* M, const float* Z, const int32_t* seg_cu, const float* init,
                                      int n_seqs, int n_segs, int H, float* starts, float* ends, int* status,
                                      cudaStream_t s) {
-    const int smem = static_cast<int>(ComposeTc<DV>::BYTES) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(compose_tc_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    CUtensorMap mm, mz;
+    memset(&mm, 0, sizeof(mm));
+    memset(&mz, 0, sizeof(mz));
+    const long long rows = static_cast<long long>(n_segs) * H * 128;
+    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;   // TMA row coordinates are 32-bit
+    if (rows > 0 && (!make_map_f32_rows(&mm, M, 128, rows) || !make_map_f32_rows(&mz, Z, DV, rows)))
+        return cudaErrorInvalidValue;
+    const int smem = static_cast<int>(ComposeTs<DV>::BYTES) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(compose_ts_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    compose_tc_kernel<DV><<<n_seqs * H, 256, smem, s>>>(M, Z, seg_cu, init, n_seqs, n_segs, H, starts, ends, status);
+    compose_ts_kernel<DV><<<n_seqs * H, 256, smem, s>>>(mm, mz, seg_cu, init, n_seqs, n_segs, H, starts, ends, status);
     return cudaGetLastError();
 }
 
@@ -321,8 +372,8 @@ cudaError_t launch_compose(const float* M, const float* Z, const int32_t* seg_cu
                            int n_segs, int H, int dk, int dv, float* starts, float* ends, int* status,
                            cudaStream_t s) {
     if (n_seqs == 0) return cudaSuccess;
-    if (dk == 128 && dv == 128) return launch_compose_tc<128>(M, Z, seg_cu, init, n_seqs, n_segs, H, starts, ends, status, s);
-    if (dk == 128 && dv == 64) return launch_compose_tc<64>(M, Z, seg_cu, init, n_seqs, n_segs, H, starts, ends, status, s);
+    if (dk == 128 && dv == 128) return launch_compose_ts<128>(M, Z, seg_cu, init, n_seqs, n_segs, H, starts, ends, status, s);
+    if (dk == 128 && dv == 64) return launch_compose_ts<64>(M, Z, seg_cu, init, n_seqs, n_segs, H, starts, ends, status, s);
     if (dk == 64 && dv == 128) return launch_compose_t<64, 128>(M, Z, seg_cu, init, n_seqs, n_segs, H, starts, ends, status, s);
     return launch_compose_t<64, 64>(M, Z, seg_cu, init, n_seqs, n_segs, H, starts, ends, status, s);
 }

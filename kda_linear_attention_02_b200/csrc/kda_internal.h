@@ -2,11 +2,15 @@
 #pragma once
 
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
 namespace kda {
+
+// The driver's tensor-map encoder (looked up once; nullptr when the driver lacks it) (kda_chunk_bf16.cu).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // Decode step (kda_decode.cu).
 cudaError_t launch_decode(float* state, const void* q, const void* k, const void* v, const float* la,
