@@ -11,8 +11,9 @@
 // into three bf16 pieces x = x1 + x2 + x3 (x1 = bf16(x), x2 = bf16(x - x1), x3 = bf16(x - x1 - x2): 24
 // significant bits) and summing the six products x1 y1 + x1 y2 + x2 y1 + x1 y3 + x3 y1 + x2 y2 in the
 // fp32 accumulator; the terms left out are below 2^-24 of |M| |X|.  M_s's pieces are the A operand in
-// tensor memory (row i in lane i, K = m), X_s's the MN-major B operand in shared memory (K rows m, N = dv
-// columns j, 128-byte swizzle).  The next segment's M and Z arrive by TMA while this one's products run.
+// tensor memory (row i in lane i, K = m; two buffers, so that M_{s+1} is split while the products of
+// segment s run), X_s's the MN-major B operand in shared memory (K rows m, N = dv columns j, 128-byte
+// swizzle); Z_s is added to the product in the epilogue.  M and Z arrive by TMA ahead of their use.
 // dk = 64 (compose_kernel): the dv columns of X evolve independently, so a CTA owns one (sequence,
 // head, 32-column slice) and walks the segments in order, staging M_s^T in shared memory and forming
 // the 64 x 32 product with 4 x 4 register blocking in fp32.
@@ -124,9 +125,11 @@ struct ComposeTs {
     static constexpr uint32_t ZS = MS + 4 * 16384;
     static constexpr uint32_t BYTES = ZS + (DV / 32) * 16384;
     static constexpr uint32_t LBO = 128 * 128;             // MN-major: 64 columns x 128 K rows per block
-    // TMEM (512 columns): the accumulator at [0, DV); piece p of M_s (A operand, row i in lane i, two bf16
-    // of K per column) at [TA + 64 p, TA + 64 p + 64)
-    static constexpr uint32_t TA = 256;
+    // TMEM (512 columns): the accumulator at [0, 128); two buffers of M's three pieces (A operand, row i in
+    // lane i, two bf16 of K per column), buffer b's piece p at [TA + 192 b + 64 p, + 64): the pieces of
+    // M_{s+1} are formed while the products of segment s read those of M_s
+    static constexpr uint32_t TA = 128;
+    __host__ __device__ static constexpr uint32_t abuf(int b) { return TA + 192u * static_cast<uint32_t>(b); }
     static_assert(MS % 1024 == 0 && ZS % 1024 == 0, "TMA boxes with the 128-byte swizzle on 1024-byte boundaries");
     static_assert(BYTES + 1024 <= 232448, "one CTA per SM");
 };
@@ -134,45 +137,57 @@ struct ComposeTs {
 template <int DV>
 __global__ void __launch_bounds__(256, 1)
 compose_ts_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_z,
+                  const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_e,
                   const int32_t* __restrict__ seg_cu, const float* __restrict__ init, int n_seqs, int n_segs, int H,
                   float* __restrict__ starts, float* __restrict__ ends, int* status) {
     using C = ComposeTs<DV>;
     constexpr int DK = 128;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_ld, bar_mma;
+    __shared__ __align__(8) uint64_t bar_m, bar_z, bar_mma;
     __shared__ uint32_t tmem_slot;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     const int seq = blockIdx.x / H, h = blockIdx.x % H;
-    const int s0 = seg_cu[seq], s1 = seg_cu[seq + 1];
+    const int s0 = seg_cu[seq];
+    int s1 = seg_cu[seq + 1];
     if (s0 < 0 || s1 < s0 || s1 > n_segs || (seq == 0 && s0 != 0) || (seq == n_seqs - 1 && s1 != n_segs)) {
         if (t == 0) set_status(status, KDA_ERR_DEVICE_INPUT);
         return;
     }
     if (t == 0) {
-        mbar_init(&bar_ld, 1);
+        mbar_init(&bar_m, 1);
+        mbar_init(&bar_z, 1);
         mbar_init(&bar_mma, 1);
         fence_barrier_init();
         prefetch_tmap(&map_m);
         prefetch_tmap(&map_z);
+        prefetch_tmap(&map_s);
+        if (ends) prefetch_tmap(&map_e);
     }
     if (w == 0) {
         tmem_alloc(&tmem_slot, 512);
         tmem_relinquish();
     }
     __syncthreads();   // the barriers are initialised before the first load completes on one
-    // M_s and Z_s of this head into MS and ZS (thread 0; one phase of bar_ld)
-    bool ld_pending = false;
-    auto issue_ld = [&](int s) {
+    // M_s of this head into MS (one phase of bar_m; thread 0) and Z_s into ZS (one phase of bar_z; thread 32,
+    // which also stores each X_{s+1} from ZS and so knows when ZS is free again)
+    bool m_pending = false, z_pending = false;
+    auto issue_m = [&](int s) {
         const int row = (s * H + h) * DK;
-        mbar_arrive_expect_tx(&bar_ld, (4 + DV / 32) * 16384);
+        mbar_arrive_expect_tx(&bar_m, 4 * 16384);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) tma_load_2d(sm + C::MS + b * 16384, &map_m, 32 * b, row, &bar_ld);
-#pragma unroll
-        for (int b = 0; b < DV / 32; ++b) tma_load_2d(sm + C::ZS + b * 16384, &map_z, 32 * b, row, &bar_ld);
-        ld_pending = true;
+        for (int b = 0; b < 4; ++b) tma_load_2d(sm + C::MS + b * 16384, &map_m, 32 * b, row, &bar_m);
+        m_pending = true;
     };
-    if (t == 0 && s1 > s0) issue_ld(s0);
+    auto issue_z = [&](int s) {
+        const int row = (s * H + h) * DK;
+        mbar_arrive_expect_tx(&bar_z, (DV / 32) * 16384);
+#pragma unroll
+        for (int b = 0; b < DV / 32; ++b) tma_load_2d(sm + C::ZS + b * 16384, &map_z, 32 * b, row, &bar_z);
+        z_pending = true;
+    };
+    if (t == 0 && s1 > s0) issue_m(s0);
+    if (t == 32 && s1 > s0) issue_z(s0);
     // X as the MN-major B operand pieces, 8 columns per 16-byte chunk of each piece
     auto put_x_row8 = [&](int i, int j, const float (&x)[8]) {
         float a[8], b[8], c[8];
@@ -219,16 +234,10 @@ compose_ts_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_consta
     // TMEM lane quarter w & 3 holds rows 32 (w & 3) ..; warp w >> 2 takes a half of the columns
     const int qw = w & 3, hh = w >> 2, i = 32 * qw + lane;
     const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
-    uint32_t ph_ld = 0, ph_mma = 0;
-    for (int s = s0; s < s1; ++s) {
-        const size_t bs = static_cast<size_t>(s) * H + h;
-        {   // M_s and Z_s have landed
-            const bool ok = mbar_wait(&bar_ld, ph_ld, status);
-            ph_ld ^= 1;
-            if (t == 0) ld_pending = false;
-            if (__syncthreads_or(!ok)) break;
-        }
-        // row i of M_s, columns [64 hh, 64 hh + 64): its three bf16 pieces into TMEM, 32 columns per box
+    uint32_t ph_m = 0, ph_z = 0, ph_mma = 0;
+    // row i of M (in MS), columns [64 hh, 64 hh + 64): its three bf16 pieces into TMEM buffer b, 32 columns of
+    // M per box
+    auto split_m = [&](int b) {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
             const uint8_t* rowp = sm + C::MS + (2 * hh + q) * 16384 + i * 128;
@@ -248,32 +257,30 @@ compose_ts_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_consta
                 p1[e] = __uint_as_float(pack_bf16x2(b0, b1));
                 p2[e] = __uint_as_float(pack_bf16x2(c0, c1));
             }
-            const uint32_t col = C::TA + 32 * hh + 16 * q;
+            const uint32_t col = C::abuf(b) + 32 * hh + 16 * q;
             tmem_st16(lane_base + col, p0);
             tmem_st16(lane_base + col + 64, p1);
             tmem_st16(lane_base + col + 128, p2);
         }
-        // row i of Z_s, columns [hh DV / 2, (hh + 1) DV / 2): the accumulator's start
-#pragma unroll
-        for (int q = 0; q < DV / 64; ++q) {
-            const uint8_t* rowp = sm + C::ZS + (hh * (DV / 64) + q) * 16384 + i * 128;
-            float z[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float4 v = *reinterpret_cast<const float4*>(rowp + ((c ^ (i & 7)) << 4));
-                z[4 * c] = v.x; z[4 * c + 1] = v.y; z[4 * c + 2] = v.z; z[4 * c + 3] = v.w;
-            }
-            tmem_st16(lane_base + hh * (DV / 2) + 32 * q, *reinterpret_cast<float(*)[16]>(z));
-            tmem_st16(lane_base + hh * (DV / 2) + 32 * q + 16, *reinterpret_cast<float(*)[16]>(z + 16));
-        }
+    };
+    // the pieces of the first segment's M
+    bool ok = true;
+    if (s1 > s0) {
+        ok = mbar_wait(&bar_m, ph_m, status);
+        ph_m ^= 1;
+        if (t == 0) m_pending = false;
+        if (ok) split_m(0);
         tmem_wait_st();
         tc_fence_before();
-        fence_proxy_async_smem();   // MS and ZS have been read: the next segment's loads may overwrite them
-        __syncthreads();
-        // D = Z_s + sum over the six piece pairs (a, b) of A_a X_b  (M = 128, N = DV, K = 128); the next
-        // segment's M and Z load meanwhile (issued first: issuing the products holds the thread)
+        fence_proxy_async_smem();   // MS has been read
+    }
+    if (__syncthreads_or(!ok)) s1 = s0;   // nothing more to do (the status word says why)
+    if (t == 0 && s0 + 1 < s1) issue_m(s0 + 1);
+    for (int s = s0; s < s1; ++s) {
+        const size_t bs = static_cast<size_t>(s) * H + h;
+        const int buf = (s - s0) & 1;
+        // D = sum over the six piece pairs (a, b) of A_a X_b  (M = 128, N = DV, K = 128), from zero
         if (t == 0) {
-            if (s + 1 < s1) issue_ld(s + 1);
             tc_fence_after();
             const uint32_t b0 = smem_u32(sm + C::B0);
             const uint32_t idesc = idesc_bf16(128, DV, false, true);
@@ -282,28 +289,54 @@ compose_ts_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_consta
             for (int p = 0; p < 6; ++p)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    umma_f16_ts(tm, tm + C::TA + 64 * pa[p] + 8 * ks,
-                                sdesc_mn_sw128(b0 + pb[p] * C::B_PIECE + ks * 2048, C::LBO), idesc, 1u);
+                    umma_f16_ts(tm, tm + C::abuf(buf) + 64 * pa[p] + 8 * ks,
+                                sdesc_mn_sw128(b0 + pb[p] * C::B_PIECE + ks * 2048, C::LBO), idesc, p > 0 || ks > 0);
             umma_commit(&bar_mma);
         }
-        {
-            const bool ok = mbar_wait(&bar_mma, ph_mma, status);
-            ph_mma ^= 1;
-            if (__syncthreads_or(!ok)) break;
+        // meanwhile the next segment's M becomes the other buffer's pieces
+        bool has_next = s + 1 < s1;
+        ok = true;
+        if (has_next) {
+            ok = mbar_wait(&bar_m, ph_m, status);
+            ph_m ^= 1;
+            if (t == 0) m_pending = false;
+            if (ok) split_m(buf ^ 1);
+            fence_proxy_async_smem();   // MS has been read
         }
+        ok = mbar_wait(&bar_mma, ph_mma, status) && ok;
+        ph_mma ^= 1;
+        ok = mbar_wait(&bar_z, ph_z, status) && ok;
+        ph_z ^= 1;
+        if (t == 32) z_pending = false;
+        if (__syncthreads_or(!ok)) break;
+        if (t == 0 && s + 2 < s1) issue_m(s + 2);
         tc_fence_after();
-        {   // X_{s+1} = D: the next start state (or the end state), and the next product's B operand
+        {   // X_{s+1} = D + Z_s, written over Z_s in ZS (each thread rewrites the values it read) for the tensor
+            // store, and the next product's B operand
             const int jh = hh * (DV / 2);
-            float* dst = s + 1 < s1 ? starts + (((bs + H) * DK) + i) * DV : (ends ? ends + (sh0 * DK + i) * DV : nullptr);
 #pragma unroll
             for (int jb = 0; jb < DV / 2; jb += 16) {
                 float d[16];
                 tmem_ld16(lane_base + jh + jb, d);
+                // Z_s row i, columns jh + jb .. + 16: box (jh + jb) / 32, 16-byte chunks from (jb % 32) / 4
+                uint8_t* zrow = sm + C::ZS + ((jh + jb) >> 5) * 16384 + i * 128;
+                float z[16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int ch = ((jb & 31) >> 2) + c;
+                    const float4 v = *reinterpret_cast<const float4*>(zrow + ((ch ^ (i & 7)) << 4));
+                    z[4 * c] = v.x; z[4 * c + 1] = v.y; z[4 * c + 2] = v.z; z[4 * c + 3] = v.w;
+                }
                 tmem_wait_ld_regs<16>(d);
 #pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    if (dst) *reinterpret_cast<float4*>(dst + jh + jb + e) = make_float4(d[e], d[e + 1], d[e + 2], d[e + 3]);
-                if (s + 1 < s1) {
+                for (int e = 0; e < 16; ++e) d[e] += z[e];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int ch = ((jb & 31) >> 2) + c;
+                    *reinterpret_cast<float4*>(zrow + ((ch ^ (i & 7)) << 4)) =
+                        make_float4(d[4 * c], d[4 * c + 1], d[4 * c + 2], d[4 * c + 3]);
+                }
+                if (has_next) {
                     float x8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) x8[e] = d[e];
@@ -314,11 +347,27 @@ compose_ts_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_consta
                 }
             }
         }
+        tmem_wait_st();   // the next buffer's pieces
         tc_fence_before();
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();   // the B pieces for the next products; X_{s+1} in ZS for the tensor store
         __syncthreads();
+        if (t == 32) {   // X_{s+1} out (the next start state, or the end state), then the next Z into ZS
+            const CUtensorMap* mo = has_next ? &map_s : (ends ? &map_e : nullptr);
+            const int row = static_cast<int>((has_next ? bs + H : sh0) * DK);
+            if (mo) {
+#pragma unroll
+                for (int b = 0; b < DV / 32; ++b) tma_store_2d(mo, 32 * b, row, sm + C::ZS + b * 16384);
+                bulk_commit();
+                bulk_wait_read0();
+            }
+            if (has_next) issue_z(s + 1);
+        }
     }
-    if (t == 0 && ld_pending) mbar_wait(&bar_ld, ph_ld, nullptr);   // never leave a TMA write in flight
+    if (t == 0 && m_pending) mbar_wait(&bar_m, ph_m, nullptr);   // never leave a TMA write in flight
+    if (t == 32) {
+        if (z_pending) mbar_wait(&bar_z, ph_z, nullptr);
+        bulk_wait0();   // nor a store
+    }
     tc_fence_before();
     __syncthreads();
     if (w == 0) tmem_dealloc(tm, 512);
@@ -341,17 +390,22 @@ template <int DV>
 static cudaError_t launch_compose_ts(const float* M, const float* Z, const int32_t* seg_cu, const float* init,
                                      int n_seqs, int n_segs, int H, float* starts, float* ends, int* status,
                                      cudaStream_t s) {
-    CUtensorMap mm, mz;
+    CUtensorMap mm, mz, ms, me;
     memset(&mm, 0, sizeof(mm));
     memset(&mz, 0, sizeof(mz));
-    const long long rows = static_cast<long long>(n_segs) * H * 128;
-    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;   // TMA row coordinates are 32-bit
-    if (rows > 0 && (!make_map_f32_rows(&mm, M, 128, rows) || !make_map_f32_rows(&mz, Z, DV, rows)))
+    memset(&ms, 0, sizeof(ms));
+    memset(&me, 0, sizeof(me));
+    const long long rows = static_cast<long long>(n_segs) * H * 128, erows = static_cast<long long>(n_seqs) * H * 128;
+    if (rows > 0x7fffffffLL || erows > 0x7fffffffLL) return cudaErrorInvalidValue;   // TMA coordinates are 32-bit
+    if (rows > 0 && (!make_map_f32_rows(&mm, M, 128, rows) || !make_map_f32_rows(&mz, Z, DV, rows) ||
+                     !make_map_f32_rows(&ms, starts, DV, rows)))
         return cudaErrorInvalidValue;
+    if (ends && !make_map_f32_rows(&me, ends, DV, erows)) return cudaErrorInvalidValue;
     const int smem = static_cast<int>(ComposeTs<DV>::BYTES) + 1024;
     cudaError_t e = cudaFuncSetAttribute(compose_ts_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    compose_ts_kernel<DV><<<n_seqs * H, 256, smem, s>>>(mm, mz, seg_cu, init, n_seqs, n_segs, H, starts, ends, status);
+    compose_ts_kernel<DV><<<n_seqs * H, 256, smem, s>>>(mm, mz, ms, me, seg_cu, init, n_seqs, n_segs, H, starts, ends,
+                                                        status);
     return cudaGetLastError();
 }
 
