@@ -107,12 +107,14 @@ compose_kernel(const float* __restrict__ M, const float* __restrict__ Z, const i
     }
 }
 
-// three bf16 pieces of x (their sum holds x to 24 significant bits)
-__device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
-    a = __bfloat162float(__float2bfloat16_rn(x));
-    const float r = x - a;
-    b = __bfloat162float(__float2bfloat16_rn(r));
-    c = r - b;
+// The three bf16 pieces a = bf16(x), b = bf16(x - a), c = bf16(x - a - b) of a pair of values (their sums
+// hold x to 24 significant bits), as packed bf16x2 words (low half = x0): each piece is rounded once and
+// its fp32 value read back from the packed word (x - a and x - a - b are exact in fp32).
+__device__ __forceinline__ void split3x2(float x0, float x1, uint32_t& pa, uint32_t& pb, uint32_t& pc) {
+    pa = pack_bf16x2(x0, x1);
+    const float r0 = x0 - __uint_as_float(pa << 16), r1 = x1 - __uint_as_float(pa & 0xFFFF0000u);
+    pb = pack_bf16x2(r0, r1);
+    pc = pack_bf16x2(r0 - __uint_as_float(pb << 16), r1 - __uint_as_float(pb & 0xFFFF0000u));
 }
 
 template <int DV>
@@ -190,16 +192,13 @@ compose_ts_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_consta
     if (t == 32 && s1 > s0) issue_z(s0);
     // X as the MN-major B operand pieces, 8 columns per 16-byte chunk of each piece
     auto put_x_row8 = [&](int i, int j, const float (&x)[8]) {
-        float a[8], b[8], c[8];
+        uint32_t a[4], b[4], c[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) split3(x[e], a[e], b[e], c[e]);
+        for (int e = 0; e < 4; ++e) split3x2(x[2 * e], x[2 * e + 1], a[e], b[e], c[e]);
         const uint32_t off = C::B0 + sw128_mn_offset(j, i, C::LBO);
-        *reinterpret_cast<uint4*>(sm + off) = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
-                                                         pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
-        *reinterpret_cast<uint4*>(sm + off + C::B_PIECE) = make_uint4(pack_bf16x2(b[0], b[1]), pack_bf16x2(b[2], b[3]),
-                                                                      pack_bf16x2(b[4], b[5]), pack_bf16x2(b[6], b[7]));
-        *reinterpret_cast<uint4*>(sm + off + 2 * C::B_PIECE) =
-            make_uint4(pack_bf16x2(c[0], c[1]), pack_bf16x2(c[2], c[3]), pack_bf16x2(c[4], c[5]), pack_bf16x2(c[6], c[7]));
+        *reinterpret_cast<uint4*>(sm + off) = make_uint4(a[0], a[1], a[2], a[3]);
+        *reinterpret_cast<uint4*>(sm + off + C::B_PIECE) = make_uint4(b[0], b[1], b[2], b[3]);
+        *reinterpret_cast<uint4*>(sm + off + 2 * C::B_PIECE) = make_uint4(c[0], c[1], c[2], c[3]);
     };
     const size_t sh0 = static_cast<size_t>(seq) * H + h;
     {   // X_0 = init (or zero): pieces, and the first segment's start state; thread = (row i = t >> 1, half)
@@ -250,12 +249,11 @@ compose_ts_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_consta
             float p0[16], p1[16], p2[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                float a0, b0, c0, a1, b1, c1;
-                split3(x[2 * e], a0, b0, c0);
-                split3(x[2 * e + 1], a1, b1, c1);
-                p0[e] = __uint_as_float(pack_bf16x2(a0, a1));
-                p1[e] = __uint_as_float(pack_bf16x2(b0, b1));
-                p2[e] = __uint_as_float(pack_bf16x2(c0, c1));
+                uint32_t a, b, c;
+                split3x2(x[2 * e], x[2 * e + 1], a, b, c);
+                p0[e] = __uint_as_float(a);
+                p1[e] = __uint_as_float(b);
+                p2[e] = __uint_as_float(c);
             }
             const uint32_t col = C::abuf(b) + 32 * hh + 16 * q;
             tmem_st16(lane_base + col, p0);
