@@ -41,13 +41,17 @@ struct F32Packet {
 
 template <int DK, int DV>
 struct PrepSmem {
+    static constexpr int TP = 64 + 4;   // pitch of the transposed factor arrays [DK][TP] (float4 rows of 4 tokens)
     static constexpr int R0 = (64 * DK > 2 * 64 * 64) ? 64 * DK : 2 * 64 * 64;   // g, later A + Aqk
-    static constexpr int KIV = 64 * (DK > DV ? DK : DV);                          // k*Einv, later beta*V
-    static constexpr size_t FLOATS = R0 + 3 * 64 * DK + KIV + 64 * 64 /*X*/ + 64 /*beta*/ + 4 * DK /*e^b*/ +
+    static constexpr int FT = DK * TP;                                             // one transposed factor array
+    static constexpr int KIV = FT > 64 * DV ? FT : 64 * DV;                        // k*Einv^T, later beta*V
+    static constexpr size_t FLOATS = R0 + 3 * FT + KIV + 64 * 64 /*X*/ + 64 /*beta*/ + 4 * DK /*e^b*/ +
                                      4 * DK /*e^(gC-b')*/ + 16 * DK /*tile pair*/ + 3 * 256 /*solve tmp*/;
     static constexpr size_t BYTES = FLOATS * 4;
 };
 
+// One CTA per (chunk, head) item.  The elementwise factors are stored transposed (channel-major, 4 tokens
+// per float4), so that the A / Aqk products, W and U run as 4 x 4 (or 4 x 8) register blocks per thread.
 template <int DK, int DV>
 __global__ void __launch_bounds__(256)
 chunk_prep_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
@@ -56,20 +60,22 @@ chunk_prep_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, 
                       int H, long long win_lo, float* __restrict__ packets) {
     using P = F32Packet<DK, DV>;
     using SM = PrepSmem<DK, DV>;
+    constexpr int TP = SM::TP;
     extern __shared__ __align__(16) float sm[];
     float* g = sm;                          // [64][DK]
     float* Am = sm;                         // [64][64]   (after g is dead)
     float* Aq = sm + 64 * 64;               // [64][64]
-    float* KE = sm + SM::R0;                // [64][DK]   k * exp(g - b_t)
-    float* QE = KE + 64 * DK;               // [64][DK]   q * exp(g - b_t)
-    float* KF = QE + 64 * DK;               // [64][DK]   k * exp(b_{t+1} - g)
-    float* KI = KF + 64 * DK;               // [64][DK]   k * exp(b_t - g); later beta*V [64][DV]
+    float* KE = sm + SM::R0;                // [DK][TP]   k * exp(g - b_t), transposed; later beta k gamma [64][DK]
+    float* QE = KE + SM::FT;                // [DK][TP]   q * exp(g - b_t), transposed
+    float* KF = QE + SM::FT;                // [DK][TP]   k * exp(b_{t+1} - g), transposed
+    float* KI = KF + SM::FT;                // [DK][TP]   k * exp(b_t - g), transposed; later beta*V [64][DV]
+    float* BK = QE;                         // [64][DK]   beta k gamma (QE is dead by then)
     float* X = KI + SM::KIV;                // [64][64]
     float* bet = X + 64 * 64;               // [64]
     float* eb = bet + 64;                   // [4][DK]    exp(b_t)
     float* ec = eb + 4 * DK;                // [4][DK]    exp(g_C - b_{t+1})
     float* ed = ec + 4 * DK;                // [4][4][DK] exp(b_i - b_jp), 1 <= jp <= i <= 3
-    float* tmp = ed + 16 * DK;              // [3][16][16] solve temporaries
+    float* tmp = ed + 16 * DK;              // [3][16][16] solve temporaries; the prefix sum's segment totals
 
     const int t = threadIdx.x;
     const long long item = blockIdx.x;
@@ -92,9 +98,17 @@ chunk_prep_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, 
     }
     if (t < 64) bet[t] = t < n ? beta[(static_cast<size_t>(loc.tok0) + t) * H + h] : 0.f;
     __syncthreads();
-    if (t < DK) {
+    {   // inclusive prefix sum along the 64 tokens: 256 / DK segments per channel, then the segments' offsets
+        constexpr int NSEG = 256 / DK, LSEG = 64 / NSEG;
+        const int c = t % DK, sg = t / DK;
         float acc = 0.f;
-        for (int r = 0; r < 64; ++r) { acc += g[r * DK + t]; g[r * DK + t] = acc; }
+        for (int r = sg * LSEG; r < (sg + 1) * LSEG; ++r) { acc += g[r * DK + c]; g[r * DK + c] = acc; }
+        tmp[sg * DK + c] = acc;
+        __syncthreads();
+        float off = 0.f;
+        for (int s2 = 0; s2 < sg; ++s2) off += tmp[s2 * DK + c];
+        if (sg > 0)
+            for (int r = sg * LSEG; r < (sg + 1) * LSEG; ++r) g[r * DK + c] += off;
     }
     __syncthreads();
     // 2. per-(tile, channel) factors
@@ -117,55 +131,71 @@ chunk_prep_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, 
         const float kv = r < n ? kb[static_cast<size_t>(r) * row_k + c] : 0.f;
         const float qv = r < n ? qb[static_cast<size_t>(r) * row_k + c] : 0.f;
         const float E = expf(gr - bt), Einv = expf(bt - gr), F = expf(bn - gr);
-        KE[e] = kv * E;
-        QE[e] = qv * E;
-        KI[e] = kv * Einv;
-        KF[e] = kv * F;
+        KE[c * TP + r] = kv * E;
+        QE[c * TP + r] = qv * E;
+        KI[c * TP + r] = kv * Einv;
+        KF[c * TP + r] = kv * F;
         pk[P::QT + e] = qv * E * eb[tl * DK + c];     // q * exp(g)
         pk[P::KD + e] = kv * F * ec[tl * DK + c];     // k * exp(g_C - g)
     }
     __syncthreads();   // g is dead from here; its space becomes A and Aqk
-    // 4. A (strict lower, beta rows) and Aqk (inclusive lower)
+    // 4. A (strict lower, beta rows) and Aqk (inclusive lower): thread = 4 x 4 block (rows r0.., keys s0..);
+    //    both lie in one 16-token tile each, so the key side is one variant for the whole block
     {
-        const int lane = t & 31, w = t >> 5;
-        for (int rr = 0; rr < 8; ++rr) {
-            const int r = w + 8 * rr, ti = r >> 4;
-            for (int half = 0; half < 2; ++half) {
-                const int s = lane + 32 * half, tj = s >> 4;
-                float ak = 0.f, aq = 0.f;
-                if (s <= r) {
-                    if (tj == ti) {
-                        for (int cc = 0; cc < DK; ++cc) {
-                            const int c = (cc + lane) & (DK - 1);
-                            const float kr = KI[s * DK + c];
-                            ak = fmaf(KE[r * DK + c], kr, ak);
-                            aq = fmaf(QE[r * DK + c], kr, aq);
-                        }
-                    } else {
-                        const float* d = ed + (ti * 4 + tj + 1) * DK;
-                        for (int cc = 0; cc < DK; ++cc) {
-                            const int c = (cc + lane) & (DK - 1);
-                            const float kr = KF[s * DK + c] * d[c];
-                            ak = fmaf(KE[r * DK + c], kr, ak);
-                            aq = fmaf(QE[r * DK + c], kr, aq);
-                        }
-                    }
+        const int rb = t >> 4, sb = t & 15, r0 = 4 * rb, s0 = 4 * sb;
+        float ak[4][4], aq[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) ak[u][x] = aq[u][x] = 0.f;
+        if (sb <= rb) {   // blocks above the diagonal are zero
+            const int ti = r0 >> 4, tj = s0 >> 4;
+            const bool diag = ti == tj;
+            const float* kside = diag ? KI : KF;
+            const float* d = ed + (ti * 4 + tj + 1) * DK;   // exp(b_ti - b_{tj+1}), read off the diagonal only
+            for (int c = 0; c < DK; ++c) {
+                const float4 ke = *reinterpret_cast<const float4*>(KE + c * TP + r0);
+                const float4 qe = *reinterpret_cast<const float4*>(QE + c * TP + r0);
+                float4 kr = *reinterpret_cast<const float4*>(kside + c * TP + s0);
+                if (!diag) {
+                    const float dc = d[c];
+                    kr = make_float4(kr.x * dc, kr.y * dc, kr.z * dc, kr.w * dc);
                 }
-                Am[r * 64 + s] = s < r ? bet[r] * ak : 0.f;
-                Aq[r * 64 + s] = aq;
+                const float kev[4] = {ke.x, ke.y, ke.z, ke.w}, qev[4] = {qe.x, qe.y, qe.z, qe.w};
+                const float krv[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        ak[u][x] = fmaf(kev[u], krv[x], ak[u][x]);
+                        aq[u][x] = fmaf(qev[u], krv[x], aq[u][x]);
+                    }
             }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u;
+            const float br = bet[r];
+            float a4[4], q4[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                a4[x] = s0 + x < r ? br * ak[u][x] : 0.f;
+                q4[x] = s0 + x <= r ? aq[u][x] : 0.f;
+            }
+            *reinterpret_cast<float4*>(Am + r * 64 + s0) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+            *reinterpret_cast<float4*>(Aq + r * 64 + s0) = make_float4(q4[0], q4[1], q4[2], q4[3]);
         }
     }
     __syncthreads();
     for (int e = t; e < 64 * 64; e += 256) pk[P::AQ + e] = Aq[e];
-    // stage beta * V over KI (dead) and beta * k * exp(g) over KE (dead)
+    // stage beta * V over KI (dead) and beta * k * exp(g) over QE (dead), both row-major
     for (int e = t; e < 64 * DV; e += 256) {
         const int r = e / DV, c = e % DV;
         KI[e] = r < n ? bet[r] * vb[static_cast<size_t>(r) * row_v + c] : 0.f;
     }
     for (int e = t; e < 64 * DK; e += 256) {
         const int r = e / DK, c = e % DK;
-        KE[e] = bet[r] * KE[e] * eb[(r >> 4) * DK + c];
+        BK[e] = bet[r] * KE[c * TP + r] * eb[(r >> 4) * DK + c];
     }
     // 5. X = (I + A)^-1: diagonal 16x16 blocks (one warp each, lane = column), then off-diagonal
     //    blocks by block-diagonal level: X_ij = -X_ii sum_{j<=m<i} A_im X_mj
@@ -204,33 +234,83 @@ chunk_prep_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, 
         }
         __syncthreads();
     }
-    // 6. W = X (beta K exp(g)),  U = X (beta V)
-    for (int e = t; e < 64 * DK; e += 256) {
-        const int r = e / DK, c = e % DK;
-        float acc = 0.f;
-        for (int s = 0; s <= r; ++s) acc = fmaf(X[r * 64 + s], KE[s * DK + c], acc);
-        pk[P::W + e] = acc;
-    }
-    for (int e = t; e < 64 * DV; e += 256) {
-        const int r = e / DV, c = e % DV;
-        float acc = 0.f;
-        for (int s = 0; s <= r; ++s) acc = fmaf(X[r * 64 + s], KI[s * DV + c], acc);
-        pk[P::U + e] = acc;
+    // 6. W = X (beta K exp(g)),  U = X (beta V): thread = 4 rows x (DK / 16 and DV / 16) columns
+    {
+        constexpr int CK = DK / 16, CV = DV / 16;
+        const int r0 = 4 * (t >> 4), cb = t & 15;
+        float aw[4][CK], au[4][CV];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int x = 0; x < CK; ++x) aw[u][x] = 0.f;
+#pragma unroll
+            for (int x = 0; x < CV; ++x) au[u][x] = 0.f;
+        }
+        for (int s2 = 0; s2 < r0 + 4; ++s2) {   // X is zero past its diagonal
+            float xr[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) xr[u] = X[(r0 + u) * 64 + s2];
+#pragma unroll
+            for (int x4 = 0; x4 < CK; x4 += 4) {
+                const float4 b = *reinterpret_cast<const float4*>(BK + s2 * DK + cb * CK + x4);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    aw[u][x4] = fmaf(xr[u], b.x, aw[u][x4]);
+                    aw[u][x4 + 1] = fmaf(xr[u], b.y, aw[u][x4 + 1]);
+                    aw[u][x4 + 2] = fmaf(xr[u], b.z, aw[u][x4 + 2]);
+                    aw[u][x4 + 3] = fmaf(xr[u], b.w, aw[u][x4 + 3]);
+                }
+            }
+#pragma unroll
+            for (int x4 = 0; x4 < CV; x4 += 4) {
+                const float4 b = *reinterpret_cast<const float4*>(KI + s2 * DV + cb * CV + x4);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    au[u][x4] = fmaf(xr[u], b.x, au[u][x4]);
+                    au[u][x4 + 1] = fmaf(xr[u], b.y, au[u][x4 + 1]);
+                    au[u][x4 + 2] = fmaf(xr[u], b.z, au[u][x4 + 2]);
+                    au[u][x4 + 3] = fmaf(xr[u], b.w, au[u][x4 + 3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int x4 = 0; x4 < CK; x4 += 4)
+                *reinterpret_cast<float4*>(pk + P::W + (r0 + u) * DK + cb * CK + x4) =
+                    make_float4(aw[u][x4], aw[u][x4 + 1], aw[u][x4 + 2], aw[u][x4 + 3]);
+#pragma unroll
+            for (int x4 = 0; x4 < CV; x4 += 4)
+                *reinterpret_cast<float4*>(pk + P::U + (r0 + u) * DV + cb * CV + x4) =
+                    make_float4(au[u][x4], au[u][x4 + 1], au[u][x4 + 2], au[u][x4 + 3]);
+        }
     }
 }
 
-constexpr int kF32Cols = 32;   // dv columns per state CTA
+constexpr int kF32Cols = 16;   // dv columns per state CTA
 
+// Shared memory of the state pass, in floats; rows of the operands read as float4 along their K index
+// are padded by 4 floats, so that the 8 rows a quarter warp reads fall on different banks.
 template <int DK, int DV>
 struct StateSmem {
-    static constexpr size_t FLOATS = DK * kF32Cols /*S*/ + 3 * 64 * DK /*W,QT,KD*/ + 2 * 64 * kF32Cols /*U,U'*/ +
-                                     64 * 64 /*Aqk*/ + DK /*G*/;
+    static constexpr int NC = kF32Cols;
+    static constexpr int PK = DK + 4, PA = 64 + 4;
+    static constexpr size_t S0 = 0;                    // S [DK][NC], two buffers (read one, write the other)
+    static constexpr size_t W = 2 * DK * NC;           // -W rows [64][PK]
+    static constexpr size_t QT = W + 64 * PK;          // Q gamma rows [64][PK]
+    static constexpr size_t KD = QT + 64 * PK;         // Kdec rows [64][DK]
+    static constexpr size_t AQ = KD + 64 * DK;         // Aqk rows [64][PA]
+    static constexpr size_t UC = AQ + 64 * PA;         // U slice [64][NC]
+    static constexpr size_t UP = UC + 64 * NC;         // U' slice [64][NC]
+    static constexpr size_t G = UP + 64 * NC;          // exp(g_C) [DK]
+    static constexpr size_t FLOATS = G + DK;
     static constexpr size_t BYTES = FLOATS * 4;
 };
 
-// One CTA per (sequence, head, 32-column slice).  Slices [0, DV/32) are state columns; with a
-// transition output, slices [DV/32, DV/32 + DK/32) carry columns of the cumulative transition
-// (same update with U = 0, identity start, no output).
+// One CTA per (sequence, head, 16-column slice).  Slices [0, DV/16) are state columns; with a
+// transition output, slices [DV/16, DV/16 + DK/16) carry columns of the cumulative transition
+// (same update with U = 0, identity start, no output).  Each thread forms four adjacent columns of one
+// row of U', O and the new S from 16-byte shared loads, summing in the same order as a plain dot product.
 template <int DK, int DV>
 __global__ void __launch_bounds__(256)
 chunk_state_f32_kernel(const float* __restrict__ packets, const int32_t* __restrict__ cu_seqlens,
@@ -240,18 +320,19 @@ chunk_state_f32_kernel(const float* __restrict__ packets, const int32_t* __restr
                        int ckpt_stride, float* __restrict__ checkpoints, const int32_t* __restrict__ ckpt_cu,
                        float* __restrict__ carry, int* status) {
     using P = F32Packet<DK, DV>;
-    constexpr int NC = kF32Cols;
+    using L = StateSmem<DK, DV>;
+    constexpr int NC = kF32Cols, PK = L::PK, PA = L::PA;
     extern __shared__ __align__(16) float sm[];
-    float* S = sm;                 // [DK][NC]
-    float* Wc = S + DK * NC;       // [64][DK]
-    float* Qc = Wc + 64 * DK;      // [64][DK]
-    float* Kc = Qc + 64 * DK;      // [64][DK]
-    float* Uc = Kc + 64 * DK;      // [64][NC]
-    float* Up = Uc + 64 * NC;      // [64][NC]
-    float* Ac = Up + 64 * NC;      // [64][64]
-    float* Gc = Ac + 64 * 64;      // [DK]
+    float* Wc = sm + L::W;
+    float* Qc = sm + L::QT;
+    float* Kc = sm + L::KD;
+    float* Ac = sm + L::AQ;
+    float* Uc = sm + L::UC;
+    float* Up = sm + L::UP;
+    float* Gc = sm + L::G;
 
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int t = threadIdx.x;
+    const int rr = t >> 2, cq = 4 * (t & 3);   // this thread's row (of U', O, S) and first column
     const int seq = blockIdx.x / H, h = blockIdx.x % H;
     const int slice = blockIdx.y;
     const bool trans = slice >= DV / NC;
@@ -267,7 +348,8 @@ chunk_state_f32_kernel(const float* __restrict__ packets, const int32_t* __restr
     const size_t sh = static_cast<size_t>(seq) * H + h;
     const int CW = DV + DK;   // carry row width
 
-    // initial state slice
+    float* S = sm + L::S0;            // the current state slice [DK][NC]
+    float* Sn = sm + L::S0 + DK * NC; // the next one
     for (int e = t; e < DK * NC; e += 256) {
         const int i = e / NC, j = e % NC;
         float x;
@@ -276,7 +358,6 @@ chunk_state_f32_kernel(const float* __restrict__ packets, const int32_t* __restr
         else x = initial_state ? initial_state[(sh * DK + i) * DV + c0 + j] : 0.f;
         S[e] = x;
     }
-    __syncthreads();
     const long long seq_tok0 = cu_seqlens[seq];
     const long long seq_len = static_cast<long long>(cu_seqlens[seq + 1]) - seq_tok0;
     for (long long gcix = lo; gcix < hi; ++gcix) {
@@ -284,46 +365,90 @@ chunk_state_f32_kernel(const float* __restrict__ packets, const int32_t* __restr
         const long long rem = seq_len - static_cast<long long>(c) * 64;
         const int n = rem < 64 ? static_cast<int>(rem) : 64;
         const float* pk = packets + static_cast<size_t>((gcix - win_lo) * H + h) * (P::BYTES / 4);
-        for (int e = t; e < 64 * DK; e += 256) {
-            Wc[e] = pk[P::W + e];
-            Qc[e] = pk[P::QT + e];
-            Kc[e] = pk[P::KD + e];
+        // this chunk's packet (16-byte loads; every offset below is a multiple of 4 floats)
+        for (int e = t; e < 64 * DK / 4; e += 256) {
+            const int r = (4 * e) / DK, i = (4 * e) % DK;
+            *reinterpret_cast<float4*>(Wc + r * PK + i) = reinterpret_cast<const float4*>(pk + P::W)[e];
+            *reinterpret_cast<float4*>(Qc + r * PK + i) = reinterpret_cast<const float4*>(pk + P::QT)[e];
+            reinterpret_cast<float4*>(Kc)[e] = reinterpret_cast<const float4*>(pk + P::KD)[e];
         }
-        for (int e = t; e < 64 * NC; e += 256) {
-            const int r = e / NC, j = e % NC;
-            Uc[e] = trans ? 0.f : pk[P::U + r * DV + c0 + j];
+        for (int e = t; e < 64 * 16; e += 256) {
+            const int r = e >> 4, s4 = 4 * (e & 15);
+            *reinterpret_cast<float4*>(Ac + r * PA + s4) = reinterpret_cast<const float4*>(pk + P::AQ)[e];
         }
-        for (int e = t; e < 64 * 64; e += 256) Ac[e] = pk[P::AQ + e];
+        for (int e = t; e < 64 * NC / 4; e += 256) {
+            const int r = (4 * e) / NC, j = (4 * e) % NC;
+            reinterpret_cast<float4*>(Uc)[e] = trans ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                                     : *reinterpret_cast<const float4*>(pk + P::U + r * DV + c0 + j);
+        }
         for (int e = t; e < DK; e += 256) Gc[e] = pk[P::G + e];
         __syncthreads();
-        // U' = U - W S
-        for (int m = 0; m < 8; ++m) {
-            const int r = w + 8 * m;
-            float acc = Uc[r * NC + lane];
-            for (int i = 0; i < DK; ++i) acc = fmaf(-Wc[r * DK + i], S[i * NC + lane], acc);
-            Up[r * NC + lane] = acc;
-        }
-        __syncthreads();
-        // O = Qt S + Aqk U'
-        if (!trans) {
-            for (int m = 0; m < 8; ++m) {
-                const int r = w + 8 * m;
-                if (r >= n) continue;
-                float acc = 0.f;
-                for (int i = 0; i < DK; ++i) acc = fmaf(Qc[r * DK + i], S[i * NC + lane], acc);
-                for (int s = 0; s <= r; ++s) acc = fmaf(Ac[r * 64 + s], Up[s * NC + lane], acc);
-                o[(static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + c0 + lane] = acc;
+        // U' = U - W S: row rr, columns cq .. cq + 3
+        {
+            float4 acc = *reinterpret_cast<const float4*>(Uc + rr * NC + cq);
+            for (int i = 0; i < DK; i += 4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(Wc + rr * PK + i);
+                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 s4 = *reinterpret_cast<const float4*>(S + (i + u) * NC + cq);
+                    acc.x = fmaf(-wv[u], s4.x, acc.x);
+                    acc.y = fmaf(-wv[u], s4.y, acc.y);
+                    acc.z = fmaf(-wv[u], s4.z, acc.z);
+                    acc.w = fmaf(-wv[u], s4.w, acc.w);
+                }
             }
+            *reinterpret_cast<float4*>(Up + rr * NC + cq) = acc;
         }
         __syncthreads();
-        // S <- Diag(exp(g_C)) S + Kdec^T U'
-        for (int m = 0; m < DK / 8; ++m) {
-            const int i = w + 8 * m;
-            float acc = Gc[i] * S[i * NC + lane];
-            for (int r = 0; r < 64; ++r) acc = fmaf(Kc[r * DK + i], Up[r * NC + lane], acc);
-            S[i * NC + lane] = acc;
+        // O = Qt S + Aqk U' (row rr) and the next state S' = Diag(exp(g_C)) S + Kdec^T U' (rows i = rr + 64 p)
+        if (!trans && rr < n) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < DK; i += 4) {
+                const float4 q4 = *reinterpret_cast<const float4*>(Qc + rr * PK + i);
+                const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 s4 = *reinterpret_cast<const float4*>(S + (i + u) * NC + cq);
+                    acc.x = fmaf(qv[u], s4.x, acc.x);
+                    acc.y = fmaf(qv[u], s4.y, acc.y);
+                    acc.z = fmaf(qv[u], s4.z, acc.z);
+                    acc.w = fmaf(qv[u], s4.w, acc.w);
+                }
+            }
+            for (int s4i = 0; s4i <= rr; s4i += 4) {   // Aqk is zero past the diagonal
+                const float4 a4 = *reinterpret_cast<const float4*>(Ac + rr * PA + s4i);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (s4i + u > rr) continue;
+                    const float4 p4 = *reinterpret_cast<const float4*>(Up + (s4i + u) * NC + cq);
+                    acc.x = fmaf(av[u], p4.x, acc.x);
+                    acc.y = fmaf(av[u], p4.y, acc.y);
+                    acc.z = fmaf(av[u], p4.z, acc.z);
+                    acc.w = fmaf(av[u], p4.w, acc.w);
+                }
+            }
+            *reinterpret_cast<float4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + rr) * H + h) * DV + c0 + cq) = acc;
         }
-        __syncthreads();
+#pragma unroll
+        for (int pp = 0; pp < DK / 64; ++pp) {
+            const int i = rr + 64 * pp;
+            const float gi = Gc[i];
+            const float4 s0 = *reinterpret_cast<const float4*>(S + i * NC + cq);
+            float4 acc = make_float4(gi * s0.x, gi * s0.y, gi * s0.z, gi * s0.w);
+            for (int r = 0; r < 64; ++r) {
+                const float kv = Kc[r * DK + i];
+                const float4 p4 = *reinterpret_cast<const float4*>(Up + r * NC + cq);
+                acc.x = fmaf(kv, p4.x, acc.x);
+                acc.y = fmaf(kv, p4.y, acc.y);
+                acc.z = fmaf(kv, p4.z, acc.z);
+                acc.w = fmaf(kv, p4.w, acc.w);
+            }
+            *reinterpret_cast<float4*>(Sn + i * NC + cq) = acc;
+        }
+        __syncthreads();   // S' complete; the packet buffers and U' free for the next chunk
+        float* tmp = S; S = Sn; Sn = tmp;
         if (!trans && ckpt_stride > 0 && checkpoints && n == 64) {
             const long long end = static_cast<long long>(c + 1) * 64;
             if (end % ckpt_stride == 0) {
