@@ -104,11 +104,11 @@ def make_inputs(lengths, H, dk, dv, *, dtype=torch.bfloat16, device="cpu", seed=
 
 
 def make_decode_inputs(n, H, dk, dv, *, dtype=torch.bfloat16, device="cpu", seed=0,
-                       steps=1, state_sd=0.02):
+                       steps=1, state_sd=0.02, alpha_mu=0.0, alpha_sd=1.5):
     """Decode workload: a state per (sequence, head) and ``steps`` single-token inputs.
 
     Returns (state0 [n,H,dk,dv] fp32, q,k [steps,n,H,dk], v [steps,n,H,dv], log_alpha [steps,n,H,dk],
-    beta [steps,n,H]); same distributions as the prefill recipe with (mu, sd) = (0, 1.5).
+    beta [steps,n,H]); same distributions as the prefill recipe, (mu, sd) = (0, 1.5) unless given.
     """
     gen = torch.Generator(device)
     gen.manual_seed(seed)
@@ -118,7 +118,7 @@ def make_decode_inputs(n, H, dk, dv, *, dtype=torch.bfloat16, device="cpu", seed
     k = (k / k.norm(dim=-1, keepdim=True).clamp_min(1e-12)).to(dtype)
     v = _draw((steps, n, H, dv), gen, device).to(dtype)
     beta = torch.sigmoid(_draw((steps, n, H), gen, device))
-    la = -5.0 * torch.sigmoid(_draw((steps, n, H, dk), gen, device, std=1.5))
+    la = -5.0 * torch.sigmoid(_draw((steps, n, H, dk), gen, device, mean=alpha_mu, std=alpha_sd))
     state0 = _draw((n, H, dk, dv), gen, device, std=state_sd)
     return state0, q, k, v, la, beta
 

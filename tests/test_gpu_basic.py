@@ -59,10 +59,13 @@ def test_bounded_wait_times_out_cleanly():
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (128, 64), (64, 64)])
-def test_decode_steps_match_oracle(dtype, dk, dv):
-    n, H, steps = 5, 3, 6
-    s0, q, k, v, la, b = synth.make_decode_inputs(n, H, dk, dv, dtype=dtype, device=DEV, seed=3, steps=steps)
+@pytest.mark.parametrize("dk,dv,steps,mu", [(128, 128, 6, 0.0), (64, 128, 6, 0.0), (128, 64, 6, 0.0), (64, 64, 6, 0.0),
+                                            (128, 128, 48, -6.0)])
+def test_decode_steps_match_oracle(dtype, dk, dv, steps, mu):
+    # mu = -6: about -0.012 per step, so the initial state still matters after all the steps
+    n, H = 5, 3
+    s0, q, k, v, la, b = synth.make_decode_inputs(n, H, dk, dv, dtype=dtype, device=DEV, seed=3, steps=steps,
+                                                  alpha_mu=mu, alpha_sd=1.5 if mu == 0.0 else 0.5)
     state = s0.clone()
     outs = []
     for t in range(steps):
@@ -191,6 +194,16 @@ def test_chunk_f32_pr1_workload():
 def test_chunk_f32_varlen_ragged(dk, dv):
     lengths = [1, 63, 64, 65, 200, 0, 130, 16]
     inp = synth.make_inputs(lengths, 2, dk, dv, dtype=torch.float32, device=DEV, seed=5, with_state0=True)
+    outs = _run_chunk(inp, torch.float32, ckpt_stride=64, transition=True)
+    _check_chunk(inp, torch.float32, outs, range(len(lengths)), [0, 1], ckpt_stride=64, transition=True)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128)])
+def test_chunk_f32_slow_decay_carries_state(dk, dv):
+    # about -0.012 per step: the state is carried across every chunk of the sequences
+    lengths = [300, 200]
+    inp = synth.make_inputs(lengths, 2, dk, dv, dtype=torch.float32, device=DEV, seed=12, alpha_mu=-6.0,
+                            alpha_sd=0.5, with_state0=True)
     outs = _run_chunk(inp, torch.float32, ckpt_stride=64, transition=True)
     _check_chunk(inp, torch.float32, outs, range(len(lengths)), [0, 1], ckpt_stride=64, transition=True)
 

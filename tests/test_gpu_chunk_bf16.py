@@ -50,6 +50,18 @@ def test_bf16_decay_near_and_at_the_floor(mu, sd):
     _check_chunk(inp, BF, outs, range(len(lengths)), [0, 1], ckpt_stride=128, transition=True)
 
 
+@pytest.mark.parametrize("mu", [-6.0, -9.0])
+def test_bf16_slow_decay_carries_state(mu):
+    # log_alpha = -5 sigmoid(N(mu, 0.5)): about -0.012 (mu = -6) or -0.0006 (mu = -9) per step, so the state
+    # is carried across many chunks (close to linear attention with the delta rule) and every output
+    # depends on the inter-chunk pass, not only those of a chunk's first tokens
+    lengths = [700, 129, 1000]
+    inp = synth.make_inputs(lengths, 2, 128, 128, dtype=BF, device=DEV, seed=11, alpha_mu=mu, alpha_sd=0.5,
+                            with_state0=True)
+    outs = _run_chunk(inp, BF, ckpt_stride=128, transition=True)
+    _check_chunk(inp, BF, outs, range(len(lengths)), [0, 1], ckpt_stride=128, transition=True)
+
+
 def test_bf16_floor_clamps_below_floor_decay():
     # log_alpha far below the floor (-50, -inf) must behave exactly like ln 0.0067
     lengths = [200]
