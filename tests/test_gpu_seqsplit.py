@@ -33,10 +33,14 @@ def _plain(f, init):
     return o, fs[0]
 
 
-def test_four_segments_match_oracle_and_unsplit_run():
+@pytest.mark.parametrize("mu", [0.0, -6.0])
+def test_four_segments_match_oracle_and_unsplit_run(mu):
+    # mu = -6 (about -0.012 per step): the segments' transitions are far from zero, so every start state
+    # depends on the composition of all earlier segments
     H, D = 4, 128
     seg = [1000, 1536, 1217, 1343]
-    inp = synth.make_inputs([sum(seg)], H, D, D, dtype=BF, device=DEV, seed=4, with_state0=True)
+    inp = synth.make_inputs([sum(seg)], H, D, D, dtype=BF, device=DEV, seed=4, with_state0=True, alpha_mu=mu,
+                            alpha_sd=1.5 if mu == 0.0 else 0.5)
     f = [inp.q, inp.k, inp.v, inp.log_alpha, inp.beta]
     init = inp.state0[0]
     bounds = np.cumsum([0] + seg).tolist()
