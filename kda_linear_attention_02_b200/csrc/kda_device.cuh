@@ -102,13 +102,6 @@ __device__ __forceinline__ void bulk_s2g(void* dst, const void* src_smem, uint32
 }
 // Warm L2 with the line holding p (no data returned; nothing waits on it).
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
-// 4-byte asynchronous copy global -> shared in the calling thread's cp.async group; src_bytes = 0 writes
-// zeros and reads nothing.  cp_async_wait_all makes the thread's copies visible to that thread.
-__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst_smem)), "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -128,13 +121,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst_smem, const CUtensorMap* m
         "[%5];" ::"r"(smem_u32(dst_smem)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
-}
-// 3D tensor TMA prefetch of a box into L2 (no shared memory written, nothing to wait for).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
 }
 // Loads of data read exactly once: bypass L1 allocation.
 __device__ __forceinline__ float2 ld_once_f2(const float* p) {
