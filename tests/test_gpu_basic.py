@@ -82,10 +82,11 @@ def test_decode_steps_match_oracle(dtype, dk, dv, steps, mu):
             assert_close(f32np(state[i, h]), r["state"], dtype, f"decode state ({i},{h})")
 
 
-@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128)])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (128, 64), (64, 128), (64, 64)])
 def test_segment_compose_matches_oracle(dk, dv):
+    # sequences of 3, 1, 0, 5 and 12 segments: the last one alternates the kernels' double buffers many times
     H = 3
-    nseg = [3, 1, 0, 5]
+    nseg = [3, 1, 0, 5, 12]
     S = sum(nseg)
     g = torch.Generator(DEV).manual_seed(11)
     M = torch.randn(S, H, dk, dk, device=DEV, generator=g) / (dk ** 0.5)
