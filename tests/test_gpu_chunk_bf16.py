@@ -33,6 +33,16 @@ def test_bf16_varlen_ragged(dv):
     _check_chunk(inp, BF, outs, range(len(lengths)), [0, 1, 2], ckpt_stride=64, transition=True)
 
 
+@pytest.mark.parametrize("n_seqs,H,dv", [(8, 8, 128), (16, 8, 64)])
+def test_bf16_64_column_state_slices(n_seqs, H, dv):
+    # 64 chains at dv = 128, or 128 chains at dv = 64: the state pass runs 64-column slices (the bench
+    # workload runs 128-column slices, the small ragged batches 32-column ones)
+    lengths = [97, 64, 130, 1, 200, 65, 150, 33] * (n_seqs // 8)
+    inp = synth.make_inputs(lengths, H, 128, dv, dtype=BF, device=DEV, seed=13, with_state0=True)
+    outs = _run_chunk(inp, BF, ckpt_stride=64, transition=True)
+    _check_chunk(inp, BF, outs, range(0, n_seqs, 3), [0, H - 1], ckpt_stride=64, transition=True)
+
+
 def test_bf16_zero_state_single_sequence():
     inp = synth.make_inputs([256], 2, 128, 128, dtype=BF, device=DEV, seed=0)
     outs = _run_chunk(inp, BF, init=False)
