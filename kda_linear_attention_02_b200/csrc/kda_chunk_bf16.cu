@@ -740,18 +740,21 @@ struct SCfg {
     static constexpr int NEW = DVS >= 64 ? 16 : 8;        // epilogue warps (NEW/4 share each TMEM lane quarter)
     static constexpr int NCW = DVS * 4 / NEW;              // state columns per epilogue warp (>= 16)
     static constexpr int NT = 32 * (NEW + 2);              // + producer warp + MMA warp
-    static constexpr bool MN = DVS >= 64;                  // S and U' staged MN-major (row = channel / token)
+    // S and U' are staged MN-major (row = channel / token) in blocks of 64 columns; a 32-column slice
+    // fills half of one block (a product with N = 32 reads just those columns)
+    static constexpr int DVA = DVS >= 64 ? DVS : 64;
+    static constexpr bool TMA_O = DVS >= 64;               // whole 64-column O tiles leave by tensor stores
     static constexpr int NST = DVS == 32 ? 3 : 2;
     static constexpr uint32_t U_BYTES = DVS >= 64 ? DVS * 128 : 8192;   // whole 64-column atoms of U
     // stage: the packet's parts for this slice (Aqk right after Kdec^T, as in the packet)
     static constexpr uint32_t AW = 0, KD = 32768, AQ = 49152, U = 57344, G = U + U_BYTES;
     static constexpr uint32_t STAGE = ((G + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SOP = NST * STAGE;      // S as B operand (N = DVS, K = 128)
-    static constexpr uint32_t UOP = SOP + DVS * 256;  // U' as B operand (N = DVS, K = 64)
+    static constexpr uint32_t UOP = SOP + DVA * 256;  // U' as B operand (N = DVS, K = 64)
     // O tile staging for the tensor store, [DVS/64][64 tokens][128 B] with the 128B swizzle (slices of whole
     // 64-column atoms only; narrower slices store O from registers)
-    static constexpr uint32_t OST = UOP + DVS * 128;
-    static constexpr uint32_t BYTES = OST + (MN ? DVS * 128 : 0);
+    static constexpr uint32_t OST = UOP + DVA * 128;
+    static constexpr uint32_t BYTES = OST + (TMA_O ? DVS * 128 : 0);
     // TMEM: D1 double-buffered at columns [0, DVS) and [2 DVS, 3 DVS), D2 at [DVS, 2 DVS)
     static constexpr uint32_t S_LBO = 128 * 128;      // MN-major: 64 columns x 128 K rows per block
     static constexpr uint32_t U_LBO = 64 * 128;       // MN-major: 64 columns x 64 K rows per block
@@ -844,10 +847,10 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
     } else if (w == NEW + 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, DVS, false, C::MN);
+            const uint32_t idesc = idesc_bf16(128, DVS, false, true);
             const uint32_t sop = smem_u32(sm + C::SOP), uop = smem_u32(sm + C::UOP);
             auto ubdesc = [&](int ks) -> uint64_t {   // U' as the B operand (K = 64 tokens)
-                return C::MN ? sdesc_mn_sw128(uop + ks * 2048, C::U_LBO) : sdesc_k_sw128(uop + ks * 32);
+                return sdesc_mn_sw128(uop + ks * 2048, C::U_LBO);
             };
             for (int ci = 0; ci < nch; ++ci) {
                 const int st = ci % NST;
@@ -860,8 +863,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
-                    const uint64_t bdesc = C::MN ? sdesc_mn_sw128(sop + ks * 2048, C::S_LBO)
-                                                 : sdesc_k_sw128(sop + ka * (DVS * 128) + kb);
+                    const uint64_t bdesc = sdesc_mn_sw128(sop + ks * 2048, C::S_LBO);
                     umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc, ks > 0);
                 }
                 umma_commit(&d1_full);
@@ -906,19 +908,12 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         }
         // S (and later U') as a B operand: MN-major rows are written 8 columns at a time
         auto write_sop = [&]() {
-            if constexpr (C::MN) {
 #pragma unroll
-                for (int j = 0; j < NCW; j += 8) {
-                    float f8[8];
+            for (int j = 0; j < NCW; j += 8) {
+                float f8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) f8[e] = S[j + e];
-                    *reinterpret_cast<uint4*>(sm + C::SOP + sw128_mn_offset(jw + j, i, C::S_LBO)) = pack8(f8);
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < NCW; ++j)
-                    *reinterpret_cast<__nv_bfloat16*>(sm + C::SOP + sw128_offset(jw + j, i, DVS)) =
-                        __float2bfloat16_rn(S[j]);
+                for (int e = 0; e < 8; ++e) f8[e] = S[j + e];
+                *reinterpret_cast<uint4*>(sm + C::SOP + sw128_mn_offset(jw + j, i, C::S_LBO)) = pack8(f8);
             }
         };
         write_sop();
@@ -934,7 +929,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             const int c = static_cast<int>(lo + ci - ch_lo);
             const long long rem = seq_len - static_cast<long long>(c) * 64;
             const int n = rem < 64 ? static_cast<int>(rem) : 64;
-            const bool full_tma = C::MN && !trans && n == 64;
+            const bool full_tma = C::TMA_O && !trans && n == 64;
             if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
             if (qw < 2) {   // U' = U - W S: U row i from the stage, -W S from D1 rows 0..63
                 uint4 ur[NCW / 8];
@@ -959,14 +954,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                     unpack8(ur[e8], u8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) u8[e] += vv[8 * e8 + e];
-                    if constexpr (C::MN) {
-                        *reinterpret_cast<uint4*>(sm + C::UOP + sw128_mn_offset(8 * cc, i, C::U_LBO)) = pack8(u8);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            *reinterpret_cast<__nv_bfloat16*>(sm + C::UOP + sw128_offset(8 * cc + e, i, DVS)) =
-                                __float2bfloat16_rn(u8[e]);
-                    }
+                    *reinterpret_cast<uint4*>(sm + C::UOP + sw128_mn_offset(8 * cc, i, C::U_LBO)) = pack8(u8);
                 }
                 tc_fence_before();
                 fence_proxy_async_smem();
