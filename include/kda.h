@@ -363,7 +363,8 @@ KDA_API kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_
  *  kda_selftest_umma: one 128 x n x 64 bf16 tcgen05 product D = A B^T through the same shared-memory
  *  descriptors, TMEM allocation and load path the chunk kernels use. a [128,64], b [n,64] bf16
  *  row-major (device), d [128,n] fp32 (device); n in {16, 32, ..., 256}.  flags: KDA_SELFTEST_B_MN_MAJOR
- *  stages B MN-major instead of K-major (then n must be a multiple of 64); KDA_SELFTEST_A_TMEM reads A
+ *  stages B MN-major in 64-column blocks instead of K-major (then n must be a multiple of 32; a last
+ *  32-column part fills half a block, as the state pass's 32-column slices do); KDA_SELFTEST_A_TMEM reads A
  *  from tensor memory (row m in lane m, two bf16 per 32-bit column), the operand form the segment
  *  compose uses, instead of shared memory.  Other flag bits: KDA_ERR_ARG.
  */

@@ -468,7 +468,7 @@ kda_status_t kda_selftest_mma_rate(int n, int k, int b_mn_major, int reps, float
 kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, int flags, kda_stream_t stream) {
     if (!a || !b || !d || n < 16 || n > 256 || (n % 16) != 0) return KDA_ERR_ARG;
     if (flags < 0 || flags > (KDA_SELFTEST_B_MN_MAJOR | KDA_SELFTEST_A_TMEM)) return KDA_ERR_ARG;
-    if ((flags & KDA_SELFTEST_B_MN_MAJOR) && (n % 64) != 0) return KDA_ERR_ARG;
+    if ((flags & KDA_SELFTEST_B_MN_MAJOR) && (n % 32) != 0) return KDA_ERR_ARG;
     if (!aligned16(a) || !aligned16(b) || !aligned16(d)) return KDA_ERR_ALIGN;
     int* st = status_ptr();
     if (!st) return KDA_ERR_CUDA;

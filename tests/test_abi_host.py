@@ -127,7 +127,7 @@ def test_decode_and_compose_host_argument_errors(lib):
     assert lib.kda_segment_compose(vp(0x1000), vp(0x2000), vp(0x4000), None, 1, 1, 1, 128, 80, vp(0x3000), None,
                                    None) == -3
     assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 20, 0, None) == -1
-    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 32, 1, None) == -1
+    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 48, 1, None) == -1   # MN-major: n % 32
     assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 64, 4, None) == -1   # unknown flag bit
     # tensor-core rate diagnostic: shape limits and the cycles buffer are checked before any launch
     assert lib.kda_selftest_mma_rate(8, 64, 0, 16, vp(0x1000), 1, None) == -1       # n below 16

@@ -21,7 +21,7 @@ def _clear_status():
 
 
 @pytest.mark.parametrize("n,mn,at", [(16, False, False), (64, False, False), (128, False, False), (256, False, False),
-                                     (64, True, False), (128, True, False),
+                                     (32, True, False), (64, True, False), (96, True, False), (128, True, False),
                                      (64, False, True), (128, True, True), (256, False, True)])
 def test_selftest_umma_matches_matmul(n, mn, at):
     # at: A read from tensor memory (row m in lane m, two bf16 per 32-bit column), as the compose issues it
