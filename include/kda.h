@@ -366,20 +366,23 @@ KDA_API kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_
  *  stages B MN-major in 64-column blocks instead of K-major (then n must be a multiple of 32; a last
  *  32-column part fills half a block, as the state pass's 32-column slices do); KDA_SELFTEST_A_TMEM reads A
  *  from tensor memory (row m in lane m, two bf16 per 32-bit column), the operand form the segment
- *  compose uses, instead of shared memory.  Other flag bits: KDA_ERR_ARG.
+ *  compose uses, instead of shared memory; KDA_SELFTEST_A_MN_MAJOR stages A in shared memory MN-major
+ *  (two 64-row blocks).  A_TMEM together with A_MN_MAJOR, or any other flag bit: KDA_ERR_ARG.
  */
 #define KDA_SELFTEST_B_MN_MAJOR 1
 #define KDA_SELFTEST_A_TMEM 2
+#define KDA_SELFTEST_A_MN_MAJOR 4
 /*
  *  kda_selftest_mma_rate: the tensor-core rate of one product shape as the chunk kernels issue it:
- *  128 x n x k bf16 (k in {64, 128}, n in {16, ..., 256}; B K-major, or MN-major when b_mn_major, then
- *  n a multiple of 64), fp32 accumulator in TMEM.  `grid` CTAs (one per SM when grid <= the SM count),
+ *  128 x n x k bf16 (k in {64, 128}, n in {16, ..., 256}), fp32 accumulator in TMEM.  majors:
+ *  KDA_SELFTEST_B_MN_MAJOR stages B MN-major (then n a multiple of 64), KDA_SELFTEST_A_MN_MAJOR stages
+ *  A MN-major; both K-major when 0; any other bit: KDA_ERR_ARG.  `grid` CTAs (one per SM when grid <= the SM count),
  *  each with one issuing thread, time `reps` products back to back and then `reps` products each
  *  waited for before the next, with the SM clock.  cycles (device, [grid][2] fp32) receives the SM
  *  cycles per product in the two modes (-1 if a bounded wait ran out).  FLOP per cycle per SM of a
  *  mode is 2 * 128 * n * k / cycles.
  */
-KDA_API kda_status_t kda_selftest_mma_rate(int n, int k, int b_mn_major, int reps, float* cycles, int grid,
+KDA_API kda_status_t kda_selftest_mma_rate(int n, int k, int majors, int reps, float* cycles, int grid,
                                            kda_stream_t stream);
 KDA_API kda_status_t kda_selftest_wait_timeout(int limit_us, kda_stream_t stream);
 KDA_API kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, int flags,

@@ -740,6 +740,12 @@ struct SCfg {
     static constexpr int NEW = DVS >= 64 ? 16 : 8;        // epilogue warps (NEW/4 share each TMEM lane quarter)
     static constexpr int NCW = DVS * 4 / NEW;              // state columns per epilogue warp (>= 16)
     static constexpr int NT = 32 * (NEW + 2);              // + producer warp + MMA warp
+    // Full 128-column slices run products 1 and 3 transposed, with the state columns on the M side:
+    // D1^T = S^T [-W; Q gamma]^T (A = S, MN-major) and O^T += U'^T Aqk^T, so that D1^T's TMEM lanes are
+    // state columns; warps 0..7 then form U' and warps 8..15 read O, 32 tokens per warp in the
+    // fragment layout of 16-lane TMEM loads and 8 x 8 matrix loads and stores.  Narrower slices cannot
+    // fill M = 128 and keep D1 = [-W; Q gamma] S.
+    static constexpr bool TR = DVS == 128;
     // S and U' are staged MN-major (row = channel / token) in blocks of 64 columns; a 32-column slice
     // fills half of one block (a product with N = 32 reads just those columns)
     static constexpr int DVA = DVS >= 64 ? DVS : 64;
@@ -808,7 +814,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         mbar_init(&d2_full, 1);
         mbar_init(&o_full, 1);
         mbar_init(&s_ready, NEW);
-        mbar_init(&up_ready, NEW / 2);   // only the warps that produce U' (TMEM lanes 0..63)
+        mbar_init(&up_ready, NEW / 2);   // the warps that produce U'
         fence_barrier_init();
     }
     if (w == 0) {
@@ -858,29 +864,56 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
                 tc_fence_after();
                 const uint32_t sb = smem_u32(sm + st * C::STAGE);
-                // D1 = [-W; Q gamma] S   (M = 128, N = DVS, K = 128).  D1[ci] was last read as chunk ci - 2's O,
-                // before the O warps' s_ready arrival for chunk ci - 1.
+                if constexpr (C::TR) {
+                    // D1^T = S^T [-W; Q gamma]^T   (M = 128 state columns, N = 128 tokens: -W rows, then Q gamma
+                    // rows; K = 128 channels), A = S MN-major, B = the packet's K-major [-W; Q gamma]
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
-                    const uint64_t bdesc = sdesc_mn_sw128(sop + ks * 2048, C::S_LBO);
-                    umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc, ks > 0);
-                }
-                umma_commit(&d1_full);
-                if (!mbar_wait(&up_ready, ci & 1, status)) break;
-                tc_fence_after();
-                // D2 = Kdec^T U'   (M = 128, N = DVS, K = 64)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), ubdesc(ks), idesc, ks > 0);
-                umma_commit(&d2_full);
-                if (!trans) {
-                    // D1 rows 64..127 += Aqk U' (O = Q gamma S + Aqk U'): the A operand starts 64 rows into Kdec^T,
-                    // so its rows 64..127 are Aqk; what it adds to rows 0..63 (U', already read) is never used
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_f16(tm + C::d1col(ci), sdesc_mn_sw128(sop + ks * 2048, C::S_LBO),
+                                 sdesc_k_sw128(sb + C::AW + (ks >> 2) * 16384 + (ks & 3) * 32),
+                                 idesc_bf16(128, 128, false, false, true), ks > 0);
+                    umma_commit(&d1_full);
+                    if (!mbar_wait(&up_ready, ci & 1, status)) break;
+                    tc_fence_after();
+                    // D2 = Kdec^T U'   (M = 128 channels, N = 128 state columns, K = 64 tokens), B = U'^T K-major
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::KD + 8192 + ks * 32), ubdesc(ks), idesc, true);
-                    umma_commit(&o_full);
+                        umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), sdesc_k_sw128(uop + ks * 32),
+                                 idesc_bf16(128, DVS), ks > 0);
+                    umma_commit(&d2_full);
+                    if (!trans) {
+                        // O^T = (Q gamma S)^T + U'^T Aqk^T: D1^T columns 64..127 (M = 128, N = 64, K = 64 tokens)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            umma_f16(tm + C::d1col(ci) + 64, sdesc_k_sw128(uop + ks * 32),
+                                     sdesc_k_sw128(sb + C::AQ + ks * 32), idesc_bf16(128, 64), true);
+                        umma_commit(&o_full);
+                    }
+                } else {
+                    // D1 = [-W; Q gamma] S   (M = 128, N = DVS, K = 128).  D1[ci] was last read as chunk ci - 2's O,
+                    // before the O warps' s_ready arrival for chunk ci - 1.
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t ka = ks >> 2, kb = (ks & 3) * 32;
+                        const uint64_t bdesc = sdesc_mn_sw128(sop + ks * 2048, C::S_LBO);
+                        umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::AW + ka * 16384 + kb), bdesc, idesc, ks > 0);
+                    }
+                    umma_commit(&d1_full);
+                    if (!mbar_wait(&up_ready, ci & 1, status)) break;
+                    tc_fence_after();
+                    // D2 = Kdec^T U'   (M = 128, N = DVS, K = 64)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), ubdesc(ks), idesc, ks > 0);
+                    umma_commit(&d2_full);
+                    if (!trans) {
+                        // D1 rows 64..127 += Aqk U' (O = Q gamma S + Aqk U'): the A operand starts 64 rows into Kdec^T,
+                        // so its rows 64..127 are Aqk; what it adds to rows 0..63 (U', already read) is never used
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            umma_f16(tm + C::d1col(ci), sdesc_k_sw128(sb + C::KD + 8192 + ks * 32), ubdesc(ks), idesc, true);
+                        umma_commit(&o_full);
+                    }
                 }
                 umma_commit(&empty[st]);
             }
@@ -888,7 +921,10 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
     } else {
         // ---------------- epilogue warps: lane quarter qw, columns [jw, jw + NCW) of the slice
         const int qw = w & 3, jw = (w >> 2) * NCW;
-        const int i = 32 * qw + lane;   // TMEM lane: row of D1 (token row / P row), channel of D2 and S
+        // TMEM lane: channel of D2 and S; row of D1 (token row), or with transposed products the slice column
+        // of D1^T, whose tokens [tk0, tk0 + 32) this warp takes (U' for warps 0..7, O for warps 8..15)
+        const int i = 32 * qw + lane;
+        const int tk0 = 32 * ((w >> 2) & 1);
         const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
         float S[NCW];
         {
@@ -922,7 +958,14 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         if (lane == 0) mbar_arrive(&s_ready);
         const int ucol = (DVS >= 64 ? 0 : (j0 & 63)) + jw;   // this warp's first column inside the stage's U atoms
         // full chunks of whole-atom slices leave through a TMA tensor store of the O tile staged in OST
-        const bool o_issuer = (w == 2) && lane == 0;
+        const bool o_issuer = (w == (C::TR ? NEW / 2 : 2)) && lane == 0;
+        // checkpoints: one after every cpe-th chunk of the sequence (ckpt_stride is a multiple of 64), counted
+        // down without divisions in the loop; ck_slot is the next one's slot
+        const int cpe = (!trans && ckpt_stride > 0 && checkpoints) ? ckpt_stride / 64 : 0;
+        const int c_first = static_cast<int>(lo - ch_lo);
+        int ck_wait = cpe > 0 ? cpe - c_first % cpe : 0;
+        long long ck_slot = cpe > 0 ? static_cast<long long>(ckpt_cu[seq]) + c_first / cpe : 0;
+        const long long ck_end = cpe > 0 ? static_cast<long long>(ckpt_cu[seq + 1]) : 0;
         for (int ci = 0; ci < nch; ++ci) {
             const int st = ci % NST;
             const uint8_t* sb = sm + st * C::STAGE;
@@ -931,7 +974,56 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             const int n = rem < 64 ? static_cast<int>(rem) : 64;
             const bool full_tma = C::TMA_O && !trans && n == 64;
             if (!mbar_wait(&full[st], (ci / NST) & 1, status)) break;
-            if (qw < 2) {   // U' = U - W S: U row i from the stage, -W S from D1 rows 0..63
+            if constexpr (C::TR) {
+                if (w < NEW / 2) {
+                    // U'^T = U^T - (W S)^T for state columns [32 qw, 32 qw + 32) and tokens [tk0, tk0 + 32), in the
+                    // fragment layout: token block tb, lane half hh and token half bb make 16 x 8 tiles, each two
+                    // 8 x 8 matrices (column half vh); U comes from the stage by transposing matrix loads, D1^T from
+                    // TMEM by 16-lane loads, and U'^T goes to row v of the K-major operand by matrix stores.
+                    const int mj = lane >> 3, mr = lane & 7;   // matrix j = 2 bb + vh, row mr: this lane's address
+                    uint32_t uf[2][2][4];
+#pragma unroll
+                    for (int tb = 0; tb < 2; ++tb)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            if (!trans) {
+                                const int v0 = 32 * qw + 16 * hh + 8 * (mj & 1), tok = tk0 + 16 * tb + 8 * (mj >> 1) + mr;
+                                ldsm_x4_trans(smem_u32(sb + C::U + (v0 >> 6) * 8192 + tok * 128 +
+                                                       ((((v0 & 63) >> 3) ^ (tok & 7)) << 4)),
+                                              uf[tb][hh]);
+                            } else {
+                                uf[tb][hh][0] = uf[tb][hh][1] = uf[tb][hh][2] = uf[tb][hh][3] = 0u;
+                            }
+                        }
+                    if (!mbar_wait(&d1_full, ci & 1, status)) break;
+                    tc_fence_after();
+                    float dv[32];
+#pragma unroll
+                    for (int tb = 0; tb < 2; ++tb) {
+                        tmem_ld_16x256b_x2(lane_base + C::d1col(ci) + tk0 + 16 * tb, dv + 16 * tb);
+                        tmem_ld_16x256b_x2(lane_base + (16u << 16) + C::d1col(ci) + tk0 + 16 * tb, dv + 16 * tb + 8);
+                    }
+                    tmem_wait_ld_regs<32>(dv);
+#pragma unroll
+                    for (int tb = 0; tb < 2; ++tb)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t pf[4];
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {   // m = 2 bb + vh
+                                const float2 u = bf2_to_f2(uf[tb][hh][m]);
+                                const int e = 16 * tb + 8 * hh + 4 * (m >> 1) + 2 * (m & 1);
+                                pf[m] = pack_bf16x2(u.x + dv[e], u.y + dv[e + 1]);
+                            }
+                            const int v = 32 * qw + 16 * hh + 8 * (mj & 1) + mr;
+                            stsm_x4(smem_u32(sm + C::UOP + v * 128 + (((((tk0 + 16 * tb) >> 3) + (mj >> 1)) ^ (v & 7)) << 4)), pf);
+                        }
+                    tc_fence_before();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&up_ready);
+                }
+            } else if (qw < 2) {   // U' = U - W S: U row i from the stage, -W S from D1 rows 0..63
                 uint4 ur[NCW / 8];
 #pragma unroll
                 for (int e8 = 0; e8 < NCW / 8; ++e8) {
@@ -983,7 +1075,63 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_ready);
-            if (qw >= 2 && !trans) {   // O = Q gamma S + Aqk U': D1 rows 64..127, read while the next product 1 runs
+            if (C::TR && !trans && w >= NEW / 2) {
+                // O^T: D1^T columns 64 + tk0 .. + 32, read while the next product 1 runs; matrix stores that
+                // transpose put O's token rows into OST, which leaves by tensor stores (whole chunks) or by
+                // 16-byte stores of its first n rows
+                if (!mbar_wait(&o_full, ci & 1, status)) break;
+                tc_fence_after();
+                float dv[32];
+#pragma unroll
+                for (int tb = 0; tb < 2; ++tb) {
+                    tmem_ld_16x256b_x2(lane_base + C::d1col(ci) + 64 + tk0 + 16 * tb, dv + 16 * tb);
+                    tmem_ld_16x256b_x2(lane_base + (16u << 16) + C::d1col(ci) + 64 + tk0 + 16 * tb, dv + 16 * tb + 8);
+                }
+                tmem_wait_ld_regs<32>(dv);
+                tc_fence_before();
+                uint32_t pf[2][2][4];
+#pragma unroll
+                for (int tb = 0; tb < 2; ++tb)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const int e = 16 * tb + 8 * hh + 4 * (m >> 1) + 2 * (m & 1);
+                            pf[tb][hh][m] = pack_bf16x2(dv[e], dv[e + 1]);
+                        }
+                if (o_issuer) bulk_wait_read0();   // the previous tile has left OST
+                named_bar_sync(2, 32 * NEW / 2);
+                {
+                    const int mj = lane >> 3, mr = lane & 7;
+#pragma unroll
+                    for (int tb = 0; tb < 2; ++tb)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int v0 = 32 * qw + 16 * hh + 8 * (mj & 1), tok = tk0 + 16 * tb + 8 * (mj >> 1) + mr;
+                            stsm_x4_trans(smem_u32(sm + C::OST + (v0 >> 6) * 8192 + tok * 128 +
+                                                   ((((v0 & 63) >> 3) ^ (tok & 7)) << 4)),
+                                          pf[tb][hh]);
+                        }
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, 32 * NEW / 2);   // every O warp has written its part of the tile
+                if (full_tma) {
+                    if (o_issuer) {
+#pragma unroll
+                        for (int b = 0; b < DVS / 64; ++b)
+                            tma_store_3d(&map_o, j0 + 64 * b, h, static_cast<int>(seq_tok0 + c * 64), sm + C::OST + b * 8192);
+                        bulk_commit();
+                    }
+                } else {   // a ragged last chunk: rows r < n, 16 bytes (8 columns) per store
+                    for (int e = t - 32 * NEW / 2; e < 64 * (DVS / 8); e += 32 * NEW / 2) {
+                        const int r = e / (DVS / 8), v0 = 8 * (e % (DVS / 8));
+                        if (r < n)
+                            *reinterpret_cast<uint4*>(o + (static_cast<size_t>(seq_tok0 + c * 64 + r) * H + h) * DV + j0 + v0) =
+                                *reinterpret_cast<const uint4*>(sm + C::OST + (v0 >> 6) * 8192 + r * 128 +
+                                                                ((((v0 & 63) >> 3) ^ (r & 7)) << 4));
+                    }
+                }
+            } else if (!C::TR && qw >= 2 && !trans) {   // O = Q gamma S + Aqk U': D1 rows 64..127, read while the next product 1 runs
                 if (!mbar_wait(&o_full, ci & 1, status)) break;
                 tc_fence_after();
                 float vv[NCW];
@@ -1026,13 +1174,12 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             }
             // the checkpoint leaves from registers after the next product has been released, so its
             // stores drain while product 1 of the next chunk runs
-            if (!trans && ckpt_stride > 0 && checkpoints && n == 64) {
-                const long long end = static_cast<long long>(c + 1) * 64;
-                if (end % ckpt_stride == 0) {
-                    const long long slot = ckpt_cu[seq] + end / ckpt_stride - 1;
-                    if (slot >= ckpt_cu[seq] && slot < ckpt_cu[seq + 1]) {
+            if (cpe > 0 && --ck_wait == 0) {   // chunk c ends at a multiple of ckpt_stride tokens
+                ck_wait = cpe;
+                if (n == 64) {
+                    if (ck_slot < ck_end) {
                         float4* dst = reinterpret_cast<float4*>(checkpoints +
-                                                                ((static_cast<size_t>(slot) * H + h) * kDK + i) * DV + j0 + jw);
+                                                                ((static_cast<size_t>(ck_slot) * H + h) * kDK + i) * DV + j0 + jw);
 #pragma unroll
                         for (int e = 0; e < NCW / 4; ++e)
                             dst[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
@@ -1040,6 +1187,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                         set_status(status, KDA_ERR_DEVICE_INPUT);
                     }
                 }
+                ++ck_slot;
             }
         }
         if (o_issuer) bulk_wait0();

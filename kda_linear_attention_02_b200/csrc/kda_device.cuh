@@ -246,6 +246,38 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
         : "r"(taddr));
 }
 
+// 16 lanes x 256 bit, twice along the columns: the accumulator fragment of a warp-level m16n8 product for
+// two blocks of 8 columns.  Thread t (g = t / 4, q = t % 4) gets, for block b (columns 8 b .. 8 b + 7 from the
+// address's column): r[4 b] = (lane g, column 2 q), r[4 b + 1] = (lane g, column 2 q + 1), r[4 b + 2] =
+// (lane g + 8, column 2 q), r[4 b + 3] = (lane g + 8, column 2 q + 1), lanes from the address's lane field.
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, float* r) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+                 : "r"(taddr));
+}
+
+// Four 8 x 8 matrices of 16-bit elements between shared memory and the fragment layout: lanes 8 j .. 8 j + 7
+// give the shared addresses of the eight 16-byte rows of matrix j, and r[j] of thread t holds the two
+// elements (row t / 4; columns 2 (t % 4), 2 (t % 4) + 1) of matrix j, the lower column in the low half.
+// The .trans forms exchange rows and columns between memory and the fragment.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t saddr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(saddr)
+                 : "memory");
+}
+__device__ __forceinline__ void stsm_x4(uint32_t saddr, const uint32_t (&r)[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+__device__ __forceinline__ void stsm_x4_trans(uint32_t saddr, const uint32_t (&r)[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+
 // Shared-memory matrix descriptor, K-major operand with the 128-byte swizzle: 8-row core groups of
 // 8 x 128 B (1024 B, SBO), rows 128 B apart, 16-byte chunks XOR-permuted by (row % 8).  The tile
 // base must be 1024-byte aligned; stepping K by 16 bf16 inside the 128-byte row adds 32 B to the
@@ -275,11 +307,13 @@ __device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo_
 }
 // Instruction descriptor: kind::f16 with A = B = bf16, D = fp32, shape M x N; A K-major, B K-major
 // unless b_mn (then MN-major).
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool negate_a = false, bool b_mn = false) {
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool negate_a = false, bool b_mn = false,
+                                                 bool a_mn = false) {
     return (1u << 4)                       // D format: f32
            | (1u << 7)                     // A format: bf16
            | (1u << 10)                    // B format: bf16
            | ((negate_a ? 1u : 0u) << 13)  // negate A
+           | ((a_mn ? 1u : 0u) << 15)      // A major-ness
            | ((b_mn ? 1u : 0u) << 16)      // B major-ness
            | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }

@@ -82,7 +82,7 @@ ChunkEvents* profile_slot();   // events for the current call, or null
 
 // Diagnostics.
 cudaError_t launch_selftest_wait(int limit_us, int* d_result, cudaStream_t s);
-cudaError_t launch_selftest_mma_rate(int n, int k, int b_mn, int reps, float* cycles, int grid, int* status,
+cudaError_t launch_selftest_mma_rate(int n, int k, int majors, int reps, float* cycles, int grid, int* status,
                                      cudaStream_t s);
 cudaError_t launch_selftest_umma(const void* a, const void* b, float* d, int n, int flags, int* status,
                                  cudaStream_t s);

@@ -1,6 +1,6 @@
 // kda_umma_selftest.cu -- diagnostics of the tcgen05 path the chunk kernels use, no KDA arithmetic:
-//  * one bf16 product through the same shared-memory descriptors (128-byte swizzle; B K-major or
-//    MN-major), TMEM allocation, commit and TMEM-load path: D[128, n] = A[128, 64] * B[n, 64]^T, with A
+//  * one bf16 product through the same shared-memory descriptors (128-byte swizzle; A and B each K-major
+//    or MN-major), TMEM allocation, commit and TMEM-load path: D[128, n] = A[128, 64] * B[n, 64]^T, with A
 //    from shared memory or from tensor memory (row m in lane m, two bf16 per 32-bit column);
 //  * the tensor-core rate of a product shape as the kernels issue it (M = 128 x N x K, one CTA per SM,
 //    timed with the SM clock): back to back, and one product at a time waited for before the next.
@@ -12,7 +12,7 @@ namespace kda {
 __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16* __restrict__ a,
                                                             const __nv_bfloat16* __restrict__ b,
                                                             float* __restrict__ d, int n, int flags, int* status) {
-    const int b_mn = flags & 1, a_tmem = flags & 2;
+    const int b_mn = flags & 1, a_tmem = flags & 2, a_mn = flags & 4;
     extern __shared__ __align__(1024) uint8_t raw[];
     uint8_t* base = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);   // stays a shared-memory pointer
     uint8_t* sA = base;                 // 128 rows x 128 B
@@ -21,13 +21,20 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
     __shared__ uint32_t tbase;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
 
-    // stage rows into the K-major 128B-swizzled layout: 16-byte chunk c of row r goes to chunk c ^ (r % 8)
-    for (int e = t; e < 128 * 8; e += 128) {
-        const int r = e >> 3, c = e & 7;
-        const uint4 x = reinterpret_cast<const uint4*>(a + r * 64)[c];
-        *reinterpret_cast<uint4*>(sA + sw128_offset(r, c * 8, 128)) = x;
-    }
     const uint32_t lbo = 8 * 1024;   // MN-major: 64 K rows = 8 atoms per 64-element MN block
+    if (a_mn) {   // two 64-row M blocks, each [64 k][128 B]
+        for (int e = t; e < 128 * 64; e += 128) {
+            const int r = e >> 6, k = e & 63;
+            *reinterpret_cast<__nv_bfloat16*>(sA + sw128_mn_offset(r, k, lbo)) = a[r * 64 + k];
+        }
+    } else {
+        // stage rows into the K-major 128B-swizzled layout: 16-byte chunk c of row r goes to chunk c ^ (r % 8)
+        for (int e = t; e < 128 * 8; e += 128) {
+            const int r = e >> 3, c = e & 7;
+            const uint4 x = reinterpret_cast<const uint4*>(a + r * 64)[c];
+            *reinterpret_cast<uint4*>(sA + sw128_offset(r, c * 8, 128)) = x;
+        }
+    }
     if (b_mn) {
         for (int e = t; e < n * 64; e += 128) {
             const int r = e >> 6, k = e & 63;
@@ -66,12 +73,14 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
         tc_fence_after();
     }
     if (t == 0) {
-        const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0);
+        const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0, a_mn != 0);
         for (int kk = 0; kk < 4; ++kk) {
             const uint64_t db = b_mn ? sdesc_mn_sw128(smem_u32(sB) + kk * 2048, lbo)
                                      : sdesc_k_sw128(smem_u32(sB) + kk * 32);
+            const uint64_t da = a_mn ? sdesc_mn_sw128(smem_u32(sA) + kk * 2048, lbo)
+                                     : sdesc_k_sw128(smem_u32(sA) + kk * 32);
             if (a_tmem) umma_f16_ts(tm, tm + 256 + kk * 8, db, idesc, kk > 0);
-            else umma_f16(tm, sdesc_k_sw128(smem_u32(sA) + kk * 32), db, idesc, kk > 0);
+            else umma_f16(tm, da, db, idesc, kk > 0);
         }
         umma_commit(&bar);
     }
@@ -94,11 +103,12 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
 // One CTA per SM; thread 0 times `reps` products of shape 128 x n x k (operands zero: only the timing
 // matters) issued back to back with one commit at the end, then `reps` products each committed and waited
 // for before the next.  cycles[2 * blockIdx.x + {0, 1}] = SM cycles per product in the two modes.
-__global__ void __launch_bounds__(128) selftest_mma_rate_kernel(int n, int k, int b_mn, int reps, float* cycles,
+__global__ void __launch_bounds__(128) selftest_mma_rate_kernel(int n, int k, int majors, int reps, float* cycles,
                                                                 int* status) {
+    const int b_mn = majors & 1, a_mn = majors & 4;
     extern __shared__ __align__(1024) uint8_t raw[];
     uint8_t* base = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
-    uint8_t* sA = base;                          // [k / 64 atoms][128 rows][128 B]
+    uint8_t* sA = base;                          // K-major [k / 64][128 rows][128 B] or MN-major [2][k][128 B]
     uint8_t* sB = base + (k / 64) * 16384;       // K-major [k / 64][n][128 B] or MN-major [n / 64][k][128 B]
     __shared__ __align__(8) uint64_t bar;
     __shared__ uint32_t tbase;
@@ -119,14 +129,15 @@ __global__ void __launch_bounds__(128) selftest_mma_rate_kernel(int n, int k, in
     tc_fence_after();
     const uint32_t tm = tbase;
     if (t == 0) {
-        const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0);
+        const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0, a_mn != 0);
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
         auto product = [&]() {
             for (int ks = 0; ks < k / 16; ++ks) {
-                const uint32_t ka = (ks >> 2) * 16384 + (ks & 3) * 32;
+                const uint64_t da = a_mn ? sdesc_mn_sw128(a0 + ks * 2048, static_cast<uint32_t>(k) * 128)
+                                         : sdesc_k_sw128(a0 + (ks >> 2) * 16384 + (ks & 3) * 32);
                 const uint64_t db = b_mn ? sdesc_mn_sw128(b0 + ks * 2048, static_cast<uint32_t>(k) * 128)
                                          : sdesc_k_sw128(b0 + (ks >> 2) * n * 128 + (ks & 3) * 32);
-                umma_f16(tm, sdesc_k_sw128(a0 + ka), db, idesc, ks > 0);
+                umma_f16(tm, da, db, idesc, ks > 0);
             }
         };
         uint32_t ph = 0;
@@ -156,12 +167,12 @@ __global__ void __launch_bounds__(128) selftest_mma_rate_kernel(int n, int k, in
     if (w == 0) tmem_dealloc(tm, 256);
 }
 
-cudaError_t launch_selftest_mma_rate(int n, int k, int b_mn, int reps, float* cycles, int grid, int* status,
+cudaError_t launch_selftest_mma_rate(int n, int k, int majors, int reps, float* cycles, int grid, int* status,
                                      cudaStream_t s) {
     const int smem = 1024 + (k / 64) * 16384 + n * k * 2;
     cudaError_t e = cudaFuncSetAttribute(selftest_mma_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    selftest_mma_rate_kernel<<<grid, 128, smem, s>>>(n, k, b_mn, reps, cycles, status);
+    selftest_mma_rate_kernel<<<grid, 128, smem, s>>>(n, k, majors, reps, cycles, status);
     return cudaGetLastError();
 }
 

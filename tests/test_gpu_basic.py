@@ -20,27 +20,32 @@ def _clear_status():
     assert kda.kda_get_device_status() == 0, "a kernel recorded an error in the status word"
 
 
-@pytest.mark.parametrize("n,mn,at", [(16, False, False), (64, False, False), (128, False, False), (256, False, False),
-                                     (32, True, False), (64, True, False), (96, True, False), (128, True, False),
-                                     (64, False, True), (128, True, True), (256, False, True)])
-def test_selftest_umma_matches_matmul(n, mn, at):
-    # at: A read from tensor memory (row m in lane m, two bf16 per 32-bit column), as the compose issues it
+@pytest.mark.parametrize("n,mn,at,amn", [(16, False, False, False), (64, False, False, False),
+                                         (128, False, False, False), (256, False, False, False),
+                                         (32, True, False, False), (64, True, False, False), (96, True, False, False),
+                                         (128, True, False, False), (64, False, True, False), (128, True, True, False),
+                                         (256, False, True, False), (64, False, False, True), (128, True, False, True),
+                                         (32, True, False, True)])
+def test_selftest_umma_matches_matmul(n, mn, at, amn):
+    # at: A read from tensor memory (row m in lane m, two bf16 per 32-bit column), as the compose issues it;
+    # amn: A staged MN-major in shared memory, as the state pass's transposed products take S
     g = torch.Generator(DEV).manual_seed(n)
     a = torch.randn(128, 64, device=DEV, generator=g).to(torch.bfloat16)
     b = torch.randn(n, 64, device=DEV, generator=g).to(torch.bfloat16)
     d = torch.full((128, n), float("nan"), device=DEV)
-    kda.kda_selftest_umma(a, b, d, b_mn_major=mn, a_tmem=at)
+    kda.kda_selftest_umma(a, b, d, b_mn_major=mn, a_tmem=at, a_mn_major=amn)
     ref = a.double().cpu() @ b.double().cpu().T
     np.testing.assert_allclose(d.cpu().numpy(), ref.numpy(), rtol=1e-4, atol=1e-4)
 
 
 
-@pytest.mark.parametrize("n,k,mn", [(160, 64, False), (64, 64, False), (128, 128, True)])
-def test_selftest_mma_rate_is_plausible(n, k, mn):
+@pytest.mark.parametrize("n,k,mn,amn", [(160, 64, False, False), (64, 64, False, False), (128, 128, True, False),
+                                        (64, 128, False, True)])
+def test_selftest_mma_rate_is_plausible(n, k, mn, amn):
     # one CTA per SM times the product shape; the rate must lie between a small fraction and about the
     # hardware's dense bf16 rate (8192 FLOP per cycle per SM), and products one at a time never beat
     # products back to back
-    cyc = kda.kda_selftest_mma_rate(n, k, b_mn_major=mn, reps=64)
+    cyc = kda.kda_selftest_mma_rate(n, k, b_mn_major=mn, a_mn_major=amn, reps=64)
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
     c = cyc.cpu()
