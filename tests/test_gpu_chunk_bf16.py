@@ -43,6 +43,29 @@ def test_bf16_64_column_state_slices(n_seqs, H, dv):
     _check_chunk(inp, BF, outs, range(0, n_seqs, 3), [0, H - 1], ckpt_stride=64, transition=True)
 
 
+def test_bf16_128_column_transposed_state_pass():
+    # 8 sequences x 16 heads = 128 chains: the state pass runs full 128-column slices with transposed
+    # products (state columns on the M side); ragged last chunks leave through the staged O tile's rows
+    lengths = [97, 64, 130, 1, 200, 65, 150, 33]
+    H = 16
+    inp = synth.make_inputs(lengths, H, 128, 128, dtype=BF, device=DEV, seed=21, with_state0=True)
+    outs = _run_chunk(inp, BF, ckpt_stride=64, transition=True)
+    _check_chunk(inp, BF, outs, range(0, 8, 3), [0, H - 1], ckpt_stride=64, transition=True)
+    # one sequence alone (16 chains) runs 32-column slices with D1 = [-W; Q gamma] S: every output element
+    # sums the same products in the same order, so the two forms agree bit for bit
+    o, fs, ck, ckcu, tr = outs
+    cu = inp.cu_seqlens.cpu().tolist()
+    for i in (2, 4):
+        a, b = cu[i], cu[i + 1]
+        one = synth.KDAInputs(inp.q[a:b].contiguous(), inp.k[a:b].contiguous(), inp.v[a:b].contiguous(),
+                              inp.log_alpha[a:b].contiguous(), inp.beta[a:b].contiguous(),
+                              synth.cu_from_lengths([b - a], DEV), inp.state0[i:i + 1].contiguous())
+        o1, fs1, ck1, _, tr1 = _run_chunk(one, BF, ckpt_stride=64, transition=True)
+        assert torch.equal(o1, o[a:b]) and torch.equal(fs1[0], fs[i]) and torch.equal(tr1[0], tr[i])
+        c0 = int(ckcu[i])
+        assert torch.equal(ck1[: (b - a) // 64], ck[c0:c0 + (b - a) // 64])
+
+
 def test_bf16_zero_state_single_sequence():
     inp = synth.make_inputs([256], 2, 128, 128, dtype=BF, device=DEV, seed=0)
     outs = _run_chunk(inp, BF, init=False)
