@@ -367,16 +367,20 @@ KDA_API kda_status_t kda_profile_end(float* ms_index, float* ms_prep, float* ms_
  *  32-column part fills half a block, as the state pass's 32-column slices do); KDA_SELFTEST_A_TMEM reads A
  *  from tensor memory (row m in lane m, two bf16 per 32-bit column), the operand form the segment
  *  compose uses, instead of shared memory; KDA_SELFTEST_A_MN_MAJOR stages A in shared memory MN-major
- *  (two 64-row blocks).  A_TMEM together with A_MN_MAJOR, or any other flag bit: KDA_ERR_ARG.
+ *  (two 64-row blocks); KDA_SELFTEST_M64 issues the product with M = 64 (rows 0..63 of A), and d then
+ *  receives all 128 TMEM lanes of the accumulator as the hardware placed them.  A_TMEM together with
+ *  A_MN_MAJOR or M64, or any other flag bit: KDA_ERR_ARG.
  */
 #define KDA_SELFTEST_B_MN_MAJOR 1
 #define KDA_SELFTEST_A_TMEM 2
 #define KDA_SELFTEST_A_MN_MAJOR 4
+#define KDA_SELFTEST_M64 8
 /*
  *  kda_selftest_mma_rate: the tensor-core rate of one product shape as the chunk kernels issue it:
  *  128 x n x k bf16 (k in {64, 128}, n in {16, ..., 256}), fp32 accumulator in TMEM.  majors:
  *  KDA_SELFTEST_B_MN_MAJOR stages B MN-major (then n a multiple of 64), KDA_SELFTEST_A_MN_MAJOR stages
- *  A MN-major; both K-major when 0; any other bit: KDA_ERR_ARG.  `grid` CTAs (one per SM when grid <= the SM count),
+ *  A MN-major; both K-major when 0; KDA_SELFTEST_M64 times M = 64 instead of 128; any other bit:
+ *  KDA_ERR_ARG.  `grid` CTAs (one per SM when grid <= the SM count),
  *  each with one issuing thread, time `reps` products back to back and then `reps` products each
  *  waited for before the next, with the SM clock.  cycles (device, [grid][2] fp32) receives the SM
  *  cycles per product in the two modes (-1 if a bounded wait ran out).  FLOP per cycle per SM of a

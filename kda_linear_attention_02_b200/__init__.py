@@ -471,14 +471,15 @@ def kda_selftest_wait_timeout(limit_us: int = 2000, stream=None) -> int:
     return int(_load().kda_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
-def kda_selftest_mma_rate(n, k, *, b_mn_major=False, a_mn_major=False, reps=256, grid=None, stream=None):
+def kda_selftest_mma_rate(n, k, *, b_mn_major=False, a_mn_major=False, m64=False, reps=256, grid=None, stream=None):
     """SM cycles per 128 x n x k bf16 tensor-core product, back to back and one at a time
     (C: kda_selftest_mma_rate): a float32 tensor [grid, 2] on the current device."""
     dev = torch.device("cuda", torch.cuda.current_device())
     if grid is None:
         grid = torch.cuda.get_device_properties(dev).multi_processor_count
     cyc = torch.empty(grid, 2, dtype=torch.float32, device=dev)
-    majors = (KDA_SELFTEST_B_MN_MAJOR if b_mn_major else 0) | (KDA_SELFTEST_A_MN_MAJOR if a_mn_major else 0)
+    majors = ((KDA_SELFTEST_B_MN_MAJOR if b_mn_major else 0) | (KDA_SELFTEST_A_MN_MAJOR if a_mn_major else 0) |
+              (KDA_SELFTEST_M64 if m64 else 0))
     _check(_load().kda_selftest_mma_rate(int(n), int(k), majors, int(reps), _p(cyc), int(grid),
                                          _stream(stream)), "kda_selftest_mma_rate")
     return cyc
@@ -487,15 +488,16 @@ def kda_selftest_mma_rate(n, k, *, b_mn_major=False, a_mn_major=False, reps=256,
 KDA_SELFTEST_B_MN_MAJOR = 1
 KDA_SELFTEST_A_TMEM = 2
 KDA_SELFTEST_A_MN_MAJOR = 4
+KDA_SELFTEST_M64 = 8
 
 
-def kda_selftest_umma(a, b, d, *, b_mn_major=False, a_tmem=False, a_mn_major=False, stream=None):
+def kda_selftest_umma(a, b, d, *, b_mn_major=False, a_tmem=False, a_mn_major=False, m64=False, stream=None):
     n = b.shape[0]
     _need(a, "a", (128, 64), torch.bfloat16)
     _need(b, "b", (n, 64), torch.bfloat16, a.device)
     _need(d, "d", (128, n), torch.float32, a.device)
     flags = ((KDA_SELFTEST_B_MN_MAJOR if b_mn_major else 0) | (KDA_SELFTEST_A_TMEM if a_tmem else 0) |
-             (KDA_SELFTEST_A_MN_MAJOR if a_mn_major else 0))
+             (KDA_SELFTEST_A_MN_MAJOR if a_mn_major else 0) | (KDA_SELFTEST_M64 if m64 else 0))
     _check(_load().kda_selftest_umma(_p(a), _p(b), _p(d), n, flags, _stream(stream)), "kda_selftest_umma")
     return d
 

@@ -457,7 +457,7 @@ kda_status_t kda_selftest_mma_rate(int n, int k, int majors, int reps, float* cy
     if (n < 16 || n > 256 || (n % 16) != 0 || (k != 64 && k != 128) || reps <= 0 || reps > (1 << 20) || grid <= 0 ||
         !cycles)
         return KDA_ERR_ARG;
-    if ((majors & ~(KDA_SELFTEST_B_MN_MAJOR | KDA_SELFTEST_A_MN_MAJOR)) != 0) return KDA_ERR_ARG;
+    if ((majors & ~(KDA_SELFTEST_B_MN_MAJOR | KDA_SELFTEST_A_MN_MAJOR | KDA_SELFTEST_M64)) != 0) return KDA_ERR_ARG;
     if ((majors & KDA_SELFTEST_B_MN_MAJOR) && (n % 64) != 0) return KDA_ERR_ARG;
     if (!aligned4(cycles)) return KDA_ERR_ALIGN;
     int* st = status_ptr();
@@ -468,8 +468,9 @@ kda_status_t kda_selftest_mma_rate(int n, int k, int majors, int reps, float* cy
 
 kda_status_t kda_selftest_umma(const void* a, const void* b, float* d, int n, int flags, kda_stream_t stream) {
     if (!a || !b || !d || n < 16 || n > 256 || (n % 16) != 0) return KDA_ERR_ARG;
-    if ((flags & ~(KDA_SELFTEST_B_MN_MAJOR | KDA_SELFTEST_A_TMEM | KDA_SELFTEST_A_MN_MAJOR)) != 0) return KDA_ERR_ARG;
-    if ((flags & KDA_SELFTEST_A_TMEM) && (flags & KDA_SELFTEST_A_MN_MAJOR)) return KDA_ERR_ARG;
+    if ((flags & ~(KDA_SELFTEST_B_MN_MAJOR | KDA_SELFTEST_A_TMEM | KDA_SELFTEST_A_MN_MAJOR | KDA_SELFTEST_M64)) != 0)
+        return KDA_ERR_ARG;
+    if ((flags & KDA_SELFTEST_A_TMEM) && (flags & (KDA_SELFTEST_A_MN_MAJOR | KDA_SELFTEST_M64))) return KDA_ERR_ARG;
     if ((flags & KDA_SELFTEST_B_MN_MAJOR) && (n % 32) != 0) return KDA_ERR_ARG;
     if (!aligned16(a) || !aligned16(b) || !aligned16(d)) return KDA_ERR_ALIGN;
     int* st = status_ptr();

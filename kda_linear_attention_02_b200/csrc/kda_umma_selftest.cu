@@ -12,7 +12,7 @@ namespace kda {
 __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16* __restrict__ a,
                                                             const __nv_bfloat16* __restrict__ b,
                                                             float* __restrict__ d, int n, int flags, int* status) {
-    const int b_mn = flags & 1, a_tmem = flags & 2, a_mn = flags & 4;
+    const int b_mn = flags & 1, a_tmem = flags & 2, a_mn = flags & 4, m64 = flags & 8;
     extern __shared__ __align__(1024) uint8_t raw[];
     uint8_t* base = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);   // stays a shared-memory pointer
     uint8_t* sA = base;                 // 128 rows x 128 B
@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
         tc_fence_after();
     }
     if (t == 0) {
-        const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0, a_mn != 0);
+        const uint32_t idesc = idesc_bf16(m64 ? 64 : 128, n, false, b_mn != 0, a_mn != 0);
         for (int kk = 0; kk < 4; ++kk) {
             const uint64_t db = b_mn ? sdesc_mn_sw128(smem_u32(sB) + kk * 2048, lbo)
                                      : sdesc_k_sw128(smem_u32(sB) + kk * 32);
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(128) selftest_umma_kernel(const __nv_bfloat16*
 // for before the next.  cycles[2 * blockIdx.x + {0, 1}] = SM cycles per product in the two modes.
 __global__ void __launch_bounds__(128) selftest_mma_rate_kernel(int n, int k, int majors, int reps, float* cycles,
                                                                 int* status) {
-    const int b_mn = majors & 1, a_mn = majors & 4;
+    const int b_mn = majors & 1, a_mn = majors & 4, m64 = majors & 8;
     extern __shared__ __align__(1024) uint8_t raw[];
     uint8_t* base = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
     uint8_t* sA = base;                          // K-major [k / 64][128 rows][128 B] or MN-major [2][k][128 B]
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(128) selftest_mma_rate_kernel(int n, int k, in
     tc_fence_after();
     const uint32_t tm = tbase;
     if (t == 0) {
-        const uint32_t idesc = idesc_bf16(128, n, false, b_mn != 0, a_mn != 0);
+        const uint32_t idesc = idesc_bf16(m64 ? 64 : 128, n, false, b_mn != 0, a_mn != 0);
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
         auto product = [&]() {
             for (int ks = 0; ks < k / 16; ++ks) {

@@ -128,13 +128,15 @@ def test_decode_and_compose_host_argument_errors(lib):
                                    None) == -3
     assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 20, 0, None) == -1
     assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 48, 1, None) == -1   # MN-major: n % 32
-    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 64, 8, None) == -1   # unknown flag bit
+    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 64, 16, None) == -1  # unknown flag bit
+    assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 64, 10, None) == -1  # A in TMEM with M = 64
     assert lib.kda_selftest_umma(vp(0x1000), vp(0x2000), vp(0x3000), 64, 6, None) == -1   # A both in TMEM and MN-major
     # tensor-core rate diagnostic: shape limits and the cycles buffer are checked before any launch
     assert lib.kda_selftest_mma_rate(8, 64, 0, 16, vp(0x1000), 1, None) == -1       # n below 16
     assert lib.kda_selftest_mma_rate(160, 96, 0, 16, vp(0x1000), 1, None) == -1     # k not 64 or 128
     assert lib.kda_selftest_mma_rate(96, 64, 1, 16, vp(0x1000), 1, None) == -1      # MN-major needs n % 64 == 0
     assert lib.kda_selftest_mma_rate(128, 64, 2, 16, vp(0x1000), 1, None) == -1     # no A from TMEM here
+    assert lib.kda_selftest_mma_rate(128, 64, 16, 16, vp(0x1000), 1, None) == -1    # unknown flag bit
     assert lib.kda_selftest_mma_rate(128, 64, 0, 0, vp(0x1000), 1, None) == -1      # no repetitions
     assert lib.kda_selftest_mma_rate(128, 64, 0, 16, None, 1, None) == -1
     assert lib.kda_selftest_mma_rate(128, 64, 0, 16, vp(0x1002), 1, None) == -2     # unaligned buffer

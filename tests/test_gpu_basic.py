@@ -39,18 +39,32 @@ def test_selftest_umma_matches_matmul(n, mn, at, amn):
 
 
 
-@pytest.mark.parametrize("n,k,mn,amn", [(160, 64, False, False), (64, 64, False, False), (128, 128, True, False),
-                                        (64, 128, False, True)])
-def test_selftest_mma_rate_is_plausible(n, k, mn, amn):
+@pytest.mark.parametrize("n,amn", [(64, False), (128, True)])
+def test_selftest_umma_m64_lane_layout(n, amn):
+    # M = 64: accumulator row 16 j + i sits in TMEM lane 32 j + i (lanes 0..15 of each 32-lane quarter)
+    g = torch.Generator(DEV).manual_seed(64 + n)
+    a = torch.randn(128, 64, device=DEV, generator=g).to(torch.bfloat16)
+    b = torch.randn(n, 64, device=DEV, generator=g).to(torch.bfloat16)
+    d = torch.full((128, n), float("nan"), device=DEV)
+    kda.kda_selftest_umma(a, b, d, a_mn_major=amn, m64=True)
+    ref = (a[:64].double() @ b.double().T).cpu().numpy()
+    lanes = [32 * (r // 16) + r % 16 for r in range(64)]
+    np.testing.assert_allclose(d.cpu().numpy()[lanes], ref, rtol=1e-4, atol=1e-4)
+
+
+@pytest.mark.parametrize("n,k,mn,amn,m64", [(160, 64, False, False, False), (64, 64, False, False, False),
+                                            (128, 128, True, False, False), (64, 128, False, True, False),
+                                            (128, 128, False, True, True)])
+def test_selftest_mma_rate_is_plausible(n, k, mn, amn, m64):
     # one CTA per SM times the product shape; the rate must lie between a small fraction and about the
     # hardware's dense bf16 rate (8192 FLOP per cycle per SM), and products one at a time never beat
     # products back to back
-    cyc = kda.kda_selftest_mma_rate(n, k, b_mn_major=mn, a_mn_major=amn, reps=64)
+    cyc = kda.kda_selftest_mma_rate(n, k, b_mn_major=mn, a_mn_major=amn, m64=m64, reps=64)
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
     c = cyc.cpu()
     assert bool((c > 0).all()), "a bounded wait ran out"
-    flop = 2.0 * 128 * n * k
+    flop = 2.0 * (64 if m64 else 128) * n * k
     rate = flop / c[:, 0]
     assert float(rate.max()) <= 8192 * 1.05 and float(rate.min()) >= 200
     assert bool((c[:, 1] >= 0.9 * c[:, 0]).all())
