@@ -240,7 +240,8 @@ template <typename T, int DK, int DV, bool VERIFY>
 __global__ void __launch_bounds__(spec_threads<DV>(), 1024 / spec_threads<DV>() / 2)
 decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T* __restrict__ k,
                     const T* __restrict__ v, const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                    int H, int n_draft, const int32_t* __restrict__ n_accept, T* __restrict__ o, int* status) {
+                    int H, int n_draft, const int32_t* __restrict__ n_accept, T* __restrict__ o, bool pre16,
+                    int* status) {
     constexpr int DVS = kSpecSlice;
     static_assert(DV % DVS == 0, "slice");
     constexpr int NT = spec_threads<DV>();
@@ -261,37 +262,64 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
         if (steps == 0) return;
     }
     auto row_of = [&](int d) { return (static_cast<size_t>(seq) * n_draft + d) * H + h; };
-    // the first draft's inputs are loaded ahead of the state stream, so that they do not queue behind it,
-    // and converted once the state loads have been issued
-    TokenIn x;
-    T rq{}, rk{}, rv{};
+    // The inputs of the first kPre drafts go to shared memory by 16-byte asynchronous copies, issued ahead
+    // of the state stream, so that no draft waits for a global load; later drafts (n_draft > kPre) are
+    // loaded into registers while the one before is applied.
+    constexpr int kPre = 4;
+    __shared__ __align__(16) float pre_la[kPre][DK];
+    __shared__ __align__(16) T pre_k[kPre][DK];
+    __shared__ __align__(16) T pre_q[kPre][DK];
+    __shared__ __align__(16) T pre_v[kPre][DVS];
+    const int npre = !pre16 ? 0 : (steps < kPre ? steps : kPre);   // pre16: q, k, v, log_alpha 16-byte aligned
     {
-        const size_t row = row_of(0);
-        if (t < DK) {
-            x.la = log_alpha[row * DK + t];
-            rk = k[row * DK + t];
-            if (VERIFY) rq = q[row * DK + t];
+        constexpr int CLA = DK * 4 / 16, CK = DK * static_cast<int>(sizeof(T)) / 16,
+                      CV = DVS * static_cast<int>(sizeof(T)) / 16;
+        constexpr int CPD = CLA + CK * (VERIFY ? 2 : 1) + CV;   // 16-byte chunks per draft
+        for (int e = t; e < npre * CPD; e += NT) {
+            const int d = e / CPD;
+            int c = e % CPD;
+            const size_t row = row_of(d);
+            if (c < CLA) {
+                cp_async16(&pre_la[d][4 * c], log_alpha + row * DK + 4 * c);
+            } else if ((c -= CLA) < CK) {
+                cp_async16(&pre_k[d][c * 16 / sizeof(T)], k + row * DK + c * 16 / sizeof(T));
+            } else if ((c -= CK) < CV) {
+                cp_async16(&pre_v[d][c * 16 / sizeof(T)], v + row * DV + j0 + c * 16 / sizeof(T));
+            } else {
+                c -= CV;
+                cp_async16(&pre_q[d][c * 16 / sizeof(T)], q + row * DK + c * 16 / sizeof(T));
+            }
         }
-        if (t < DVS) rv = v[row * DV + j0 + t];
-        if (t == 0) x.beta = beta[row];
     }
+    float beta_pre = 0.f;   // thread d < npre: beta of draft d
+    if (t < npre) beta_pre = beta[row_of(t)];
     asm volatile("" ::: "memory");
     // state rows are DV wide; this CTA's float4 column groups start at j0
     float4* S = reinterpret_cast<float4*>(state + static_cast<size_t>(head) * DK * DV + j0);
     float4 s[DT::RPT];
 #pragma unroll
     for (int r = 0; r < DT::RPT; ++r) s[r] = __ldcs(S + (rg * DT::RPT + r) * (DV / 4) + cg);
-    if (t < DK) {
-        x.k = to_f32(rk);
-        if (VERIFY) x.q = to_f32(rq);
-    }
-    if (t < DVS) x.v = to_f32(rv);
-    // token d + 1's inputs are loaded into registers while token d is applied, then staged
+    cp_async_wait_all();
+    __shared__ float pre_beta[kPre];
+    if (t < npre) pre_beta[t] = beta_pre;
+    __syncthreads();
+    TokenIn x;
     auto load = [&](TokenIn& x, int d) {
-        const size_t row = row_of(d);
-        load_token<T, DK, DVS, VERIFY>(x, VERIFY ? q + row * DK : nullptr, k + row * DK, v + row * DV + j0,
-                                       log_alpha + row * DK, beta + row);
+        if (d < npre) {   // this thread's elements of a preloaded draft
+            if (t < DK) {
+                x.la = pre_la[d][t];
+                x.k = to_f32(pre_k[d][t]);
+                if (VERIFY) x.q = to_f32(pre_q[d][t]);
+            }
+            if (t < DVS) x.v = to_f32(pre_v[d][t]);
+            if (t == 0) x.beta = pre_beta[d];
+        } else {
+            const size_t row = row_of(d);
+            load_token<T, DK, DVS, VERIFY>(x, VERIFY ? q + row * DK : nullptr, k + row * DK, v + row * DV + j0,
+                                           log_alpha + row * DK, beta + row);
+        }
     };
+    load(x, 0);
     stage_token<DK, DVS, NT, VERIFY>(sh, 0, x);
     for (int d = 0; d < steps; ++d) {
         const int par = d & 1;
@@ -341,11 +369,15 @@ cudaError_t launch_multi_t(float* state, const void* q, const void* k, const voi
     const T* kk = static_cast<const T*>(k);
     const T* vv = static_cast<const T*>(v);
     const dim3 grid(n * H, DV / kSpecSlice), block(spec_threads<DV>());
+    // the first drafts' inputs are copied to shared memory 16 bytes at a time when every base is 16-byte
+    // aligned (every row and slice offset is a multiple of 16 bytes); otherwise they are loaded per element
+    auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    const bool pre16 = a16(kk) && a16(vv) && a16(la) && (n_accept || a16(qq));
     if (n_accept)
         return launch_chained(decode_multi_kernel<T, DK, DV, false>, grid, block, s, state, qq, kk, vv, la, beta, H,
-                              n_draft, n_accept, static_cast<T*>(nullptr), status);
+                              n_draft, n_accept, static_cast<T*>(nullptr), pre16, status);
     return launch_chained(decode_multi_kernel<T, DK, DV, true>, grid, block, s, state, qq, kk, vv, la, beta, H,
-                          n_draft, static_cast<const int32_t*>(nullptr), static_cast<T*>(o), status);
+                          n_draft, static_cast<const int32_t*>(nullptr), static_cast<T*>(o), pre16, status);
 }
 
 }  // namespace

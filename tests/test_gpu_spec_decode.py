@@ -64,6 +64,38 @@ def test_verify_and_commit_equal_sequential_steps(dtype, dk, dv):
         assert torch.equal(state[i], snaps[a][i]), f"sequence {i}, {a} accepted"
 
 
+def _unaligned(x):
+    """The same values one element past a 16-byte boundary (element-aligned, not 16-byte aligned)."""
+    buf = torch.empty(x.numel() + 1, dtype=x.dtype, device=x.device)
+    y = buf[1:].view(x.shape)
+    y.copy_(x)
+    return y
+
+
+@pytest.mark.parametrize("nd,unaligned", [(6, False), (4, True), (7, True)])
+def test_verify_and_commit_more_drafts_and_unaligned_inputs(nd, unaligned):
+    # the first four drafts' inputs are copied to shared memory when q, k, v and log_alpha are 16-byte
+    # aligned; later drafts, and every draft of unaligned inputs, are loaded element by element
+    n, H, d = 5, 2, 128
+    s0, steps_in = _inputs(n, H, d, d, nd, BF, seed=17 + nd)
+    q, k, v, la, b = (synth.draft_layout(x) for x in steps_in)
+    if unaligned:
+        q, k, v, la = (_unaligned(x) for x in (q, k, v, la))
+        assert all(x.data_ptr() % 16 != 0 for x in (q, k, v, la))
+    ref_o, snaps = _sequential(s0, steps_in, nd)
+    state = s0.clone()
+    o = torch.empty(n * nd, H, d, dtype=BF, device=DEV)
+    kda.kda_decode_verify(state, q, k, v, la, b, o)
+    torch.cuda.synchronize()
+    assert torch.equal(state, s0)
+    assert torch.equal(o.view(n, nd, H, d).transpose(0, 1), ref_o)
+    acc = [nd, 0, 1, nd - 1, min(5, nd)][:n]
+    kda.kda_decode_commit(state, k, v, la, b, torch.tensor(acc, dtype=torch.int32, device=DEV))
+    assert kda.kda_get_device_status() == 0
+    for i, a in enumerate(acc):
+        assert torch.equal(state[i], snaps[a][i]), f"sequence {i}, {a} accepted"
+
+
 def test_single_draft_is_one_decode_step():
     n, H, d = 4, 2, 128
     s0, steps_in = _inputs(n, H, d, d, 1, BF, seed=5)
