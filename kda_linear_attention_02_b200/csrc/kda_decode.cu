@@ -168,6 +168,80 @@ __device__ __forceinline__ void token_step(float4 (&s)[DecodeTiling<DK, DV, NT>:
     }
 }
 
+// k . q of one token from its staged k and q (thread t < 32 sums elements t, t + 32, .. with fmaf, then
+// a butterfly over the warp), as token_step forms it; lane 0's value is the one used.
+template <int DK>
+__device__ __forceinline__ float token_kq(const float* __restrict__ kk, const float* __restrict__ qq, int lane) {
+    float kq = 0.f;
+    for (int i = lane; i < DK; i += 32) kq = fmaf(kk[i], qq[i], kq);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    return kq;
+}
+
+// token_step for the speculative kernels: the same arithmetic in the same order, arranged for a chain of
+// drafts.  k . q comes ready in *kq (staged with the token) unless kq_here, when warp 0 forms it as
+// token_step does; with OUT the output's column sums run on threads DV .. 2 DV - 1 beside u's on threads
+// 0 .. DV - 1, and those threads form o = u (k . q) + (Diag(a) S)^T q after the second barrier.
+template <typename T, int DK, int DV, int NT, bool OUT>
+__device__ __forceinline__ void draft_step(float4 (&s)[DecodeTiling<DK, DV, NT>::RPT], DecodeSmem<DK, DV, NT>& sh,
+                                           int par, float* kq, bool kq_here, T* __restrict__ o, bool update) {
+    using DT = DecodeTiling<DK, DV, NT>;
+    constexpr int CG = DT::CG, RG = DT::RG, RPT = DT::RPT;
+    static_assert(!OUT || NT >= 2 * DV, "threads for both reductions");
+    const int t = threadIdx.x, cg = t % CG, rg = t / CG;
+    float2 pk01 = make_float2(0.f, 0.f), pk23 = pk01, pq01 = pk01, pq23 = pk01;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = rg * RPT + r;
+        const float ak = sh.ak[par][i];
+        pk01 = __ffma2_rn(make_float2(ak, ak), make_float2(s[r].x, s[r].y), pk01);
+        pk23 = __ffma2_rn(make_float2(ak, ak), make_float2(s[r].z, s[r].w), pk23);
+        if (OUT) {
+            const float aq = sh.aq[par][i];
+            pq01 = __ffma2_rn(make_float2(aq, aq), make_float2(s[r].x, s[r].y), pq01);
+            pq23 = __ffma2_rn(make_float2(aq, aq), make_float2(s[r].z, s[r].w), pq23);
+        }
+    }
+    sh.red[0][rg][cg] = make_float4(pk01.x, pk01.y, pk23.x, pk23.y);
+    if (OUT) {
+        sh.red[1][rg][cg] = make_float4(pq01.x, pq01.y, pq23.x, pq23.y);
+        if (kq_here && t < 32) {
+            const float v = token_kq<DK>(sh.k[par], sh.q[par], t);
+            if (t == 0) *kq = v;
+        }
+    }
+    __syncthreads();
+
+    float pqj = 0.f;
+    if (t < DV) {
+        const float* red0 = reinterpret_cast<const float*>(sh.red[0]);
+        float p = 0.f;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) p += red0[g * DV + t];
+        sh.u[par][t] = sh.beta[par] * (sh.v[par][t] - p);
+    } else if (OUT && t < 2 * DV) {
+        const float* red1 = reinterpret_cast<const float*>(sh.red[1]);
+#pragma unroll
+        for (int g = 0; g < RG; ++g) pqj += red1[g * DV + t - DV];
+    }
+    __syncthreads();
+    if (OUT && t >= DV && t < 2 * DV) o[t - DV] = from_f32<T>(fmaf(sh.u[par][t - DV], *kq, pqj));
+    if (!update) return;
+
+    const float4 u4 = reinterpret_cast<const float4*>(sh.u[par])[cg];
+    const float2 u01 = make_float2(u4.x, u4.y), u23 = make_float2(u4.z, u4.w);
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = rg * RPT + r;
+        const float a = sh.a[par][i], kk = sh.k[par][i];
+        const float2 a2 = make_float2(a, a), k2 = make_float2(kk, kk);
+        const float2 s01 = __ffma2_rn(a2, make_float2(s[r].x, s[r].y), __fmul2_rn(k2, u01));
+        const float2 s23 = __ffma2_rn(a2, make_float2(s[r].z, s[r].w), __fmul2_rn(k2, u23));
+        s[r] = make_float4(s01.x, s01.y, s23.x, s23.y);
+    }
+}
+
 // MX: q, k, v are MXFP8 codes with their scale arrays (q_scale, k_scale [n, H, dk / 32], v_scale
 // [n, H, dv / 32]) and T is the type of o (bf16).
 template <typename T, int DK, int DV, bool MX>
@@ -319,6 +393,24 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
                                            log_alpha + row * DK, beta + row);
         }
     };
+    // k . q of the preloaded drafts, formed once by warp 0 (the other drafts' in their own step)
+    __shared__ float pre_kq[kPre];
+    if (VERIFY && t < 32) {
+        for (int d = 0; d < npre; ++d) {
+            float kf[DK / 32], qf[DK / 32];
+#pragma unroll
+            for (int m = 0; m < DK / 32; ++m) {
+                kf[m] = to_f32(pre_k[d][t + 32 * m]);
+                qf[m] = to_f32(pre_q[d][t + 32 * m]);
+            }
+            float kq = 0.f;
+#pragma unroll
+            for (int m = 0; m < DK / 32; ++m) kq = fmaf(kf[m], qf[m], kq);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+            if (t == 0) pre_kq[d] = kq;
+        }
+    }
     load(x, 0);
     stage_token<DK, DVS, NT, VERIFY>(sh, 0, x);
     for (int d = 0; d < steps; ++d) {
@@ -326,8 +418,8 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
         if (d + 1 < steps) load(x, d + 1);
         __syncthreads();   // token d staged (and every reader of the other half is past token d - 1)
         // verify discards the state: the last draft needs its output only
-        token_step<T, DK, DVS, NT, VERIFY>(s, sh, par, VERIFY ? o + row_of(d) * DV + j0 : nullptr,
-                                           !VERIFY || d + 1 < steps);
+        draft_step<T, DK, DVS, NT, VERIFY>(s, sh, par, d < npre ? &pre_kq[d] : &sh.kq, d >= npre,
+                                           VERIFY ? o + row_of(d) * DV + j0 : nullptr, !VERIFY || d + 1 < steps);
         if (d + 1 < steps) stage_token<DK, DVS, NT, VERIFY>(sh, par ^ 1, x);
     }
     if (!VERIFY) {
