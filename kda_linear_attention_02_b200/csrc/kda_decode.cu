@@ -393,23 +393,24 @@ decode_multi_kernel(float* __restrict__ state, const T* __restrict__ q, const T*
                                            log_alpha + row * DK, beta + row);
         }
     };
-    // k . q of the preloaded drafts, formed once by warp 0 (the other drafts' in their own step)
+    // k . q of preloaded draft d, formed once by warp d (the other drafts' in their own step); read after
+    // the barriers ahead of each draft's output
     __shared__ float pre_kq[kPre];
-    if (VERIFY && t < 32) {
-        for (int d = 0; d < npre; ++d) {
-            float kf[DK / 32], qf[DK / 32];
+    static_assert(NT / 32 >= kPre, "a warp per preloaded draft");
+    if (VERIFY && (t >> 5) < npre) {
+        const int d = t >> 5, lane = t & 31;
+        float kf[DK / 32], qf[DK / 32];
 #pragma unroll
-            for (int m = 0; m < DK / 32; ++m) {
-                kf[m] = to_f32(pre_k[d][t + 32 * m]);
-                qf[m] = to_f32(pre_q[d][t + 32 * m]);
-            }
-            float kq = 0.f;
-#pragma unroll
-            for (int m = 0; m < DK / 32; ++m) kq = fmaf(kf[m], qf[m], kq);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-            if (t == 0) pre_kq[d] = kq;
+        for (int m = 0; m < DK / 32; ++m) {
+            kf[m] = to_f32(pre_k[d][lane + 32 * m]);
+            qf[m] = to_f32(pre_q[d][lane + 32 * m]);
         }
+        float kq = 0.f;
+#pragma unroll
+        for (int m = 0; m < DK / 32; ++m) kq = fmaf(kf[m], qf[m], kq);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+        if (lane == 0) pre_kq[d] = kq;
     }
     load(x, 0);
     stage_token<DK, DVS, NT, VERIFY>(sh, 0, x);
