@@ -278,13 +278,15 @@ def prefill_roofline(token_heads, ms, hbm, extra_bytes=0, read_b=PREFILL_READ_B,
 
 # The tcgen05 products of one (chunk, head) item and one chunk step, as the kernels issue them:
 # (phase, N, K, B MN-major, products of that shape per unit).  M = 128 throughout.
+# (name, N, K, B MN-major, A MN-major, products per unit); M = 128.  The state products are those of the
+# 128-column slices the prefill workload runs: products 1 and 3 transposed (state columns on the M side).
 MMA_PHASES = [
-    ("prep A: [K e^(g-b); Q e^(g-b)] x 160 anchored key rows, per 64-channel half", 160, 64, False, 2),
-    ("prep B, K part: [X; X] diag(beta) x -(K gamma)^T", 128, 64, False, 1),
-    ("prep B, V part: [X; X] diag(beta) x V (MN-major)", 128, 64, True, 1),
-    ("state 1: [-W; Q gamma] S (S MN-major)", 128, 128, True, 1),
-    ("state 2: Kdec^T U' (U' MN-major)", 128, 64, True, 1),
-    ("state 3: Aqk U' (U' MN-major)", 128, 64, True, 1),
+    ("prep A: [K e^(g-b); Q e^(g-b)] x 160 anchored key rows, per 64-channel half", 160, 64, False, False, 2),
+    ("prep B, K part: [X; X] diag(beta) x -(K gamma)^T", 128, 64, False, False, 1),
+    ("prep B, V part: [X; X] diag(beta) x V (MN-major)", 128, 64, True, False, 1),
+    ("state 1: S^T [-W; Q gamma]^T (S the MN-major A operand)", 128, 128, False, True, 1),
+    ("state 2: Kdec^T U' (U'^T the K-major B operand)", 128, 64, False, False, 1),
+    ("state 3: U'^T Aqk^T (N = 64 tokens)", 64, 64, False, False, 1),
 ]
 
 
@@ -294,14 +296,14 @@ def mma_phase_rates(kda, tc_tflops, n_sms, sm_mhz):
     import torch
     peak_fc = tc_tflops * 1e12 / (n_sms * sm_mhz * 1e6)
     rows = []
-    for name, n, k, mn, per_unit in MMA_PHASES:
-        cyc = kda.kda_selftest_mma_rate(n, k, b_mn_major=mn, reps=512)
+    for name, n, k, mn, amn, per_unit in MMA_PHASES:
+        cyc = kda.kda_selftest_mma_rate(n, k, b_mn_major=mn, a_mn_major=amn, reps=512)
         torch.cuda.synchronize()
         c = cyc.cpu()
         ok = c[:, 0] > 0
         b2b, single = float(c[ok, 0].mean()), float(c[ok, 1].mean())
         fl = 2.0 * 128 * n * k
-        rows.append({"phase": name, "M": 128, "N": n, "K": k, "b_mn_major": mn, "per_unit": per_unit,
+        rows.append({"phase": name, "M": 128, "N": n, "K": k, "b_mn_major": mn, "a_mn_major": amn, "per_unit": per_unit,
                      "cycles_back_to_back": round(b2b, 1), "cycles_single": round(single, 1),
                      "flop_per_cycle_sm_back_to_back": round(fl / b2b, 1),
                      "flop_per_cycle_sm_single": round(fl / single, 1),
