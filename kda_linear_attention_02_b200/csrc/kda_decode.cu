@@ -180,8 +180,8 @@ __device__ __forceinline__ float token_kq(const float* __restrict__ kk, const fl
 }
 
 // token_step for the speculative kernels: the same arithmetic in the same order, arranged for a chain of
-// drafts.  k . q comes ready in *kq (staged with the token) unless kq_here, when warp 0 forms it as
-// token_step does; with OUT the output's column sums run on threads DV .. 2 DV - 1 beside u's on threads
+// drafts.  k . q comes ready in *kq (formed ahead, for a preloaded draft) unless kq_here, when warp 0
+// forms it as token_step does; with OUT the output's column sums run on threads DV .. 2 DV - 1 beside u's on threads
 // 0 .. DV - 1, and those threads form o = u (k . q) + (Diag(a) S)^T q after the second barrier.
 template <typename T, int DK, int DV, int NT, bool OUT>
 __device__ __forceinline__ void draft_step(float4 (&s)[DecodeTiling<DK, DV, NT>::RPT], DecodeSmem<DK, DV, NT>& sh,
