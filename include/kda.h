@@ -137,8 +137,8 @@ KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v,
  * is as for kda_chunk_fwd with dtype KDA_BF16, and so are the supported sizes (dk = 128, dv in {64, 128}).
  * The codes are decoded in the kernel that reads them; the values are exact (E4M3 has 4 significant bits)
  * as long as X * E4M3 stays inside the fp32 range, so the results equal kda_chunk_fwd's on the decoded
- * values given as bf16.  NaN inputs are outside the contract: a NaN code (E4M3 S.1111.111) is read as
- * +-480 and a NaN scale (0xFF) gives NaN results.
+ * values given as bf16.  NaN inputs are outside the contract: a NaN code (E4M3 S.1111.111) or a NaN
+ * scale (0xFF) gives NaN results.
  */
 KDA_API kda_status_t kda_chunk_fwd_mxfp8(const uint8_t* q, const uint8_t* q_scale,
                            const uint8_t* k, const uint8_t* k_scale,

@@ -358,14 +358,13 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 float2 kf, qf;
                 if constexpr (MX) {   // code x shared scale of the 32-channel block holding c0
                     const float* scf = reinterpret_cast<const float*>(sm + ps::SCF) + (c0 >> 5);
-                    const float2 un = f2(kE4M3Unscale);
                     // rows past n hold other tokens' (finite) codes, which nothing below lets through
                     const uint32_t kc = *reinterpret_cast<const uint16_t*>(kq_stage + r * 64 + (c0 & 63));
                     const uint32_t qc = *reinterpret_cast<const uint16_t*>(kq_stage + kKQ + r * 64 + (c0 & 63));
-                    kf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(kc), un), f2(scf[4 * (64 + r)]));
-                    qf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(qc), un), f2(scf[4 * r]));
+                    kf = __fmul2_rn(e4m3x2_to_f2(kc), f2(scf[4 * (64 + r)]));
+                    qf = __fmul2_rn(e4m3x2_to_f2(qc), f2(scf[4 * r]));
                     if (c0 < DV) {   // V as product B's MN-major operand
-                        const float2 vf = __fmul2_rn(__fmul2_rn(e4m3x2_scaled(vb8[j]), un), f2(scf[4 * (128 + r)]));
+                        const float2 vf = __fmul2_rn(e4m3x2_to_f2(vb8[j]), f2(scf[4 * (128 + r)]));
                         st_b32(sm + ps::VOP + (c0 >> 6) * 8192 + (r >> 3) * 1024 + (r & 7) * 128 +
                                    ((kk ^ static_cast<uint32_t>(r & 7)) << 4) + kb,
                                pack2(vf));

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -365,25 +366,22 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// MXFP8 inputs (OCP Microscaling Formats v1.0).  Two E4M3 codes (the first in the low byte) -> 2^-120
-// times their values as fp32, with integer operations only: a code's 7 magnitude bits placed at bits
-// 20..26 of an fp32 make exponent field e and mantissa m << 20, which reads 2^(e - 127) (1 + m / 8) for
-// e > 0 and m 2^-129 (an fp32 subnormal) for e = 0 -- exactly 2^-120 times the E4M3 magnitude either way;
-// the sign moves to bit 31.  (The NaN codes S.1111.111 read as +-480.)  Multiplying by 2^120 and then by
-// the shared scale is exact unless the value leaves the fp32 range.
-__device__ __forceinline__ float2 e4m3x2_scaled(uint32_t u) {
-    const uint32_t lo = ((u << 20) & 0x07F00000u) | ((u << 24) & 0x80000000u);
-    const uint32_t hi = ((u << 12) & 0x07F00000u) | ((u << 16) & 0x80000000u);
-    return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+// MXFP8 inputs (OCP Microscaling Formats v1.0).  Two E4M3 codes (the first in the low byte of u) to
+// fp32 by the hardware conversion to an f16 pair: every E4M3 value is exact in f16 (|x| <= 448, finest step
+// 2^-9), the NaN codes S.1111.111 become NaN, and the widening to fp32 is exact.  The shared scale then
+// follows as one power-of-two multiply, exact unless the value leaves the fp32 range.
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t u) {
+    uint32_t h;
+    asm("{\n .reg .b16 c;\n cvt.u16.u32 c, %1;\n cvt.rn.f16x2.e4m3x2 %0, c;\n}" : "=r"(h) : "r"(u));
+    return __half22float2(*reinterpret_cast<__half2*>(&h));
 }
-constexpr float kE4M3Unscale = 1.329227995784916e36f;   // 2^120
 // E8M0 shared scale -> 2^(e - 127) (code 0 is the fp32 subnormal 2^-127, code 255 is NaN)
 __device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
     return e == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float(e ? e << 23 : 0x00400000u);
 }
 // One MXFP8 element: code c with the shared scale code e of its 32-element block.
 __device__ __forceinline__ float mx8_value(uint32_t c, uint32_t e) {
-    return e4m3x2_scaled(c).x * kE4M3Unscale * e8m0_to_f32(e);
+    return e4m3x2_to_f2(c).x * e8m0_to_f32(e);
 }
 
 template <typename T>

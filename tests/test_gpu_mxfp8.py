@@ -211,3 +211,29 @@ def test_mxfp8_decode_equals_bf16_decode_on_decoded_inputs():
         torch.cuda.synchronize()
         assert torch.equal(oa, ob), f"step {t}: o differs from the bf16 decode on the decoded inputs"
     assert torch.equal(sa, sb)
+
+
+def test_mxfp8_nan_codes_read_as_nan():
+    # OCP MX v1.0: the E4M3 codes S.1111.111 are NaN.  One such code in v of token 70, head 1 makes that
+    # head's outputs NaN from the chunk holding it on (the chunk's products take 0 x NaN = NaN, and the state
+    # carries it), in the chunk path and in the decode step; the other heads are unchanged
+    lengths = [200]
+    inp, mx = _mx_inputs(lengths, 3, 128, seed=41, skew=False, with_state0=True)
+    base = _run_mx(inp, mx)
+    vc = mx[4].clone()
+    vc[70, 1, 5] = 0x7F
+    bad = _run_mx(inp, (mx[0], mx[1], mx[2], mx[3], vc, mx[5]))
+    assert torch.equal(bad[0][:, 0], base[0][:, 0]) and torch.equal(bad[0][:, 2], base[0][:, 2])
+    assert torch.equal(bad[0][:64, 1], base[0][:64, 1])
+    assert bool(torch.isnan(bad[0][64:, 1].float()).any(dim=-1).all()), "every output from token 64 on has a NaN"
+    assert bool(torch.isnan(bad[1][0, 1]).any())
+    n, H, steps = 3, 2, 2
+    s0, dmx, la, b = _mx_decode_inputs(n, H, 128, 128, steps, seed=42)
+    dvc = dmx[4].clone()
+    dvc[0, 1, 0, 9] = 0xFF   # step 0, sequence 1, head 0
+    state = s0.clone()
+    o = torch.empty(n, H, 128, dtype=BF, device=DEV)
+    kda.kda_recurrent_step_mxfp8(state, dmx[0][0], dmx[1][0], dmx[2][0], dmx[3][0], dvc[0], dmx[5][0], la[0], b[0], o)
+    torch.cuda.synchronize()
+    assert bool(torch.isnan(o[1, 0].float()).any()) and bool(torch.isnan(state[1, 0]).any())
+    assert not bool(torch.isnan(o[0]).any()) and not bool(torch.isnan(state[0]).any())
