@@ -220,6 +220,8 @@ KDA_API kda_status_t kda_recurrent_step_mxfp8(float* state, const uint8_t* q, co
  *   beta [n*n_draft, H] fp32; o [n*n_draft, H, dv] of `dtype`;
  *   state [n, H, dk, dv] fp32 (16-byte aligned); n_accept: device int32 [n], each in 0..n_draft.
  * Supported: dk, dv in {64, 128}; n_draft >= 1.  Host-detectable errors return before any launch.
+ * q, k, v and log_alpha need element alignment only; when all four start on 16-byte boundaries the
+ * first four drafts' inputs are copied into the kernel's shared memory ahead of the state (faster).
  * A sequence whose n_accept is out of range keeps its state unchanged and sets the status word to
  * KDA_ERR_DEVICE_INPUT (read it with kda_get_device_status); the other sequences are committed.
  * Applying commit with n_accept[i] = a gives, bit for bit, the state of a consecutive
