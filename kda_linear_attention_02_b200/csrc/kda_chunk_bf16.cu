@@ -234,11 +234,16 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     // everything above is private set-up; the chunk table and the inputs come from earlier launches
     grid_dependency_wait();
-    // chunk table entry {first token, valid tokens} of a window item (n = 0: past the last chunk)
-    auto entry = [&](long long it) -> int2 { return it < n_items ? chunk_tab[it / H] : make_int2(0, 0); };
+    // Item it = window chunk c times H plus head h; a CTA's next item is gridDim.x further on, so (c, h)
+    // advance by (gridDim.x / H, gridDim.x % H) with a carry, without a 64-bit division per item.
+    // entry(c): the chunk table entry {first token, valid tokens} (n = 0: past the window's last chunk).
+    const long long n_chunks_win = n_items / H;
+    const int step_c = static_cast<int>(gridDim.x) / H, step_h = static_cast<int>(gridDim.x) % H;
+    auto entry = [&](long long ch) -> int2 { return ch < n_chunks_win ? chunk_tab[ch] : make_int2(0, 0); };
     long long item = blockIdx.x;
-    int2 loc = entry(item);
-    int h = static_cast<int>(item % H);
+    long long c = static_cast<int>(blockIdx.x) / H;
+    int h = static_cast<int>(blockIdx.x) % H;
+    int2 loc = entry(c);
     bool valid = loc.y > 0;
     if (valid) {
         if (t == 0) issue_kq(loc.x, h, 0);
@@ -249,8 +254,13 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int n = loc.y;
         uint8_t* pkt = packets + static_cast<size_t>(item) * P::BYTES;
         const long long nitem = item + gridDim.x;   // this CTA's next item
-        const int2 nloc = entry(nitem);
-        const int nh = static_cast<int>(nitem % H);
+        long long nc = c + step_c;
+        int nh = h + step_h;
+        if (nh >= H) {
+            nh -= H;
+            ++nc;
+        }
+        const int2 nloc = entry(nc);
         const bool nvalid = nloc.y > 0;
         // beta (threads 0..63) and the MXFP8 scale words (threads 64..255) of the chunk's rows go to shared
         // memory only later in the column pass, so that no thread waits for these loads before its first barrier
@@ -721,6 +731,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
         }
         item = nitem;
+        c = nc;
         loc = nloc;
         h = nh;
         valid = nvalid;
