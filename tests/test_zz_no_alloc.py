@@ -49,6 +49,30 @@ def test_noalloc_matches_workspace_entry_point_twice():
             assert torch.equal(a, b), f"no-alloc call {call}: {name} differs from kda_chunk_fwd"
 
 
+def test_noalloc_full_width_state_slices_over_windows():
+    # 4 sequences x 32 heads = 128 chains: the state pass runs full 128-column slices (transposed products);
+    # the packets (about 100 MB) exceed the 64 MiB array, so the call also runs window by window
+    H, D, S = 32, 128, 512
+    lengths = [700, 1300, 64, 513]
+    assert kda.kda_chunk_fwd_workspace_bytes(sum(lengths), 4, H, D, D) > (64 << 20)
+    inp = synth.make_inputs(lengths, H, D, D, dtype=BF, device=DEV, seed=23, with_state0=True)
+    ckcu = kda.kda_ckpt_offsets(inp.cu_seqlens.cpu(), S)
+    ckcu_d = ckcu.to(DEV)
+    ref = _outputs(inp, H, D, ckcu)
+    kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.state0, inp.cu_seqlens, ref[0], ref[1],
+                      ckpt_stride=S, checkpoints=ref[2], ckpt_cu=ckcu_d, final_transition=ref[3])
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    got = _outputs(inp, H, D, ckcu)
+    kda.kda_chunk_fwd_noalloc(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.state0, inp.cu_seqlens,
+                              got[0], got[1], ckpt_stride=S, checkpoints=got[2], ckpt_cu=ckcu_d,
+                              final_transition=got[3])
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    for name, a, b in zip(("o", "final_state", "checkpoints", "transition"), got, ref):
+        assert torch.equal(a, b), f"no-alloc call: {name} differs from kda_chunk_fwd"
+
+
 def test_noalloc_windows_over_the_fixed_array():
     # one 4096-token sequence at H=32: the full scratch (~172 MB of packets) exceeds the 64 MiB array while
     # its minimum (carried state + one chunk of packets) fits, so the call runs window by window and carries
