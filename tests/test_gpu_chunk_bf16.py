@@ -66,6 +66,20 @@ def test_bf16_128_column_transposed_state_pass():
         assert torch.equal(ck1[: (b - a) // 64], ck[c0:c0 + (b - a) // 64])
 
 
+def test_bf16_transposed_state_pass_with_empty_sequences():
+    # 4 sequences x 32 heads = 128 chains (128-column slices): an empty sequence keeps its start state and
+    # its transition is the identity; the others match the oracle
+    lengths = [0, 200, 0, 65]
+    H = 32
+    inp = synth.make_inputs(lengths, H, 128, 128, dtype=BF, device=DEV, seed=24, with_state0=True)
+    outs = _run_chunk(inp, BF, ckpt_stride=64, transition=True)
+    o, fs, ck, ckcu, tr = outs
+    for i in (0, 2):
+        assert torch.equal(fs[i], inp.state0[i])
+        assert torch.equal(tr[i], torch.eye(128, device=DEV).expand(H, 128, 128))
+    _check_chunk(inp, BF, outs, [1, 3], [0, 17, H - 1], ckpt_stride=64, transition=True)
+
+
 def test_bf16_zero_state_single_sequence():
     inp = synth.make_inputs([256], 2, 128, 128, dtype=BF, device=DEV, seed=0)
     outs = _run_chunk(inp, BF, init=False)
