@@ -234,12 +234,21 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     // everything above is private set-up; the chunk table and the inputs come from earlier launches
     grid_dependency_wait();
-    // Item it = window chunk c times H plus head h; a CTA's next item is gridDim.x further on, so (c, h)
-    // advance by (gridDim.x / H, gridDim.x % H) with a carry, without a 64-bit division per item.
-    // entry(c): the chunk table entry {first token, valid tokens} (n = 0: past the window's last chunk).
+    // Item it = c H + h; a CTA's next item is gridDim.x further on, so (c, h) advance by
+    // (gridDim.x / H, gridDim.x % H) with a carry, without a 64-bit division per item.  Item c takes the
+    // window's chunk n_valid - 1 - c: the chunks are prepared last to first, so that the state pass, which
+    // walks every chain from its first chunk, finds the packets written last (its first ones) still in L2.
+    // The window's valid chunks (n > 0) are a prefix of its table, the rest lying past the batch's last
+    // chunk, so a binary search over the table finds their count n_valid.
+    // entry(c): the chunk table entry {first token, valid tokens} of item c (n = 0: none).
     const long long n_chunks_win = n_items / H;
+    long long n_valid = 0;
+    for (long long hi = n_chunks_win; n_valid < hi;) {
+        const long long mid = (n_valid + hi) / 2;
+        if (chunk_tab[mid].y > 0) n_valid = mid + 1; else hi = mid;
+    }
     const int step_c = static_cast<int>(gridDim.x) / H, step_h = static_cast<int>(gridDim.x) % H;
-    auto entry = [&](long long ch) -> int2 { return ch < n_chunks_win ? chunk_tab[ch] : make_int2(0, 0); };
+    auto entry = [&](long long ch) -> int2 { return ch < n_valid ? chunk_tab[n_valid - 1 - ch] : make_int2(0, 0); };
     long long item = blockIdx.x;
     long long c = static_cast<int>(blockIdx.x) / H;
     int h = static_cast<int>(blockIdx.x) % H;
@@ -252,7 +261,7 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     while (valid) {
         const int n = loc.y;
-        uint8_t* pkt = packets + static_cast<size_t>(item) * P::BYTES;
+        uint8_t* pkt = packets + static_cast<size_t>((n_valid - 1 - c) * H + h) * P::BYTES;
         const long long nitem = item + gridDim.x;   // this CTA's next item
         long long nc = c + step_c;
         int nh = h + step_h;
