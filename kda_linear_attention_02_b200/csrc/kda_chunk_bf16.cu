@@ -166,7 +166,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // transposed into its upper triangle (AM[s][r] for s < r in the same tile)
     float* AM = reinterpret_cast<float*>(sm + ps::AM);
     float* XF = reinterpret_cast<float*>(sm + ps::XF);    // X = (I + A)^-1, fp32, pitch LDX
-    float* TT = reinterpret_cast<float*>(sm + ps::TOT);   // T = A_10 X_00 of a merge, pitch LDTT
+    float* TT = reinterpret_cast<float*>(sm + ps::TOT);   // T = A_10 X_00 of a level-1 merge, pitch LDTT
+    float* TS = AM;                                       // T of the level-2 merge, pitch LDTT (rows 0..31 of A)
 
     if (t == 0) {
         mbar_init(&bar_in, 1);
@@ -529,114 +530,130 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
         }
         tc_fence_before();
-        fence_proxy_async_smem();   // Aqk leaves by a bulk copy
-        __syncthreads();
-        // Aqk and Q gamma are final: warp 4 sends them to the packet (waited for before the next column pass)
-        if (t == 128) {
-            bulk_s2g(pkt + P::AQ, sm + ps::IAQ + 8192, 8192);
-            bulk_s2g(pkt + P::AW + 8192, sm + ps::QG, 8192);
-            bulk_s2g(pkt + P::AW + 16384 + 8192, sm + ps::QG + 8192, 8192);
-            bulk_commit();
-        }
-
-        // ---------------- X = (I + A)^-1 by blocked forward substitution over 16 x 16 tiles.
-        // Level 0: each diagonal block by forward substitution, one warp per block, lane = column, the
-        // column held in registers; a column of A comes as float4 broadcasts of a row of the transposed block.
-        if (w < 4) {
-            const int o0 = 16 * w, col = lane & 15;
-            float x[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) x[r] = (r == col) ? 1.f : 0.f;
-            float4 cur[4], nxt[4];
-#pragma unroll
-            for (int r4 = 0; r4 < 4; ++r4) cur[r4] = reinterpret_cast<const float4*>(AM + o0 * LDM + o0)[r4];
-#pragma unroll
-            for (int m = 0; m < 15; ++m) {
-                if (m + 1 < 15) {
-#pragma unroll
-                    for (int r4 = (m + 2) >> 2; r4 < 4; ++r4)
-                        nxt[r4] = reinterpret_cast<const float4*>(AM + (o0 + m + 1) * LDM + o0)[r4];
-                }
-                const float xm = x[m];
-#pragma unroll
-                for (int r4 = (m + 1) >> 2; r4 < 4; ++r4) {
-                    const float4 a = cur[r4];
-                    if (4 * r4 + 0 > m) x[4 * r4 + 0] = fmaf(-a.x, xm, x[4 * r4 + 0]);
-                    if (4 * r4 + 1 > m) x[4 * r4 + 1] = fmaf(-a.y, xm, x[4 * r4 + 1]);
-                    if (4 * r4 + 2 > m) x[4 * r4 + 2] = fmaf(-a.z, xm, x[4 * r4 + 2]);
-                    if (4 * r4 + 3 > m) x[4 * r4 + 3] = fmaf(-a.w, xm, x[4 * r4 + 3]);
-                }
-#pragma unroll
-                for (int r4 = 0; r4 < 4; ++r4) cur[r4] = nxt[r4];
+        // ---------------- X = (I + A)^-1 by blocked forward substitution over 16 x 16 tiles, each lane quarter's
+        // warps on their own: the K-row warps of quarter kq (warps kq and kq + 4, rows 32 kq .. 32 kq + 31 of A)
+        // invert the quarter's two diagonal blocks and merge them (levels 0 and 1) as soon as their own rows of
+        // A are written, while the Q-row warps (quarters 2, 3) finish Aqk, send it, and clear X above its
+        // diagonal blocks.  Level 2 follows a CTA barrier.
+        const int fg = lane >> 2, ft = lane & 3;   // fragment row group and column pair of this lane
+        if ((w & 3) >= 2) {
+            fence_proxy_async_smem();   // Aqk leaves by a bulk copy
+            named_bar_sync(1, 128);     // the four Q-row warps have written Aqk
+            // Aqk and Q gamma are final: warp 2 sends them to the packet (waited for before the next column pass)
+            if (t == 64) {
+                bulk_s2g(pkt + P::AQ, sm + ps::IAQ + 8192, 8192);
+                bulk_s2g(pkt + P::AW + 8192, sm + ps::QG, 8192);
+                bulk_s2g(pkt + P::AW + 16384 + 8192, sm + ps::QG + 8192, 8192);
+                bulk_commit();
             }
-            if (lane < 16) {
-#pragma unroll
-                for (int r = 0; r < 16; ++r) XF[(o0 + r) * LDX + o0 + col] = x[r];
-            }
-        } else {
-            for (int e = t - 128; e < 64 * 64; e += 128) {   // the blocks above the diagonal are zero
+            const int zt = 32 * (2 * (w >> 2) + (w & 1)) + lane;   // 0..127 over warps 2, 3, 6, 7
+            for (int e = zt; e < 64 * 64; e += 128) {   // the blocks above the diagonal are zero
                 const int r = e >> 6, c = e & 63;
                 if ((c >> 4) > (r >> 4)) XF[r * LDX + c] = 0.f;
             }
+        } else {
+            const int kq = w & 3, hb = w >> 2;   // lane quarter (0, 1) and which of its two warps
+            if (kq == 1) named_bar_arrive(4, 128);   // rows 32..63 of A (A_10 of level 2) are written
+            named_bar_sync(2 + kq, 64);          // this quarter's rows of A are written
+            {   // level 0: diagonal block 2 kq + hb by forward substitution, lane = column, the column held in
+                // registers; a column of A comes as float4 broadcasts of a row of the transposed block
+                const int o0 = 16 * (2 * kq + hb), col = lane & 15;
+                float x[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) x[r] = (r == col) ? 1.f : 0.f;
+                float4 cur[4], nxt[4];
+#pragma unroll
+                for (int r4 = 0; r4 < 4; ++r4) cur[r4] = reinterpret_cast<const float4*>(AM + o0 * LDM + o0)[r4];
+#pragma unroll
+                for (int m = 0; m < 15; ++m) {
+                    if (m + 1 < 15) {
+#pragma unroll
+                        for (int r4 = (m + 2) >> 2; r4 < 4; ++r4)
+                            nxt[r4] = reinterpret_cast<const float4*>(AM + (o0 + m + 1) * LDM + o0)[r4];
+                    }
+                    const float xm = x[m];
+#pragma unroll
+                    for (int r4 = (m + 1) >> 2; r4 < 4; ++r4) {
+                        const float4 a = cur[r4];
+                        if (4 * r4 + 0 > m) x[4 * r4 + 0] = fmaf(-a.x, xm, x[4 * r4 + 0]);
+                        if (4 * r4 + 1 > m) x[4 * r4 + 1] = fmaf(-a.y, xm, x[4 * r4 + 1]);
+                        if (4 * r4 + 2 > m) x[4 * r4 + 2] = fmaf(-a.z, xm, x[4 * r4 + 2]);
+                        if (4 * r4 + 3 > m) x[4 * r4 + 3] = fmaf(-a.w, xm, x[4 * r4 + 3]);
+                    }
+#pragma unroll
+                    for (int r4 = 0; r4 < 4; ++r4) cur[r4] = nxt[r4];
+                }
+                if (lane < 16) {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) XF[(o0 + r) * LDX + o0 + col] = x[r];
+                }
+            }
+            named_bar_sync(2 + kq, 64);   // both diagonal blocks of the quarter are inverted
+            // Levels 1 and 2 merge two inverted diagonal blocks: X_10 = -X_11 (A_10 X_00).  The products are
+            // 16- and 32-row tiles, below the tensor-core MMA's smallest M, so they run as warp-level tf32
+            // m16n8k8 MMAs with fp32 accumulation on fragments loaded straight from shared memory.
+            {   // level 1: 16 -> 32, pair kq (rows 32 kq + 16 .., cols 32 kq ..), column tile hb of 8
+                const int nt = hb, rb = 32 * kq + 16, c0 = 32 * kq;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    if (ks < nt) continue;   // X_00 is zero above its diagonal
+                    const uint32_t a[4] = {to_tf32(AM[(rb + fg) * LDM + c0 + 8 * ks + ft]),
+                                           to_tf32(AM[(rb + fg + 8) * LDM + c0 + 8 * ks + ft]),
+                                           to_tf32(AM[(rb + fg) * LDM + c0 + 8 * ks + ft + 4]),
+                                           to_tf32(AM[(rb + fg + 8) * LDM + c0 + 8 * ks + ft + 4])};
+                    const uint32_t b[2] = {to_tf32(XF[(c0 + 8 * ks + ft) * LDX + c0 + 8 * nt + fg]),
+                                           to_tf32(XF[(c0 + 8 * ks + ft + 4) * LDX + c0 + 8 * nt + fg])};
+                    mma_tf32(d, a, b);
+                }
+                float* tt = TT + 16 * kq * LDTT + 8 * nt;
+                *reinterpret_cast<float2*>(tt + fg * LDTT + 2 * ft) = make_float2(d[0], d[1]);
+                *reinterpret_cast<float2*>(tt + (fg + 8) * LDTT + 2 * ft) = make_float2(d[2], d[3]);
+                __syncwarp();
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    const uint32_t a[4] = {to_tf32(XF[(rb + fg) * LDX + rb + 8 * ks + ft]),
+                                           to_tf32(XF[(rb + fg + 8) * LDX + rb + 8 * ks + ft]),
+                                           to_tf32(XF[(rb + fg) * LDX + rb + 8 * ks + ft + 4]),
+                                           to_tf32(XF[(rb + fg + 8) * LDX + rb + 8 * ks + ft + 4])};
+                    const uint32_t b[2] = {to_tf32(tt[(8 * ks + ft) * LDTT + fg]), to_tf32(tt[(8 * ks + ft + 4) * LDTT + fg])};
+                    mma_tf32(e, a, b);
+                }
+                float* xo = XF + rb * LDX + c0 + 8 * nt + 2 * ft;
+                xo[fg * LDX] = -e[0];
+                xo[fg * LDX + 1] = -e[1];
+                xo[(fg + 8) * LDX] = -e[2];
+                xo[(fg + 8) * LDX + 1] = -e[3];
+            }
+            if (kq == 0) {
+                // Level 2's first product, T = A_10 X_00 (32 x 32, K = 32), needs only X_00 and rows 32..63 of A,
+                // so quarter 0's warps form it (row tile hb) while quarter 1 is still inverting X_11.  T goes
+                // to rows 0..31 of A, which levels 0 and 1 of quarter 0 no longer read.
+                named_bar_sync(4, 128);   // both warps of quarter 0 are through level 1; quarter 1 has arrived
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        if (ks < nt) continue;   // X_00 is zero above its diagonal
+                        const int ra = 32 + 16 * hb + fg;
+                        const uint32_t a[4] = {to_tf32(AM[ra * LDM + 8 * ks + ft]), to_tf32(AM[(ra + 8) * LDM + 8 * ks + ft]),
+                                               to_tf32(AM[ra * LDM + 8 * ks + ft + 4]),
+                                               to_tf32(AM[(ra + 8) * LDM + 8 * ks + ft + 4])};
+                        const uint32_t b[2] = {to_tf32(XF[(8 * ks + ft) * LDX + 8 * nt + fg]),
+                                               to_tf32(XF[(8 * ks + ft + 4) * LDX + 8 * nt + fg])};
+                        mma_tf32(d, a, b);
+                    }
+                    float* ts = TS + 16 * hb * LDTT + 8 * nt;
+                    *reinterpret_cast<float2*>(ts + fg * LDTT + 2 * ft) = make_float2(d[0], d[1]);
+                    *reinterpret_cast<float2*>(ts + (fg + 8) * LDTT + 2 * ft) = make_float2(d[2], d[3]);
+                }
+            }
         }
         __syncthreads();
-        // Levels 1 and 2 merge two inverted diagonal blocks: X_10 = -X_11 (A_10 X_00).  The products are
-        // 16- and 32-row tiles, below the tensor-core MMA's smallest M, so they run as warp-level tf32
-        // m16n8k8 MMAs with fp32 accumulation on fragments loaded straight from shared memory.
-        const int fg = lane >> 2, ft = lane & 3;   // fragment row group and column pair of this lane
-        if (w < 4) {   // level 1: 16 -> 32, pair p (rows 32 p + 16 .., cols 32 p ..), column tile nt of 8
-            const int p = w >> 1, nt = w & 1, rb = 32 * p + 16, c0 = 32 * p;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                if (ks < nt) continue;   // X_00 is zero above its diagonal
-                const uint32_t a[4] = {to_tf32(AM[(rb + fg) * LDM + c0 + 8 * ks + ft]),
-                                       to_tf32(AM[(rb + fg + 8) * LDM + c0 + 8 * ks + ft]),
-                                       to_tf32(AM[(rb + fg) * LDM + c0 + 8 * ks + ft + 4]),
-                                       to_tf32(AM[(rb + fg + 8) * LDM + c0 + 8 * ks + ft + 4])};
-                const uint32_t b[2] = {to_tf32(XF[(c0 + 8 * ks + ft) * LDX + c0 + 8 * nt + fg]),
-                                       to_tf32(XF[(c0 + 8 * ks + ft + 4) * LDX + c0 + 8 * nt + fg])};
-                mma_tf32(d, a, b);
-            }
-            float* tt = TT + 16 * p * LDTT + 8 * nt;
-            *reinterpret_cast<float2*>(tt + fg * LDTT + 2 * ft) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2*>(tt + (fg + 8) * LDTT + 2 * ft) = make_float2(d[2], d[3]);
-            __syncwarp();
-            float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                const uint32_t a[4] = {to_tf32(XF[(rb + fg) * LDX + rb + 8 * ks + ft]),
-                                       to_tf32(XF[(rb + fg + 8) * LDX + rb + 8 * ks + ft]),
-                                       to_tf32(XF[(rb + fg) * LDX + rb + 8 * ks + ft + 4]),
-                                       to_tf32(XF[(rb + fg + 8) * LDX + rb + 8 * ks + ft + 4])};
-                const uint32_t b[2] = {to_tf32(tt[(8 * ks + ft) * LDTT + fg]), to_tf32(tt[(8 * ks + ft + 4) * LDTT + fg])};
-                mma_tf32(e, a, b);
-            }
-            float* xo = XF + rb * LDX + c0 + 8 * nt + 2 * ft;
-            xo[fg * LDX] = -e[0];
-            xo[fg * LDX + 1] = -e[1];
-            xo[(fg + 8) * LDX] = -e[2];
-            xo[(fg + 8) * LDX + 1] = -e[3];
-        }
-        __syncthreads();
-        {   // level 2: 32 -> 64, row tile mt of 16 and column tile nt of 8
+        {   // level 2: 32 -> 64, X_10 = -X_11 T: row tile mt of 16 and column tile nt of 8
             const int nt = w & 3, mt = w >> 2;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                if (ks < nt) continue;   // X_00 is zero above its diagonal
-                const int ra = 32 + 16 * mt + fg;
-                const uint32_t a[4] = {to_tf32(AM[ra * LDM + 8 * ks + ft]), to_tf32(AM[(ra + 8) * LDM + 8 * ks + ft]),
-                                       to_tf32(AM[ra * LDM + 8 * ks + ft + 4]),
-                                       to_tf32(AM[(ra + 8) * LDM + 8 * ks + ft + 4])};
-                const uint32_t b[2] = {to_tf32(XF[(8 * ks + ft) * LDX + 8 * nt + fg]),
-                                       to_tf32(XF[(8 * ks + ft + 4) * LDX + 8 * nt + fg])};
-                mma_tf32(d, a, b);
-            }
-            float* tt = TT + 16 * mt * LDTT + 8 * nt;
-            *reinterpret_cast<float2*>(tt + fg * LDTT + 2 * ft) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2*>(tt + (fg + 8) * LDTT + 2 * ft) = make_float2(d[2], d[3]);
-            named_bar_sync(1 + nt, 64);   // the two row tiles of this column tile of T are written
             float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
@@ -646,8 +663,8 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                                        to_tf32(XF[(ra + 8) * LDX + 32 + 8 * ks + ft]),
                                        to_tf32(XF[ra * LDX + 32 + 8 * ks + ft + 4]),
                                        to_tf32(XF[(ra + 8) * LDX + 32 + 8 * ks + ft + 4])};
-                const uint32_t b[2] = {to_tf32(TT[(8 * ks + ft) * LDTT + 8 * nt + fg]),
-                                       to_tf32(TT[(8 * ks + ft + 4) * LDTT + 8 * nt + fg])};
+                const uint32_t b[2] = {to_tf32(TS[(8 * ks + ft) * LDTT + 8 * nt + fg]),
+                                       to_tf32(TS[(8 * ks + ft + 4) * LDTT + 8 * nt + fg])};
                 mma_tf32(e, a, b);
             }
             float* xo = XF + (32 + 16 * mt) * LDX + 8 * nt + 2 * ft;

@@ -167,6 +167,11 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int c0, int
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Arrive at named barrier `id` (of `count` threads) without waiting: writes before it are visible to the
+// threads that pass the barrier with named_bar_sync.
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 // Programmatic dependent launch: a kernel launched with programmatic stream serialization may start
 // while the previous kernel of the stream is still finishing; this waits until that kernel has
 // completed and its memory is visible (a no-op for an ordinary launch).
