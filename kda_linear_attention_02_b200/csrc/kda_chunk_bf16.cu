@@ -801,9 +801,13 @@ struct SCfg {
     static constexpr uint32_t S_LBO = 128 * 128;      // MN-major: 64 columns x 128 K rows per block
     static constexpr uint32_t U_LBO = 64 * 128;       // MN-major: 64 columns x 64 K rows per block
     static constexpr uint32_t TMEM_COLS = 3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512);
+    // Transposed path: S^T in bf16 (lane = state column, two channels per 32-bit column) as product 1's A
+    // operand in TMEM, so that S never passes through shared memory
+    static constexpr uint32_t SA_COL = 3 * DVS;
     static __host__ __device__ constexpr uint32_t d1col(int ci) { return (ci & 1) ? 2 * DVS : 0; }
     static_assert(BYTES + 1024 <= 232448, "one CTA per SM");
-    static_assert(STAGE % 1024 == 0 && SOP % 1024 == 0 && UOP % 1024 == 0 && OST % 1024 == 0,
+    static_assert(!TR || SA_COL + kDK / 2 <= TMEM_COLS, "S^T operand inside the TMEM allocation");
+    static_assert(STAGE % 1024 == 0 && SOP % 1024 == 0 && UOP % 1024 == 0 && OST % 1024 == 0 && S_LBO % 1024 == 0,
                   "128B-swizzle operands and tiles on 1024-byte atoms");
 };
 
@@ -902,20 +906,21 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 const uint32_t sb = smem_u32(sm + st * C::STAGE);
                 if constexpr (C::TR) {
                     // D1^T = S^T [-W; Q gamma]^T   (M = 128 state columns, N = 128 tokens: -W rows, then Q gamma
-                    // rows; K = 128 channels), A = S MN-major, B = the packet's K-major [-W; Q gamma]
+                    // rows; K = 128 channels), A = S^T in TMEM, B = the packet's K-major [-W; Q gamma]
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        umma_f16(tm + C::d1col(ci), sdesc_mn_sw128(sop + ks * 2048, C::S_LBO),
-                                 sdesc_k_sw128(sb + C::AW + (ks >> 2) * 16384 + (ks & 3) * 32),
-                                 idesc_bf16(128, 128, false, false, true), ks > 0);
+                        umma_f16_ts(tm + C::d1col(ci), tm + C::SA_COL + ks * 8,
+                                    sdesc_k_sw128(sb + C::AW + (ks >> 2) * 16384 + (ks & 3) * 32), idesc_bf16(128, 128),
+                                    ks > 0);
                     umma_commit(&d1_full);
                     if (!mbar_wait(&up_ready, ci & 1, status)) break;
                     tc_fence_after();
-                    // D2 = Kdec^T U'   (M = 128 channels, N = 128 state columns, K = 64 tokens), B = U'^T K-major
+                    // D2^T = U'^T Kdec   (M = 128 state columns, N = 128 channels, K = 64 tokens): A = U'^T K-major,
+                    // B = the packet's Kdec^T rows (K-major)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        umma_f16(tm + DVS, sdesc_k_sw128(sb + C::KD + ks * 32), sdesc_k_sw128(uop + ks * 32),
-                                 idesc_bf16(128, DVS), ks > 0);
+                        umma_f16(tm + DVS, sdesc_k_sw128(uop + ks * 32), sdesc_k_sw128(sb + C::KD + ks * 32),
+                                 idesc_bf16(128, 128), ks > 0);
                     umma_commit(&d2_full);
                     if (!trans) {
                         // O^T = (Q gamma S)^T + U'^T Aqk^T: D1^T columns 64..127 (M = 128, N = 64, K = 64 tokens)
@@ -962,33 +967,60 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
         const int i = 32 * qw + lane;
         const int tk0 = 32 * ((w >> 2) & 1);
         const uint32_t lane_base = tm + (static_cast<uint32_t>(32 * qw) << 16);
+        // S[e]: element (channel i, slice column jw + e); transposed path: S^T, element (slice column i,
+        // channel jw + e), the layout of D2^T and of product 1's A operand in TMEM.  srow / scol: the state
+        // row (channel) and slice column of element e.
         float S[NCW];
+        auto srow = [&](int e) { return C::TR ? jw + e : i; };
+        auto scol = [&](int e) { return C::TR ? i : jw + e; };
         {
             const float* src = nullptr;
-            if (!first) src = carry + (sh * kDK + i) * CW + (trans ? DV : 0) + j0 + jw;
-            else if (!trans && initial_state) src = initial_state + (sh * kDK + i) * DV + j0 + jw;
+            size_t pitch = 0;
+            if (!first) {
+                src = carry + sh * kDK * CW + (trans ? DV : 0) + j0;
+                pitch = CW;
+            } else if (!trans && initial_state) {
+                src = initial_state + sh * kDK * DV + j0;
+                pitch = DV;
+            }
+            if constexpr (C::TR) {
 #pragma unroll
-            for (int e = 0; e < NCW / 4; ++e) {
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (src) x = reinterpret_cast<const float4*>(src)[e];
-                S[4 * e] = x.x; S[4 * e + 1] = x.y; S[4 * e + 2] = x.z; S[4 * e + 3] = x.w;
+                for (int e = 0; e < NCW; ++e) S[e] = src ? src[srow(e) * pitch + scol(e)] : 0.f;
+            } else {
+#pragma unroll
+                for (int e = 0; e < NCW / 4; ++e) {
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (src) x = reinterpret_cast<const float4*>(src + i * pitch + jw)[e];
+                    S[4 * e] = x.x; S[4 * e + 1] = x.y; S[4 * e + 2] = x.z; S[4 * e + 3] = x.w;
+                }
             }
             if (first && trans) {
 #pragma unroll
-                for (int j = 0; j < NCW; ++j) S[j] = (i == j0 + jw + j) ? 1.f : 0.f;
+                for (int e = 0; e < NCW; ++e) S[e] = (srow(e) == j0 + scol(e)) ? 1.f : 0.f;
             }
         }
-        // S (and later U') as a B operand: MN-major rows are written 8 columns at a time
+        // S as product 1's operand: MN-major rows of the B operand in shared memory, written 8 columns at a
+        // time; transposed path: S^T in bf16 into TMEM (this warp's lanes, channels jw .. jw + NCW)
         auto write_sop = [&]() {
+            if constexpr (C::TR) {
+                float p16[NCW / 2];
 #pragma unroll
-            for (int j = 0; j < NCW; j += 8) {
-                float f8[8];
+                for (int e = 0; e < NCW / 2; ++e) p16[e] = __uint_as_float(pack_bf16x2(S[2 * e], S[2 * e + 1]));
+                static_assert(NCW == 32, "one 16-column TMEM store per warp");
+                tmem_st16(lane_base + C::SA_COL + jw / 2, p16);
+                tmem_wait_st();
+            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f8[e] = S[j + e];
-                *reinterpret_cast<uint4*>(sm + C::SOP + sw128_mn_offset(jw + j, i, C::S_LBO)) = pack8(f8);
+                for (int j = 0; j < NCW; j += 8) {
+                    float f8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f8[e] = S[j + e];
+                    *reinterpret_cast<uint4*>(sm + C::SOP + sw128_mn_offset(jw + j, i, C::S_LBO)) = pack8(f8);
+                }
             }
         };
         write_sop();
+        tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_ready);
@@ -1091,16 +1123,26 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             }
             if (!mbar_wait(&d2_full, ci & 1, status)) break;
             tc_fence_after();
-            const float gam = *reinterpret_cast<const float*>(sb + C::G + i * 4);
-            {
+            {   // S = diag(gamma_C) S + D2 (transposed path: S^T = S^T diag(gamma_C) + D2^T, gamma per channel jw + e)
                 float vv[NCW];
 #pragma unroll
                 for (int cb = 0; cb < NCW; cb += 16)
                     tmem_ld16(lane_base + DVS + jw + cb, *reinterpret_cast<float(*)[16]>(vv + cb));
+                float gm[C::TR ? NCW : 1];
+                if constexpr (C::TR) {
+#pragma unroll
+                    for (int e = 0; e < NCW / 4; ++e) {
+                        const float4 g4 = *reinterpret_cast<const float4*>(sb + C::G + (jw + 4 * e) * 4);
+                        gm[4 * e] = g4.x; gm[4 * e + 1] = g4.y; gm[4 * e + 2] = g4.z; gm[4 * e + 3] = g4.w;
+                    }
+                } else {
+                    gm[0] = *reinterpret_cast<const float*>(sb + C::G + i * 4);
+                }
                 tmem_wait_ld_regs<NCW>(vv);
 #pragma unroll
                 for (int e = 0; e < NCW; e += 2) {
-                    const float2 a = __ffma2_rn(f2(gam), make_float2(S[e], S[e + 1]), make_float2(vv[e], vv[e + 1]));
+                    const float2 g2 = C::TR ? make_float2(gm[C::TR ? e : 0], gm[C::TR ? e + 1 : 0]) : f2(gm[0]);
+                    const float2 a = __ffma2_rn(g2, make_float2(S[e], S[e + 1]), make_float2(vv[e], vv[e + 1]));
                     S[e] = a.x; S[e + 1] = a.y;
                 }
             }
@@ -1108,7 +1150,7 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             if (lane == 0) mbar_arrive(&empty[st]);   // done with this stage
             write_sop();
             tc_fence_before();
-            fence_proxy_async_smem();
+            if constexpr (!C::TR) fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_ready);
             if (C::TR && !trans && w >= NEW / 2) {
@@ -1214,11 +1256,16 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
                 ck_wait = cpe;
                 if (n == 64) {
                     if (ck_slot < ck_end) {
-                        float4* dst = reinterpret_cast<float4*>(checkpoints +
-                                                                ((static_cast<size_t>(ck_slot) * H + h) * kDK + i) * DV + j0 + jw);
+                        float* ck = checkpoints + (static_cast<size_t>(ck_slot) * H + h) * kDK * DV + j0;
+                        if constexpr (C::TR) {   // one 128-byte row segment per element index and warp
 #pragma unroll
-                        for (int e = 0; e < NCW / 4; ++e)
-                            dst[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
+                            for (int e = 0; e < NCW; ++e) ck[srow(e) * DV + scol(e)] = S[e];
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(ck + i * DV + jw);
+#pragma unroll
+                            for (int e = 0; e < NCW / 4; ++e)
+                                dst[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
+                        }
                     } else if (lane == 0) {
                         set_status(status, KDA_ERR_DEVICE_INPUT);
                     }
@@ -1227,18 +1274,26 @@ state_bf16_kernel(const uint8_t* __restrict__ packets, const int32_t* __restrict
             }
         }
         if (o_issuer) bulk_wait0();
-        // row i, columns j0 + jw .. + NCW: 16-byte stores (every row start and column offset is a multiple of 4)
+        // the state (or transition) rows of this slice: pitch is the row length of the destination
         float* dst = nullptr;
+        size_t pitch = 0;
         if (last) {
-            if (trans) dst = final_transition + (sh * kDK + i) * kDK + j0 + jw;
-            else if (final_state) dst = final_state + (sh * kDK + i) * DV + j0 + jw;
+            if (trans) { dst = final_transition + sh * kDK * kDK + j0; pitch = kDK; }
+            else if (final_state) { dst = final_state + sh * kDK * DV + j0; pitch = DV; }
         } else {
-            dst = carry + (sh * kDK + i) * CW + (trans ? DV : 0) + j0 + jw;
+            dst = carry + sh * kDK * CW + (trans ? DV : 0) + j0;
+            pitch = CW;
         }
         if (dst) {
+            if constexpr (C::TR) {   // element e of every lane: one 128-byte row segment per warp
 #pragma unroll
-            for (int e = 0; e < NCW / 4; ++e)
-                reinterpret_cast<float4*>(dst)[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
+                for (int e = 0; e < NCW; ++e) dst[srow(e) * pitch + scol(e)] = S[e];
+            } else {   // row i, columns jw .. + NCW: 16-byte stores (row starts and column offsets are multiples of 4)
+#pragma unroll
+                for (int e = 0; e < NCW / 4; ++e)
+                    reinterpret_cast<float4*>(dst + i * pitch + jw)[e] =
+                        make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
+            }
         }
     }
     tc_fence_before();
