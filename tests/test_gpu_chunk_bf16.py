@@ -141,6 +141,26 @@ def test_bf16_windows_are_bit_identical():
             assert torch.equal(a, b)
 
 
+def test_bf16_transposed_state_pass_windows_are_bit_identical():
+    # 8 sequences x 16 heads = 128 chains run 128-column slices with S^T in tensor memory; over 3-chunk
+    # windows the state, the transition columns and the checkpoints pass from window to window through the
+    # carry, in the transposed layout, and must give what one window gives
+    lengths = [300, 5, 129, 64, 0, 700, 191, 1]
+    N, H = len(lengths), 16
+    inp = synth.make_inputs(lengths, H, 128, 128, dtype=BF, device=DEV, seed=23, with_state0=True)
+    full = _run_chunk(inp, BF, ckpt_stride=128, transition=True)
+    ub = (inp.total_tokens + 63) // 64 + N
+    index = ((N + 1) * 4 + 255) // 256 * 256
+    pk = (kda.kda_chunk_fwd_workspace_bytes(inp.total_tokens, N, H, 128, 128, kda.KDA_BF16) - index) // (ub * H)
+    small = kda.kda_chunk_fwd_min_workspace_bytes(N, H, 128, 128, kda.KDA_BF16) + 2 * H * pk
+    win = _run_chunk(inp, BF, ckpt_stride=128, transition=True, ws_bytes=small)
+    for a, b in zip(full, win):
+        if a is not None and a.dtype != torch.int32:
+            assert torch.equal(a, b)
+    _check_chunk(inp, BF, win, [0, 2, 5, 6, 7], [0, 9, H - 1], ckpt_stride=128, transition=True)
+    assert kda.kda_get_device_status() == 0
+
+
 def test_bf16_resume_from_checkpoint_matches_unsplit():
     # prefix reuse: run [0, len), take the checkpoint at b (a 512 boundary), run [b, len) from it
     lengths = [1536 + 77]
