@@ -64,16 +64,19 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
 }
 __device__ __forceinline__ uint32_t pack2(float2 f) { return pack_bf16x2(f.x, f.y); }
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
-// 2^x by the ex2.approx instruction; e^x is taken as 2^(x log2 e) with the scaling done two lanes at a time.
-// The flush-to-zero form: its callers pass log-decays inside one 16-token tile, |x| <= 16 |ln 0.0067| log2 e
-// < 116, so neither the argument nor the result is ever subnormal and the form without flushing (which
-// adds instructions to handle subnormals) would give the same values.
+constexpr float kLog2e = 1.4426950408889634f;
+// 2^x by the ex2.approx instruction in its flush-to-zero form (the form without flushing adds instructions
+// to handle subnormals); e^x is taken as 2^(x log2 e), with the scaling done two lanes at a time where it can.
+// The in-tile factors pass log-decays inside one 16-token tile, |x| <= 16 |ln 0.0067| log2 e < 116, so
+// neither argument nor result is ever subnormal there.  The anchors' factors (exp_ftz) span up to a whole
+// chunk and can underflow: a result below 2^-126 becomes 0 instead of a subnormal, which is the deep-underflow
+// limit of a decay product (the values it replaces are below 1.2e-38).
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float exp_ftz(float x) { return ex2_approx(x * kLog2e); }
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                       pack_bf16x2(f[6], f[7]));
@@ -355,17 +358,17 @@ prep_bf16_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 if (i == tq) { btx = bx[i]; bty = by[i]; bnx = bx[i + 1]; bny = by[i + 1]; }
-            const float ebx = __expf(btx), eby = __expf(bty);                 // e^{b_t}
-            const float ftx = __expf(bnx - btx), fty = __expf(bny - bty);     // e^{b_{t+1}-b_t}
-            const float ecx = __expf(bx[4] - bnx), ecy = __expf(by[4] - bny); // e^{g_C-b_{t+1}}
+            const float ebx = exp_ftz(btx), eby = exp_ftz(bty);                 // e^{b_t}
+            const float ftx = exp_ftz(bnx - btx), fty = exp_ftz(bny - bty);     // e^{b_{t+1}-b_t}
+            const float ecx = exp_ftz(bx[4] - bnx), ecy = exp_ftz(by[4] - bny); // e^{g_C-b_{t+1}}
             float dvx[4], dvy[4];   // e^{b_i - b_{t+1}}, i > t
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                dvx[i] = i > tq ? __expf(bx[i] - bnx) : 0.f;
-                dvy[i] = i > tq ? __expf(by[i] - bny) : 0.f;
+                dvx[i] = i > tq ? exp_ftz(bx[i] - bnx) : 0.f;
+                dvy[i] = i > tq ? exp_ftz(by[i] - bny) : 0.f;
             }
             if (w == 7)
-                *reinterpret_cast<float2*>(pkt + P::G + c0 * 4) = make_float2(__expf(bx[4]), __expf(by[4]));
+                *reinterpret_cast<float2*>(pkt + P::G + c0 * 4) = make_float2(exp_ftz(bx[4]), exp_ftz(by[4]));
 
             // -K gamma and Kdec along the 8 tokens, packed to bf16 pairs of consecutive tokens as they are made
             uint32_t tkw[2][4], tdw[2][4];
