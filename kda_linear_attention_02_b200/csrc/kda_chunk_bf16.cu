@@ -782,14 +782,15 @@ struct SCfg {
     static constexpr int NEW = DVS >= 64 ? 16 : 8;        // epilogue warps (NEW/4 share each TMEM lane quarter)
     static constexpr int NCW = DVS * 4 / NEW;              // state columns per epilogue warp (>= 16)
     static constexpr int NT = 32 * (NEW + 2);              // + producer warp + MMA warp
-    // Full 128-column slices run products 1 and 3 transposed, with the state columns on the M side:
-    // D1^T = S^T [-W; Q gamma]^T (A = S, MN-major) and O^T += U'^T Aqk^T, so that D1^T's TMEM lanes are
-    // state columns; warps 0..7 then form U' and warps 8..15 read O, 32 tokens per warp in the
-    // fragment layout of 16-lane TMEM loads and 8 x 8 matrix loads and stores.  Narrower slices cannot
-    // fill M = 128 and keep D1 = [-W; Q gamma] S.
+    // Full 128-column slices run all three products transposed, with the state columns on the M side:
+    // D1^T = S^T [-W; Q gamma]^T (A = S^T in TMEM), D2^T = U'^T Kdec and O^T += U'^T Aqk^T, so that D1^T's
+    // TMEM lanes are state columns; warps 0..7 then form U' and warps 8..15 read O, 32 tokens per warp in
+    // the fragment layout of 16-lane TMEM loads and 8 x 8 matrix loads and stores.  Narrower slices cannot
+    // fill M = 128 and keep D1 = [-W; Q gamma] S and D2 = Kdec^T U' (S and U' as MN-major B operands).
     static constexpr bool TR = DVS == 128;
-    // S and U' are staged MN-major (row = channel / token) in blocks of 64 columns; a 32-column slice
-    // fills half of one block (a product with N = 32 reads just those columns)
+    // Narrower slices stage S and U' MN-major (row = channel / token) in blocks of 64 columns; a 32-column
+    // slice fills half of one block (a product with N = 32 reads just those columns).  The transposed path
+    // stages U'^T K-major (row = state column) and keeps S out of shared memory (SOP unused)
     static constexpr int DVA = DVS >= 64 ? DVS : 64;
     static constexpr bool TMA_O = DVS >= 64;               // whole 64-column O tiles leave by tensor stores
     static constexpr int NST = DVS == 32 ? 3 : 2;
@@ -798,12 +799,13 @@ struct SCfg {
     static constexpr uint32_t AW = 0, KD = 32768, AQ = 49152, U = 57344, G = U + U_BYTES;
     static constexpr uint32_t STAGE = ((G + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SOP = NST * STAGE;      // S as B operand (N = DVS, K = 128)
-    static constexpr uint32_t UOP = SOP + DVA * 256;  // U' as B operand (N = DVS, K = 64)
+    static constexpr uint32_t UOP = SOP + DVA * 256;  // U' as B operand (N = DVS, K = 64); transposed: U'^T as A
     // O tile staging for the tensor store, [DVS/64][64 tokens][128 B] with the 128B swizzle (slices of whole
     // 64-column atoms only; narrower slices store O from registers)
     static constexpr uint32_t OST = UOP + DVA * 128;
     static constexpr uint32_t BYTES = OST + (TMA_O ? DVS * 128 : 0);
-    // TMEM: D1 double-buffered at columns [0, DVS) and [2 DVS, 3 DVS), D2 at [DVS, 2 DVS)
+    // TMEM: D1 double-buffered at columns [0, DVS) and [2 DVS, 3 DVS), D2 at [DVS, 2 DVS); transposed path:
+    // S^T in bf16 at [3 DVS, 3 DVS + 64)
     static constexpr uint32_t S_LBO = 128 * 128;      // MN-major: 64 columns x 128 K rows per block
     static constexpr uint32_t U_LBO = 64 * 128;       // MN-major: 64 columns x 64 K rows per block
     static constexpr uint32_t TMEM_COLS = 3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512);
