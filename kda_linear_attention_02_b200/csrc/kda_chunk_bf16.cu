@@ -22,18 +22,20 @@
 // finite (|.| <= 128 e^80.09 < fp32 max) and are dropped after the product.
 //
 // Kernels:
-//  prep_bf16_kernel   persistent, one (chunk, head) item at a time per CTA: TMA tensor loads of the
-//                     raw tiles (prefetched one item ahead), SIMT exponentials and operand
-//                     construction, tcgen05 products for A/Aqk (4 anchored variants) and for
-//                     X diag(beta) (-K gamma | V) (which yields -W and U), X by forward substitution
-//                     of the four 16 x 16 diagonal blocks and two merge levels on warp-level tf32
-//                     MMAs, and bulk TMA stores of the MMA-ready packet.
+//  prep_bf16_kernel   persistent, two CTAs per SM, one (chunk, head) item at a time per CTA, a window's
+//                     chunks taken last to first: TMA tensor loads of the raw tiles (prefetched one item
+//                     ahead), SIMT exponentials and operand construction, tcgen05 products for A/Aqk
+//                     (4 anchored variants) and for X diag(beta) (-K gamma | V) (which yields -W and U),
+//                     X by forward substitution of the four 16 x 16 diagonal blocks and two merge levels
+//                     on warp-level tf32 MMAs (the first two per TMEM lane quarter), and bulk TMA stores
+//                     of the MMA-ready packet.
 //  state_bf16_kernel  one CTA per (sequence, head, dv-slice), warp-specialised: a producer warp
 //                     streams packets through a shared-memory ring with bulk TMA, one thread issues
 //                     the tcgen05 products per chunk ([-W; Q gamma] S into a double-buffered
-//                     accumulator, then Kdec^T U' and Aqk U'), 8 or 16 epilogue warps
-//                     hold the fp32 state in registers and feed bf16 copies of S and U' back as the
-//                     next operands.
+//                     accumulator, then Kdec^T U' and Aqk U'; all three transposed on 128-column
+//                     slices), 8 or 16 epilogue warps hold the fp32 state in registers and feed bf16
+//                     copies of S and U' back as the next operands (S^T through tensor memory on
+//                     128-column slices).
 #include <cudaTypedefs.h>
 
 #include <cstring>
