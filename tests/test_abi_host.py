@@ -86,6 +86,29 @@ def test_workspace_sizes(lib):
     assert kda.kda_chunk_fwd_workspace_bytes(100, 1, 2, 64, 64, kda.KDA_BF16) == 0
 
 
+def test_workspace_layout_matches_the_documented_one(lib):
+    # workspace = chunk index (n + 1 int32, rounded to 256 B) + per chunk of the bound ceil(T / 64) + n:
+    # H packet slots and one 8-byte chunk-table entry; the windowed minimum holds the carried states
+    # [n, H, dk, dv + dk] fp32 (rounded to 256 B) and one chunk's worth.  A bf16 packet slot at dk = dv = 128
+    # is 74,752 bytes.
+    r256 = lambda x: (x + 255) // 256 * 256
+    for n, H in [(1, 1), (4, 32), (7, 3)]:
+        index = r256((n + 1) * 4)
+        per_chunk = kda.kda_chunk_fwd_workspace_bytes(64 * 10, n, H, 128, 128, kda.KDA_BF16) - \
+            kda.kda_chunk_fwd_workspace_bytes(64 * 9, n, H, 128, 128, kda.KDA_BF16)
+        assert per_chunk == H * 74752 + 8
+        for T in (0, 1, 64, 65, 4096, 100000):
+            ub = (T + 63) // 64 + n
+            assert kda.kda_chunk_fwd_workspace_bytes(T, n, H, 128, 128, kda.KDA_BF16) == index + ub * per_chunk
+            assert kda.kda_chunk_fwd_workspace_bytes(T, n, H, 128, 128, kda.KDA_MXFP8) == index + ub * per_chunk
+        carry = r256(n * H * 128 * (128 + 128) * 4)
+        assert kda.kda_chunk_fwd_min_workspace_bytes(n, H, 128, 128, kda.KDA_BF16) == index + carry + per_chunk
+        for dt, dk, dv in [(kda.KDA_BF16, 128, 64), (kda.KDA_F32, 64, 64), (kda.KDA_F32, 128, 128), (kda.KDA_F32, 64, 128)]:
+            pc = kda.kda_chunk_fwd_workspace_bytes(640, n, H, dk, dv, dt) - kda.kda_chunk_fwd_workspace_bytes(576, n, H, dk, dv, dt)
+            assert pc > 8 and (pc - 8) % H == 0
+            assert kda.kda_chunk_fwd_min_workspace_bytes(n, H, dk, dv, dt) == index + r256(n * H * dk * (dv + dk) * 4) + pc
+
+
 def _call_chunk(lib, **over):
     """Raw C call with fake (never dereferenced) pointers: all of these must fail on the host."""
     a = dict(q=0x1000, k=0x2000, v=0x3000, la=0x4000, b=0x5000, s0=None, cu=0x6000, n=2, T=100, H=4, dk=128,
